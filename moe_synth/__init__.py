@@ -1,0 +1,150 @@
+"""Seeded synthetic inputs for the routed MoE FFN layer.
+
+This module only draws random numbers and stores them in the layer's input formats; it holds
+none of the layer's own arithmetic (routing, permutation, activation quantisation, the expert
+contractions, the combine).  Both the CUDA path's tests/benchmark and the CPU oracle consume
+the same bytes produced here.
+
+Recipe (every tensor has its own seeded torch generator on the chosen device):
+  * x       ~ N(0, 1), rounded to bf16 (RNE) -- the hidden states;
+  * logits  ~ N(0, 1) fp32, plus a per-expert bias for two workloads:
+      - "normal": bias_e ~ N(0, 0.5) (0.5 read as the variance);
+      - "zipf":   bias_e = -1.2 * ln(rank_e), rank a seeded permutation of 1..E
+                  (the log of a Zipf(s = 1.2) probability up to a constant), so a few
+                  experts take most tokens;
+  * weights W ~ N(0, 1/fan_in) fp32 (fan_in = H for gate/up, I for down), stored quantised:
+      - FP8: one fp32 scale per (row, 512-element K block), s = amax/448 (1 when amax = 0),
+             codes = e4m3(W/s) by torch's float8_e4m3fn conversion (round to nearest even);
+      - int4: one bf16 scale per (row, 128-element K group), s = bf16(amax/7) (1 when 0),
+             q = clamp(round_half_even(W/s), -7, 7), two's-complement nibbles, the even K
+             index in the low nibble.
+Shapes follow the pages' models: a Qwen3.5-397B-shaped layer (512 experts x 1024, top-10,
+one shared expert of 1024, hidden 4096) at decode and prefill sizes; a DeepSeek-R1-shaped
+layer (hidden 7168, 256 experts x 2048, top-8, shared 2048) with skewed routing; a 4-bit
+128-expert layer; and a tiny layer for the oracle.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+CONFIGS = {
+    "tiny": dict(T=16, H=512, E=8, I=256, k=2, Is=0, wfmt="fp8", seed=0, bias=None,
+                 workload="tiny MoE layer T=16 H=512 E=8 I=256 top-2, FP8 e4m3 sc512"),
+    "decode": dict(T=512, H=4096, E=512, I=1024, k=10, Is=1024, wfmt="fp8", seed=1, bias=None,
+                   workload="Qwen3.5-397B-shaped MoE decode step T=512 H=4096 E=512 I=1024 "
+                            "top-10 + shared 1024, FP8 e4m3 sc512"),
+    "prefill": dict(T=8192, H=4096, E=512, I=1024, k=10, Is=1024, wfmt="fp8", seed=2,
+                    bias="normal",
+                    workload="Qwen3.5-397B-shaped MoE prefill T=8192 H=4096 E=512 I=1024 "
+                             "top-10 + shared 1024, FP8 e4m3 sc512, biased logits"),
+    "skewed": dict(T=4096, H=7168, E=256, I=2048, k=8, Is=2048, wfmt="fp8", seed=3, bias="zipf",
+                   workload="DeepSeek-R1-shaped MoE T=4096 H=7168 E=256 I=2048 top-8 + shared "
+                            "2048, FP8 e4m3 sc512, Zipf-skewed routing"),
+    "int4": dict(T=1024, H=4096, E=128, I=1536, k=8, Is=0, wfmt="int4", seed=4, bias=None,
+                 workload="4-bit-weight MoE T=1024 H=4096 E=128 I=1536 top-8, int4 g128 bf16"),
+}
+
+# tensor ids for the per-tensor generators
+_TID = {"x": 1, "logits": 2, "bias": 3, "rank": 4, "w_gate": 5, "w_up": 6, "w_down": 7,
+        "ws_gate": 8, "ws_up": 9, "ws_down": 10}
+
+
+def _gen(seed: int, tid: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(seed * 1_000_003 + tid * 7919 + 17)
+    return g
+
+
+def _quant_fp8(w: torch.Tensor):
+    """W [..., N, K] fp32 -> (codes uint8 [..., N, K], scales fp32 [..., N, ceil(K/512)])."""
+    K = w.shape[-1]
+    nb = (K + 511) // 512
+    pad = nb * 512 - K
+    wp = torch.nn.functional.pad(w, (0, pad)) if pad else w
+    blk = wp.reshape(*w.shape[:-1], nb, 512)
+    amax = blk.abs().amax(dim=-1)
+    s = torch.where(amax == 0, torch.ones_like(amax), amax / 448.0)
+    q = (blk / s.unsqueeze(-1)).clamp(-448.0, 448.0).to(torch.float8_e4m3fn)
+    q = q.reshape(*w.shape[:-1], nb * 512)[..., :K].contiguous().view(torch.uint8)
+    return q, s.contiguous()
+
+
+def _quant_int4(w: torch.Tensor):
+    """W [..., N, K] fp32 -> (packed uint8 [..., N, K/2], scales bf16 [..., N, K/128])."""
+    K = w.shape[-1]
+    assert K % 128 == 0
+    blk = w.reshape(*w.shape[:-1], K // 128, 128)
+    amax = blk.abs().amax(dim=-1)
+    s = (amax / 7.0).to(torch.bfloat16)
+    s = torch.where(s == 0, torch.ones_like(s), s)
+    q = torch.round(blk / s.float().unsqueeze(-1)).clamp(-7, 7).to(torch.int16)
+    q = q.reshape(*w.shape[:-1], K) & 0xF
+    packed = (q[..., 0::2] | (q[..., 1::2] << 4)).to(torch.uint8)
+    return packed.contiguous(), s.contiguous()
+
+
+def _weights(seed, tid, shape, fan_in, wfmt, device, chunk_elems=1 << 28):
+    """Draw W ~ N(0, 1/fan_in) of `shape` [E, N, K] in expert chunks and quantise."""
+    E, N, K = shape
+    g = _gen(seed, tid, device)
+    per = max(1, chunk_elems // (N * K))
+    qs, ss = [], []
+    for e0 in range(0, E, per):
+        e1 = min(E, e0 + per)
+        w = torch.randn((e1 - e0, N, K), generator=g, device=device, dtype=torch.float32)
+        w.mul_(1.0 / math.sqrt(fan_in))
+        q, s = _quant_fp8(w) if wfmt == "fp8" else _quant_int4(w)
+        qs.append(q)
+        ss.append(s)
+        del w
+    return torch.cat(qs, 0), torch.cat(ss, 0)
+
+
+def make_layer(name_or_cfg, device="cpu", **overrides) -> dict:
+    """Build one synthetic layer.  Returns a dict of torch tensors on `device` plus "dims"."""
+    cfg = dict(CONFIGS[name_or_cfg]) if isinstance(name_or_cfg, str) else dict(name_or_cfg)
+    cfg.update(overrides)
+    T, H, E, I, k, Is = (cfg[n] for n in ("T", "H", "E", "I", "k", "Is"))
+    seed, wfmt = cfg["seed"], cfg["wfmt"]
+    out = {"dims": dict(T=T, H=H, E=E, I=I, k=k, Is=Is, wfmt=wfmt), "cfg": cfg}
+    x = torch.randn((T, H), generator=_gen(seed, _TID["x"], device), device=device)
+    out["x"] = x.to(torch.bfloat16)
+    logits = torch.randn((T, E), generator=_gen(seed, _TID["logits"], device), device=device)
+    if cfg.get("bias") == "normal":
+        b = torch.randn((E,), generator=_gen(seed, _TID["bias"], device), device=device)
+        logits = logits + b * math.sqrt(0.5)
+    elif cfg.get("bias") == "zipf":
+        rank = torch.randperm(E, generator=_gen(seed, _TID["rank"], device), device=device) + 1
+        logits = logits + (-1.2) * torch.log(rank.to(torch.float32))
+    out["logits"] = logits.contiguous()
+    out["w_gate"], out["s_gate"] = _weights(seed, _TID["w_gate"], (E, I, H), H, wfmt, device)
+    out["w_up"], out["s_up"] = _weights(seed, _TID["w_up"], (E, I, H), H, wfmt, device)
+    out["w_down"], out["s_down"] = _weights(seed, _TID["w_down"], (E, H, I), I, wfmt, device)
+    if Is > 0:
+        out["ws_gate"], out["ss_gate"] = _weights(seed, _TID["ws_gate"], (1, Is, H), H, wfmt, device)
+        out["ws_up"], out["ss_up"] = _weights(seed, _TID["ws_up"], (1, Is, H), H, wfmt, device)
+        out["ws_down"], out["ss_down"] = _weights(seed, _TID["ws_down"], (1, H, Is), Is, wfmt, device)
+    return out
+
+
+def to_numpy(layer: dict) -> dict:
+    """Host copies with bf16 tensors as uint16 bit patterns (the oracle's input format)."""
+    res = {"dims": dict(layer["dims"])}
+    for key, v in layer.items():
+        if not isinstance(v, torch.Tensor):
+            continue
+        v = v.detach().cpu().contiguous()
+        if v.dtype == torch.bfloat16:
+            v = v.view(torch.int16).numpy().view(np.uint16)
+        else:
+            v = v.numpy()
+        res[key] = v
+    return res
+
+
+def weight_bytes(layer: dict) -> int:
+    return sum(v.numel() * v.element_size() for key, v in layer.items()
+               if isinstance(v, torch.Tensor) and key[:2] in ("w_", "s_", "ws", "ss"))

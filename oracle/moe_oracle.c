@@ -1,0 +1,558 @@
+/*
+ * moe_oracle.c -- plain fp64 CPU oracle of the routed Mixture-of-Experts FFN layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file defines what the layer computes so that the
+ * CUDA path can be checked against it.  Only the tests, the package entry's smoke
+ * check and the benchmark's CPU-baseline leg may load it.  It shares no code, header,
+ * table or constant with the CUDA library, and the CUDA library never calls it.
+ *
+ * Sources (page title, section):
+ *  [P1] "把 397B MoE 榨進 TPU7x：Google 拿到 4.7 倍加速" -- section "稀疏在哪裡：397B 參數、
+ *       17B 啟動": 512 routed experts, top-10 chosen by softmax probability, plus one
+ *       shared expert that runs for every token whatever the routing says.
+ *  [P1] same page, section "Kernel 手術台：RPA、Grouped GEMM v2、GDN 融合": the expert FFN is
+ *       a SwiGLU (gate and up projections, then down) over FP8 weights quantised with
+ *       512-element sub-channels.
+ *  [P1] same page, section "數值驗證：省下來的效能有沒有偷跑": the lowered path is audited
+ *       against a high-precision reference; the gating weights must not deviate.
+ *  [P2] "TPU推理外部化全面加速：InferenceX首份第三方性能數據發布" -- section "优化 MoE 路由与
+ *       专家内核": tokens are gathered into contiguous per-expert groups; the sort key packs
+ *       (expert id, token index); the combine is an un-permute weighted by the top-k weights.
+ *  [P4] "设计 AI 芯片的硬件与软件" -- section "数值格式，或如何制造便宜的脉动阵列": FP8 means the
+ *       E4M3 and E5M2 formats; products are accumulated at higher precision.
+ *  [P5] "Flash-Next 在 GPU 上到底在算什麼" -- section "① 專家 FFN": each expert computes
+ *       input x matrix A -> activation -> x matrix B, with 4/8-bit weights dequantised
+ *       to 16-bit before the multiply-adds.
+ *
+ * Readings where the pages are silent (each also listed in the design notes):
+ *  R1/R2  top-k ties: equal logits -> the lower expert index wins; the k chosen experts
+ *         are ordered by (logit descending, index ascending).
+ *  R3     p_hat = softmax over the k selected logits (= full softmax renormalised over top-k).
+ *  R4     permutation order = assignments sorted by the key (expert, token) ascending.
+ *  R5/R6  activation quantiser per (row, 512-block): s = fl32(amax / 448), q = e4m3(fl32(x/s));
+ *         amax == 0 -> s = 1, q = 0.
+ *  R7     activations are quantised for every FP8 layer.
+ *  R8     the shared expert has no gate; its output is added with weight 1.
+ *  R9     gate is the first projection, up the second; h = silu(G) * U.
+ *  R10    h is rounded to fp32 then quantised with the R5/R6 rule per 512-block of I.
+ *  R11    4-bit layers keep activations in bf16: h is rounded to bf16 (RNE).
+ *  R12    outputs are summed in fp64 here and rounded to bf16 (RNE) once.
+ *  R13    e4m3 = OCP FP8 E4M3: bias 7, no infinities, max finite 448, subnormal step 2^-9,
+ *         round-to-nearest-even, finite values beyond 448 saturate to 448.
+ *  R14    int4 weights are symmetric two's-complement nibbles, the even K index in the
+ *         low nibble; the weight is q * s with one bf16 s per (row, 128-element K group).
+ *
+ * Every sum below is written out in the order the definition states; nothing is blocked,
+ * fused or reordered beyond it.  Build: gcc -O2 -fno-fast-math -ffp-contract=off.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_FP8_SC512 1
+#define ORC_INT4_G128 2
+
+typedef struct {
+    int T, H, E, I, k, Is; /* Is = 0: no shared expert */
+    int wfmt;              /* ORC_FP8_SC512 or ORC_INT4_G128 */
+} orc_dims;
+
+typedef struct {
+    /* FP8: codes [E,I,H], [E,I,H], [E,H,I]; scales fp32 [E,I,nb(H)], [E,I,nb(H)], [E,H,nb(I)]
+     * int4: packed bytes [E,I,H/2], [E,I,H/2], [E,H,I/2]; scales bf16 [E,I,H/128] ... */
+    const uint8_t *w_gate, *w_up, *w_down;
+    const void *s_gate, *s_up, *s_down;
+    /* shared expert, same formats with E = 1 and I -> Is (NULL when Is == 0) */
+    const uint8_t *ws_gate, *ws_up, *ws_down;
+    const void *ss_gate, *ss_up, *ss_down;
+} orc_weights;
+
+/* ------------------------------------------------------------------------------------ */
+/* number formats                                                                       */
+/* ------------------------------------------------------------------------------------ */
+
+/* E4M3 decode from the format definition (R13): S.EEEE.MMM, bias 7; exponent field 0 is
+ * subnormal (0.MMM x 2^-6); S.1111.111 is NaN; there is no infinity. */
+double orc_e4m3_decode(uint8_t code)
+{
+    int sign = code >> 7;
+    int e = (code >> 3) & 0xF;
+    int m = code & 0x7;
+    double v;
+    if (e == 0xF && m == 0x7) return NAN;
+    if (e == 0)
+        v = ldexp((double)m / 8.0, -6);
+    else
+        v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+/* E4M3 encode of an fp32 value, round-to-nearest-even with saturation of finite values
+ * (R13).  Works on the exact value in fp64: the quantum of the binade is 2^(e-3) for
+ * normal numbers (2^-6 <= |x|) and 2^-9 below, and rint() rounds half to even under the
+ * default rounding mode. */
+uint8_t orc_e4m3_encode(float xf)
+{
+    double x = (double)xf;
+    uint8_t sign = signbit(xf) ? 0x80 : 0x00;
+    double a = fabs(x);
+    if (isnan(xf)) return 0x7F;
+    if (a > 448.0) a = 448.0; /* finite values and +-inf saturate to the largest finite */
+    double quantum;
+    if (a < ldexp(1.0, -6)) {
+        quantum = ldexp(1.0, -9);
+    } else {
+        int e2;
+        frexp(a, &e2); /* a = f * 2^e2 with f in [0.5, 1): leading bit weight 2^(e2-1) */
+        quantum = ldexp(1.0, (e2 - 1) - 3);
+    }
+    double r = rint(a / quantum) * quantum; /* exact: a/quantum and the product are exact */
+    if (r > 448.0) r = 448.0;               /* cannot happen after the clamp, kept for clarity */
+    /* encode r: exponent field 0 holds 0.MMM x 2^-6, field E >= 1 holds 1.MMM x 2^(E-7) */
+    int code;
+    if (r < ldexp(1.0, -6)) {
+        code = (int)(r / ldexp(1.0, -9)); /* 0..7, exact */
+    } else {
+        int e2;
+        double f = frexp(r, &e2); /* r = f * 2^e2, f in [0.5, 1) */
+        int lead = e2 - 1;
+        int mant = (int)((2.0 * f - 1.0) * 8.0); /* exact: r has at most 4 significant bits */
+        code = ((lead + 7) << 3) | mant;
+    }
+    return (uint8_t)(sign | code);
+}
+
+void orc_e4m3_encode_n(int n, const float *x, uint8_t *q)
+{
+    for (int i = 0; i < n; ++i) q[i] = orc_e4m3_encode(x[i]);
+}
+
+double orc_bf16_to_double(uint16_t b)
+{
+    uint32_t u = ((uint32_t)b) << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+/* fp64 -> bf16 with one round-to-nearest-even (no double rounding through fp32).
+ * bf16 carries 8 significant bits and fp32's exponent range; its subnormal step is 2^-133. */
+uint16_t orc_double_to_bf16(double x)
+{
+    if (isnan(x)) return 0x7FC0;
+    int neg = signbit(x) ? 1 : 0;
+    double a = fabs(x);
+    double r;
+    if (a == 0.0) {
+        r = 0.0;
+    } else {
+        int e2;
+        frexp(a, &e2);
+        int lead = e2 - 1; /* exponent of the leading bit */
+        if (lead < -126) lead = -126;
+        double quantum = ldexp(1.0, lead - 7);
+        r = rint(a / quantum) * quantum;
+    }
+    uint16_t bits;
+    if (r >= ldexp(1.0, 128)) {
+        bits = 0x7F80; /* overflow to infinity */
+    } else {
+        float f = (float)r; /* exact: r has at most 8 significant bits */
+        uint32_t u;
+        memcpy(&u, &f, 4);
+        bits = (uint16_t)(u >> 16);
+    }
+    return neg ? (uint16_t)(bits | 0x8000) : bits;
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* A1: route -- [P1] top-k by softmax probability; R1-R3                                 */
+/* ------------------------------------------------------------------------------------ */
+
+typedef struct {
+    float v;
+    int e;
+} orc_cand;
+
+static int orc_cand_cmp(const void *pa, const void *pb)
+{
+    const orc_cand *a = (const orc_cand *)pa, *b = (const orc_cand *)pb;
+    if (a->v > b->v) return -1;
+    if (a->v < b->v) return 1;
+    return (a->e < b->e) ? -1 : (a->e > b->e);
+}
+
+/* One token: sort all E logits by (value desc, index asc), keep the first k; p_hat is the
+ * softmax over those k logits in fp64.  Selection uses the fp32 logits themselves: exp is
+ * monotone, so the top-k by probability is the top-k by logit. */
+static void orc_route_token(int E, int k, const float *L, int32_t *idx, double *w)
+{
+    orc_cand *c = (orc_cand *)malloc(sizeof(orc_cand) * (size_t)E);
+    for (int e = 0; e < E; ++e) {
+        c[e].v = L[e];
+        c[e].e = e;
+    }
+    qsort(c, (size_t)E, sizeof(orc_cand), orc_cand_cmp);
+    double lmax = (double)c[0].v;
+    double denom = 0.0;
+    for (int j = 0; j < k; ++j) denom += exp((double)c[j].v - lmax);
+    for (int j = 0; j < k; ++j) {
+        idx[j] = c[j].e;
+        w[j] = exp((double)c[j].v - lmax) / denom;
+    }
+    free(c);
+}
+
+int orc_route(int T, int E, int k, const float *logits, int32_t *topk_idx, double *topk_w)
+{
+    if (T < 0 || E < 1 || k < 1 || k > E) return -1;
+    for (int t = 0; t < T; ++t)
+        orc_route_token(E, k, logits + (size_t)t * E, topk_idx + (size_t)t * k,
+                        topk_w + (size_t)t * k);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* A3: permute -- [P2] contiguous per-expert groups, packed (expert, token) sort key; R4  */
+/* ------------------------------------------------------------------------------------ */
+
+typedef struct {
+    int32_t e, t, j;
+} orc_asg;
+
+static int orc_asg_cmp(const void *pa, const void *pb)
+{
+    const orc_asg *a = (const orc_asg *)pa, *b = (const orc_asg *)pb;
+    if (a->e != b->e) return (a->e < b->e) ? -1 : 1;
+    if (a->t != b->t) return (a->t < b->t) ? -1 : 1;
+    return (a->j < b->j) ? -1 : (a->j > b->j);
+}
+
+/* counts[e] = number of assignments to e; offsets = exclusive prefix sum (E+1 entries);
+ * perm_tok[r] = token of the r-th assignment in (expert, token) order; pos[t*k+j] = row r of
+ * assignment (t, j). */
+int orc_permute(int T, int E, int k, const int32_t *topk_idx, int32_t *counts, int32_t *offsets,
+                int32_t *perm_tok, int32_t *pos)
+{
+    size_t n = (size_t)T * (size_t)k;
+    orc_asg *a = (orc_asg *)malloc(sizeof(orc_asg) * (n ? n : 1));
+    for (int e = 0; e < E; ++e) counts[e] = 0;
+    for (int t = 0; t < T; ++t)
+        for (int j = 0; j < k; ++j) {
+            int e = topk_idx[(size_t)t * k + j];
+            if (e < 0 || e >= E) {
+                free(a);
+                return -1;
+            }
+            counts[e] += 1;
+            a[(size_t)t * k + j].e = e;
+            a[(size_t)t * k + j].t = t;
+            a[(size_t)t * k + j].j = j;
+        }
+    offsets[0] = 0;
+    for (int e = 0; e < E; ++e) offsets[e + 1] = offsets[e] + counts[e];
+    qsort(a, n, sizeof(orc_asg), orc_asg_cmp);
+    for (size_t r = 0; r < n; ++r) {
+        perm_tok[r] = a[r].t;
+        pos[(size_t)a[r].t * k + a[r].j] = (int32_t)r;
+    }
+    free(a);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* A2: FP8 512-sub-channel quantiser -- [P1] Kernel section; R5, R6, R13                  */
+/* ------------------------------------------------------------------------------------ */
+
+/* x: K fp32 values of one row; q: K e4m3 codes; s: ceil(K/512) fp32 scales.  The last
+ * block may be shorter than 512. */
+void orc_quant_row_fp8(int K, const float *x, uint8_t *q, float *s)
+{
+    int nb = (K + 511) / 512;
+    for (int kb = 0; kb < nb; ++kb) {
+        int i0 = kb * 512, i1 = (kb + 1) * 512 < K ? (kb + 1) * 512 : K;
+        float amax = 0.0f;
+        for (int i = i0; i < i1; ++i) {
+            float a = fabsf(x[i]);
+            if (a > amax) amax = a;
+        }
+        if (amax == 0.0f) {
+            s[kb] = 1.0f;
+            for (int i = i0; i < i1; ++i) q[i] = 0;
+            continue;
+        }
+        volatile float sc = amax / 448.0f; /* fp32 IEEE division */
+        s[kb] = sc;
+        for (int i = i0; i < i1; ++i) {
+            volatile float v = x[i] / sc; /* fp32 IEEE division */
+            q[i] = orc_e4m3_encode(v);
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* A4-A6: one expert on one activation row, FP8 weights -- [P1] Kernel section, [P5] ①    */
+/* ------------------------------------------------------------------------------------ */
+
+static double orc_dec_tab[256];
+static pthread_once_t orc_tab_once = PTHREAD_ONCE_INIT;
+static void orc_tab_init(void)
+{
+    for (int c = 0; c < 256; ++c) orc_dec_tab[c] = orc_e4m3_decode((uint8_t)c);
+}
+
+/* y[n] = sum_kb sx[kb] * sw[n,kb] * sum_{i in kb} dec(qx[i]) * dec(qw[n,i]),  n < N.
+ * The inner sum is exact in fp64 (each product of two e4m3 values has at most 8
+ * significant bits and lies in [2^-18, 2^18)). */
+static void orc_proj_fp8(int N, int K, const uint8_t *qx, const float *sx, const uint8_t *qw,
+                         const float *sw, double *y)
+{
+    int nb = (K + 511) / 512;
+    for (int n = 0; n < N; ++n) {
+        const uint8_t *row = qw + (size_t)n * K;
+        double acc = 0.0;
+        for (int kb = 0; kb < nb; ++kb) {
+            int i0 = kb * 512, i1 = (kb + 1) * 512 < K ? (kb + 1) * 512 : K;
+            double part = 0.0;
+            for (int i = i0; i < i1; ++i) part += orc_dec_tab[qx[i]] * orc_dec_tab[row[i]];
+            acc += (double)sx[kb] * (double)sw[(size_t)n * nb + kb] * part;
+        }
+        y[n] = acc;
+    }
+}
+
+static double orc_silu(double z) { return z * (1.0 / (1.0 + exp(-z))); }
+
+/* One FP8 expert (gate/up/down already offset to that expert) on one quantised row.
+ * h_out (optional, I values) receives h rounded to fp32 before its quantisation (R10). */
+static void orc_expert_fp8(int H, int I, const uint8_t *qx, const float *sx, const uint8_t *wg,
+                           const float *sg, const uint8_t *wu, const float *su, const uint8_t *wd,
+                           const float *sd, double *y, float *h_out)
+{
+    double *G = (double *)malloc(sizeof(double) * (size_t)I);
+    double *U = (double *)malloc(sizeof(double) * (size_t)I);
+    float *h = (float *)malloc(sizeof(float) * (size_t)I);
+    uint8_t *qh = (uint8_t *)malloc((size_t)I);
+    float *sh = (float *)malloc(sizeof(float) * (size_t)((I + 511) / 512));
+    orc_proj_fp8(I, H, qx, sx, wg, sg, G);
+    orc_proj_fp8(I, H, qx, sx, wu, su, U);
+    for (int n = 0; n < I; ++n) h[n] = (float)(orc_silu(G[n]) * U[n]);
+    if (h_out) memcpy(h_out, h, sizeof(float) * (size_t)I);
+    orc_quant_row_fp8(I, h, qh, sh);
+    orc_proj_fp8(H, I, qh, sh, wd, sd, y);
+    free(G);
+    free(U);
+    free(h);
+    free(qh);
+    free(sh);
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* int4 experts -- [P5] ① (4-bit weights dequantised to 16-bit, then multiply-add); R11, R14 */
+/* ------------------------------------------------------------------------------------ */
+
+static int orc_nib(const uint8_t *packed_row, int i)
+{
+    int b = packed_row[i >> 1];
+    int v = (i & 1) ? (b >> 4) : (b & 0xF);
+    return v >= 8 ? v - 16 : v;
+}
+
+/* y[n] = sum_i a[i] * (q[n,i] * s[n, i/128])  with a in fp64 (bf16 values, exact). */
+static void orc_proj_int4(int N, int K, const double *a, const uint8_t *qw, const uint16_t *sw,
+                          double *y)
+{
+    int ng = K / 128;
+    for (int n = 0; n < N; ++n) {
+        const uint8_t *row = qw + (size_t)n * (K / 2);
+        double acc = 0.0;
+        for (int i = 0; i < K; ++i) {
+            double w = (double)orc_nib(row, i) * orc_bf16_to_double(sw[(size_t)n * ng + i / 128]);
+            acc += a[i] * w;
+        }
+        y[n] = acc;
+    }
+}
+
+static void orc_expert_int4(int H, int I, const double *x, const uint8_t *wg, const uint16_t *sg,
+                            const uint8_t *wu, const uint16_t *su, const uint8_t *wd,
+                            const uint16_t *sd, double *y, double *h_out)
+{
+    double *G = (double *)malloc(sizeof(double) * (size_t)I);
+    double *U = (double *)malloc(sizeof(double) * (size_t)I);
+    double *h = (double *)malloc(sizeof(double) * (size_t)I);
+    orc_proj_int4(I, H, x, wg, sg, G);
+    orc_proj_int4(I, H, x, wu, su, U);
+    for (int n = 0; n < I; ++n) h[n] = orc_bf16_to_double(orc_double_to_bf16(orc_silu(G[n]) * U[n]));
+    if (h_out) memcpy(h_out, h, sizeof(double) * (size_t)I);
+    orc_proj_int4(H, I, h, wd, sd, y);
+    free(G);
+    free(U);
+    free(h);
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* the layer on a chosen set of tokens -- route, quantise, experts, weighted combine       */
+/* ------------------------------------------------------------------------------------ */
+
+typedef struct {
+    const orc_dims *d;
+    const orc_weights *w;
+    const uint16_t *x;    /* [T,H] bf16 bits */
+    const float *logits;  /* [T,E] */
+    const int32_t *sel;   /* tokens to evaluate */
+    int n_sel;
+    double *out;          /* [n_sel,H] fp64 before the final rounding */
+    uint16_t *out_bf16;   /* [n_sel,H] */
+    int next;             /* next index of sel to take (guarded by mu) */
+    pthread_mutex_t mu;
+} orc_job;
+
+static void orc_layer_token(const orc_dims *d, const orc_weights *w, const uint16_t *xrow,
+                            const float *lrow, double *out)
+{
+    int H = d->H, I = d->I, E = d->E, k = d->k, Is = d->Is;
+    int32_t *idx = (int32_t *)malloc(sizeof(int32_t) * (size_t)k);
+    double *p = (double *)malloc(sizeof(double) * (size_t)k);
+    double *y = (double *)malloc(sizeof(double) * (size_t)H);
+    orc_route_token(E, k, lrow, idx, p);
+    for (int n = 0; n < H; ++n) out[n] = 0.0;
+
+    if (d->wfmt == ORC_FP8_SC512) {
+        int nbH = (H + 511) / 512, nbI = (I + 511) / 512, nbIs = (Is + 511) / 512;
+        float *xf = (float *)malloc(sizeof(float) * (size_t)H);
+        uint8_t *qx = (uint8_t *)malloc((size_t)H);
+        float *sx = (float *)malloc(sizeof(float) * (size_t)nbH);
+        for (int i = 0; i < H; ++i) xf[i] = (float)orc_bf16_to_double(xrow[i]);
+        orc_quant_row_fp8(H, xf, qx, sx);
+        const float *sg = (const float *)w->s_gate, *su = (const float *)w->s_up,
+                    *sd = (const float *)w->s_down;
+        for (int j = 0; j < k; ++j) {
+            size_t e = (size_t)idx[j];
+            orc_expert_fp8(H, I, qx, sx, w->w_gate + e * I * H, sg + e * I * nbH,
+                           w->w_up + e * I * H, su + e * I * nbH, w->w_down + e * H * I,
+                           sd + e * H * nbI, y, NULL);
+            for (int n = 0; n < H; ++n) out[n] += p[j] * y[n];
+        }
+        if (Is > 0) {
+            orc_expert_fp8(H, Is, qx, sx, w->ws_gate, (const float *)w->ss_gate, w->ws_up,
+                           (const float *)w->ss_up, w->ws_down, (const float *)w->ss_down, y, NULL);
+            for (int n = 0; n < H; ++n) out[n] += y[n];
+        }
+        (void)nbIs;
+        free(xf);
+        free(qx);
+        free(sx);
+    } else {
+        double *xd = (double *)malloc(sizeof(double) * (size_t)H);
+        for (int i = 0; i < H; ++i) xd[i] = orc_bf16_to_double(xrow[i]);
+        const uint16_t *sg = (const uint16_t *)w->s_gate, *su = (const uint16_t *)w->s_up,
+                       *sd = (const uint16_t *)w->s_down;
+        for (int j = 0; j < k; ++j) {
+            size_t e = (size_t)idx[j];
+            orc_expert_int4(H, I, xd, w->w_gate + e * I * (H / 2), sg + e * I * (H / 128),
+                            w->w_up + e * I * (H / 2), su + e * I * (H / 128),
+                            w->w_down + e * H * (I / 2), sd + e * H * (I / 128), y, NULL);
+            for (int n = 0; n < H; ++n) out[n] += p[j] * y[n];
+        }
+        if (Is > 0) {
+            orc_expert_int4(H, Is, xd, w->ws_gate, (const uint16_t *)w->ss_gate, w->ws_up,
+                            (const uint16_t *)w->ss_up, w->ws_down, (const uint16_t *)w->ss_down,
+                            y, NULL);
+            for (int n = 0; n < H; ++n) out[n] += y[n];
+        }
+        free(xd);
+    }
+    free(idx);
+    free(p);
+    free(y);
+}
+
+static void *orc_worker(void *arg)
+{
+    orc_job *jb = (orc_job *)arg;
+    pthread_once(&orc_tab_once, orc_tab_init);
+    for (;;) {
+        pthread_mutex_lock(&jb->mu);
+        int i = jb->next++;
+        pthread_mutex_unlock(&jb->mu);
+        if (i >= jb->n_sel) break;
+        int t = jb->sel[i];
+        const orc_dims *d = jb->d;
+        double *o = jb->out + (size_t)i * d->H;
+        orc_layer_token(d, jb->w, jb->x + (size_t)t * d->H, jb->logits + (size_t)t * d->E, o);
+        for (int n = 0; n < d->H; ++n) jb->out_bf16[(size_t)i * d->H + n] = orc_double_to_bf16(o[n]);
+    }
+    return NULL;
+}
+
+/* The layer output for the tokens sel[0..n_sel): out (fp64, before rounding) and out_bf16
+ * (R12).  Tokens are independent, so any subset is exact; nthreads workers take tokens in
+ * turn.  Returns 0, or -1 on bad dims. */
+int orc_layer(const orc_dims *d, const orc_weights *w, const uint16_t *x, const float *logits,
+              int n_sel, const int32_t *sel, double *out, uint16_t *out_bf16, int nthreads)
+{
+    if (d->E < 1 || d->k < 1 || d->k > d->E || d->H < 1 || d->I < 1 || d->Is < 0) return -1;
+    if (d->wfmt == ORC_INT4_G128 && (d->H % 128 || d->I % 128 || d->Is % 128)) return -1;
+    if (d->wfmt != ORC_FP8_SC512 && d->wfmt != ORC_INT4_G128) return -1;
+    for (int i = 0; i < n_sel; ++i)
+        if (sel[i] < 0 || sel[i] >= d->T) return -1;
+    pthread_once(&orc_tab_once, orc_tab_init);
+    orc_job jb;
+    jb.d = d;
+    jb.w = w;
+    jb.x = x;
+    jb.logits = logits;
+    jb.sel = sel;
+    jb.n_sel = n_sel;
+    jb.out = out;
+    jb.out_bf16 = out_bf16;
+    jb.next = 0;
+    pthread_mutex_init(&jb.mu, NULL);
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    pthread_t th[256];
+    for (int i = 0; i < nthreads; ++i) pthread_create(&th[i], NULL, orc_worker, &jb);
+    for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
+    pthread_mutex_destroy(&jb.mu);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* single steps, exposed for step-by-step parity                                        */
+/* ------------------------------------------------------------------------------------ */
+
+/* x (bf16 bits) rows -> quantised rows, FP8 layers (A2). */
+void orc_quant_rows_bf16(int R, int K, const uint16_t *x, uint8_t *q, float *s)
+{
+    int nb = (K + 511) / 512;
+    float *xf = (float *)malloc(sizeof(float) * (size_t)K);
+    for (int r = 0; r < R; ++r) {
+        for (int i = 0; i < K; ++i) xf[i] = (float)orc_bf16_to_double(x[(size_t)r * K + i]);
+        orc_quant_row_fp8(K, xf, q + (size_t)r * K, s + (size_t)r * nb);
+    }
+    free(xf);
+}
+
+/* One FP8 expert on one quantised row: y (H values, fp64) and h (I values, fp32 before
+ * its quantisation). */
+void orc_expert_fp8_row(int H, int I, const uint8_t *qx, const float *sx, const uint8_t *wg,
+                        const float *sg, const uint8_t *wu, const float *su, const uint8_t *wd,
+                        const float *sd, double *y, float *h)
+{
+    pthread_once(&orc_tab_once, orc_tab_init);
+    orc_expert_fp8(H, I, qx, sx, wg, sg, wu, su, wd, sd, y, h);
+}
+
+/* One int4 expert on one bf16 row: y (H values) and h (I values, bf16-rounded). */
+void orc_expert_int4_row(int H, int I, const uint16_t *x, const uint8_t *wg, const uint16_t *sg,
+                         const uint8_t *wu, const uint16_t *su, const uint8_t *wd,
+                         const uint16_t *sd, double *y, double *h)
+{
+    double *xd = (double *)malloc(sizeof(double) * (size_t)H);
+    for (int i = 0; i < H; ++i) xd[i] = orc_bf16_to_double(x[i]);
+    orc_expert_int4(H, I, xd, wg, sg, wu, su, wd, sd, y, h);
+    free(xd);
+}
