@@ -1,0 +1,366 @@
+#!/usr/bin/env python
+"""Benchmark of the routed MoE FFN layer on B200: one JSON line on rank 0.
+
+A step is one moe_forward call (route, permute, quantise, gate|up GEMM, down GEMM, combine)
+over one batch of seeded synthetic inputs already resident in HBM.  The default workload is
+the Qwen3.5-397B-shaped decode step (T=512, H=4096, 512 experts x 1024, top-10 + shared
+1024, FP8 512-sub-channel).  Multi-GPU runs are independent replicas (one process per GPU,
+each with its own batch; nothing is exchanged on the data path), so scaling is weak.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config decode] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s; % HBM roofline (decode) / % FP8 tensor peak (prefill)"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM bytes per launch of the gate|up GEMM on the decode workload, from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum), with the hash of the kernel source it was
+# taken on; reported as null once the source changes.
+TRAFFIC = {"decode": {"kernel": "gemm_gateup", "bytes": None, "src_sha": None}}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="decode")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target oracle time for cpu_baseline")
+    return ap.parse_args()
+
+
+def peaks():
+    p = dict(FALLBACK_PEAKS)
+    src = "fallback"
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            m = json.load(f)
+        for k in FALLBACK_PEAKS:
+            if k in m:
+                p[k] = float(m[k])
+        src = "measured"
+    return p, src
+
+
+def src_sha(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def dist_setup(args):
+    import torch
+    import torch.distributed as dist
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(ws, v):
+    if ws == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"moe_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def algorithmic(cfg, counts):
+    """Algorithmic bytes and flops of one layer call (experts with >= 1 token only)."""
+    H, I, Is, T, k = cfg["H"], cfg["I"], cfg["Is"], cfg["T"], cfg["k"]
+    touched = int((counts > 0).sum())
+    if cfg["wfmt"] == "fp8":
+        nbH, nbI, nbIs = -(-H // 512), -(-I // 512), -(-Is // 512)
+        gu = touched * 2 * (I * H + I * nbH * 4) + (2 * (Is * H + Is * nbH * 4) if Is else 0)
+        dn = touched * (H * I + H * nbI * 4) + ((H * Is + H * nbIs * 4) if Is else 0)
+    else:
+        gu = touched * 2 * (I * H // 2 + I * (H // 128) * 2) + (2 * (Is * H // 2 + Is * (H // 128) * 2) if Is else 0)
+        dn = touched * (H * I // 2 + H * (I // 128) * 2) + ((H * Is // 2 + H * (Is // 128) * 2) if Is else 0)
+    act = T * H * 2 + T * H * 2 + T * cfg["E"] * 4  # x in, out, logits
+    flops = 2 * 3 * H * I * T * k + (2 * 3 * H * Is * T if Is else 0)
+    return {"gemm_gateup": gu, "gemm_down": dn, "layer": gu + dn + act, "touched": touched, "flops": flops}
+
+
+def make_host_layer(name, device):
+    import moe_synth
+    layer = moe_synth.make_layer(name, device=device)
+    return moe_synth.to_numpy(layer), layer
+
+
+def time_oracle(Lnp, n_tokens, seed=7):
+    import numpy as np
+    import oracle
+    T = Lnp["dims"]["T"]
+    rng = np.random.default_rng(seed)
+    sel = np.sort(rng.choice(T, min(n_tokens, T), replace=False)).astype(np.int32)
+    threads = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    oracle.layer(Lnp, sel, nthreads=threads)
+    return time.perf_counter() - t0, len(sel), threads
+
+
+def cpu_baseline(Lnp, target_s):
+    """The oracle, as it stands, on a bounded sample of the workload's tokens."""
+    dt, n, thr = time_oracle(Lnp, 4)
+    per_tok = dt / n
+    n2 = max(4, min(Lnp["dims"]["T"], int(target_s / max(per_tok, 1e-6))))
+    dt, n, thr = time_oracle(Lnp, n2, seed=8)
+    return {"value": n / dt, "unit": UNIT, "cores": thr, "kind": "oracle",
+            "sample": f"{n} of {Lnp['dims']['T']} tokens (random, seeded) through the fp64 oracle, {dt:.1f} s"}
+
+
+def run_reference(args, ws, rank, cfg_name):
+    import moe_synth
+    import oracle  # noqa: F401  (the reference arm times the oracle)
+    import torch
+    if rank != 0:
+        return
+    cfg = moe_synth.CONFIGS[cfg_name]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    Lnp, _ = make_host_layer(cfg_name, dev)
+    if dev == "cuda":
+        torch.cuda.empty_cache()
+    # size a step to ~2 s of oracle work
+    dt, n, thr = time_oracle(Lnp, 2)
+    per_tok = dt / n
+    S = max(2, min(cfg["T"], int(2.0 / max(per_tok, 1e-6))))
+    for w in range(args.warmup):
+        time_oracle(Lnp, S, seed=100 + w)
+    total, toks = 0.0, 0
+    for s in range(args.steps):
+        dt, n, thr = time_oracle(Lnp, S, seed=1000 + s)
+        total += dt
+        toks += n
+    v = toks / total
+    line = {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": cfg["workload"], "T": cfg["T"], "H": cfg["H"], "E": cfg["E"], "I": cfg["I"],
+                       "k": cfg["k"], "I_shared": cfg["Is"], "wfmt": cfg["wfmt"],
+                       "sample_tokens_per_step": S},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": thr, "kind": "oracle",
+                             "sample": f"{S} random tokens of {cfg['T']} per step through the fp64 oracle"},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, ws, rank, local, cfg_name):
+    import numpy as np
+    import torch
+
+    import moe_synth
+    import mixture_experts_ffn_13_b200 as moe
+    from mixture_experts_ffn_13_b200 import build as moe_build
+
+    moe_build.build()
+    cfg = moe_synth.CONFIGS[cfg_name]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    layer = moe_synth.make_layer(cfg_name, device=dev)
+    m = moe.MoELayer(layer)
+    x, logits = layer["x"], layer["logits"]
+    out = torch.empty_like(x)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > 126 MB L2
+    moe.moe_profile_enable(m.plan, True)
+
+    for _ in range(args.warmup):
+        m(x, logits, out=out)
+    torch.cuda.synchronize()
+    rc = moe.moe_get_status(m.plan)
+    if rc != 0:
+        raise RuntimeError(f"device status after warm-up: {moe.moe_strerror(rc)}")
+
+    clocks = ClockSampler(local) if rank == 0 else None
+    if clocks:
+        clocks.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    stage_ms = {s: 0.0 for s in moe.STAGES}
+    launches = 0
+    barrier(ws)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        m(x, logits, out=out)
+        ev[i][1].record(stream)
+        launches += moe.moe_launch_count(m.plan)
+        for kname, v in moe.moe_profile_read(m.plan).items():
+            stage_ms[kname] += v
+    torch.cuda.synchronize()
+    barrier(ws)
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    clk = clocks.stop() if clocks else None
+    rc = moe.moe_get_status(m.plan)
+    if rc != 0:
+        raise RuntimeError(f"device status after timing: {moe.moe_strerror(rc)}")
+    total_ms = max_over_ranks(ws, sum(step_ms))
+
+    # end to end through the public API with host buffers: H2D of x and logits from pinned
+    # memory, the layer, D2H of the output, every step inside the timed region
+    xh = x.cpu().pin_memory()
+    lh = logits.cpu().pin_memory()
+    oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    xd, ld = torch.empty_like(x), torch.empty_like(logits)
+    moe.moe_profile_enable(m.plan, False)
+    for _ in range(max(1, args.warmup)):
+        xd.copy_(xh, non_blocking=True)
+        ld.copy_(lh, non_blocking=True)
+        m(xd, ld, out=out)
+        oh.copy_(out, non_blocking=True)
+    torch.cuda.synchronize()
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier(ws)
+    for i in range(args.steps):
+        flush.zero_()
+        e2e_ev[i][0].record(stream)
+        xd.copy_(xh, non_blocking=True)
+        ld.copy_(lh, non_blocking=True)
+        m(xd, ld, out=out)
+        oh.copy_(out, non_blocking=True)
+        e2e_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    e2e_ms = max_over_ranks(ws, sum(a.elapsed_time(b) for a, b in e2e_ev))
+
+    r = m.route(logits)
+    counts = r["counts"].cpu().numpy()
+    alg = algorithmic(cfg, counts)
+    pk, pk_src = peaks()
+    T = cfg["T"]
+    value = ws * T * args.steps / (total_ms / 1e3)
+    e2e_value = ws * T * args.steps / (e2e_ms / 1e3)
+    ms_step = total_ms / args.steps
+    mean_stage = {k: v / args.steps for k, v in stage_ms.items()}
+    dom = max(("gemm_gateup", "gemm_down"), key=lambda s: mean_stage[s])
+    achieved = alg[dom] / (mean_stage[dom] / 1e3) / 1e9
+    tr = TRAFFIC.get(cfg_name)
+    traffic = None
+    if tr and tr["bytes"] and tr["kernel"] == dom and tr["src_sha"] == src_sha(
+            os.path.join(ROOT, "mixture_experts_ffn_13_b200", "csrc", "gemm_fp8.cu")):
+        traffic = tr["bytes"]
+    layer_gbs = alg["layer"] / (ms_step / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8_e4m3" if cfg["wfmt"] == "fp8" else "bf16", "data": "synthetic",
+        "config": {"workload": cfg["workload"], "T": T, "H": cfg["H"], "E": cfg["E"], "I": cfg["I"], "k": cfg["k"],
+                   "I_shared": cfg["Is"], "wfmt": cfg["wfmt"], "seed": cfg["seed"],
+                   "parallelism": f"replicas x{ws}", "l2": "flushed (256 MiB write) before every timed step",
+                   "experts_touched": alg["touched"], "max_tokens_per_expert": int(counts.max())},
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
+                     "algorithmic_bytes": alg[dom], "peak_source": pk_src,
+                     "layer_achieved_gbs": layer_gbs, "layer_frac": layer_gbs / pk["hbm_gbs"]},
+        "stages_ms": mean_stage,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": x.numel() * 2 + logits.numel() * 4,
+                "d2h_bytes_per_step": out.numel() * 2},
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        del layer, m, flush
+        torch.cuda.empty_cache()
+        Lnp, _ = make_host_layer(cfg_name, dev)
+        line["cpu_baseline"] = cpu_baseline(Lnp, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    ws, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, ws, rank, args.config)
+        else:
+            run_ours(args, ws, rank, local, args.config)
+    finally:
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

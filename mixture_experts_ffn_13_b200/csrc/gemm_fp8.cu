@@ -1,0 +1,327 @@
+// gemm_fp8.cu -- steps A4 and A5: persistent grouped GEMMs over FP8 expert weights with
+// 512-element sub-channel scales, on the 5th-generation tensor cores (tcgen05, TMEM, TMA).
+//
+// Page "把 397B MoE 榨進 TPU7x：Google 拿到 4.7 倍加速", section "Kernel 手術台": the grouped GEMM
+// fuses the gate and up projections in one tile, uses 512-sub-channel FP8, and sizes each
+// expert's work by its real row count instead of a padded maximum.  Page "Flash-Next 在 GPU 上
+// 到底在算什麼", section "① 專家 FFN": each expert is input x A -> activation -> x B.
+//
+// Design (B200):
+//  * Operand roles are swapped: the MMA's M side (128 rows) is a tile of WEIGHT rows and its N
+//    side is a tile of BN token rows of one expert group, so a decode-sized group (a handful
+//    of tokens) still fills the 128-row MMA and the kernel streams weights at full width.
+//  * One CTA per SM, persistent over a flat list of (group, weight-row tile, token tile)
+//    work items; per group the list is built from the routed row counts, so empty experts
+//    cost nothing and hot experts get many token tiles.
+//  * Warp roles: warp 0 issues TMA loads of 128-byte-wide K slices (weights with an
+//    evict-first L2 hint, activations evict-last) into an NS-deep ring of shared-memory
+//    stages; warp 1 issues tcgen05.mma (E4M3 x E4M3 -> F32) from one thread; warps 2-5 are
+//    the epilogue.
+//  * Sub-channel promotion: the scales change every 512 elements of K for both operands, so
+//    each 512-block gets its own TMEM accumulator slot (a ring of slots covering all 512
+//    TMEM columns).  The epilogue reads a finished slot, multiplies it by
+//    s_w[row, kb] * s_x[token, kb] and adds it into fp32 registers, then frees the slot, so
+//    the MMAs of the next blocks overlap the promotion of the previous ones.
+//  * gate|up: two weight tiles per stage share one activation tile; the epilogue computes
+//    h = silu(G) * U in fp32 and stores it.  down: one weight tile; y is stored in fp32.
+#include "moe_internal.h"
+#include "sm100.cuh"
+
+#include <algorithm>
+
+namespace moe {
+
+namespace {
+
+constexpr int kTileM = 128;  // weight rows per tile (MMA M)
+constexpr int kKC = 128;     // K elements (bytes) per pipeline stage = one 128-byte swizzle row
+constexpr int kStagesPerBlock = kBlockK / kKC;
+constexpr int kSmemBudget = 200 * 1024;
+
+template <int BN, bool GATEUP>
+struct Fp8Cfg {
+    static constexpr int NA = GATEUP ? 2 : 1;
+    static constexpr int A_BYTES = kTileM * kKC;
+    static constexpr int B_BYTES = BN * kKC;
+    static constexpr int STAGE_BYTES = NA * A_BYTES + B_BYTES;
+    static constexpr int NS = (kSmemBudget / STAGE_BYTES) < 16 ? (kSmemBudget / STAGE_BYTES) : 16;
+    static constexpr int SLOT_COLS = NA * BN;
+    static constexpr int NSLOT = 512 / SLOT_COLS;
+    static constexpr int EPI_WARPS = 4;
+    static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+    static constexpr int BAR_BYTES = 8 * (2 * NS + 2 * NSLOT) + 16;
+    static constexpr int SMEM = 1024 + NS * STAGE_BYTES + BAR_BYTES;
+    static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "stage tiles must stay 1024-byte aligned");
+    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M=128 is a multiple of 16 in [16, 256]");
+    static_assert(NSLOT >= 1, "TMEM slots");
+};
+
+struct TileInfo {
+    int seg;    // 0 routed, 1 shared
+    int nt;     // weight-row tile index within the group
+    int row0;   // first activation row (segment-relative)
+    int nrows;  // valid activation rows in this tile (<= BN)
+    int wrow;   // first weight row in the segment's 2-D weight view
+};
+
+// Work item w -> tile.  Routed items come first: group g owns items
+// [ttile[g]*nT, ttile[g+1]*nT), laid out n-tile major so consecutive items reuse the same
+// weight tile across the group's token tiles.  Shared-expert items follow.
+template <int BN>
+__device__ __forceinline__ TileInfo decode_tile(const GemmArgs &a, int w, int tot0)
+{
+    TileInfo t;
+    if (w < tot0) {
+        const int nT = a.seg[0].N / kTileM;
+        int lo = 0, hi = a.E - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (__ldg(a.ttile + mid) * nT <= w)
+                lo = mid;
+            else
+                hi = mid - 1;
+        }
+        const int g = lo;
+        const int t0 = __ldg(a.ttile + g);
+        const int ntt = __ldg(a.ttile + g + 1) - t0;
+        const int local = w - t0 * nT;
+        const int nt = local / ntt;
+        const int tt = local - nt * ntt;
+        const int rbeg = __ldg(a.offsets + g) + tt * BN;
+        const int rend = __ldg(a.offsets + g + 1);
+        t.seg = 0;
+        t.nt = nt;
+        t.row0 = rbeg;
+        t.nrows = min(BN, rend - rbeg);
+        t.wrow = g * a.seg[0].N + nt * kTileM;
+    } else {
+        const int ww = w - tot0;
+        const int ntt = (a.T + BN - 1) / BN;
+        const int nt = ww / ntt;
+        const int tt = ww - nt * ntt;
+        t.seg = 1;
+        t.nt = nt;
+        t.row0 = tt * BN;
+        t.nrows = min(BN, a.T - t.row0);
+        t.wrow = nt * kTileM;
+    }
+    return t;
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
+
+template <int BN, bool GATEUP>
+__global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP>::THREADS, 1)
+    gemm_fp8_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmArgs args)
+{
+    using C = Fp8Cfg<BN, GATEUP>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::NS * C::STAGE_BYTES);
+    uint64_t *empty = full + C::NS;
+    uint64_t *accf = empty + C::NS;
+    uint64_t *acce = accf + C::NSLOT;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(acce + C::NSLOT);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::NS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int s = 0; s < C::NSLOT; ++s) {
+            mbar_init(&accf[s], 1);
+            mbar_init(&acce[s], C::EPI_WARPS);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        for (int i = 0; i < args.nseg; ++i) {
+            tma_prefetch_desc(&maps.a0[i]);
+            if (GATEUP) tma_prefetch_desc(&maps.a1[i]);
+            tma_prefetch_desc(&maps.b[i]);
+        }
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    const int tot0 = __ldg(args.ttile + args.E) * (args.seg[0].N / kTileM);
+    const int tot1 = args.nseg > 1 ? ((args.T + BN - 1) / BN) * (args.seg[1].N / kTileM) : 0;
+    const int total = tot0 + tot1;
+    int *status = args.status;
+    const uint64_t tmo = args.timeout_ns;
+
+    if (warp == 0) {
+        // ------------------------------ TMA producer ------------------------------
+        if (lane == 0) {
+            const uint64_t pol_w = l2_policy_evict_first();
+            const uint64_t pol_x = l2_policy_evict_last();
+            uint32_t it = 0;
+            for (int w = blockIdx.x; w < total; w += gridDim.x) {
+                const TileInfo tl = decode_tile<BN>(args, w, tot0);
+                const int nkc = args.seg[tl.seg].K / kKC;
+                for (int kc = 0; kc < nkc; ++kc, ++it) {
+                    const int s = it % C::NS;
+                    const uint32_t ph = (it / C::NS) & 1;
+                    if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, status, tmo)) goto done;
+                    uint8_t *st = smem + s * C::STAGE_BYTES;
+                    mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+                    tma_load_2d_hint(st, &maps.a0[tl.seg], &full[s], kc * kKC, tl.wrow, pol_w);
+                    if (GATEUP) tma_load_2d_hint(st + C::A_BYTES, &maps.a1[tl.seg], &full[s], kc * kKC, tl.wrow, pol_w);
+                    tma_load_2d_hint(st + C::NA * C::A_BYTES, &maps.b[tl.seg], &full[s], kc * kKC, tl.row0, pol_x);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------ MMA issuer --------------------------------
+        if (lane == 0) {
+            constexpr uint32_t kIdesc = instr_desc(kTileM, BN, 0, 0);
+            uint32_t it = 0, ai = 0;
+            for (int w = blockIdx.x; w < total; w += gridDim.x) {
+                const TileInfo tl = decode_tile<BN>(args, w, tot0);
+                const int K = args.seg[tl.seg].K;
+                const int nkc = K / kKC;
+                const int nkb = (K + kBlockK - 1) / kBlockK;
+                for (int kb = 0; kb < nkb; ++kb, ++ai) {
+                    const int slot = ai % C::NSLOT;
+                    const uint32_t aph = (ai / C::NSLOT) & 1;
+                    if (!mbar_wait(&acce[slot], aph ^ 1, abort_flag, status, tmo)) goto done;
+                    tc_fence_after();
+                    const uint32_t d0 = tmem_base + slot * C::SLOT_COLS;
+                    const uint32_t d1 = d0 + BN;
+                    const int kc_end = min(nkc, (kb + 1) * kStagesPerBlock);
+                    for (int kc = kb * kStagesPerBlock; kc < kc_end; ++kc, ++it) {
+                        const int s = it % C::NS;
+                        const uint32_t ph = (it / C::NS) & 1;
+                        if (!mbar_wait(&full[s], ph, abort_flag, status, tmo)) goto done;
+                        tc_fence_after();
+                        uint8_t *st = smem + s * C::STAGE_BYTES;
+                        const uint64_t da0 = smem_desc_sw128(st);
+                        const uint64_t da1 = smem_desc_sw128(st + C::A_BYTES);
+                        const uint64_t db = smem_desc_sw128(st + C::NA * C::A_BYTES);
+#pragma unroll
+                        for (int kk = 0; kk < kKC / 32; ++kk) {
+                            const uint32_t acc = (kc > kb * kStagesPerBlock || kk > 0) ? 1u : 0u;
+                            mma_f8(d0, da0 + 2 * kk, db + 2 * kk, kIdesc, acc);
+                            if (GATEUP) mma_f8(d1, da1 + 2 * kk, db + 2 * kk, kIdesc, acc);
+                        }
+                        mma_commit(&empty[s]);
+                    }
+                    mma_commit(&accf[slot]);
+                }
+            }
+        }
+    } else {
+        // ------------------------------ epilogue ----------------------------------
+        const int q = warp & 3;  // TMEM lanes 32q..32q+31 are reachable from this warp
+        const int r = q * 32 + lane;
+        uint32_t ai = 0;
+        for (int w = blockIdx.x; w < total; w += gridDim.x) {
+            const TileInfo tl = decode_tile<BN>(args, w, tot0);
+            const GemmSeg &sg = args.seg[tl.seg];
+            const int K = sg.K;
+            const int nkb = (K + kBlockK - 1) / kBlockK;
+            const float *sw0 = static_cast<const float *>(sg.sw0) + (size_t)(tl.wrow + r) * nkb;
+            const float *sw1 = GATEUP ? static_cast<const float *>(sg.sw1) + (size_t)(tl.wrow + r) * nkb : nullptr;
+            float acc0[BN], acc1[GATEUP ? BN : 1];
+#pragma unroll
+            for (int c = 0; c < BN; ++c) acc0[c] = 0.0f;
+            if constexpr (GATEUP) {
+#pragma unroll
+                for (int c = 0; c < BN; ++c) acc1[c] = 0.0f;
+            }
+            for (int kb = 0; kb < nkb; ++kb, ++ai) {
+                const int slot = ai % C::NSLOT;
+                const uint32_t aph = (ai / C::NSLOT) & 1;
+                const float s0 = __ldg(sw0 + kb);
+                const float s1 = GATEUP ? __ldg(sw1 + kb) : 0.0f;
+                const bool ok = mbar_wait(&accf[slot], aph, abort_flag, status, tmo);
+                if (!__all_sync(0xffffffffu, ok)) goto done;
+                tc_fence_after();
+                const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + slot * C::SLOT_COLS;
+#pragma unroll
+                for (int c0 = 0; c0 < BN; c0 += 16) {
+                    float v[16], u[16];
+                    tmem_ld16(tb + c0, v);
+                    if constexpr (GATEUP) {
+                        tmem_ld16(tb + BN + c0, u);
+                        tmem_wait_ld2(v, u);
+                    } else {
+                        tmem_wait_ld(v);
+                    }
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        const int row = min(tl.row0 + c0 + c, sg.rows - 1);
+                        const float sx = __ldg(sg.sx + (size_t)row * nkb + kb);
+                        acc0[c0 + c] = fmaf(v[c], s0 * sx, acc0[c0 + c]);
+                        if constexpr (GATEUP) acc1[c0 + c] = fmaf(u[c], s1 * sx, acc1[c0 + c]);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acce[slot]);
+            }
+            float *out = static_cast<float *>(sg.out);
+            const int n = tl.nt * kTileM + r;
+#pragma unroll
+            for (int c = 0; c < BN; ++c) {
+                if (c < tl.nrows) {
+                    float v;
+                    if constexpr (GATEUP)
+                        v = silu_mul(acc0[c], acc1[c]);
+                    else
+                        v = acc0[c];
+                    out[(size_t)(tl.row0 + c) * sg.N + n] = v;
+                }
+            }
+        }
+    }
+done:
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem_base, 512);
+    }
+}
+
+template <int BN, bool GATEUP>
+cudaError_t launch_t(const GemmMaps &maps, const GemmArgs &args, int num_sms, cudaStream_t s)
+{
+    using C = Fp8Cfg<BN, GATEUP>;
+    auto kern = gemm_fp8_kernel<BN, GATEUP>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    kern<<<num_sms, C::THREADS, C::SMEM, s>>>(maps, args);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_fp8(bool gateup, int bn, const GemmMaps &maps, const GemmArgs &args, int num_sms,
+                            cudaStream_t s)
+{
+    if (gateup) {
+        switch (bn) {
+            case 32: return launch_t<32, true>(maps, args, num_sms, s);
+            case 64: return launch_t<64, true>(maps, args, num_sms, s);
+            default: return cudaErrorInvalidValue;
+        }
+    }
+    switch (bn) {
+        case 32: return launch_t<32, false>(maps, args, num_sms, s);
+        case 64: return launch_t<64, false>(maps, args, num_sms, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace moe

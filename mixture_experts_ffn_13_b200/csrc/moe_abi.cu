@@ -1,0 +1,410 @@
+// moe_abi.cu -- the C ABI (include/moe_b200.h): plan validation, workspace carving, tensor-map
+// encoding and the launch sequence of one layer call.  Host code only.
+#include "moe_internal.h"
+
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+#include <new>
+
+struct moe_plan_s {
+    moe_dims d;
+    int device;
+    int num_sms;
+    int *d_status;  // device status word (4 ints), allocated by moe_plan
+    int last_cuda_error;
+    size_t ws_bytes;
+    int launches;             // kernels launched by the last route/forward call
+    bool prof;                // stage events enabled
+    bool prof_recorded;       // the last forward recorded them
+    cudaEvent_t ev[8];        // stage boundaries 0..7
+};
+
+namespace moe {
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
+
+int nb512(int K) { return (K + kBlockK - 1) / kBlockK; }
+
+// Byte offsets of every workspace buffer for a token count of Tm (the plan's T_max).
+struct Layout {
+    size_t topk_idx, topk_w, counts, offsets, perm, pos, chunk_hist, ttile_a, ttile_b;
+    size_t act, act_scale;       // permuted activations (+ scales for FP8)
+    size_t h, h_sh;              // gate|up output, routed / shared
+    size_t hq, hq_sh, sh, sh_sh; // quantised h (FP8)
+    size_t y;                    // down output rows (routed then shared), fp32
+    size_t total;
+};
+
+Layout make_layout(const moe_dims &d)
+{
+    const size_t Tm = (size_t)d.T_max, k = (size_t)d.k, E = (size_t)d.E;
+    const size_t H = (size_t)d.H, I = (size_t)d.I, Is = (size_t)d.I_shared;
+    const size_t A = Tm * k;
+    const size_t R = A + (Is > 0 ? Tm : 0);
+    const size_t nch = (Tm + kChunk - 1) / kChunk;
+    const bool fp8 = d.wfmt == MOE_W_FP8_SC512;
+    Layout L{};
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = o;
+        o = align_up(o + std::max<size_t>(bytes, 1));
+        return at;
+    };
+    L.topk_idx = take(A * 4);
+    L.topk_w = take(A * 4);
+    L.counts = take(E * 4);
+    L.offsets = take((E + 1) * 4);
+    L.perm = take(A * 4);
+    L.pos = take(A * 4);
+    L.chunk_hist = take(nch * E * 4);
+    L.ttile_a = take((E + 1) * 4);
+    L.ttile_b = take((E + 1) * 4);
+    if (fp8) {
+        L.act = take(R * H);
+        L.act_scale = take(R * nb512(d.H) * 4);
+        L.h = take(A * I * 4);
+        L.h_sh = take(Tm * Is * 4);
+        L.hq = take(A * I);
+        L.hq_sh = take(Tm * Is);
+        L.sh = take(A * nb512(d.I) * 4);
+        L.sh_sh = take(Tm * nb512(d.I_shared) * 4);
+    } else {
+        L.act = take(R * H * 2);
+        L.act_scale = 0;
+        L.h = take(A * I * 2);
+        L.h_sh = take(Tm * Is * 2);
+        L.hq = L.hq_sh = L.sh = L.sh_sh = 0;
+    }
+    L.y = take(R * H * 4);
+    L.total = o;
+    return L;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+void load_encode()
+{
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+int fail_cuda(moe_plan_t *p, cudaError_t e)
+{
+    p->last_cuda_error = (int)e;
+    return MOE_ERR_CUDA;
+}
+
+// Tile size along the token dimension for a given token count per group.
+int pick_bn(int T, int k, int E)
+{
+    const long avg = ((long)T * k + E - 1) / E;
+    return avg > 48 ? 64 : 32;
+}
+
+}  // namespace
+
+int encode_map_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, int elem_bytes, uint64_t inner,
+                  uint64_t outer, uint32_t box_inner, uint32_t box_outer, bool swizzle128)
+{
+    std::call_once(g_encode_once, load_encode);
+    if (!g_encode) return MOE_ERR_CUDA;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {inner * (uint64_t)elem_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = g_encode(map, dtype, 2, const_cast<void *>(base), dims, strides, box, estr,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char *moe_strerror(int code)
+{
+    switch (code) {
+        case MOE_OK: return "MOE_OK";
+        case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+        case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+        case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+        case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+        case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT";
+        case MOE_ERR_BOUNDS: return "MOE_ERR_BOUNDS";
+        default: return "MOE_ERR_UNKNOWN";
+    }
+}
+
+int moe_plan(const moe_dims *dims, moe_plan_t **out_plan, size_t *workspace_bytes)
+{
+    if (!dims || !out_plan || !workspace_bytes) return MOE_ERR_INVALID_ARG;
+    *out_plan = nullptr;
+    const moe_dims d = *dims;
+    if (d.T_max < 1 || d.H < 1 || d.E < 1 || d.I < 1 || d.k < 1 || d.I_shared < 0) return MOE_ERR_INVALID_ARG;
+    if (d.wfmt != MOE_W_FP8_SC512 && d.wfmt != MOE_W_INT4_G128) return MOE_ERR_INVALID_ARG;
+    if (d.k > d.E) return MOE_ERR_INVALID_ARG;
+    if (d.E > kMaxE || d.k > kMaxK || d.T_max > (1 << 20)) return MOE_ERR_UNSUPPORTED;
+    if (d.H % 128 || d.I % 128 || d.I_shared % 128) return MOE_ERR_UNSUPPORTED;
+    // 32-bit row arithmetic inside the kernels
+    if ((long long)d.E * std::max(d.I, d.H) >= (1ll << 31) ||
+        (long long)d.T_max * (d.k + 1) * std::max(d.I, d.H) >= (1ll << 40))
+        return MOE_ERR_UNSUPPORTED;
+    moe_plan_t *p = new (std::nothrow) moe_plan_s();
+    if (!p) return MOE_ERR_INVALID_ARG;
+    p->d = d;
+    cudaError_t e = cudaGetDevice(&p->device);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&p->num_sms, cudaDevAttrMultiProcessorCount, p->device);
+    if (e == cudaSuccess) e = cudaMalloc(&p->d_status, 4 * sizeof(int));
+    if (e == cudaSuccess) e = cudaMemset(p->d_status, 0, 4 * sizeof(int));
+    if (e != cudaSuccess) {
+        if (p->d_status) cudaFree(p->d_status);
+        delete p;
+        return MOE_ERR_CUDA;
+    }
+    p->ws_bytes = make_layout(d).total;
+    *workspace_bytes = p->ws_bytes;
+    *out_plan = p;
+    return MOE_OK;
+}
+
+void moe_destroy(moe_plan_t *p)
+{
+    if (!p) return;
+    if (p->prof)
+        for (cudaEvent_t &e : p->ev) cudaEventDestroy(e);
+    if (p->d_status) cudaFree(p->d_status);
+    delete p;
+}
+
+static const char *kStageNames[7] = {"route", "permute", "quant_x", "gemm_gateup", "quant_h", "gemm_down", "combine"};
+
+const char *moe_profile_stage_name(int i) { return (i >= 0 && i < 7) ? kStageNames[i] : nullptr; }
+
+int moe_launch_count(const moe_plan_t *p) { return p ? p->launches : 0; }
+
+int moe_profile_enable(moe_plan_t *p, int enable)
+{
+    if (!p) return MOE_ERR_INVALID_ARG;
+    if (enable && !p->prof) {
+        for (int i = 0; i < 8; ++i) {
+            const cudaError_t e = cudaEventCreate(&p->ev[i]);
+            if (e != cudaSuccess) {
+                for (int j = 0; j < i; ++j) cudaEventDestroy(p->ev[j]);
+                return fail_cuda(p, e);
+            }
+        }
+        p->prof = true;
+    } else if (!enable && p->prof) {
+        for (cudaEvent_t &e : p->ev) cudaEventDestroy(e);
+        p->prof = false;
+    }
+    p->prof_recorded = false;
+    return MOE_OK;
+}
+
+int moe_profile_read(moe_plan_t *p, float *ms, int max_stages)
+{
+    if (!p || !ms || max_stages < 0 || !p->prof || !p->prof_recorded) return MOE_ERR_INVALID_ARG;
+    const int n = std::min(max_stages, 7);
+    cudaError_t e = cudaEventSynchronize(p->ev[7]);
+    for (int i = 0; i < n && e == cudaSuccess; ++i) e = cudaEventElapsedTime(&ms[i], p->ev[i], p->ev[i + 1]);
+    if (e != cudaSuccess) return fail_cuda(p, e);
+    return n;
+}
+
+int moe_last_cuda_error(const moe_plan_t *p) { return p ? p->last_cuda_error : 0; }
+
+int moe_get_status(moe_plan_t *p, moe_stream_t stream)
+{
+    if (!p) return MOE_ERR_INVALID_ARG;
+    int h[4] = {0, 0, 0, 0};
+    cudaError_t e = cudaMemcpyAsync(h, p->d_status, sizeof(h), cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e == cudaSuccess && h[0] != 0) e = cudaMemsetAsync(p->d_status, 0, sizeof(h), (cudaStream_t)stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return fail_cuda(p, e);
+    return h[0];
+}
+
+static int check_ws(const moe_plan_t *p, void *ws, size_t ws_bytes)
+{
+    if (!ws || ws_bytes < p->ws_bytes) return MOE_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(ws) % kAlign) return MOE_ERR_WORKSPACE;
+    return MOE_OK;
+}
+
+static RouteBufs route_bufs(const Layout &L, uint8_t *ws)
+{
+    RouteBufs b;
+    b.topk_idx = reinterpret_cast<int32_t *>(ws + L.topk_idx);
+    b.topk_w = reinterpret_cast<float *>(ws + L.topk_w);
+    b.counts = reinterpret_cast<int32_t *>(ws + L.counts);
+    b.offsets = reinterpret_cast<int32_t *>(ws + L.offsets);
+    b.perm_tok = reinterpret_cast<int32_t *>(ws + L.perm);
+    b.pos = reinterpret_cast<int32_t *>(ws + L.pos);
+    b.chunk_hist = reinterpret_cast<int32_t *>(ws + L.chunk_hist);
+    b.ttile_a = reinterpret_cast<int32_t *>(ws + L.ttile_a);
+    b.ttile_b = reinterpret_cast<int32_t *>(ws + L.ttile_b);
+    return b;
+}
+
+int moe_route(moe_plan_t *p, int32_t T, const float *logits, int32_t *topk_idx, float *topk_w, int32_t *counts,
+              int32_t *offsets, int32_t *perm_tok, void *workspace, size_t ws_bytes, moe_stream_t stream)
+{
+    if (!p) return MOE_ERR_INVALID_ARG;
+    if (T < 0 || T > p->d.T_max) return MOE_ERR_INVALID_ARG;
+    if (!counts || !offsets || (T > 0 && (!logits || !topk_idx || !topk_w || !perm_tok))) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(logits) || !aligned16(topk_idx) || !aligned16(topk_w) || !aligned16(counts) ||
+        !aligned16(offsets) || !aligned16(perm_tok))
+        return MOE_ERR_INVALID_ARG;
+    int rc = check_ws(p, workspace, ws_bytes);
+    if (rc) return rc;
+    const moe_dims &d = p->d;
+    const Layout L = make_layout(d);
+    RouteBufs b = route_bufs(L, static_cast<uint8_t *>(workspace));
+    b.topk_idx = topk_idx;
+    b.topk_w = topk_w;
+    b.counts = counts;
+    b.offsets = offsets;
+    b.perm_tok = perm_tok;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int bn = pick_bn(T, d.k, d.E);
+    p->launches = 0;
+    cudaError_t e = launch_route(logits, T, d.E, d.k, topk_idx, topk_w, s);
+    if (e == cudaSuccess) e = launch_permute(b, T, d.E, d.k, bn, bn, s);
+    p->launches = (T > 0 ? 1 : 0) + (T > 0 ? 3 : 1);
+    return e == cudaSuccess ? MOE_OK : fail_cuda(p, e);
+}
+
+int moe_forward(moe_plan_t *p, int32_t T, const uint16_t *x, const float *logits, const moe_weights *w,
+                uint16_t *out, void *workspace, size_t ws_bytes, moe_stream_t stream)
+{
+    if (!p || !w) return MOE_ERR_INVALID_ARG;
+    const moe_dims &d = p->d;
+    if (T < 0 || T > d.T_max) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!x || !logits || !out)) return MOE_ERR_INVALID_ARG;
+    if (!w->w_gate || !w->w_up || !w->w_down || !w->s_gate || !w->s_up || !w->s_down) return MOE_ERR_INVALID_ARG;
+    const bool shared = d.I_shared > 0;
+    if (shared && (!w->ws_gate || !w->ws_up || !w->ws_down || !w->ss_gate || !w->ss_up || !w->ss_down))
+        return MOE_ERR_INVALID_ARG;
+    const void *ptrs[] = {x, logits, out, w->w_gate, w->w_up, w->w_down, w->s_gate, w->s_up, w->s_down,
+                          w->ws_gate, w->ws_up, w->ws_down, w->ss_gate, w->ss_up, w->ss_down};
+    for (const void *q : ptrs)
+        if (!aligned16(q)) return MOE_ERR_INVALID_ARG;
+    int rc = check_ws(p, workspace, ws_bytes);
+    if (rc) return rc;
+    p->launches = 0;
+    p->prof_recorded = false;
+    if (T == 0) return MOE_OK;
+    if (d.wfmt != MOE_W_FP8_SC512) return MOE_ERR_UNSUPPORTED;
+
+    cudaStream_t s = (cudaStream_t)stream;
+    auto mark = [&](int i) {
+        if (p->prof) cudaEventRecord(p->ev[i], s);
+    };
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    const Layout L = make_layout(d);
+    const RouteBufs b = route_bufs(L, ws);
+    const int H = d.H, I = d.I, Is = d.I_shared, k = d.k, E = d.E;
+    const int A = T * k;
+    const int bn_a = pick_bn(T, k, E), bn_b = bn_a;
+
+    mark(0);
+    cudaError_t e = launch_route(logits, T, E, k, b.topk_idx, b.topk_w, s);
+    mark(1);
+    if (e == cudaSuccess) e = launch_permute(b, T, E, k, bn_a, bn_b, s);
+    mark(2);
+    if (e != cudaSuccess) return fail_cuda(p, e);
+
+    // A2: quantise x into permuted rows [0, A) and shared rows [A, A + T)
+    uint8_t *xq = ws + L.act;
+    float *sx = reinterpret_cast<float *>(ws + L.act_scale);
+    const int nbH = nb512(H);
+    uint8_t *xq_sh = shared ? xq + (size_t)A * H : nullptr;
+    float *sx_sh = shared ? sx + (size_t)A * nbH : nullptr;
+    e = launch_quant_x_fp8(x, T, H, k, b.pos, xq, sx, xq_sh, sx_sh, s);
+    mark(3);
+    if (e != cudaSuccess) return fail_cuda(p, e);
+
+    float *h = reinterpret_cast<float *>(ws + L.h);
+    float *h_sh = reinterpret_cast<float *>(ws + L.h_sh);
+    uint8_t *hq = ws + L.hq, *hq_sh = ws + L.hq_sh;
+    float *sh = reinterpret_cast<float *>(ws + L.sh), *sh_sh = reinterpret_cast<float *>(ws + L.sh_sh);
+    float *y = reinterpret_cast<float *>(ws + L.y);
+    float *y_sh = shared ? y + (size_t)A * H : nullptr;
+    const CUtensorMapDataType U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+
+    // A4: gate|up
+    GemmMaps mg{};
+    GemmArgs ag{};
+    ag.nseg = shared ? 2 : 1;
+    ag.E = E;
+    ag.T = T;
+    ag.offsets = b.offsets;
+    ag.ttile = b.ttile_a;
+    ag.status = p->d_status;
+    ag.timeout_ns = kDefaultTimeoutNs;
+    ag.seg[0] = GemmSeg{I, H, A, w->s_gate, w->s_up, sx, h};
+    rc = encode_map_2d(&mg.a0[0], w->w_gate, U8, 1, H, (uint64_t)E * I, 128, 128, true);
+    rc |= encode_map_2d(&mg.a1[0], w->w_up, U8, 1, H, (uint64_t)E * I, 128, 128, true);
+    rc |= encode_map_2d(&mg.b[0], xq, U8, 1, H, A, 128, bn_a, true);
+    if (shared) {
+        ag.seg[1] = GemmSeg{Is, H, T, w->ss_gate, w->ss_up, sx_sh, h_sh};
+        rc |= encode_map_2d(&mg.a0[1], w->ws_gate, U8, 1, H, Is, 128, 128, true);
+        rc |= encode_map_2d(&mg.a1[1], w->ws_up, U8, 1, H, Is, 128, 128, true);
+        rc |= encode_map_2d(&mg.b[1], xq_sh, U8, 1, H, T, 128, bn_a, true);
+    }
+    if (rc) return MOE_ERR_CUDA;
+    e = launch_gemm_fp8(true, bn_a, mg, ag, p->num_sms, s);
+    mark(4);
+    if (e != cudaSuccess) return fail_cuda(p, e);
+
+    // quantise h per (row, 512-block)
+    e = launch_quant_rows_fp8(h, A, I, hq, sh, s);
+    if (e == cudaSuccess && shared) e = launch_quant_rows_fp8(h_sh, T, Is, hq_sh, sh_sh, s);
+    mark(5);
+    if (e != cudaSuccess) return fail_cuda(p, e);
+
+    // A5: down
+    GemmMaps md{};
+    GemmArgs ad = ag;
+    ad.ttile = b.ttile_b;
+    ad.seg[0] = GemmSeg{H, I, A, w->s_down, nullptr, sh, y};
+    rc = encode_map_2d(&md.a0[0], w->w_down, U8, 1, I, (uint64_t)E * H, 128, 128, true);
+    rc |= encode_map_2d(&md.b[0], hq, U8, 1, I, A, 128, bn_b, true);
+    if (shared) {
+        ad.seg[1] = GemmSeg{H, Is, T, w->ss_down, nullptr, sh_sh, y_sh};
+        rc |= encode_map_2d(&md.a0[1], w->ws_down, U8, 1, Is, H, 128, 128, true);
+        rc |= encode_map_2d(&md.b[1], hq_sh, U8, 1, Is, T, 128, bn_b, true);
+    }
+    if (rc) return MOE_ERR_CUDA;
+    e = launch_gemm_fp8(false, bn_b, md, ad, p->num_sms, s);
+    mark(6);
+    if (e != cudaSuccess) return fail_cuda(p, e);
+
+    // A6: combine
+    e = launch_combine(y, y_sh, b.pos, b.topk_w, T, H, k, out, s);
+    mark(7);
+    if (e != cudaSuccess) return fail_cuda(p, e);
+    p->launches = 1 + 3 + 1 + 1 + (shared ? 2 : 1) + 1 + 1;
+    p->prof_recorded = p->prof;
+    return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,96 @@
+// moe_internal.h -- declarations shared by the library's translation units (not part of the ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/moe_b200.h"
+
+namespace moe {
+
+constexpr int kMaxE = 1024;   // router: at most 32 logits per lane
+constexpr int kMaxK = 32;     // router: one lane per selected expert
+constexpr int kChunk = 256;   // permutation: tokens per chunk (8 warps x 32)
+constexpr int kBlockK = 512;  // FP8 sub-channel block along K
+constexpr int kGroupK = 128;  // int4 scale group along K
+constexpr uint64_t kDefaultTimeoutNs = 1000000000ull;  // device-side waits give up after 1 s
+
+// ---- routing / permutation (route.cu) ---------------------------------------------------
+
+struct RouteBufs {
+    int32_t *topk_idx;    // [T, k]
+    float *topk_w;        // [T, k]
+    int32_t *counts;      // [E]
+    int32_t *offsets;     // [E + 1]
+    int32_t *perm_tok;    // [T * k]
+    int32_t *pos;         // [T, k]
+    int32_t *chunk_hist;  // [nchunks, E]
+    int32_t *ttile_a;     // [E + 1] token-tile prefix for the gate|up GEMM tile size
+    int32_t *ttile_b;     // [E + 1] token-tile prefix for the down GEMM tile size
+};
+
+cudaError_t launch_route(const float *logits, int T, int E, int k, int32_t *topk_idx, float *topk_w,
+                         cudaStream_t s);
+cudaError_t launch_permute(const RouteBufs &b, int T, int E, int k, int bn_a, int bn_b, cudaStream_t s);
+
+// ---- activation quantisation and gathers (quant.cu) --------------------------------------
+
+// FP8: quantise each bf16 token row of x (per 512-block) and write it to the permuted rows
+// pos[t, 0..k) and, when shared_rows != nullptr, to shared row t.
+cudaError_t launch_quant_x_fp8(const uint16_t *x, int T, int H, int k, const int32_t *pos, uint8_t *xq,
+                               float *sx, uint8_t *xq_shared, float *sx_shared, cudaStream_t s);
+// FP8: quantise fp32 rows (h) per 512-block.
+cudaError_t launch_quant_rows_fp8(const float *h, int R, int K, uint8_t *q, float *sq, cudaStream_t s);
+// int4 layers: copy bf16 token rows into the permuted rows (and the shared rows).
+cudaError_t launch_gather_x_bf16(const uint16_t *x, int T, int H, int k, const int32_t *pos, uint16_t *xp,
+                                 uint16_t *xp_shared, cudaStream_t s);
+
+// ---- combine (combine.cu) ----------------------------------------------------------------
+
+cudaError_t launch_combine(const float *y, const float *y_shared, const int32_t *pos, const float *topk_w,
+                           int T, int H, int k, uint16_t *out, cudaStream_t s);
+
+// ---- grouped GEMMs (gemm_fp8.cu, gemm_int4.cu) -------------------------------------------
+
+// One segment of a grouped GEMM: either the routed experts (E groups whose activation rows
+// are given by offsets) or the shared expert (one group over T rows).
+struct GemmSeg {
+    int N;          // weight rows (output features) per group, multiple of 128
+    int K;          // reduction length, multiple of 128
+    int rows;       // activation rows of this segment
+    const void *sw0;  // scales of the first weight matrix  (gate, or down)
+    const void *sw1;  // scales of the second weight matrix (up), gate|up only
+    const float *sx;  // activation scales [rows, ceil(K/512)] (FP8 only)
+    void *out;        // gate|up: h [rows, N]; down: y [rows, N]
+};
+
+struct GemmArgs {
+    GemmSeg seg[2];
+    int nseg;                // 1 (routed only) or 2 (routed + shared)
+    int E;                   // routed groups
+    int T;                   // shared-expert rows
+    const int32_t *offsets;  // [E + 1] routed group row offsets
+    const int32_t *ttile;    // [E + 1] routed token-tile prefix for this GEMM's tile size
+    int *status;             // device status word
+    uint64_t timeout_ns;
+};
+
+// Tensor maps of one GEMM launch: A (weights) 0 and 1 per segment, B (activations) per segment.
+struct GemmMaps {
+    CUtensorMap a0[2], a1[2], b[2];
+};
+
+// FP8 grouped GEMMs.  gateup: h = silu(x Wg^T) * (x Wu^T) in fp32; down: y = h Wd^T in fp32.
+cudaError_t launch_gemm_fp8(bool gateup, int bn, const GemmMaps &maps, const GemmArgs &args, int num_sms,
+                            cudaStream_t s);
+// int4 grouped GEMMs over bf16 activations: gate|up writes h as bf16, down writes y fp32.
+cudaError_t launch_gemm_int4(bool gateup, int bn, const GemmMaps &maps, const GemmArgs &args,
+                             int num_sms, cudaStream_t s);
+
+// Tensor-map encoding through the driver entry point (host).
+int encode_map_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, int elem_bytes,
+                  uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_outer, bool swizzle128);
+
+}  // namespace moe

@@ -1,0 +1,169 @@
+// quant.cu -- step A2: FP8 activation quantisation with 512-element sub-channels, and the
+// gathers that place activation rows in permuted (per-expert) order.
+//
+// Page "把 397B MoE 榨進 TPU7x：Google 拿到 4.7 倍加速", section "Kernel 手術台": the expert FFN
+// runs on FP8 with 512-element sub-channel quantisation.  Per (row, 512-block):
+// s = amax / 448 in fp32 (1 when amax == 0) and q = e4m3(x / s), rounded to nearest even
+// with saturation (cvt.rn.satfinite).  Both divisions are IEEE round-to-nearest; an all-zero
+// block stores zero codes.
+#include "moe_internal.h"
+
+#include <cuda_bf16.h>
+
+namespace moe {
+
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+__device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi)
+{
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t b) { return __uint_as_float(b << 16); }
+
+// Quantise 16 values (one lane's share of a 512-block held by one warp); returns the 16
+// codes as a uint4 and the block scale.
+__device__ __forceinline__ uint4 quant16(const float (&f)[16], bool valid, float *scale_out)
+{
+    float amax = 0.0f;
+    if (valid)
+#pragma unroll
+        for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, off));
+    uint4 q = make_uint4(0, 0, 0, 0);
+    float s = 1.0f;
+    if (amax > 0.0f) {
+        s = __fdiv_rn(amax, 448.0f);
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t lo = cvt_e4m3x2(__fdiv_rn(f[4 * i + 0], s), __fdiv_rn(f[4 * i + 1], s));
+            const uint32_t hi = cvt_e4m3x2(__fdiv_rn(f[4 * i + 2], s), __fdiv_rn(f[4 * i + 3], s));
+            w[i] = lo | (hi << 16);
+        }
+        q = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    *scale_out = s;
+    return q;
+}
+
+// 1-D grid of T * ceil(nb/4) blocks, 4 warps: warp w of block (t, bx) quantises 512-block
+// bx*4+w of token row t and writes it to the k permuted rows pos[t, :] and to shared row t.
+__global__ void __launch_bounds__(128) quant_x_fp8_kernel(const uint16_t *__restrict__ x, int H, int k,
+                                                          const int32_t *__restrict__ pos, uint8_t *__restrict__ xq,
+                                                          float *__restrict__ sx, uint8_t *__restrict__ xq_sh,
+                                                          float *__restrict__ sx_sh)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nb = (H + kBlockK - 1) / kBlockK;
+    const int nbx = (nb + 3) / 4;
+    const int t = blockIdx.x / nbx;
+    const int kb = (blockIdx.x - t * nbx) * 4 + warp;
+    if (kb >= nb) return;
+    const int i0 = kb * kBlockK + lane * 16;
+    const bool valid = i0 < H;
+    float f[16] = {};
+    if (valid) {
+        const uint4 *p = reinterpret_cast<const uint4 *>(x + (size_t)t * H + i0);
+        const uint4 a = __ldg(p), b = __ldg(p + 1);
+        const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            f[2 * i] = bf16_bits_to_float(w[i] & 0xffffu);
+            f[2 * i + 1] = bf16_bits_to_float(w[i] >> 16);
+        }
+    }
+    float s;
+    const uint4 q = quant16(f, valid, &s);
+    for (int j = 0; j < k; ++j) {
+        const int r = pos[(size_t)t * k + j];
+        if (valid) *reinterpret_cast<uint4 *>(xq + (size_t)r * H + i0) = q;
+        if (lane == 0) sx[(size_t)r * nb + kb] = s;
+    }
+    if (xq_sh) {
+        if (valid) *reinterpret_cast<uint4 *>(xq_sh + (size_t)t * H + i0) = q;
+        if (lane == 0) sx_sh[(size_t)t * nb + kb] = s;
+    }
+}
+
+// 1-D grid of R * ceil(nb/4) blocks: fp32 rows -> e4m3 rows + scales.
+__global__ void __launch_bounds__(128) quant_rows_fp8_kernel(const float *__restrict__ h, int K,
+                                                             uint8_t *__restrict__ q, float *__restrict__ sq)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nb = (K + kBlockK - 1) / kBlockK;
+    const int nbx = (nb + 3) / 4;
+    const int r = blockIdx.x / nbx;
+    const int kb = (blockIdx.x - r * nbx) * 4 + warp;
+    if (kb >= nb) return;
+    const int i0 = kb * kBlockK + lane * 16;
+    const bool valid = i0 < K;
+    float f[16] = {};
+    if (valid) {
+        const float4 *p = reinterpret_cast<const float4 *>(h + (size_t)r * K + i0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float4 v = __ldg(p + i);
+            f[4 * i] = v.x;
+            f[4 * i + 1] = v.y;
+            f[4 * i + 2] = v.z;
+            f[4 * i + 3] = v.w;
+        }
+    }
+    float s;
+    const uint4 qq = quant16(f, valid, &s);
+    if (valid) *reinterpret_cast<uint4 *>(q + (size_t)r * K + i0) = qq;
+    if (lane == 0) sq[(size_t)r * nb + kb] = s;
+}
+
+// grid T: copy bf16 token row t to the permuted rows pos[t, :] and to shared row t.
+__global__ void __launch_bounds__(128) gather_x_bf16_kernel(const uint16_t *__restrict__ x, int H, int k,
+                                                            const int32_t *__restrict__ pos, uint16_t *__restrict__ xp,
+                                                            uint16_t *__restrict__ xp_sh)
+{
+    const int t = blockIdx.x;
+    const int n16 = H / 8;  // uint4 chunks of 8 bf16
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * H);
+    for (int c = threadIdx.x; c < n16; c += blockDim.x) {
+        const uint4 v = __ldg(src + c);
+        for (int j = 0; j < k; ++j) {
+            const int r = pos[(size_t)t * k + j];
+            reinterpret_cast<uint4 *>(xp + (size_t)r * H)[c] = v;
+        }
+        if (xp_sh) reinterpret_cast<uint4 *>(xp_sh + (size_t)t * H)[c] = v;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_quant_x_fp8(const uint16_t *x, int T, int H, int k, const int32_t *pos, uint8_t *xq, float *sx,
+                               uint8_t *xq_shared, float *sx_shared, cudaStream_t s)
+{
+    if (T <= 0) return cudaSuccess;
+    const int nb = (H + kBlockK - 1) / kBlockK;
+    quant_x_fp8_kernel<<<(unsigned)(T * ((nb + 3) / 4)), 128, 0, s>>>(x, H, k, pos, xq, sx, xq_shared, sx_shared);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quant_rows_fp8(const float *h, int R, int K, uint8_t *q, float *sq, cudaStream_t s)
+{
+    if (R <= 0) return cudaSuccess;
+    const int nb = (K + kBlockK - 1) / kBlockK;
+    quant_rows_fp8_kernel<<<(unsigned)(R * ((nb + 3) / 4)), 128, 0, s>>>(h, K, q, sq);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather_x_bf16(const uint16_t *x, int T, int H, int k, const int32_t *pos, uint16_t *xp,
+                                 uint16_t *xp_shared, cudaStream_t s)
+{
+    if (T <= 0) return cudaSuccess;
+    gather_x_bf16_kernel<<<T, 128, 0, s>>>(x, H, k, pos, xp, xp_shared);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

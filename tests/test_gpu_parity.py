@@ -1,0 +1,159 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 CPU oracle.
+
+Bar (the layer's statement of correctness): routing indices, expert counts, offsets and the
+permutation bit-exact given the same fp32 logits; outputs within
+|gpu - oracle| <= 2e-3 + 1e-2 * |oracle| per element (bf16 out, fp32 accumulation).
+"""
+import numpy as np
+import pytest
+import torch
+
+import moe_synth
+import oracle
+import mixture_experts_ffn_13_b200 as moe
+
+pytestmark = pytest.mark.gpu
+
+ATOL, RTOL = 2e-3, 1e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    moe.load_library()
+
+
+def _bf16_to_f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def check_out(got_bf16: torch.Tensor, want: np.ndarray, what: str):
+    got = _bf16_to_f64(got_bf16)
+    err = np.abs(got - want)
+    bound = ATOL + RTOL * np.abs(want)
+    bad = err > bound
+    assert not bad.any(), (f"{what}: {bad.sum()} of {bad.size} outside tolerance; "
+                           f"worst excess {(err - bound).max():.3e} at {np.unravel_index(np.argmax(err - bound), err.shape)}")
+
+
+def check_route(plan, ws, logits: torch.Tensor, k: int):
+    r = moe.moe_route(plan, logits, ws)
+    torch.cuda.synchronize()
+    L = logits.cpu().numpy()
+    idx, w = oracle.route(L, k)
+    E = L.shape[1]
+    counts, offsets, perm, _ = oracle.permute(idx, E)
+    T = L.shape[0]
+    assert np.array_equal(r["topk_idx"].cpu().numpy(), idx)
+    assert np.array_equal(r["counts"].cpu().numpy(), counts)
+    assert np.array_equal(r["offsets"].cpu().numpy(), offsets)
+    assert np.array_equal(r["perm_tok"].cpu().numpy()[:T * k], perm)
+    assert np.allclose(r["topk_w"].cpu().numpy(), w, rtol=2e-6, atol=1e-7)
+    return r
+
+
+# ---------------------------------------------------------------------------------------
+# routing and permutation
+# ---------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("T,E,k", [(1, 8, 2), (16, 8, 2), (300, 64, 6), (513, 512, 10), (1000, 1024, 32),
+                                   (77, 5, 5), (257, 3, 1), (4096, 256, 8)])
+def test_route_random(T, E, k):
+    plan = moe.Plan(T, 128, E, 128, k)
+    ws = plan.new_workspace()
+    g = torch.Generator(device="cuda").manual_seed(T * 7 + E)
+    logits = torch.randn((T, E), generator=g, device="cuda")
+    check_route(plan, ws, logits, k)
+
+
+def test_route_ties_and_plateaus():
+    T, E, k = 600, 96, 7
+    plan = moe.Plan(T, 128, E, 128, k)
+    ws = plan.new_workspace()
+    g = torch.Generator(device="cuda").manual_seed(3)
+    # logits drawn from a handful of values: many exact ties, broken by the lower index
+    logits = torch.randint(0, 4, (T, E), generator=g, device="cuda").float() * 0.5
+    logits[0] = 1.0  # a row of all-equal logits
+    check_route(plan, ws, logits, k)
+
+
+def test_route_empty_batch():
+    plan = moe.Plan(8, 128, 16, 128, 2)
+    ws = plan.new_workspace()
+    r = moe.moe_route(plan, torch.zeros((0, 16), device="cuda"), ws)
+    torch.cuda.synchronize()
+    assert int(r["counts"].sum()) == 0 and int(r["offsets"][-1]) == 0
+
+
+@pytest.mark.parametrize("name", list(moe_synth.CONFIGS))
+def test_route_configs_full_size(name):
+    cfg = moe_synth.CONFIGS[name]
+    layer = moe_synth.make_layer(dict(cfg, E=cfg["E"], I=128, Is=0, H=128), device="cuda")
+    plan = moe.Plan(cfg["T"], 128, cfg["E"], 128, cfg["k"], 0, cfg["wfmt"])
+    ws = plan.new_workspace()
+    check_route(plan, ws, layer["logits"], cfg["k"])
+
+
+# ---------------------------------------------------------------------------------------
+# the whole layer
+# ---------------------------------------------------------------------------------------
+
+SMALL_FP8 = [
+    dict(T=16, H=512, E=8, I=256, k=2, Is=0, seed=0, bias=None),          # the tiny layer
+    dict(T=1, H=512, E=4, I=128, k=2, Is=128, seed=21, bias=None),        # one token
+    dict(T=37, H=1024, E=16, I=384, k=4, Is=256, seed=22, bias="normal"),  # ragged groups, partial h block
+    dict(T=200, H=768, E=8, I=640, k=3, Is=0, seed=23, bias="zipf"),       # partial K blocks, >1 token tile
+    dict(T=130, H=512, E=2, I=128, k=1, Is=512, seed=24, bias=None),       # groups of ~65 rows
+    dict(T=64, H=1536, E=64, I=256, k=8, Is=0, seed=25, bias="zipf"),      # empty experts
+]
+
+
+@pytest.mark.parametrize("cfg", SMALL_FP8, ids=lambda c: f"T{c['T']}-H{c['H']}-E{c['E']}-I{c['I']}-k{c['k']}-Is{c['Is']}")
+def test_layer_fp8_small(cfg):
+    cfg = dict(cfg, wfmt="fp8")
+    layer = moe_synth.make_layer(cfg, device="cuda")
+    m = moe.MoELayer(layer)
+    out = m(layer["x"], layer["logits"])
+    assert moe.moe_get_status(m.plan) == 0
+    want, _ = oracle.layer(moe_synth.to_numpy(layer))
+    check_out(out, want, "layer")
+    # a second call on the same workspace gives the same bits
+    out2 = m(layer["x"], layer["logits"])
+    torch.cuda.synchronize()
+    assert torch.equal(out, out2)
+
+
+def test_layer_fp8_variable_T_within_plan():
+    cfg = dict(T=100, H=512, E=8, I=256, k=2, Is=128, wfmt="fp8", seed=31, bias=None)
+    layer = moe_synth.make_layer(cfg, device="cuda")
+    m = moe.MoELayer(layer, T_max=100)
+    L = moe_synth.to_numpy(layer)
+    want, _ = oracle.layer(L)
+    for T in (100, 3, 57):
+        out = m(layer["x"][:T].contiguous(), layer["logits"][:T].contiguous())
+        check_out(out, want[:T], f"T={T}")
+    out0 = m(layer["x"][:0], layer["logits"][:0])
+    assert out0.shape == (0, 512)
+
+
+def _sampled_parity(name, n_sample=12):
+    cfg = moe_synth.CONFIGS[name]
+    layer = moe_synth.make_layer(name, device="cuda")
+    m = moe.MoELayer(layer)
+    out = m(layer["x"], layer["logits"])
+    assert moe.moe_get_status(m.plan) == 0
+    torch.cuda.synchronize()
+    T = cfg["T"]
+    rng = np.random.default_rng(99)
+    sel = np.unique(np.concatenate([[0, T - 1], rng.choice(T, n_sample, replace=False)])).astype(np.int32)
+    L = moe_synth.to_numpy(layer)
+    want, _ = oracle.layer(L, sel)
+    check_out(out[torch.from_numpy(sel).long().cuda()], want, name)
+    # the routing of the whole batch is bit-exact as well
+    check_route(m.plan, m.workspace, layer["logits"], cfg["k"])
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode", "prefill", "skewed"])
+def test_layer_fp8_configs_sampled(name):
+    _sampled_parity(name)
