@@ -66,7 +66,7 @@ def lib():
             L.orc_quant_rows_bf16.argtypes = [I, I, P, P, P]
             L.orc_expert_fp8_row.argtypes = [I, I] + [P] * 10
             L.orc_expert_int4_row.argtypes = [I, I] + [P] * 9
-            L.orc_layer.argtypes = [ctypes.POINTER(Dims), ctypes.POINTER(Weights), P, P, I, P, P, P, I]
+            L.orc_layer.argtypes = [ctypes.POINTER(Dims), ctypes.POINTER(Weights), P, P, I, P, P, P, P, I]
             _lib = L
     return _lib
 
@@ -186,8 +186,10 @@ def expert_int4_row(x_bits, wg, sg, wu, su, wd, sd):
 # the layer
 # --------------------------------------------------------------------------------------
 
-def layer(layer_np: dict, tokens=None, nthreads: int | None = None):
-    """Layer output for ``tokens`` (default: all) -> (out float64 [n,H], out_bf16 uint16 [n,H]).
+def layer(layer_np: dict, tokens=None, nthreads: int | None = None, ambiguity: bool = False):
+    """Layer output for ``tokens`` (default: all) -> (out float64 [n,H], out_bf16 uint16 [n,H]),
+    plus, with ``ambiguity=True``, the envelope float64 [n,H] of the equally valid outputs
+    that an h code sitting on a rounding midpoint allows (see moe_oracle.c, reading R10a).
 
     ``layer_np`` holds numpy arrays with the keys of ``moe_synth`` (x as bf16 bit patterns).
     """
@@ -217,10 +219,13 @@ def layer(layer_np: dict, tokens=None, nthreads: int | None = None):
     n = tokens.size
     out = np.empty((n, d["H"]), np.float64)
     outb = np.empty((n, d["H"]), np.uint16)
+    amb = np.empty((n, d["H"]), np.float64) if ambiguity else None
     if nthreads is None:
         nthreads = os.cpu_count() or 1
     rc = lib().orc_layer(ctypes.byref(dims), ctypes.byref(W), _p(x), _p(logits), n, _p(tokens),
-                         _p(out), _p(outb), int(nthreads))
+                         _p(out), _p(outb), _p(amb), int(nthreads))
     if rc != 0:
         raise ValueError("oracle layer: bad dims or token index")
+    if ambiguity:
+        return out, outb, amb
     return out, outb

@@ -325,11 +325,49 @@ static void orc_proj_fp8(int N, int K, const uint8_t *qx, const float *sx, const
 
 static double orc_silu(double z) { return z * (1.0 / (1.0 + exp(-z))); }
 
+/* R10a -- which h codes are not unique.  The layer rounds h to fp32 before quantising it
+ * (R10), and an fp32 h obtained with another (equally valid) summation order can sit on the
+ * other side of an e4m3 rounding midpoint, which moves that code by one step.  A code counts
+ * as ambiguous when fl32(h/s) lies within a relative distance ORC_AMBIG_REL of the midpoint
+ * between its e4m3 value and the neighbour on that side; the neighbour is then an equally
+ * valid result.  For each ambiguous element i the down projection can move by
+ * |dec(q_alt) - dec(q)| * s * |Wd[n, i] * sd[n, block(i)]| in output n; env[n] receives the
+ * sum of those bounds (the envelope of the valid outputs around y).  ORC_AMBIG_REL = 2^-16
+ * bounds the relative error of an fp32 accumulation of these dot products with margin. */
+#define ORC_AMBIG_REL (1.0 / 65536.0)
+
+static void orc_h_ambiguity(int H, int I, const float *h, const uint8_t *qh, const float *sh,
+                            const uint8_t *wd, const float *sd, double *env)
+{
+    int nbI = (I + 511) / 512;
+    for (int i = 0; i < I; ++i) {
+        int code = qh[i] & 0x7F;
+        float sc = sh[i / 512];
+        double a = fabs((double)(float)(h[i] / sc)); /* the value the rounding decided on */
+        double r = orc_dec_tab[code];
+        int nb_code;
+        if (a >= r)
+            nb_code = code + 1;
+        else
+            nb_code = code - 1;
+        if (nb_code < 0 || nb_code > 0x7E) continue; /* no neighbour (zero side or saturated) */
+        double rn = orc_dec_tab[nb_code];
+        double mid = 0.5 * (r + rn);
+        if (fabs(a - mid) > ORC_AMBIG_REL * a) continue;
+        double dh = fabs(rn - r) * (double)sc;
+        for (int n = 0; n < H; ++n) {
+            double wv = orc_dec_tab[wd[(size_t)n * I + i]] * (double)sd[(size_t)n * nbI + i / 512];
+            env[n] += dh * fabs(wv);
+        }
+    }
+}
+
 /* One FP8 expert (gate/up/down already offset to that expert) on one quantised row.
- * h_out (optional, I values) receives h rounded to fp32 before its quantisation (R10). */
+ * h_out (optional, I values) receives h rounded to fp32 before its quantisation (R10);
+ * env (optional, H values) is cleared and receives the R10a envelope. */
 static void orc_expert_fp8(int H, int I, const uint8_t *qx, const float *sx, const uint8_t *wg,
                            const float *sg, const uint8_t *wu, const float *su, const uint8_t *wd,
-                           const float *sd, double *y, float *h_out)
+                           const float *sd, double *y, float *h_out, double *env)
 {
     double *G = (double *)malloc(sizeof(double) * (size_t)I);
     double *U = (double *)malloc(sizeof(double) * (size_t)I);
@@ -342,6 +380,10 @@ static void orc_expert_fp8(int H, int I, const uint8_t *qx, const float *sx, con
     if (h_out) memcpy(h_out, h, sizeof(float) * (size_t)I);
     orc_quant_row_fp8(I, h, qh, sh);
     orc_proj_fp8(H, I, qh, sh, wd, sd, y);
+    if (env) {
+        for (int n = 0; n < H; ++n) env[n] = 0.0;
+        orc_h_ambiguity(H, I, h, qh, sh, wd, sd, env);
+    }
     free(G);
     free(U);
     free(h);
@@ -376,20 +418,51 @@ static void orc_proj_int4(int N, int K, const double *a, const uint8_t *qw, cons
     }
 }
 
+/* R10a for 4-bit layers: h is rounded to bf16, so an h within ORC_AMBIG_REL of a bf16
+ * rounding midpoint may round either way; env[n] gets |h_alt - h| * |W[n, i]| for each such i. */
+static void orc_h_ambiguity_bf16(int H, int I, const double *hx, const uint8_t *wd,
+                                 const uint16_t *sd, double *env)
+{
+    for (int i = 0; i < I; ++i) {
+        double a = fabs(hx[i]);
+        if (a == 0.0) continue;
+        int e2;
+        frexp(a, &e2);
+        int lead = e2 - 1 < -126 ? -126 : e2 - 1;
+        double quantum = ldexp(1.0, lead - 7);
+        double frac = a / quantum - floor(a / quantum); /* position between two bf16 values */
+        if (fabs(frac - 0.5) * quantum > ORC_AMBIG_REL * a) continue;
+        for (int n = 0; n < H; ++n) {
+            const uint8_t *row = wd + (size_t)n * (I / 2);
+            double wv = (double)orc_nib(row, i) * orc_bf16_to_double(sd[(size_t)n * (I / 128) + i / 128]);
+            env[n] += quantum * fabs(wv);
+        }
+    }
+}
+
 static void orc_expert_int4(int H, int I, const double *x, const uint8_t *wg, const uint16_t *sg,
                             const uint8_t *wu, const uint16_t *su, const uint8_t *wd,
-                            const uint16_t *sd, double *y, double *h_out)
+                            const uint16_t *sd, double *y, double *h_out, double *env)
 {
     double *G = (double *)malloc(sizeof(double) * (size_t)I);
     double *U = (double *)malloc(sizeof(double) * (size_t)I);
+    double *hx = (double *)malloc(sizeof(double) * (size_t)I);
     double *h = (double *)malloc(sizeof(double) * (size_t)I);
     orc_proj_int4(I, H, x, wg, sg, G);
     orc_proj_int4(I, H, x, wu, su, U);
-    for (int n = 0; n < I; ++n) h[n] = orc_bf16_to_double(orc_double_to_bf16(orc_silu(G[n]) * U[n]));
+    for (int n = 0; n < I; ++n) {
+        hx[n] = orc_silu(G[n]) * U[n];
+        h[n] = orc_bf16_to_double(orc_double_to_bf16(hx[n]));
+    }
     if (h_out) memcpy(h_out, h, sizeof(double) * (size_t)I);
     orc_proj_int4(H, I, h, wd, sd, y);
+    if (env) {
+        for (int n = 0; n < H; ++n) env[n] = 0.0;
+        orc_h_ambiguity_bf16(H, I, hx, wd, sd, env);
+    }
     free(G);
     free(U);
+    free(hx);
     free(h);
 }
 
@@ -406,19 +479,23 @@ typedef struct {
     int n_sel;
     double *out;          /* [n_sel,H] fp64 before the final rounding */
     uint16_t *out_bf16;   /* [n_sel,H] */
+    double *amb;          /* [n_sel,H] R10a envelope, or NULL */
     int next;             /* next index of sel to take (guarded by mu) */
     pthread_mutex_t mu;
 } orc_job;
 
 static void orc_layer_token(const orc_dims *d, const orc_weights *w, const uint16_t *xrow,
-                            const float *lrow, double *out)
+                            const float *lrow, double *out, double *amb)
 {
     int H = d->H, I = d->I, E = d->E, k = d->k, Is = d->Is;
     int32_t *idx = (int32_t *)malloc(sizeof(int32_t) * (size_t)k);
     double *p = (double *)malloc(sizeof(double) * (size_t)k);
     double *y = (double *)malloc(sizeof(double) * (size_t)H);
+    double *env = amb ? (double *)malloc(sizeof(double) * (size_t)H) : NULL;
     orc_route_token(E, k, lrow, idx, p);
     for (int n = 0; n < H; ++n) out[n] = 0.0;
+    if (amb)
+        for (int n = 0; n < H; ++n) amb[n] = 0.0;
 
     if (d->wfmt == ORC_FP8_SC512) {
         int nbH = (H + 511) / 512, nbI = (I + 511) / 512, nbIs = (Is + 511) / 512;
@@ -433,13 +510,18 @@ static void orc_layer_token(const orc_dims *d, const orc_weights *w, const uint1
             size_t e = (size_t)idx[j];
             orc_expert_fp8(H, I, qx, sx, w->w_gate + e * I * H, sg + e * I * nbH,
                            w->w_up + e * I * H, su + e * I * nbH, w->w_down + e * H * I,
-                           sd + e * H * nbI, y, NULL);
+                           sd + e * H * nbI, y, NULL, env);
             for (int n = 0; n < H; ++n) out[n] += p[j] * y[n];
+            if (amb)
+                for (int n = 0; n < H; ++n) amb[n] += p[j] * env[n];
         }
         if (Is > 0) {
             orc_expert_fp8(H, Is, qx, sx, w->ws_gate, (const float *)w->ss_gate, w->ws_up,
-                           (const float *)w->ss_up, w->ws_down, (const float *)w->ss_down, y, NULL);
+                           (const float *)w->ss_up, w->ws_down, (const float *)w->ss_down, y, NULL,
+                           env);
             for (int n = 0; n < H; ++n) out[n] += y[n];
+            if (amb)
+                for (int n = 0; n < H; ++n) amb[n] += env[n];
         }
         (void)nbIs;
         free(xf);
@@ -454,20 +536,25 @@ static void orc_layer_token(const orc_dims *d, const orc_weights *w, const uint1
             size_t e = (size_t)idx[j];
             orc_expert_int4(H, I, xd, w->w_gate + e * I * (H / 2), sg + e * I * (H / 128),
                             w->w_up + e * I * (H / 2), su + e * I * (H / 128),
-                            w->w_down + e * H * (I / 2), sd + e * H * (I / 128), y, NULL);
+                            w->w_down + e * H * (I / 2), sd + e * H * (I / 128), y, NULL, env);
             for (int n = 0; n < H; ++n) out[n] += p[j] * y[n];
+            if (amb)
+                for (int n = 0; n < H; ++n) amb[n] += p[j] * env[n];
         }
         if (Is > 0) {
             orc_expert_int4(H, Is, xd, w->ws_gate, (const uint16_t *)w->ss_gate, w->ws_up,
                             (const uint16_t *)w->ss_up, w->ws_down, (const uint16_t *)w->ss_down,
-                            y, NULL);
+                            y, NULL, env);
             for (int n = 0; n < H; ++n) out[n] += y[n];
+            if (amb)
+                for (int n = 0; n < H; ++n) amb[n] += env[n];
         }
         free(xd);
     }
     free(idx);
     free(p);
     free(y);
+    free(env);
 }
 
 static void *orc_worker(void *arg)
@@ -482,17 +569,21 @@ static void *orc_worker(void *arg)
         int t = jb->sel[i];
         const orc_dims *d = jb->d;
         double *o = jb->out + (size_t)i * d->H;
-        orc_layer_token(d, jb->w, jb->x + (size_t)t * d->H, jb->logits + (size_t)t * d->E, o);
+        orc_layer_token(d, jb->w, jb->x + (size_t)t * d->H, jb->logits + (size_t)t * d->E, o,
+                        jb->amb ? jb->amb + (size_t)i * d->H : NULL);
         for (int n = 0; n < d->H; ++n) jb->out_bf16[(size_t)i * d->H + n] = orc_double_to_bf16(o[n]);
     }
     return NULL;
 }
 
 /* The layer output for the tokens sel[0..n_sel): out (fp64, before rounding) and out_bf16
- * (R12).  Tokens are independent, so any subset is exact; nthreads workers take tokens in
- * turn.  Returns 0, or -1 on bad dims. */
+ * (R12); amb (optional) receives the R10a envelope per output (zero where no h value sits
+ * at a rounding boundary).  Tokens are
+ * independent, so any subset is exact; nthreads workers take tokens in turn.  Returns 0, or
+ * -1 on bad dims. */
 int orc_layer(const orc_dims *d, const orc_weights *w, const uint16_t *x, const float *logits,
-              int n_sel, const int32_t *sel, double *out, uint16_t *out_bf16, int nthreads)
+              int n_sel, const int32_t *sel, double *out, uint16_t *out_bf16, double *amb,
+              int nthreads)
 {
     if (d->E < 1 || d->k < 1 || d->k > d->E || d->H < 1 || d->I < 1 || d->Is < 0) return -1;
     if (d->wfmt == ORC_INT4_G128 && (d->H % 128 || d->I % 128 || d->Is % 128)) return -1;
@@ -509,6 +600,7 @@ int orc_layer(const orc_dims *d, const orc_weights *w, const uint16_t *x, const 
     jb.n_sel = n_sel;
     jb.out = out;
     jb.out_bf16 = out_bf16;
+    jb.amb = amb;
     jb.next = 0;
     pthread_mutex_init(&jb.mu, NULL);
     if (nthreads < 1) nthreads = 1;
@@ -543,7 +635,7 @@ void orc_expert_fp8_row(int H, int I, const uint8_t *qx, const float *sx, const 
                         const float *sd, double *y, float *h)
 {
     pthread_once(&orc_tab_once, orc_tab_init);
-    orc_expert_fp8(H, I, qx, sx, wg, sg, wu, su, wd, sd, y, h);
+    orc_expert_fp8(H, I, qx, sx, wg, sg, wu, su, wd, sd, y, h, NULL);
 }
 
 /* One int4 expert on one bf16 row: y (H values) and h (I values, bf16-rounded). */
@@ -553,6 +645,6 @@ void orc_expert_int4_row(int H, int I, const uint16_t *x, const uint8_t *wg, con
 {
     double *xd = (double *)malloc(sizeof(double) * (size_t)H);
     for (int i = 0; i < H; ++i) xd[i] = orc_bf16_to_double(x[i]);
-    orc_expert_int4(H, I, xd, wg, sg, wu, su, wd, sd, y, h);
+    orc_expert_int4(H, I, xd, wg, sg, wu, su, wd, sd, y, h, NULL);
     free(xd);
 }

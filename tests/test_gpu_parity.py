@@ -28,10 +28,12 @@ def _bf16_to_f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
-def check_out(got_bf16: torch.Tensor, want: np.ndarray, what: str):
+def check_out(got_bf16: torch.Tensor, want: np.ndarray, what: str, amb: np.ndarray | None = None):
+    """Per-element bound ATOL + RTOL*|oracle|, widened only by the oracle's envelope of equally
+    valid outputs where an h value sits on an FP8/bf16 rounding midpoint (zero elsewhere)."""
     got = _bf16_to_f64(got_bf16)
     err = np.abs(got - want)
-    bound = ATOL + RTOL * np.abs(want)
+    bound = ATOL + RTOL * np.abs(want) + (amb if amb is not None else 0.0)
     bad = err > bound
     assert not bad.any(), (f"{what}: {bad.sum()} of {bad.size} outside tolerance; "
                            f"worst excess {(err - bound).max():.3e} at {np.unravel_index(np.argmax(err - bound), err.shape)}")
@@ -116,8 +118,8 @@ def test_layer_fp8_small(cfg):
     m = moe.MoELayer(layer)
     out = m(layer["x"], layer["logits"])
     assert moe.moe_get_status(m.plan) == 0
-    want, _ = oracle.layer(moe_synth.to_numpy(layer))
-    check_out(out, want, "layer")
+    want, _, amb = oracle.layer(moe_synth.to_numpy(layer), ambiguity=True)
+    check_out(out, want, "layer", amb)
     # a second call on the same workspace gives the same bits
     out2 = m(layer["x"], layer["logits"])
     torch.cuda.synchronize()
@@ -129,10 +131,10 @@ def test_layer_fp8_variable_T_within_plan():
     layer = moe_synth.make_layer(cfg, device="cuda")
     m = moe.MoELayer(layer, T_max=100)
     L = moe_synth.to_numpy(layer)
-    want, _ = oracle.layer(L)
+    want, _, amb = oracle.layer(L, ambiguity=True)
     for T in (100, 3, 57):
         out = m(layer["x"][:T].contiguous(), layer["logits"][:T].contiguous())
-        check_out(out, want[:T], f"T={T}")
+        check_out(out, want[:T], f"T={T}", amb[:T])
     out0 = m(layer["x"][:0], layer["logits"][:0])
     assert out0.shape == (0, 512)
 
@@ -148,8 +150,8 @@ def _sampled_parity(name, n_sample=12):
     rng = np.random.default_rng(99)
     sel = np.unique(np.concatenate([[0, T - 1], rng.choice(T, n_sample, replace=False)])).astype(np.int32)
     L = moe_synth.to_numpy(layer)
-    want, _ = oracle.layer(L, sel)
-    check_out(out[torch.from_numpy(sel).long().cuda()], want, name)
+    want, _, amb = oracle.layer(L, sel, ambiguity=True)
+    check_out(out[torch.from_numpy(sel).long().cuda()], want, name, amb)
     # the routing of the whole batch is bit-exact as well
     check_route(m.plan, m.workspace, layer["logits"], cfg["k"])
 

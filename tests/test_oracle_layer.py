@@ -258,3 +258,41 @@ def test_shared_expert_adds_with_weight_one(orc):
     Ls["logits"] = np.zeros((cfg["T"], 1), np.float32)
     shared, _ = orc.layer(Ls)
     assert np.allclose(with_shared, routed + shared, rtol=1e-14, atol=1e-14)
+
+
+def test_h_on_a_rounding_midpoint_reports_the_envelope(orc):
+    """G = 64 (silu(64) = 64 in fp64), U = (7, 2.625): h = (448, 168) exactly, so s_h = 1 and
+    h[1] = 168 is the midpoint between the e4m3 values 160 and 176.  Round-to-nearest-even
+    takes 160; 176 is an equally valid outcome for an fp32 h one ulp higher, so the envelope
+    of output n is 16 * |Wd[n, 1]|, and zero in every output that h[1] does not reach."""
+    H, I = 512, 2
+    x = np.zeros((1, H), np.float32)
+    x[0, 0], x[0, 1], x[0, 511] = 1.0, 1.0, 448.0
+    wg = np.zeros((1, I, H), np.uint8)
+    wu = np.zeros((1, I, H), np.uint8)
+    wg[0, :, 0] = _code(orc, 64.0)
+    wu[0, 0, 0] = _code(orc, 7.0)
+    wu[0, 1, 0], wu[0, 1, 1] = _code(orc, 2.5), _code(orc, 0.125)
+    rng = np.random.default_rng(5)
+    wd = np.zeros((1, H, I), np.uint8)
+    wd[0, :, 0] = rng.integers(0x10, 0x30, H)
+    wd[0, :200, 1] = rng.integers(0x10, 0x30, 200) | (rng.integers(0, 2, 200) << 7).astype(np.uint8)
+    ones = lambda *s: np.ones(s, np.float32)
+    L = dict(dims=dict(T=1, H=H, E=1, I=I, k=1, Is=0, wfmt="fp8"), x=_bits(x),
+             logits=np.zeros((1, 1), np.float32), w_gate=wg, w_up=wu, w_down=wd,
+             s_gate=ones(1, I, 1), s_up=ones(1, I, 1), s_down=ones(1, H, 1))
+    out, _, amb = orc.layer(L, ambiguity=True)
+    dec = lambda c: np.array([orc.e4m3_decode(int(v)) for v in c])
+    d0, d1 = dec(wd[0, :, 0]), dec(wd[0, :, 1])
+    assert np.array_equal(out[0], 448.0 * d0 + 160.0 * d1)
+    assert np.array_equal(amb[0], 16.0 * np.abs(d1))
+    assert np.all(amb[0, 200:] == 0) and np.all(amb[0, :200] > 0)
+
+
+def test_envelope_is_zero_off_the_midpoints(orc):
+    L = moe_synth.to_numpy(moe_synth.make_layer(SMALL[0]))
+    out, outb, amb = orc.layer(L, ambiguity=True)
+    out2, _ = orc.layer(L)
+    assert np.array_equal(out, out2)
+    # random data essentially never puts an h within 2^-16 of a midpoint
+    assert (amb != 0).mean() < 0.05
