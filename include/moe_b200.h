@@ -111,6 +111,23 @@ MOE_API int moe_route(moe_plan_t *plan, int32_t T, const float *logits, int32_t 
               int32_t *counts, int32_t *offsets, int32_t *perm_tok, void *workspace,
               size_t ws_bytes, moe_stream_t stream);
 
+/* Routing and permutation without any allocation, for callers that cannot call cudaMalloc
+ * (code inside an allocator or pool callback, serving loops that forbid allocation after
+ * start-up, embedders whose device memory another allocator has reserved).  The pages have no
+ * counterpart: this is a library convenience.  Same outputs and argument rules as moe_route,
+ * but no plan and no workspace: its scratch is one fixed 2 MiB __device__ array in the library
+ * (held by every GPU that loads it until the process exits), so
+ *   T*k + ceil(T/256)*E + 2*(E+1) <= 2^19 is required (else MOE_ERR_UNSUPPORTED, before any
+ *   device work), with 1 <= k <= min(E, 32) and E <= 1024;
+ *   the first call on a device looks up the array's address (cudaGetSymbolAddress, once per
+ *   device, with it current) -- make that first call before any stream capture;
+ *   all calls share the array: calls whose kernels may overlap on the GPU race and must be
+ *   serialised by the caller.
+ * Returns MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED or MOE_ERR_CUDA. */
+MOE_API int moe_route_static(int32_t T, int32_t E, int32_t k, const float *logits, int32_t *topk_idx,
+                             float *topk_w, int32_t *counts, int32_t *offsets, int32_t *perm_tok,
+                             moe_stream_t stream);
+
 /* The whole layer: out[T, H] (bf16) from x[T, H] (bf16), logits[T, E] (fp32) and the
  * weights.  0 <= T <= T_max.  The workspace (>= the size moe_plan reported, 256-byte
  * aligned) holds every intermediate; its contents are undefined after the call. */

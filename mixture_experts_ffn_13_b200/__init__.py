@@ -25,7 +25,7 @@ ERRORS = {-1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED", -3: "MOE_ERR_WOR
           -4: "MOE_ERR_CUDA", -5: "MOE_ERR_DEVICE_TIMEOUT", -6: "MOE_ERR_BOUNDS"}
 EXPORTS = ("moe_plan", "moe_route", "moe_forward", "moe_get_status", "moe_last_cuda_error",
            "moe_destroy", "moe_strerror", "moe_profile_enable", "moe_profile_read",
-           "moe_profile_stage_name", "moe_launch_count")
+           "moe_profile_stage_name", "moe_launch_count", "moe_route_static")
 STAGES = ("route", "permute", "quant_x", "gemm_gateup", "quant_h", "gemm_down", "combine")
 
 
@@ -84,6 +84,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             L.moe_profile_stage_name.restype = ctypes.c_char_p
             L.moe_launch_count.argtypes = [P]
             L.moe_launch_count.restype = ctypes.c_int
+            L.moe_route_static.argtypes = [I32, I32, I32, P, P, P, P, P, P, P]
+            L.moe_route_static.restype = ctypes.c_int
             _lib = L
     return _lib
 
@@ -198,6 +200,26 @@ def moe_route(plan: Plan, logits: torch.Tensor, workspace: torch.Tensor, out: di
                                   _ptr(out["counts"]), _ptr(out["offsets"]), _ptr(out["perm_tok"]),
                                   _ptr(workspace), workspace.numel(), _stream(stream))
     _check(rc, "moe_route", plan.handle)
+    return out
+
+
+def moe_route_static(logits: torch.Tensor, k: int, out: dict | None = None, stream=None) -> dict:
+    """moe_route without a plan or workspace (fixed static scratch inside the library; for
+    callers that cannot allocate device memory -- see include/moe_b200.h for its limits)."""
+    T, E = logits.shape
+    if logits.dtype != torch.float32 or logits.dim() != 2:
+        raise ValueError("logits must be fp32 [T, E]")
+    dev = logits.device
+    if out is None:
+        out = dict(topk_idx=torch.empty((T, k), dtype=torch.int32, device=dev),
+                   topk_w=torch.empty((T, k), dtype=torch.float32, device=dev),
+                   counts=torch.empty((E,), dtype=torch.int32, device=dev),
+                   offsets=torch.empty((E + 1,), dtype=torch.int32, device=dev),
+                   perm_tok=torch.empty((max(T * k, 1),), dtype=torch.int32, device=dev))
+    rc = load_library().moe_route_static(T, E, k, _ptr(logits), _ptr(out["topk_idx"]), _ptr(out["topk_w"]),
+                                         _ptr(out["counts"]), _ptr(out["offsets"]), _ptr(out["perm_tok"]),
+                                         _stream(stream))
+    _check(rc, "moe_route_static")
     return out
 
 
