@@ -17,7 +17,6 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -97,53 +96,65 @@ def max_over_ranks(ws, v):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms during the timed region."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event reasons read through NVML (read-only) every ~2 ms by a background
+    thread while the timed region runs; falls back to nothing if NVML is unavailable."""
 
-    def __init__(self, gpu_index):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = os.path.join("/tmp", f"moe_clocks_{os.getpid()}.csv")
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
+
+    def __init__(self, cuda_index):
+        import threading
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.stop_ev = threading.Event()
+        self.thread = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(cuda_index)
+            try:
+                bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(cuda_index)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        masks = [(n, getattr(nv, a, 0)) for n, a in self.REASONS]
+        while not self.stop_ev.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for n, m in masks:
+                    if m and (r & m):
+                        self.reasons.add(n)
+            except Exception:
+                pass
+            self.stop_ev.wait(0.002)
 
     def start(self):
-        try:
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=self.f, stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+        if self.nv is None:
+            return
+        import threading
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
 
     def stop(self):
-        if self.proc is None:
+        if self.thread is None:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.f.close()
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        os.unlink(self.path)
-        if not sm:
+        self.stop_ev.set()
+        self.thread.join()
+        if not self.samples:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples), "source": "nvml"}
 
 
 def algorithmic(cfg, counts):
@@ -196,7 +207,7 @@ def run_reference(args, ws, rank, cfg_name):
     import torch
     if rank != 0:
         return
-    cfg = moe_synth.CONFIGS[cfg_name]
+    cfg = {**moe_synth.CONFIGS, **moe_synth.PROFILE_CONFIGS}[cfg_name]
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     Lnp, _ = make_host_layer(cfg_name, dev)
     if dev == "cuda":
@@ -235,7 +246,7 @@ def run_ours(args, ws, rank, local, cfg_name):
     from mixture_experts_ffn_13_b200 import build as moe_build
 
     moe_build.build()
-    cfg = moe_synth.CONFIGS[cfg_name]
+    cfg = {**moe_synth.CONFIGS, **moe_synth.PROFILE_CONFIGS}[cfg_name]
     dev = torch.device("cuda", torch.cuda.current_device())
     layer = moe_synth.make_layer(cfg_name, device=dev)
     m = moe.MoELayer(layer)

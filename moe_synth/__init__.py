@@ -47,6 +47,17 @@ CONFIGS = {
                  workload="4-bit-weight MoE T=1024 H=4096 E=128 I=1536 top-8, int4 g128 bf16"),
 }
 
+# Smaller layers with the same per-expert shapes, for profiler captures (weights still far
+# larger than the 126 MB L2, a few GB on the device at most).
+PROFILE_CONFIGS = {
+    "profile-decode": dict(T=64, H=4096, E=64, I=1024, k=10, Is=1024, wfmt="fp8", seed=5, bias=None,
+                           workload="decode-shaped MoE T=64 H=4096 E=64 I=1024 top-10 + shared 1024, FP8"),
+    "profile-prefill": dict(T=1024, H=4096, E=64, I=1024, k=10, Is=1024, wfmt="fp8", seed=6, bias="normal",
+                            workload="prefill-shaped MoE T=1024 H=4096 E=64 I=1024 top-10 + shared 1024, FP8"),
+    "profile-int4": dict(T=128, H=4096, E=16, I=1536, k=8, Is=0, wfmt="int4", seed=7, bias=None,
+                         workload="4-bit MoE T=128 H=4096 E=16 I=1536 top-8, int4 g128"),
+}
+
 # tensor ids for the per-tensor generators
 _TID = {"x": 1, "logits": 2, "bias": 3, "rank": 4, "w_gate": 5, "w_up": 6, "w_down": 7,
         "ws_gate": 8, "ws_up": 9, "ws_down": 10}
@@ -105,7 +116,10 @@ def _weights(seed, tid, shape, fan_in, wfmt, device, chunk_elems=1 << 28):
 
 def make_layer(name_or_cfg, device="cpu", **overrides) -> dict:
     """Build one synthetic layer.  Returns a dict of torch tensors on `device` plus "dims"."""
-    cfg = dict(CONFIGS[name_or_cfg]) if isinstance(name_or_cfg, str) else dict(name_or_cfg)
+    if isinstance(name_or_cfg, str):
+        cfg = dict(CONFIGS[name_or_cfg] if name_or_cfg in CONFIGS else PROFILE_CONFIGS[name_or_cfg])
+    else:
+        cfg = dict(name_or_cfg)
     cfg.update(overrides)
     T, H, E, I, k, Is = (cfg[n] for n in ("T", "H", "E", "I", "k", "Is"))
     seed, wfmt = cfg["seed"], cfg["wfmt"]
