@@ -27,16 +27,18 @@ METRIC = "MoE-layer tokens/s; % HBM roofline (decode) / % FP8 tensor peak (prefi
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM bytes per launch of the gate|up GEMM on the decode workload, from one ncu capture
-# (dram__bytes_read.sum + dram__bytes_write.sum), with the hash of the kernel source it was
-# taken on; reported as null once the source changes.
-TRAFFIC = {"decode": {"kernel": "gemm_gateup", "bytes": None, "src_sha": None}}
+# DRAM traffic of the gate|up GEMM per algorithmic byte, from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum) of the decode-shaped profiling workload
+# (profiles/gemm_fp8_profile-decode_full.md), scaled to a decode launch by its algorithmic
+# bytes, with the hash of the kernel source it was taken on; null once the source changes.
+TRAFFIC = {"decode": {"kernel": "gemm_gateup", "ratio": (552.47872e6 + 4.306944e6) / 557973504.0,
+                      "src_sha": "d2072a50228e4526"}}
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default="decode")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -328,9 +330,9 @@ def run_ours(args, ws, rank, local, cfg_name):
     achieved = alg[dom] / (mean_stage[dom] / 1e3) / 1e9
     tr = TRAFFIC.get(cfg_name)
     traffic = None
-    if tr and tr["bytes"] and tr["kernel"] == dom and tr["src_sha"] == src_sha(
+    if tr and tr["kernel"] == dom and tr["src_sha"] == src_sha(
             os.path.join(ROOT, "mixture_experts_ffn_13_b200", "csrc", "gemm_fp8.cu")):
-        traffic = tr["bytes"]
+        traffic = tr["ratio"] * alg[dom]
     layer_gbs = alg["layer"] / (ms_step / 1e3) / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
