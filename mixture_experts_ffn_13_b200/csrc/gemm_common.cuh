@@ -1,0 +1,72 @@
+// gemm_common.cuh -- the work decomposition shared by the grouped GEMMs: a flat list of
+// (group, weight-row tile, token tile) items built from the per-expert row counts.
+#pragma once
+
+#include "moe_internal.h"
+
+namespace moe {
+
+constexpr int kTileM = 128;  // weight rows per tile (the MMA's M side)
+
+struct TileInfo {
+    int seg;    // 0 routed, 1 shared
+    int nt;     // weight-row tile index within the group
+    int row0;   // first activation row (segment-relative)
+    int nrows;  // valid activation rows in this tile (<= BN)
+    int wrow;   // first weight row in the segment's 2-D weight view
+};
+
+// Work item w -> tile.  Routed items come first: group g owns items
+// [ttile[g]*nT, ttile[g+1]*nT), laid out n-tile major so consecutive items reuse the same
+// weight tile across the group's token tiles.  Shared-expert items follow.
+template <int BN>
+__device__ __forceinline__ TileInfo decode_tile(const GemmArgs &a, int w, int tot0)
+{
+    TileInfo t;
+    if (w < tot0) {
+        const int nT = a.seg[0].N / kTileM;
+        int lo = 0, hi = a.E - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (__ldg(a.ttile + mid) * nT <= w)
+                lo = mid;
+            else
+                hi = mid - 1;
+        }
+        const int g = lo;
+        const int t0 = __ldg(a.ttile + g);
+        const int ntt = __ldg(a.ttile + g + 1) - t0;
+        const int local = w - t0 * nT;
+        const int nt = local / ntt;
+        const int tt = local - nt * ntt;
+        const int rbeg = __ldg(a.offsets + g) + tt * BN;
+        const int rend = __ldg(a.offsets + g + 1);
+        t.seg = 0;
+        t.nt = nt;
+        t.row0 = rbeg;
+        t.nrows = min(BN, rend - rbeg);
+        t.wrow = g * a.seg[0].N + nt * kTileM;
+    } else {
+        const int ww = w - tot0;
+        const int ntt = (a.T + BN - 1) / BN;
+        const int nt = ww / ntt;
+        const int tt = ww - nt * ntt;
+        t.seg = 1;
+        t.nt = nt;
+        t.row0 = tt * BN;
+        t.nrows = min(BN, a.T - t.row0);
+        t.wrow = nt * kTileM;
+    }
+    return t;
+}
+
+__device__ __forceinline__ int total_tiles(const GemmArgs &a, int BN, int *tot0)
+{
+    *tot0 = __ldg(a.ttile + a.E) * (a.seg[0].N / kTileM);
+    const int tot1 = a.nseg > 1 ? ((a.T + BN - 1) / BN) * (a.seg[1].N / kTileM) : 0;
+    return *tot0 + tot1;
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
+
+}  // namespace moe

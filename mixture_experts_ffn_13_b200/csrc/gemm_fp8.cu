@@ -25,6 +25,7 @@
 //  * gate|up: two weight tiles per stage share one activation tile; the epilogue computes
 //    h = silu(G) * U in fp32 and stores it.  down: one weight tile; y is stored in fp32.
 #include "moe_internal.h"
+#include "gemm_common.cuh"
 #include "sm100.cuh"
 
 #include <algorithm>
@@ -33,7 +34,6 @@ namespace moe {
 
 namespace {
 
-constexpr int kTileM = 128;  // weight rows per tile (MMA M)
 constexpr int kKC = 128;     // K elements (bytes) per pipeline stage = one 128-byte swizzle row
 constexpr int kStagesPerBlock = kBlockK / kKC;
 constexpr int kSmemBudget = 200 * 1024;
@@ -55,60 +55,6 @@ struct Fp8Cfg {
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M=128 is a multiple of 16 in [16, 256]");
     static_assert(NSLOT >= 1, "TMEM slots");
 };
-
-struct TileInfo {
-    int seg;    // 0 routed, 1 shared
-    int nt;     // weight-row tile index within the group
-    int row0;   // first activation row (segment-relative)
-    int nrows;  // valid activation rows in this tile (<= BN)
-    int wrow;   // first weight row in the segment's 2-D weight view
-};
-
-// Work item w -> tile.  Routed items come first: group g owns items
-// [ttile[g]*nT, ttile[g+1]*nT), laid out n-tile major so consecutive items reuse the same
-// weight tile across the group's token tiles.  Shared-expert items follow.
-template <int BN>
-__device__ __forceinline__ TileInfo decode_tile(const GemmArgs &a, int w, int tot0)
-{
-    TileInfo t;
-    if (w < tot0) {
-        const int nT = a.seg[0].N / kTileM;
-        int lo = 0, hi = a.E - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (__ldg(a.ttile + mid) * nT <= w)
-                lo = mid;
-            else
-                hi = mid - 1;
-        }
-        const int g = lo;
-        const int t0 = __ldg(a.ttile + g);
-        const int ntt = __ldg(a.ttile + g + 1) - t0;
-        const int local = w - t0 * nT;
-        const int nt = local / ntt;
-        const int tt = local - nt * ntt;
-        const int rbeg = __ldg(a.offsets + g) + tt * BN;
-        const int rend = __ldg(a.offsets + g + 1);
-        t.seg = 0;
-        t.nt = nt;
-        t.row0 = rbeg;
-        t.nrows = min(BN, rend - rbeg);
-        t.wrow = g * a.seg[0].N + nt * kTileM;
-    } else {
-        const int ww = w - tot0;
-        const int ntt = (a.T + BN - 1) / BN;
-        const int nt = ww / ntt;
-        const int tt = ww - nt * ntt;
-        t.seg = 1;
-        t.nt = nt;
-        t.row0 = tt * BN;
-        t.nrows = min(BN, a.T - t.row0);
-        t.wrow = nt * kTileM;
-    }
-    return t;
-}
-
-__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
 
 template <int BN, bool GATEUP>
 __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP>::THREADS, 1)

@@ -1,11 +1,316 @@
-// gemm_int4.cu -- steps A4/A5 for 4-bit weights (filled in below the FP8 path).
-#include "moe_internal.h"
+// gemm_int4.cu -- steps A4/A5 for 4-bit expert weights: persistent grouped GEMMs that
+// dequantise int4 weights into shared memory and run bf16 x bf16 -> fp32 tcgen05 MMAs.
+//
+// Page "Flash-Next 在 GPU 上到底在算什麼", section "① 專家 FFN" (and its NVIDIA table): expert
+// weights are stored in 4/8 bits and must be decompressed to 16-bit before the tensor units
+// can use them; on consumer GPUs that decompress-then-FMA runs on the CUDA cores with the
+// tensor cores idle.  Here the decompression feeds the tensor cores instead:
+//  * warp 0 streams raw int4 weight tiles (128 rows x 32 bytes = 64 K-elements per matrix) by
+//    TMA into a deep ring of raw stages (evict-first);
+//  * warps 2-5 (one thread per weight row) turn each raw tile into a bf16 tile in the
+//    128-byte-swizzled K-major layout the MMA reads: flip each nibble's sign bit, place it in
+//    the mantissa of the bf16 value 128 (so the bf16 reads 128 + q + 8), subtract 136 (exact),
+//    multiply by the row's group scale (one rounding to bf16, nearest-even), store 16 bytes per
+//    8 values at the swizzled chunk; the first of these warps also loads the activation tile
+//    (bf16, TMA) of the same stage;
+//  * warp 1 issues tcgen05.mma.kind::f16 (BF16 x BF16 -> F32) from one thread: 4 MMAs of
+//    K = 16 per stage per matrix, all of K into one TMEM accumulator (no promotion: the scales
+//    are already in the weights);
+//  * warps 6-9 read the finished accumulators: gate|up writes h = silu(G) * U rounded to bf16
+//    (the 4-bit layer keeps activations in bf16), down writes y in fp32.
+// Two TMEM accumulator sets alternate so the epilogue of one tile overlaps the next tile.
+#include "gemm_common.cuh"
+#include "sm100.cuh"
+
+#include <cuda_bf16.h>
 
 namespace moe {
 
-cudaError_t launch_gemm_int4(bool, int, const GemmMaps &, const GemmArgs &, int, cudaStream_t)
+namespace {
+
+constexpr int kKE = 64;                // K elements per stage (one 128-byte bf16 swizzle row)
+constexpr int kRawRow = kKE / 2;       // raw bytes per weight row per stage
+constexpr int kConvWarps = 4;
+constexpr int kEpiWarps = 4;
+constexpr int kThreads = 32 * (2 + kConvWarps + kEpiWarps);
+
+template <int BN, bool GATEUP>
+struct I4Cfg {
+    static constexpr int NA = GATEUP ? 2 : 1;
+    static constexpr int RAW_BYTES = kTileM * kRawRow;      // 4 KB per matrix
+    static constexpr int A_BYTES = kTileM * kKE * 2;        // 16 KB per matrix
+    static constexpr int B_BYTES = BN * kKE * 2;
+    static constexpr int NR = 8;                            // raw stages
+    static constexpr int MSTAGE = NA * A_BYTES + B_BYTES;
+    static constexpr int NM = GATEUP ? 3 : 4;               // MMA stages
+    static constexpr int ACC_COLS = NA * BN;
+    static constexpr int TMEM_COLS = 2 * ACC_COLS <= 32 ? 32 : (2 * ACC_COLS <= 64 ? 64 : (2 * ACC_COLS <= 128 ? 128 : (2 * ACC_COLS <= 256 ? 256 : 512)));
+    static constexpr int BAR_BYTES = 8 * (2 * NR + 2 * NM + 4) + 16;
+    static constexpr int SMEM = 1024 + NM * MSTAGE + NR * NA * RAW_BYTES + BAR_BYTES;
+    static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "1024-byte aligned tiles");
+    static_assert(SMEM <= 227 * 1024, "shared memory");
+};
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
 {
-    return cudaErrorNotSupported;
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t bf2_bits(__nv_bfloat162 v) { return *reinterpret_cast<uint32_t *>(&v); }
+
+__device__ __forceinline__ __nv_bfloat162 bits_bf2(uint32_t u) { return *reinterpret_cast<__nv_bfloat162 *>(&u); }
+
+// 8 two's-complement nibbles (element 2i in the low nibble of byte i) -> 8 bf16 values
+// bf16(q * s), returned as 4 words of bf16 pairs in element order.
+__device__ __forceinline__ uint4 dequant8(uint32_t w, __nv_bfloat162 s2)
+{
+    const uint32_t t = w ^ 0x88888888u;      // q + 8 in every nibble (0..15)
+    const uint32_t lo = t & 0x0F0F0F0Fu;     // elements 0, 2, 4, 6 (one per byte)
+    const uint32_t hi = (t >> 4) & 0x0F0F0F0Fu;  // elements 1, 3, 5, 7
+    const __nv_bfloat162 off = bits_bf2(0x43084308u);  // (136, 136)
+    uint32_t r[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        // bytes: lo.byte_i -> result byte 0, hi.byte_i -> result byte 2
+        const uint32_t p = prmt(lo, hi, 0x0400u | (0x0101u * i));
+        const uint32_t v = (p & 0x00FF00FFu) | 0x43004300u;  // bf16 pair (128 + q + 8)
+        r[i] = bf2_bits(__hmul2(__hsub2(bits_bf2(v), off), s2));
+    }
+    return make_uint4(r[0], r[1], r[2], r[3]);
+}
+
+template <int BN, bool GATEUP>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_int4_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmArgs args)
+{
+    using C = I4Cfg<BN, GATEUP>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *mst = smem;                                   // NM MMA stages [A0 | A1 | B]
+    uint8_t *raw = smem + C::NM * C::MSTAGE;               // NR raw stages [raw0 | raw1]
+    uint64_t *rfull = reinterpret_cast<uint64_t *>(raw + C::NR * C::NA * C::RAW_BYTES);
+    uint64_t *rempty = rfull + C::NR;
+    uint64_t *mfull = rempty + C::NR;
+    uint64_t *mempty = mfull + C::NM;
+    uint64_t *accf = mempty + C::NM;   // 2
+    uint64_t *acce = accf + 2;         // 2
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(acce + 2);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::NR; ++s) {
+            mbar_init(&rfull[s], 1);
+            mbar_init(&rempty[s], kConvWarps);
+        }
+        for (int s = 0; s < C::NM; ++s) {
+            mbar_init(&mfull[s], kConvWarps + 1);
+            mbar_init(&mempty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&accf[s], 1);
+            mbar_init(&acce[s], kEpiWarps);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    int tot0;
+    const int total = total_tiles(args, BN, &tot0);
+    int *status = args.status;
+    const uint64_t tmo = args.timeout_ns;
+
+    if (warp == 0) {
+        // ------------------------------ raw weight producer -----------------------
+        if (lane == 0) {
+            const uint64_t pol_w = l2_policy_evict_first();
+            uint32_t it = 0;
+            for (int w = blockIdx.x; w < total; w += gridDim.x) {
+                const TileInfo tl = decode_tile<BN>(args, w, tot0);
+                const int nkc = args.seg[tl.seg].K / kKE;
+                for (int kc = 0; kc < nkc; ++kc, ++it) {
+                    const int s = it % C::NR;
+                    const uint32_t ph = (it / C::NR) & 1;
+                    if (!mbar_wait(&rempty[s], ph ^ 1, abort_flag, status, tmo)) goto done;
+                    uint8_t *rs = raw + s * C::NA * C::RAW_BYTES;
+                    mbar_arrive_expect_tx(&rfull[s], C::NA * C::RAW_BYTES);
+                    tma_load_2d_hint(rs, &maps.a0[tl.seg], &rfull[s], kc * kRawRow, tl.wrow, pol_w);
+                    if (GATEUP)
+                        tma_load_2d_hint(rs + C::RAW_BYTES, &maps.a1[tl.seg], &rfull[s], kc * kRawRow, tl.wrow, pol_w);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------ MMA issuer --------------------------------
+        if (lane == 0) {
+            constexpr uint32_t kIdesc = instr_desc(kTileM, BN, 1, 1);
+            uint32_t it = 0, ti = 0;
+            for (int w = blockIdx.x; w < total; w += gridDim.x, ++ti) {
+                const TileInfo tl = decode_tile<BN>(args, w, tot0);
+                const int nkc = args.seg[tl.seg].K / kKE;
+                const int slot = ti & 1;
+                if (!mbar_wait(&acce[slot], ((ti >> 1) & 1) ^ 1, abort_flag, status, tmo)) goto done;
+                tc_fence_after();
+                const uint32_t d0 = tmem_base + slot * C::ACC_COLS;
+                const uint32_t d1 = d0 + BN;
+                for (int kc = 0; kc < nkc; ++kc, ++it) {
+                    const int s = it % C::NM;
+                    if (!mbar_wait(&mfull[s], (it / C::NM) & 1, abort_flag, status, tmo)) goto done;
+                    tc_fence_after();
+                    uint8_t *st = mst + s * C::MSTAGE;
+                    const uint64_t da0 = smem_desc_sw128(st);
+                    const uint64_t da1 = smem_desc_sw128(st + C::A_BYTES);
+                    const uint64_t db = smem_desc_sw128(st + C::NA * C::A_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < kKE / 16; ++kk) {
+                        const uint32_t acc = (kc > 0 || kk > 0) ? 1u : 0u;
+                        mma_bf16(d0, da0 + 2 * kk, db + 2 * kk, kIdesc, acc);
+                        if (GATEUP) mma_bf16(d1, da1 + 2 * kk, db + 2 * kk, kIdesc, acc);
+                    }
+                    mma_commit(&mempty[s]);
+                }
+                mma_commit(&accf[slot]);
+            }
+        }
+    } else if (warp < 2 + kConvWarps) {
+        // ------------------------------ dequantisers ------------------------------
+        const int cw = warp - 2;
+        const int r = cw * 32 + lane;  // weight row of the tile handled by this thread
+        uint32_t it = 0;
+        for (int w = blockIdx.x; w < total; w += gridDim.x) {
+            const TileInfo tl = decode_tile<BN>(args, w, tot0);
+            const GemmSeg &sg = args.seg[tl.seg];
+            const int nkc = sg.K / kKE;
+            const int ng = sg.K / kGroupK;
+            const __nv_bfloat16 *s0 = static_cast<const __nv_bfloat16 *>(sg.sw0) + (size_t)(tl.wrow + r) * ng;
+            const __nv_bfloat16 *s1 =
+                GATEUP ? static_cast<const __nv_bfloat16 *>(sg.sw1) + (size_t)(tl.wrow + r) * ng : nullptr;
+            for (int kc = 0; kc < nkc; ++kc, ++it) {
+                const int rs_i = it % C::NR;
+                const int ms_i = it % C::NM;
+                const int grp = (kc * kKE) / kGroupK;
+                const __nv_bfloat16 sc0 = s0[grp];
+                const __nv_bfloat16 sc1 = GATEUP ? s1[grp] : sc0;
+                bool ok = mbar_wait(&mempty[ms_i], ((it / C::NM) & 1) ^ 1, abort_flag, status, tmo);
+                if (!__all_sync(0xffffffffu, ok)) goto done;
+                uint8_t *st = mst + ms_i * C::MSTAGE;
+                if (cw == 0 && lane == 0) {
+                    mbar_arrive_expect_tx(&mfull[ms_i], C::B_BYTES);
+                    tma_load_2d_hint(st + C::NA * C::A_BYTES, &maps.b[tl.seg], &mfull[ms_i], kc * kKE, tl.row0,
+                                     l2_policy_evict_last());
+                }
+                ok = mbar_wait(&rfull[rs_i], (it / C::NR) & 1, abort_flag, status, tmo);
+                if (!__all_sync(0xffffffffu, ok)) goto done;
+                const uint8_t *rs = raw + rs_i * C::NA * C::RAW_BYTES;
+#pragma unroll
+                for (int m = 0; m < C::NA; ++m) {
+                    const uint4 *src = reinterpret_cast<const uint4 *>(rs + m * C::RAW_BYTES + r * kRawRow);
+                    const uint4 q0 = src[0], q1 = src[1];
+                    const __nv_bfloat16 sc = m == 0 ? sc0 : sc1;
+                    const __nv_bfloat162 s2 = __halves2bfloat162(sc, sc);
+                    uint8_t *dst = st + m * C::A_BYTES + r * 128;
+                    const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        *reinterpret_cast<uint4 *>(dst + ((j ^ (r & 7)) << 4)) = dequant8(words[j], s2);
+                }
+                // make the generic-proxy shared-memory writes visible to the tensor core
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&rempty[rs_i]);
+                    mbar_arrive(&mfull[ms_i]);
+                }
+            }
+        }
+    } else {
+        // ------------------------------ epilogue ----------------------------------
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        uint32_t ti = 0;
+        for (int w = blockIdx.x; w < total; w += gridDim.x, ++ti) {
+            const TileInfo tl = decode_tile<BN>(args, w, tot0);
+            const GemmSeg &sg = args.seg[tl.seg];
+            const int slot = ti & 1;
+            const bool ok = mbar_wait(&accf[slot], (ti >> 1) & 1, abort_flag, status, tmo);
+            if (!__all_sync(0xffffffffu, ok)) goto done;
+            tc_fence_after();
+            const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + slot * C::ACC_COLS;
+            const int n = tl.nt * kTileM + r;
+#pragma unroll
+            for (int c0 = 0; c0 < BN; c0 += 16) {
+                float v[16], u[16];
+                tmem_ld16(tb + c0, v);
+                if constexpr (GATEUP) {
+                    tmem_ld16(tb + BN + c0, u);
+                    tmem_wait_ld2(v, u);
+                } else {
+                    tmem_wait_ld(v);
+                }
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    if (c0 + c < tl.nrows) {
+                        const size_t o = (size_t)(tl.row0 + c0 + c) * sg.N + n;
+                        if constexpr (GATEUP)
+                            static_cast<__nv_bfloat16 *>(sg.out)[o] = __float2bfloat16_rn(silu_mul(v[c], u[c]));
+                        else
+                            static_cast<float *>(sg.out)[o] = v[c];
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acce[slot]);
+        }
+    }
+done:
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+template <int BN, bool GATEUP>
+cudaError_t launch_t(const GemmMaps &maps, const GemmArgs &args, int num_sms, cudaStream_t s)
+{
+    using C = I4Cfg<BN, GATEUP>;
+    auto kern = gemm_int4_kernel<BN, GATEUP>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    kern<<<num_sms, kThreads, C::SMEM, s>>>(maps, args);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_int4(bool gateup, int bn, const GemmMaps &maps, const GemmArgs &args, int num_sms,
+                             cudaStream_t s)
+{
+    if (gateup) {
+        switch (bn) {
+            case 32: return launch_t<32, true>(maps, args, num_sms, s);
+            case 64: return launch_t<64, true>(maps, args, num_sms, s);
+            default: return cudaErrorInvalidValue;
+        }
+    }
+    switch (bn) {
+        case 32: return launch_t<32, false>(maps, args, num_sms, s);
+        case 64: return launch_t<64, false>(maps, args, num_sms, s);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace moe

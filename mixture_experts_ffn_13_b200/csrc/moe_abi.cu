@@ -292,6 +292,88 @@ int moe_route(moe_plan_t *p, int32_t T, const float *logits, int32_t *topk_idx, 
     return e == cudaSuccess ? MOE_OK : fail_cuda(p, e);
 }
 
+// The 4-bit layer: route, permute, gather bf16 rows, int4 gate|up (h in bf16), int4 down,
+// combine.  Stage events: 0 route | 1 permute | 2 gather | 3 gate|up | 4 (no h quantiser) |
+// 5 down | 6 combine | 7.
+static int forward_int4(moe_plan_t *p, int T, const uint16_t *x, const float *logits, const moe_weights *w,
+                        uint16_t *out, uint8_t *ws, cudaStream_t s)
+{
+    const moe_dims &d = p->d;
+    auto mark = [&](int i) {
+        if (p->prof) cudaEventRecord(p->ev[i], s);
+    };
+    const Layout L = make_layout(d);
+    const RouteBufs b = route_bufs(L, ws);
+    const int H = d.H, I = d.I, Is = d.I_shared, k = d.k, E = d.E;
+    const bool shared = Is > 0;
+    const int A = T * k;
+    const int bn = pick_bn(T, k, E);
+    mark(0);
+    cudaError_t e = launch_route(logits, T, E, k, b.topk_idx, b.topk_w, s);
+    mark(1);
+    if (e == cudaSuccess) e = launch_permute(b, T, E, k, bn, bn, s);
+    mark(2);
+    if (e != cudaSuccess) return fail_cuda(p, e);
+    uint16_t *xp = reinterpret_cast<uint16_t *>(ws + L.act);
+    uint16_t *xp_sh = shared ? xp + (size_t)A * H : nullptr;
+    e = launch_gather_x_bf16(x, T, H, k, b.pos, xp, xp_sh, s);
+    mark(3);
+    if (e != cudaSuccess) return fail_cuda(p, e);
+
+    uint16_t *h = reinterpret_cast<uint16_t *>(ws + L.h);
+    uint16_t *h_sh = reinterpret_cast<uint16_t *>(ws + L.h_sh);
+    float *y = reinterpret_cast<float *>(ws + L.y);
+    float *y_sh = shared ? y + (size_t)A * H : nullptr;
+    const CUtensorMapDataType U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8, BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+
+    GemmMaps mg{};
+    GemmArgs ag{};
+    ag.nseg = shared ? 2 : 1;
+    ag.E = E;
+    ag.T = T;
+    ag.offsets = b.offsets;
+    ag.ttile = b.ttile_a;
+    ag.status = p->d_status;
+    ag.timeout_ns = kDefaultTimeoutNs;
+    ag.seg[0] = GemmSeg{I, H, A, w->s_gate, w->s_up, nullptr, h};
+    int rc = encode_map_2d(&mg.a0[0], w->w_gate, U8, 1, H / 2, (uint64_t)E * I, 32, 128, false);
+    rc |= encode_map_2d(&mg.a1[0], w->w_up, U8, 1, H / 2, (uint64_t)E * I, 32, 128, false);
+    rc |= encode_map_2d(&mg.b[0], xp, BF, 2, H, A, 64, bn, true);
+    if (shared) {
+        ag.seg[1] = GemmSeg{Is, H, T, w->ss_gate, w->ss_up, nullptr, h_sh};
+        rc |= encode_map_2d(&mg.a0[1], w->ws_gate, U8, 1, H / 2, Is, 32, 128, false);
+        rc |= encode_map_2d(&mg.a1[1], w->ws_up, U8, 1, H / 2, Is, 32, 128, false);
+        rc |= encode_map_2d(&mg.b[1], xp_sh, BF, 2, H, T, 64, bn, true);
+    }
+    if (rc) return MOE_ERR_CUDA;
+    e = launch_gemm_int4(true, bn, mg, ag, p->num_sms, s);
+    mark(4);
+    mark(5);
+    if (e != cudaSuccess) return fail_cuda(p, e);
+
+    GemmMaps md{};
+    GemmArgs ad = ag;
+    ad.ttile = b.ttile_b;
+    ad.seg[0] = GemmSeg{H, I, A, w->s_down, nullptr, nullptr, y};
+    rc = encode_map_2d(&md.a0[0], w->w_down, U8, 1, I / 2, (uint64_t)E * H, 32, 128, false);
+    rc |= encode_map_2d(&md.b[0], h, BF, 2, I, A, 64, bn, true);
+    if (shared) {
+        ad.seg[1] = GemmSeg{H, Is, T, w->ss_down, nullptr, nullptr, y_sh};
+        rc |= encode_map_2d(&md.a0[1], w->ws_down, U8, 1, Is / 2, H, 32, 128, false);
+        rc |= encode_map_2d(&md.b[1], h_sh, BF, 2, Is, T, 64, bn, true);
+    }
+    if (rc) return MOE_ERR_CUDA;
+    e = launch_gemm_int4(false, bn, md, ad, p->num_sms, s);
+    mark(6);
+    if (e != cudaSuccess) return fail_cuda(p, e);
+    e = launch_combine(y, y_sh, b.pos, b.topk_w, T, H, k, out, s);
+    mark(7);
+    if (e != cudaSuccess) return fail_cuda(p, e);
+    p->launches = 1 + 3 + 1 + 1 + 1 + 1;
+    p->prof_recorded = p->prof;
+    return MOE_OK;
+}
+
 int moe_forward(moe_plan_t *p, int32_t T, const uint16_t *x, const float *logits, const moe_weights *w,
                 uint16_t *out, void *workspace, size_t ws_bytes, moe_stream_t stream)
 {
@@ -312,12 +394,12 @@ int moe_forward(moe_plan_t *p, int32_t T, const uint16_t *x, const float *logits
     p->launches = 0;
     p->prof_recorded = false;
     if (T == 0) return MOE_OK;
-    if (d.wfmt != MOE_W_FP8_SC512) return MOE_ERR_UNSUPPORTED;
 
     cudaStream_t s = (cudaStream_t)stream;
     auto mark = [&](int i) {
         if (p->prof) cudaEventRecord(p->ev[i], s);
     };
+    if (d.wfmt == MOE_W_INT4_G128) return forward_int4(p, T, x, logits, w, out, static_cast<uint8_t *>(workspace), s);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     const Layout L = make_layout(d);
     const RouteBufs b = route_bufs(L, ws);

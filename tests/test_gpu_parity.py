@@ -139,6 +139,28 @@ def test_layer_fp8_variable_T_within_plan():
     assert out0.shape == (0, 512)
 
 
+SMALL_INT4 = [
+    dict(T=16, H=256, E=4, I=128, k=2, Is=0, seed=41, bias=None),
+    dict(T=37, H=512, E=8, I=384, k=3, Is=256, seed=42, bias="normal"),   # shared expert, ragged groups
+    dict(T=200, H=1024, E=4, I=256, k=2, Is=0, seed=43, bias="zipf"),     # 64-row token tiles, several per group
+    dict(T=3, H=128, E=16, I=128, k=4, Is=128, seed=44, bias=None),       # mostly empty experts
+]
+
+
+@pytest.mark.parametrize("cfg", SMALL_INT4, ids=lambda c: f"T{c['T']}-H{c['H']}-E{c['E']}-I{c['I']}-k{c['k']}-Is{c['Is']}")
+def test_layer_int4_small(cfg):
+    cfg = dict(cfg, wfmt="int4")
+    layer = moe_synth.make_layer(cfg, device="cuda")
+    m = moe.MoELayer(layer)
+    out = m(layer["x"], layer["logits"])
+    assert moe.moe_get_status(m.plan) == 0
+    want, _, amb = oracle.layer(moe_synth.to_numpy(layer), ambiguity=True)
+    check_out(out, want, "int4 layer", amb)
+    out2 = m(layer["x"], layer["logits"])
+    torch.cuda.synchronize()
+    assert torch.equal(out, out2)
+
+
 def _sampled_parity(name, n_sample=12):
     cfg = moe_synth.CONFIGS[name]
     layer = moe_synth.make_layer(name, device="cuda")
@@ -156,6 +178,6 @@ def _sampled_parity(name, n_sample=12):
     check_route(m.plan, m.workspace, layer["logits"], cfg["k"])
 
 
-@pytest.mark.parametrize("name", ["tiny", "decode", "prefill", "skewed"])
-def test_layer_fp8_configs_sampled(name):
+@pytest.mark.parametrize("name", ["tiny", "decode", "prefill", "skewed", "int4"])
+def test_layer_configs_sampled(name):
     _sampled_parity(name)
