@@ -4,21 +4,25 @@
 // Page "Flash-Next 在 GPU 上到底在算什麼", section "① 專家 FFN" (and its NVIDIA table): expert
 // weights are stored in 4/8 bits and must be decompressed to 16-bit before the tensor units
 // can use them; on consumer GPUs that decompress-then-FMA runs on the CUDA cores with the
-// tensor cores idle.  Here the decompression feeds the tensor cores instead:
+// tensor cores idle.  Here the decompression feeds the tensor cores instead, and keeps the
+// weights exact:
 //  * warp 0 streams raw int4 weight tiles (128 rows x 32 bytes = 64 K-elements per matrix) by
 //    TMA into a deep ring of raw stages (evict-first);
-//  * warps 2-5 (one thread per weight row) turn each raw tile into a bf16 tile in the
-//    128-byte-swizzled K-major layout the MMA reads: flip each nibble's sign bit, place it in
-//    the mantissa of the bf16 value 128 (so the bf16 reads 128 + q + 8), subtract 136 (exact),
-//    multiply by the row's group scale (one rounding to bf16, nearest-even), store 16 bytes per
-//    8 values at the swizzled chunk; the first of these warps also loads the activation tile
-//    (bf16, TMA) of the same stage;
+//  * warps 2-5 (one thread per weight row) turn each raw tile into the integers q as bf16
+//    (exact: |q| <= 8) in the 128-byte-swizzled K-major layout the MMA reads: flip each
+//    nibble's sign bit, place it in the mantissa of the bf16 value 128 (so it reads
+//    128 + q + 8), subtract 136, store 16 bytes per 8 values at the swizzled chunk; the first
+//    of these warps also loads the stage's activation tile (bf16, TMA);
 //  * warp 1 issues tcgen05.mma.kind::f16 (BF16 x BF16 -> F32) from one thread: 4 MMAs of
-//    K = 16 per stage per matrix, all of K into one TMEM accumulator (no promotion: the scales
-//    are already in the weights);
-//  * warps 6-9 read the finished accumulators: gate|up writes h = silu(G) * U rounded to bf16
-//    (the 4-bit layer keeps activations in bf16), down writes y in fp32.
-// Two TMEM accumulator sets alternate so the epilogue of one tile overlaps the next tile.
+//    K = 16 per stage per matrix; each 128-element K group (2 stages) accumulates into its own
+//    TMEM slot, because the weight scale changes per (row, group);
+//  * warps 6-9 promote each finished group, acc += D_g * s[row, g] in fp32 registers, and at
+//    the end of the tile write gate|up h = silu(G) * U rounded to bf16 (the 4-bit layer keeps
+//    activations in bf16) or down y in fp32.
+// Multiplying the exact integers on the tensor cores and applying the bf16 scale to fp32
+// partial sums reproduces sum_i x_i * q_i * s_i up to fp32 rounding; rounding q * s to bf16
+// before the MMA would not (that costs ~2^-9 relative per weight and fails the layer's
+// tolerance at these sizes).
 #include "gemm_common.cuh"
 #include "sm100.cuh"
 
@@ -43,9 +47,10 @@ struct I4Cfg {
     static constexpr int NR = 8;                            // raw stages
     static constexpr int MSTAGE = NA * A_BYTES + B_BYTES;
     static constexpr int NM = GATEUP ? 3 : 4;               // MMA stages
-    static constexpr int ACC_COLS = NA * BN;
-    static constexpr int TMEM_COLS = 2 * ACC_COLS <= 32 ? 32 : (2 * ACC_COLS <= 64 ? 64 : (2 * ACC_COLS <= 128 ? 128 : (2 * ACC_COLS <= 256 ? 256 : 512)));
-    static constexpr int BAR_BYTES = 8 * (2 * NR + 2 * NM + 4) + 16;
+    static constexpr int SLOT_COLS = NA * BN;               // one 128-element K group
+    static constexpr int NSLOT = 512 / SLOT_COLS;
+    static constexpr int STAGES_PER_GROUP = kGroupK / kKE;  // 2
+    static constexpr int BAR_BYTES = 8 * (2 * NR + 2 * NM + 2 * NSLOT) + 16;
     static constexpr int SMEM = 1024 + NM * MSTAGE + NR * NA * RAW_BYTES + BAR_BYTES;
     static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "1024-byte aligned tiles");
     static_assert(SMEM <= 227 * 1024, "shared memory");
@@ -62,12 +67,12 @@ __device__ __forceinline__ uint32_t bf2_bits(__nv_bfloat162 v) { return *reinter
 
 __device__ __forceinline__ __nv_bfloat162 bits_bf2(uint32_t u) { return *reinterpret_cast<__nv_bfloat162 *>(&u); }
 
-// 8 two's-complement nibbles (element 2i in the low nibble of byte i) -> 8 bf16 values
-// bf16(q * s), returned as 4 words of bf16 pairs in element order.
-__device__ __forceinline__ uint4 dequant8(uint32_t w, __nv_bfloat162 s2)
+// 8 two's-complement nibbles (element 2i in the low nibble of byte i) -> the 8 integers as
+// bf16 (exact), returned as 4 words of bf16 pairs in element order.
+__device__ __forceinline__ uint4 unpack8(uint32_t w)
 {
-    const uint32_t t = w ^ 0x88888888u;      // q + 8 in every nibble (0..15)
-    const uint32_t lo = t & 0x0F0F0F0Fu;     // elements 0, 2, 4, 6 (one per byte)
+    const uint32_t t = w ^ 0x88888888u;          // q + 8 in every nibble (0..15)
+    const uint32_t lo = t & 0x0F0F0F0Fu;         // elements 0, 2, 4, 6 (one per byte)
     const uint32_t hi = (t >> 4) & 0x0F0F0F0Fu;  // elements 1, 3, 5, 7
     const __nv_bfloat162 off = bits_bf2(0x43084308u);  // (136, 136)
     uint32_t r[4];
@@ -76,7 +81,7 @@ __device__ __forceinline__ uint4 dequant8(uint32_t w, __nv_bfloat162 s2)
         // bytes: lo.byte_i -> result byte 0, hi.byte_i -> result byte 2
         const uint32_t p = prmt(lo, hi, 0x0400u | (0x0101u * i));
         const uint32_t v = (p & 0x00FF00FFu) | 0x43004300u;  // bf16 pair (128 + q + 8)
-        r[i] = bf2_bits(__hmul2(__hsub2(bits_bf2(v), off), s2));
+        r[i] = bf2_bits(__hsub2(bits_bf2(v), off));
     }
     return make_uint4(r[0], r[1], r[2], r[3]);
 }
@@ -94,9 +99,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *rempty = rfull + C::NR;
     uint64_t *mfull = rempty + C::NR;
     uint64_t *mempty = mfull + C::NM;
-    uint64_t *accf = mempty + C::NM;   // 2
-    uint64_t *acce = accf + 2;         // 2
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(acce + 2);
+    uint64_t *accf = mempty + C::NM;
+    uint64_t *acce = accf + C::NSLOT;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(acce + C::NSLOT);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -109,7 +114,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&mfull[s], kConvWarps + 1);
             mbar_init(&mempty[s], 1);
         }
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < C::NSLOT; ++s) {
             mbar_init(&accf[s], 1);
             mbar_init(&acce[s], kEpiWarps);
         }
@@ -117,7 +122,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(tmem_holder, C::TMEM_COLS);
+        tmem_alloc(tmem_holder, 512);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -154,32 +159,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------ MMA issuer --------------------------------
         if (lane == 0) {
             constexpr uint32_t kIdesc = instr_desc(kTileM, BN, 1, 1);
-            uint32_t it = 0, ti = 0;
-            for (int w = blockIdx.x; w < total; w += gridDim.x, ++ti) {
+            uint32_t it = 0, ai = 0;
+            for (int w = blockIdx.x; w < total; w += gridDim.x) {
                 const TileInfo tl = decode_tile<BN>(args, w, tot0);
-                const int nkc = args.seg[tl.seg].K / kKE;
-                const int slot = ti & 1;
-                if (!mbar_wait(&acce[slot], ((ti >> 1) & 1) ^ 1, abort_flag, status, tmo)) goto done;
-                tc_fence_after();
-                const uint32_t d0 = tmem_base + slot * C::ACC_COLS;
-                const uint32_t d1 = d0 + BN;
-                for (int kc = 0; kc < nkc; ++kc, ++it) {
-                    const int s = it % C::NM;
-                    if (!mbar_wait(&mfull[s], (it / C::NM) & 1, abort_flag, status, tmo)) goto done;
+                const int ngrp = args.seg[tl.seg].K / kGroupK;
+                for (int g = 0; g < ngrp; ++g, ++ai) {
+                    const int slot = ai % C::NSLOT;
+                    if (!mbar_wait(&acce[slot], ((ai / C::NSLOT) & 1) ^ 1, abort_flag, status, tmo)) goto done;
                     tc_fence_after();
-                    uint8_t *st = mst + s * C::MSTAGE;
-                    const uint64_t da0 = smem_desc_sw128(st);
-                    const uint64_t da1 = smem_desc_sw128(st + C::A_BYTES);
-                    const uint64_t db = smem_desc_sw128(st + C::NA * C::A_BYTES);
+                    const uint32_t d0 = tmem_base + slot * C::SLOT_COLS;
+                    const uint32_t d1 = d0 + BN;
+                    for (int sk = 0; sk < C::STAGES_PER_GROUP; ++sk, ++it) {
+                        const int s = it % C::NM;
+                        if (!mbar_wait(&mfull[s], (it / C::NM) & 1, abort_flag, status, tmo)) goto done;
+                        tc_fence_after();
+                        uint8_t *st = mst + s * C::MSTAGE;
+                        const uint64_t da0 = smem_desc_sw128(st);
+                        const uint64_t da1 = smem_desc_sw128(st + C::A_BYTES);
+                        const uint64_t db = smem_desc_sw128(st + C::NA * C::A_BYTES);
 #pragma unroll
-                    for (int kk = 0; kk < kKE / 16; ++kk) {
-                        const uint32_t acc = (kc > 0 || kk > 0) ? 1u : 0u;
-                        mma_bf16(d0, da0 + 2 * kk, db + 2 * kk, kIdesc, acc);
-                        if (GATEUP) mma_bf16(d1, da1 + 2 * kk, db + 2 * kk, kIdesc, acc);
+                        for (int kk = 0; kk < kKE / 16; ++kk) {
+                            const uint32_t acc = (sk > 0 || kk > 0) ? 1u : 0u;
+                            mma_bf16(d0, da0 + 2 * kk, db + 2 * kk, kIdesc, acc);
+                            if (GATEUP) mma_bf16(d1, da1 + 2 * kk, db + 2 * kk, kIdesc, acc);
+                        }
+                        mma_commit(&mempty[s]);
                     }
-                    mma_commit(&mempty[s]);
+                    mma_commit(&accf[slot]);
                 }
-                mma_commit(&accf[slot]);
             }
         }
     } else if (warp < 2 + kConvWarps) {
@@ -191,16 +198,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const TileInfo tl = decode_tile<BN>(args, w, tot0);
             const GemmSeg &sg = args.seg[tl.seg];
             const int nkc = sg.K / kKE;
-            const int ng = sg.K / kGroupK;
-            const __nv_bfloat16 *s0 = static_cast<const __nv_bfloat16 *>(sg.sw0) + (size_t)(tl.wrow + r) * ng;
-            const __nv_bfloat16 *s1 =
-                GATEUP ? static_cast<const __nv_bfloat16 *>(sg.sw1) + (size_t)(tl.wrow + r) * ng : nullptr;
             for (int kc = 0; kc < nkc; ++kc, ++it) {
                 const int rs_i = it % C::NR;
                 const int ms_i = it % C::NM;
-                const int grp = (kc * kKE) / kGroupK;
-                const __nv_bfloat16 sc0 = s0[grp];
-                const __nv_bfloat16 sc1 = GATEUP ? s1[grp] : sc0;
                 bool ok = mbar_wait(&mempty[ms_i], ((it / C::NM) & 1) ^ 1, abort_flag, status, tmo);
                 if (!__all_sync(0xffffffffu, ok)) goto done;
                 uint8_t *st = mst + ms_i * C::MSTAGE;
@@ -216,13 +216,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int m = 0; m < C::NA; ++m) {
                     const uint4 *src = reinterpret_cast<const uint4 *>(rs + m * C::RAW_BYTES + r * kRawRow);
                     const uint4 q0 = src[0], q1 = src[1];
-                    const __nv_bfloat16 sc = m == 0 ? sc0 : sc1;
-                    const __nv_bfloat162 s2 = __halves2bfloat162(sc, sc);
                     uint8_t *dst = st + m * C::A_BYTES + r * 128;
                     const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
                     for (int j = 0; j < 8; ++j)
-                        *reinterpret_cast<uint4 *>(dst + ((j ^ (r & 7)) << 4)) = dequant8(words[j], s2);
+                        *reinterpret_cast<uint4 *>(dst + ((j ^ (r & 7)) << 4)) = unpack8(words[j]);
                 }
                 // make the generic-proxy shared-memory writes visible to the tensor core
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -237,40 +235,60 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------ epilogue ----------------------------------
         const int q = warp & 3;
         const int r = q * 32 + lane;
-        uint32_t ti = 0;
-        for (int w = blockIdx.x; w < total; w += gridDim.x, ++ti) {
+        uint32_t ai = 0;
+        for (int w = blockIdx.x; w < total; w += gridDim.x) {
             const TileInfo tl = decode_tile<BN>(args, w, tot0);
             const GemmSeg &sg = args.seg[tl.seg];
-            const int slot = ti & 1;
-            const bool ok = mbar_wait(&accf[slot], (ti >> 1) & 1, abort_flag, status, tmo);
-            if (!__all_sync(0xffffffffu, ok)) goto done;
-            tc_fence_after();
-            const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + slot * C::ACC_COLS;
-            const int n = tl.nt * kTileM + r;
+            const int ngrp = sg.K / kGroupK;
+            const __nv_bfloat16 *sw0 = static_cast<const __nv_bfloat16 *>(sg.sw0) + (size_t)(tl.wrow + r) * ngrp;
+            const __nv_bfloat16 *sw1 =
+                GATEUP ? static_cast<const __nv_bfloat16 *>(sg.sw1) + (size_t)(tl.wrow + r) * ngrp : nullptr;
+            float acc0[BN], acc1[GATEUP ? BN : 1];
 #pragma unroll
-            for (int c0 = 0; c0 < BN; c0 += 16) {
-                float v[16], u[16];
-                tmem_ld16(tb + c0, v);
-                if constexpr (GATEUP) {
-                    tmem_ld16(tb + BN + c0, u);
-                    tmem_wait_ld2(v, u);
-                } else {
-                    tmem_wait_ld(v);
-                }
+            for (int c = 0; c < BN; ++c) acc0[c] = 0.0f;
+            if constexpr (GATEUP) {
 #pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    if (c0 + c < tl.nrows) {
-                        const size_t o = (size_t)(tl.row0 + c0 + c) * sg.N + n;
-                        if constexpr (GATEUP)
-                            static_cast<__nv_bfloat16 *>(sg.out)[o] = __float2bfloat16_rn(silu_mul(v[c], u[c]));
-                        else
-                            static_cast<float *>(sg.out)[o] = v[c];
+                for (int c = 0; c < BN; ++c) acc1[c] = 0.0f;
+            }
+            for (int g = 0; g < ngrp; ++g, ++ai) {
+                const int slot = ai % C::NSLOT;
+                const float s0 = __bfloat162float(sw0[g]);
+                const float s1 = GATEUP ? __bfloat162float(sw1[g]) : 0.0f;
+                const bool ok = mbar_wait(&accf[slot], (ai / C::NSLOT) & 1, abort_flag, status, tmo);
+                if (!__all_sync(0xffffffffu, ok)) goto done;
+                tc_fence_after();
+                const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + slot * C::SLOT_COLS;
+#pragma unroll
+                for (int c0 = 0; c0 < BN; c0 += 16) {
+                    float v[16], u[16];
+                    tmem_ld16(tb + c0, v);
+                    if constexpr (GATEUP) {
+                        tmem_ld16(tb + BN + c0, u);
+                        tmem_wait_ld2(v, u);
+                    } else {
+                        tmem_wait_ld(v);
+                    }
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        acc0[c0 + c] = fmaf(v[c], s0, acc0[c0 + c]);
+                        if constexpr (GATEUP) acc1[c0 + c] = fmaf(u[c], s1, acc1[c0 + c]);
                     }
                 }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acce[slot]);
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acce[slot]);
+            const int n = tl.nt * kTileM + r;
+#pragma unroll
+            for (int c = 0; c < BN; ++c) {
+                if (c < tl.nrows) {
+                    const size_t o = (size_t)(tl.row0 + c) * sg.N + n;
+                    if constexpr (GATEUP)
+                        static_cast<__nv_bfloat16 *>(sg.out)[o] = __float2bfloat16_rn(silu_mul(acc0[c], acc1[c]));
+                    else
+                        static_cast<float *>(sg.out)[o] = acc0[c];
+                }
+            }
         }
     }
 done:
@@ -279,7 +297,7 @@ done:
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
-        tmem_dealloc(tmem_base, C::TMEM_COLS);
+        tmem_dealloc(tmem_base, 512);
     }
 }
 
