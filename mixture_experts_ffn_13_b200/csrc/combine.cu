@@ -5,6 +5,7 @@
 // shared expert's output is added with weight 1 (page "把 397B MoE 榨進 TPU7x", section
 // "稀疏在哪裡": the shared expert runs for every token).  Sums are fp32, in slot order j = 0..k-1
 // then the shared term; the result is rounded to bf16 (round to nearest even).
+#include "launch.cuh"
 #include "moe_internal.h"
 
 #include <cuda_bf16.h>
@@ -13,39 +14,40 @@ namespace moe {
 
 namespace {
 
-// grid T, 256 threads; each thread handles 4 consecutive hidden features at a time.
+// grid (T, ceil(H/1024)), 256 threads: each thread owns 4 consecutive hidden features.
 __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ y, const float *__restrict__ ysh,
                                                       const int32_t *__restrict__ pos,
                                                       const float *__restrict__ topk_w, int H, int k,
                                                       uint16_t *__restrict__ out)
 {
+    griddep_wait();
+    griddep_launch_dependents();
     const int t = blockIdx.x;
-    const int n4 = H / 4;
-    for (int c = threadIdx.x; c < n4; c += blockDim.x) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int j = 0; j < k; ++j) {
-            const int r = __ldg(pos + (size_t)t * k + j);
-            const float w = __ldg(topk_w + (size_t)t * k + j);
-            const float4 v = __ldg(reinterpret_cast<const float4 *>(y + (size_t)r * H) + c);
-            acc.x = fmaf(w, v.x, acc.x);
-            acc.y = fmaf(w, v.y, acc.y);
-            acc.z = fmaf(w, v.z, acc.z);
-            acc.w = fmaf(w, v.w, acc.w);
-        }
-        if (ysh) {
-            const float4 v = __ldg(reinterpret_cast<const float4 *>(ysh + (size_t)t * H) + c);
-            acc.x += v.x;
-            acc.y += v.y;
-            acc.z += v.z;
-            acc.w += v.w;
-        }
-        const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-        const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-        uint2 o;
-        o.x = *reinterpret_cast<const uint32_t *>(&lo);
-        o.y = *reinterpret_cast<const uint32_t *>(&hi);
-        reinterpret_cast<uint2 *>(out + (size_t)t * H)[c] = o;
+    const int c = blockIdx.y * blockDim.x + threadIdx.x;  // float4 index within the row
+    if (c >= H / 4) return;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < k; ++j) {
+        const int r = __ldg(pos + (size_t)t * k + j);
+        const float w = __ldg(topk_w + (size_t)t * k + j);
+        const float4 v = __ldg(reinterpret_cast<const float4 *>(y + (size_t)r * H) + c);
+        acc.x = fmaf(w, v.x, acc.x);
+        acc.y = fmaf(w, v.y, acc.y);
+        acc.z = fmaf(w, v.z, acc.z);
+        acc.w = fmaf(w, v.w, acc.w);
     }
+    if (ysh) {
+        const float4 v = __ldg(reinterpret_cast<const float4 *>(ysh + (size_t)t * H) + c);
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+    }
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+    uint2 o;
+    o.x = *reinterpret_cast<const uint32_t *>(&lo);
+    o.y = *reinterpret_cast<const uint32_t *>(&hi);
+    reinterpret_cast<uint2 *>(out + (size_t)t * H)[c] = o;
 }
 
 }  // namespace
@@ -54,8 +56,8 @@ cudaError_t launch_combine(const float *y, const float *y_shared, const int32_t 
                            int H, int k, uint16_t *out, cudaStream_t s)
 {
     if (T <= 0) return cudaSuccess;
-    combine_kernel<<<T, 256, 0, s>>>(y, y_shared, pos, topk_w, H, k, out);
-    return cudaGetLastError();
+    return launch_pdl(combine_kernel, dim3(T, (H / 4 + 255) / 256), dim3(256), 0, s, y, y_shared, pos, topk_w, H, k,
+                      out);
 }
 
 }  // namespace moe

@@ -26,6 +26,7 @@
 //    h = silu(G) * U in fp32 and stores it.  down: one weight tile; y is stored in fp32.
 #include "moe_internal.h"
 #include "gemm_common.cuh"
+#include "launch.cuh"
 #include "sm100.cuh"
 
 #include <algorithm>
@@ -98,6 +99,10 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP>::THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
+    // everything above overlaps the previous kernel's tail; activations, offsets and tile
+    // prefixes are read only after it has completed
+    griddep_wait();
+    griddep_launch_dependents();
 
     const int tot0 = __ldg(args.ttile + args.E) * (args.seg[0].N / kTileM);
     const int tot1 = args.nseg > 1 ? ((args.T + BN - 1) / BN) * (args.seg[1].N / kTileM) : 0;
@@ -247,8 +252,7 @@ cudaError_t launch_t(const GemmMaps &maps, const GemmArgs &args, int num_sms, cu
     auto kern = gemm_fp8_kernel<BN, GATEUP>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
-    kern<<<num_sms, C::THREADS, C::SMEM, s>>>(maps, args);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(num_sms), dim3(C::THREADS), C::SMEM, s, maps, args);
 }
 
 }  // namespace

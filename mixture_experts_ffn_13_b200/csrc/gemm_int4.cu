@@ -24,6 +24,7 @@
 // before the MMA would not (that costs ~2^-9 relative per weight and fails the layer's
 // tolerance at these sizes).
 #include "gemm_common.cuh"
+#include "launch.cuh"
 #include "sm100.cuh"
 
 #include <cuda_bf16.h>
@@ -129,6 +130,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
+    // everything above overlaps the previous kernel's tail; activations, offsets and tile
+    // prefixes are read only after it has completed
+    griddep_wait();
+    griddep_launch_dependents();
 
     int tot0;
     const int total = total_tiles(args, BN, &tot0);
@@ -308,8 +313,7 @@ cudaError_t launch_t(const GemmMaps &maps, const GemmArgs &args, int num_sms, cu
     auto kern = gemm_int4_kernel<BN, GATEUP>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
-    kern<<<num_sms, kThreads, C::SMEM, s>>>(maps, args);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(num_sms), dim3(kThreads), C::SMEM, s, maps, args);
 }
 
 }  // namespace

@@ -286,9 +286,8 @@ int moe_route(moe_plan_t *p, int32_t T, const float *logits, int32_t *topk_idx, 
     cudaStream_t s = (cudaStream_t)stream;
     const int bn = pick_bn(T, d.k, d.E);
     p->launches = 0;
-    cudaError_t e = launch_route(logits, T, d.E, d.k, topk_idx, topk_w, s);
-    if (e == cudaSuccess) e = launch_permute(b, T, d.E, d.k, bn, bn, s);
-    p->launches = (T > 0 ? 1 : 0) + (T > 0 ? 3 : 1);
+    cudaError_t e = launch_route_permute(logits, b, T, d.E, d.k, bn, bn, s);
+    p->launches = route_permute_launches(T, d.E, d.k);
     return e == cudaSuccess ? MOE_OK : fail_cuda(p, e);
 }
 
@@ -309,9 +308,8 @@ static int forward_int4(moe_plan_t *p, int T, const uint16_t *x, const float *lo
     const int A = T * k;
     const int bn = pick_bn(T, k, E);
     mark(0);
-    cudaError_t e = launch_route(logits, T, E, k, b.topk_idx, b.topk_w, s);
+    cudaError_t e = launch_route_permute(logits, b, T, E, k, bn, bn, s);
     mark(1);
-    if (e == cudaSuccess) e = launch_permute(b, T, E, k, bn, bn, s);
     mark(2);
     if (e != cudaSuccess) return fail_cuda(p, e);
     uint16_t *xp = reinterpret_cast<uint16_t *>(ws + L.act);
@@ -369,7 +367,7 @@ static int forward_int4(moe_plan_t *p, int T, const uint16_t *x, const float *lo
     e = launch_combine(y, y_sh, b.pos, b.topk_w, T, H, k, out, s);
     mark(7);
     if (e != cudaSuccess) return fail_cuda(p, e);
-    p->launches = 1 + 3 + 1 + 1 + 1 + 1;
+    p->launches = route_permute_launches(T, E, k) + 1 + 1 + 1 + 1;
     p->prof_recorded = p->prof;
     return MOE_OK;
 }
@@ -408,9 +406,8 @@ int moe_forward(moe_plan_t *p, int32_t T, const uint16_t *x, const float *logits
     const int bn_a = pick_bn(T, k, E), bn_b = bn_a;
 
     mark(0);
-    cudaError_t e = launch_route(logits, T, E, k, b.topk_idx, b.topk_w, s);
+    cudaError_t e = launch_route_permute(logits, b, T, E, k, bn_a, bn_b, s);
     mark(1);
-    if (e == cudaSuccess) e = launch_permute(b, T, E, k, bn_a, bn_b, s);
     mark(2);
     if (e != cudaSuccess) return fail_cuda(p, e);
 
@@ -484,7 +481,7 @@ int moe_forward(moe_plan_t *p, int32_t T, const uint16_t *x, const float *logits
     e = launch_combine(y, y_sh, b.pos, b.topk_w, T, H, k, out, s);
     mark(7);
     if (e != cudaSuccess) return fail_cuda(p, e);
-    p->launches = 1 + 3 + 1 + 1 + (shared ? 2 : 1) + 1 + 1;
+    p->launches = route_permute_launches(T, E, k) + 1 + 1 + (shared ? 2 : 1) + 1 + 1;
     p->prof_recorded = p->prof;
     return MOE_OK;
 }

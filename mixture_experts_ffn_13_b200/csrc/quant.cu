@@ -6,6 +6,7 @@
 // s = amax / 448 in fp32 (1 when amax == 0) and q = e4m3(x / s), rounded to nearest even
 // with saturation (cvt.rn.satfinite).  Both divisions are IEEE round-to-nearest; an all-zero
 // block stores zero codes.
+#include "launch.cuh"
 #include "moe_internal.h"
 
 #include <cuda_bf16.h>
@@ -52,19 +53,21 @@ __device__ __forceinline__ uint4 quant16(const float (&f)[16], bool valid, float
     return q;
 }
 
-// 1-D grid of T * ceil(nb/4) blocks, 4 warps: warp w of block (t, bx) quantises 512-block
-// bx*4+w of token row t and writes it to the k permuted rows pos[t, :] and to shared row t.
-__global__ void __launch_bounds__(128) quant_x_fp8_kernel(const uint16_t *__restrict__ x, int H, int k,
+// One warp per (token row t, 512-block kb), 8 warps per block over the flattened (t, kb)
+// range: quantise the block and write it to the k permuted rows pos[t, :] and to shared row t.
+__global__ void __launch_bounds__(256) quant_x_fp8_kernel(const uint16_t *__restrict__ x, int T, int H, int k,
                                                           const int32_t *__restrict__ pos, uint8_t *__restrict__ xq,
                                                           float *__restrict__ sx, uint8_t *__restrict__ xq_sh,
                                                           float *__restrict__ sx_sh)
 {
+    griddep_wait();
+    griddep_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nb = (H + kBlockK - 1) / kBlockK;
-    const int nbx = (nb + 3) / 4;
-    const int t = blockIdx.x / nbx;
-    const int kb = (blockIdx.x - t * nbx) * 4 + warp;
-    if (kb >= nb) return;
+    const long wid = (long)blockIdx.x * 8 + warp;
+    if (wid >= (long)T * nb) return;
+    const int t = (int)(wid / nb);
+    const int kb = (int)(wid - (long)t * nb);
     const int i0 = kb * kBlockK + lane * 16;
     const bool valid = i0 < H;
     float f[16] = {};
@@ -81,7 +84,7 @@ __global__ void __launch_bounds__(128) quant_x_fp8_kernel(const uint16_t *__rest
     float s;
     const uint4 q = quant16(f, valid, &s);
     for (int j = 0; j < k; ++j) {
-        const int r = pos[(size_t)t * k + j];
+        const int r = __ldg(pos + (size_t)t * k + j);
         if (valid) *reinterpret_cast<uint4 *>(xq + (size_t)r * H + i0) = q;
         if (lane == 0) sx[(size_t)r * nb + kb] = s;
     }
@@ -91,16 +94,18 @@ __global__ void __launch_bounds__(128) quant_x_fp8_kernel(const uint16_t *__rest
     }
 }
 
-// 1-D grid of R * ceil(nb/4) blocks: fp32 rows -> e4m3 rows + scales.
-__global__ void __launch_bounds__(128) quant_rows_fp8_kernel(const float *__restrict__ h, int K,
+// One warp per (row, 512-block), 8 warps per block: fp32 rows -> e4m3 rows + scales.
+__global__ void __launch_bounds__(256) quant_rows_fp8_kernel(const float *__restrict__ h, int R, int K,
                                                              uint8_t *__restrict__ q, float *__restrict__ sq)
 {
+    griddep_wait();
+    griddep_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nb = (K + kBlockK - 1) / kBlockK;
-    const int nbx = (nb + 3) / 4;
-    const int r = blockIdx.x / nbx;
-    const int kb = (blockIdx.x - r * nbx) * 4 + warp;
-    if (kb >= nb) return;
+    const long wid = (long)blockIdx.x * 8 + warp;
+    if (wid >= (long)R * nb) return;
+    const int r = (int)(wid / nb);
+    const int kb = (int)(wid - (long)r * nb);
     const int i0 = kb * kBlockK + lane * 16;
     const bool valid = i0 < K;
     float f[16] = {};
@@ -126,6 +131,8 @@ __global__ void __launch_bounds__(128) gather_x_bf16_kernel(const uint16_t *__re
                                                             const int32_t *__restrict__ pos, uint16_t *__restrict__ xp,
                                                             uint16_t *__restrict__ xp_sh)
 {
+    griddep_wait();
+    griddep_launch_dependents();
     const int t = blockIdx.x;
     const int n16 = H / 8;  // uint4 chunks of 8 bf16
     const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * H);
@@ -145,25 +152,23 @@ cudaError_t launch_quant_x_fp8(const uint16_t *x, int T, int H, int k, const int
                                uint8_t *xq_shared, float *sx_shared, cudaStream_t s)
 {
     if (T <= 0) return cudaSuccess;
-    const int nb = (H + kBlockK - 1) / kBlockK;
-    quant_x_fp8_kernel<<<(unsigned)(T * ((nb + 3) / 4)), 128, 0, s>>>(x, H, k, pos, xq, sx, xq_shared, sx_shared);
-    return cudaGetLastError();
+    const long warps = (long)T * ((H + kBlockK - 1) / kBlockK);
+    return launch_pdl(quant_x_fp8_kernel, dim3((unsigned)((warps + 7) / 8)), dim3(256), 0, s, x, T, H, k, pos, xq, sx,
+                      xq_shared, sx_shared);
 }
 
 cudaError_t launch_quant_rows_fp8(const float *h, int R, int K, uint8_t *q, float *sq, cudaStream_t s)
 {
     if (R <= 0) return cudaSuccess;
-    const int nb = (K + kBlockK - 1) / kBlockK;
-    quant_rows_fp8_kernel<<<(unsigned)(R * ((nb + 3) / 4)), 128, 0, s>>>(h, K, q, sq);
-    return cudaGetLastError();
+    const long warps = (long)R * ((K + kBlockK - 1) / kBlockK);
+    return launch_pdl(quant_rows_fp8_kernel, dim3((unsigned)((warps + 7) / 8)), dim3(256), 0, s, h, R, K, q, sq);
 }
 
 cudaError_t launch_gather_x_bf16(const uint16_t *x, int T, int H, int k, const int32_t *pos, uint16_t *xp,
                                  uint16_t *xp_shared, cudaStream_t s)
 {
     if (T <= 0) return cudaSuccess;
-    gather_x_bf16_kernel<<<T, 128, 0, s>>>(x, H, k, pos, xp, xp_shared);
-    return cudaGetLastError();
+    return launch_pdl(gather_x_bf16_kernel, dim3(T), dim3(128), 0, s, x, H, k, pos, xp, xp_shared);
 }
 
 }  // namespace moe

@@ -10,6 +10,7 @@
 // (expert, token) key.  Here that order is produced without a sort: a per-chunk histogram,
 // one prefix sum over (expert, chunk), and an in-order scatter inside each chunk, so the
 // result is deterministic and equal to sorting by (expert, token).
+#include "launch.cuh"
 #include "moe_internal.h"
 
 #include <math.h>
@@ -20,16 +21,14 @@ namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
 
-// One warp per token.  Lane l holds the logits of experts l, l+32, ...; k rounds of a warp
-// arg-max (value desc, index asc) pick the experts; lane j keeps the j-th pick.
+// Top-k of one token's logits by one warp.  Lane l holds the logits of experts l, l+32, ...;
+// k rounds of a warp arg-max (value desc, index asc) pick the experts; lane j < k returns the
+// j-th pick in *sel_e and its weight p_hat_j = exp(L_j - L_max) / sum_i exp(L_i - L_max) (the
+// sum taken in selection order) in *sel_w.
 template <int EPL>
-__global__ void __launch_bounds__(256) route_kernel(const float *__restrict__ logits, int T, int E, int k,
-                                                    int32_t *__restrict__ topk_idx, float *__restrict__ topk_w)
+__device__ __forceinline__ void route_one(const float *__restrict__ L, int E, int k, int lane, int *sel_e_out,
+                                          float *sel_w_out)
 {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t = blockIdx.x * 8 + warp;
-    if (t >= T) return;
-    const float *L = logits + (size_t)t * E;
     float v[EPL];
     uint32_t taken = 0;  // bit i: element i of this lane is absent or already chosen
 #pragma unroll
@@ -66,14 +65,30 @@ __global__ void __launch_bounds__(256) route_kernel(const float *__restrict__ lo
             sel_e = be;
         }
     }
-    // p_hat_j = exp(L_j - L_max) / sum_i exp(L_i - L_max), the sum taken in selection order.
     const float lmax = __shfl_sync(kFull, sel_v, 0);
     const float ex = (lane < k) ? expf(sel_v - lmax) : 0.0f;
     float denom = 0.0f;
     for (int j = 0; j < k; ++j) denom += __shfl_sync(kFull, ex, j);
+    *sel_e_out = sel_e;
+    *sel_w_out = ex / denom;
+}
+
+// One warp per token.
+template <int EPL>
+__global__ void __launch_bounds__(256) route_kernel(const float *__restrict__ logits, int T, int E, int k,
+                                                    int32_t *__restrict__ topk_idx, float *__restrict__ topk_w)
+{
+    griddep_wait();
+    griddep_launch_dependents();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = blockIdx.x * 8 + warp;
+    if (t >= T) return;
+    int e;
+    float w;
+    route_one<EPL>(logits + (size_t)t * E, E, k, lane, &e, &w);
     if (lane < k) {
-        topk_idx[(size_t)t * k + lane] = sel_e;
-        topk_w[(size_t)t * k + lane] = ex / denom;
+        topk_idx[(size_t)t * k + lane] = e;
+        topk_w[(size_t)t * k + lane] = w;
     }
 }
 
@@ -82,6 +97,8 @@ __global__ void __launch_bounds__(kChunk) hist_kernel(const int32_t *__restrict_
                                                       int32_t *__restrict__ chunk_hist)
 {
     __shared__ int h[kMaxE];
+    griddep_wait();
+    griddep_launch_dependents();
     for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
     __syncthreads();
     const int t = blockIdx.x * kChunk + threadIdx.x;
@@ -132,6 +149,8 @@ __global__ void __launch_bounds__(1024) scan_kernel(int nchunks, int E, int32_t 
                                                     int32_t *__restrict__ ttile_b)
 {
     __shared__ int scratch[33];
+    griddep_wait();
+    griddep_launch_dependents();
     const int e = threadIdx.x;
     int c = 0;
     if (e < E) {
@@ -160,26 +179,33 @@ __global__ void __launch_bounds__(1024) scan_kernel(int nchunks, int E, int32_t 
 }
 
 // Scatter of one chunk of 256 tokens (8 warps x 32).  Rows of expert e inside the chunk are
-// handed out in token order: warp-level counts, an exclusive scan over the 8 warps, then each
-// warp walks its 32 tokens in order (lane j < k handles slot j; the k experts of a token are
-// distinct, so the k lanes never touch the same counter).
+// handed out in token order: warp-level counts, an exclusive scan over the 8 warps (plus the
+// chunk's base row), then each warp walks its 32 tokens in order (lane j < k handles slot j;
+// the k experts of a token are distinct, so the k lanes never touch the same counter).  Each
+// lane loads its 32 expert ids up front so the in-order walks touch shared memory only.
 __global__ void __launch_bounds__(kChunk) scatter_kernel(const int32_t *__restrict__ topk_idx, int T, int E, int k,
                                                          const int32_t *__restrict__ chunk_base,
                                                          int32_t *__restrict__ perm_tok, int32_t *__restrict__ pos)
 {
     __shared__ int cnt[kChunk / 32][kMaxE];
+    griddep_wait();
+    griddep_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t0 = blockIdx.x * kChunk + warp * 32;
+    int ids[32];
+#pragma unroll
+    for (int l = 0; l < 32; ++l) ids[l] = (t0 + l < T && lane < k) ? __ldg(topk_idx + (size_t)(t0 + l) * k + lane) : -1;
     for (int i = threadIdx.x; i < (kChunk / 32) * E; i += blockDim.x) cnt[i / E][i % E] = 0;
     __syncthreads();
-    const int t0 = blockIdx.x * kChunk + warp * 32;
+#pragma unroll
     for (int l = 0; l < 32; ++l) {
-        const int t = t0 + l;
-        if (t < T && lane < k) cnt[warp][topk_idx[(size_t)t * k + lane]] += 1;
+        if (ids[l] >= 0) cnt[warp][ids[l]] += 1;
         __syncwarp();
     }
     __syncthreads();
+    const int32_t *base = chunk_base + (size_t)blockIdx.x * E;
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int run = 0;
+        int run = __ldg(base + e);
         for (int w = 0; w < kChunk / 32; ++w) {
             const int c = cnt[w][e];
             cnt[w][e] = run;
@@ -187,21 +213,123 @@ __global__ void __launch_bounds__(kChunk) scatter_kernel(const int32_t *__restri
         }
     }
     __syncthreads();
-    const int32_t *base = chunk_base + (size_t)blockIdx.x * E;
+#pragma unroll
     for (int l = 0; l < 32; ++l) {
-        const int t = t0 + l;
-        if (t < T && lane < k) {
-            const int e = topk_idx[(size_t)t * k + lane];
-            const int r = base[e] + cnt[warp][e];
-            cnt[warp][e] += 1;
-            perm_tok[r] = t;
-            pos[(size_t)t * k + lane] = r;
+        if (ids[l] >= 0) {
+            const int r = cnt[warp][ids[l]]++;
+            perm_tok[r] = t0 + l;
+            pos[(size_t)(t0 + l) * k + lane] = r;
         }
         __syncwarp();
     }
 }
 
+// Small batches: route and permute in one block of 1024 threads.  Routing as above (warp w
+// takes tokens w, w+32, ...); each assignment sets bit t of its expert's token bitmap
+// (E x ceil(T/32) words in shared memory).  The row of assignment (t, e) is then
+// offsets[e] + (tokens below t that chose e) = a per-(expert, word) prefix of bit counts plus
+// the popcount of the bits below t in t's word, which is the (expert, token) order without a
+// sort or a serial pass.
+template <int EPL>
+__global__ void __launch_bounds__(1024) route_permute_small_kernel(
+    const float *__restrict__ logits, int T, int E, int k, int32_t *__restrict__ topk_idx,
+    float *__restrict__ topk_w, int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
+    int32_t *__restrict__ perm_tok, int32_t *__restrict__ pos, int bn_a, int32_t *__restrict__ ttile_a, int bn_b,
+    int32_t *__restrict__ ttile_b)
+{
+    extern __shared__ int sm[];
+    const int W = (T + 31) >> 5;
+    int *s_scr = sm;                                      // 33
+    int *s_cnt = s_scr + 64;                              // E
+    uint32_t *mask = reinterpret_cast<uint32_t *>(s_cnt + E);  // E * W
+    int *pre = reinterpret_cast<int *>(mask + (size_t)E * W);  // E * W
+    int *s_idx = pre + (size_t)E * W;                     // T * k
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    griddep_wait();
+    griddep_launch_dependents();
+    for (int i = tid; i < E; i += 1024) s_cnt[i] = 0;
+    for (int i = tid; i < E * W; i += 1024) mask[i] = 0;
+    __syncthreads();
+    for (int t = warp; t < T; t += 32) {
+        int e;
+        float w;
+        route_one<EPL>(logits + (size_t)t * E, E, k, lane, &e, &w);
+        if (lane < k) {
+            topk_idx[(size_t)t * k + lane] = e;
+            topk_w[(size_t)t * k + lane] = w;
+            s_idx[t * k + lane] = e;
+            atomicOr(&mask[e * W + (t >> 5)], 1u << (t & 31));
+            atomicAdd(&s_cnt[e], 1);
+        }
+    }
+    __syncthreads();
+    const int c = tid < E ? s_cnt[tid] : 0;
+    int total;
+    const int off = block_exclusive_scan(c, s_scr, &total);
+    if (tid < E) {
+        counts[tid] = c;
+        offsets[tid] = off;
+        int run = off;
+        for (int w = 0; w < W; ++w) {
+            pre[tid * W + w] = run;
+            run += __popc(mask[tid * W + w]);
+        }
+    }
+    if (tid == 0) offsets[E] = total;
+    const int oa = block_exclusive_scan(tid < E ? (c + bn_a - 1) / bn_a : 0, s_scr, &total);
+    if (tid < E) ttile_a[tid] = oa;
+    if (tid == 0) ttile_a[E] = total;
+    const int ob = block_exclusive_scan(tid < E ? (c + bn_b - 1) / bn_b : 0, s_scr, &total);
+    if (tid < E) ttile_b[tid] = ob;
+    if (tid == 0) ttile_b[E] = total;
+    __syncthreads();
+    for (int i = tid; i < T * k; i += 1024) {
+        const int t = i / k;
+        const int e = s_idx[i];
+        const int w = t >> 5;
+        const int r = pre[e * W + w] + __popc(mask[e * W + w] & ((1u << (t & 31)) - 1u));
+        perm_tok[r] = t;
+        pos[i] = r;
+    }
+}
+
+size_t small_route_smem(int T, int E, int k)
+{
+    const size_t W = ((size_t)T + 31) / 32;
+    return 4 * (64 + (size_t)E + 2 * (size_t)E * W + (size_t)T * k);
+}
+
 }  // namespace
+
+cudaError_t launch_route_permute(const float *logits, const RouteBufs &b, int T, int E, int k, int bn_a, int bn_b,
+                                 cudaStream_t s)
+{
+    const size_t smem = small_route_smem(T, E, k);
+    if (T < 1 || T > 2048 || smem > 160 * 1024) {
+        cudaError_t e = launch_route(logits, T, E, k, b.topk_idx, b.topk_w, s);
+        if (e != cudaSuccess) return e;
+        return launch_permute(b, T, E, k, bn_a, bn_b, s);
+    }
+    const int epl = (E + 31) / 32;
+    auto go = [&](auto kern) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        return launch_pdl(kern, dim3(1), dim3(1024), smem, s, logits, T, E, k, b.topk_idx, b.topk_w, b.counts,
+                          b.offsets, b.perm_tok, b.pos, bn_a, b.ttile_a, bn_b, b.ttile_b);
+    };
+    if (epl <= 1) return go(route_permute_small_kernel<1>);
+    if (epl <= 2) return go(route_permute_small_kernel<2>);
+    if (epl <= 4) return go(route_permute_small_kernel<4>);
+    if (epl <= 8) return go(route_permute_small_kernel<8>);
+    if (epl <= 16) return go(route_permute_small_kernel<16>);
+    return go(route_permute_small_kernel<32>);
+}
+
+int route_permute_launches(int T, int E, int k)
+{
+    if (T < 1 || T > 2048 || small_route_smem(T, E, k) > 160 * 1024) return (T > 0 ? 1 : 0) + (T > 0 ? 3 : 1);
+    return 1;
+}
 
 cudaError_t launch_route(const float *logits, int T, int E, int k, int32_t *topk_idx, float *topk_w,
                          cudaStream_t s)
@@ -209,28 +337,27 @@ cudaError_t launch_route(const float *logits, int T, int E, int k, int32_t *topk
     if (T <= 0) return cudaSuccess;
     const dim3 grid((T + 7) / 8), block(256);
     const int epl = (E + 31) / 32;
-    if (epl <= 1)
-        route_kernel<1><<<grid, block, 0, s>>>(logits, T, E, k, topk_idx, topk_w);
-    else if (epl <= 2)
-        route_kernel<2><<<grid, block, 0, s>>>(logits, T, E, k, topk_idx, topk_w);
-    else if (epl <= 4)
-        route_kernel<4><<<grid, block, 0, s>>>(logits, T, E, k, topk_idx, topk_w);
-    else if (epl <= 8)
-        route_kernel<8><<<grid, block, 0, s>>>(logits, T, E, k, topk_idx, topk_w);
-    else if (epl <= 16)
-        route_kernel<16><<<grid, block, 0, s>>>(logits, T, E, k, topk_idx, topk_w);
-    else
-        route_kernel<32><<<grid, block, 0, s>>>(logits, T, E, k, topk_idx, topk_w);
-    return cudaGetLastError();
+    auto go = [&](auto kern) { return launch_pdl(kern, grid, block, 0, s, logits, T, E, k, topk_idx, topk_w); };
+    if (epl <= 1) return go(route_kernel<1>);
+    if (epl <= 2) return go(route_kernel<2>);
+    if (epl <= 4) return go(route_kernel<4>);
+    if (epl <= 8) return go(route_kernel<8>);
+    if (epl <= 16) return go(route_kernel<16>);
+    return go(route_kernel<32>);
 }
 
 cudaError_t launch_permute(const RouteBufs &b, int T, int E, int k, int bn_a, int bn_b, cudaStream_t s)
 {
     const int nchunks = (T + kChunk - 1) / kChunk;
-    if (nchunks > 0) hist_kernel<<<nchunks, kChunk, 0, s>>>(b.topk_idx, T, E, k, b.chunk_hist);
-    scan_kernel<<<1, 1024, 0, s>>>(nchunks, E, b.chunk_hist, b.counts, b.offsets, bn_a, b.ttile_a, bn_b, b.ttile_b);
-    if (nchunks > 0) scatter_kernel<<<nchunks, kChunk, 0, s>>>(b.topk_idx, T, E, k, b.chunk_hist, b.perm_tok, b.pos);
-    return cudaGetLastError();
+    cudaError_t e = cudaSuccess;
+    if (nchunks > 0) e = launch_pdl(hist_kernel, dim3(nchunks), dim3(kChunk), 0, s, b.topk_idx, T, E, k, b.chunk_hist);
+    if (e == cudaSuccess)
+        e = launch_pdl(scan_kernel, dim3(1), dim3(1024), 0, s, nchunks, E, b.chunk_hist, b.counts, b.offsets, bn_a,
+                       b.ttile_a, bn_b, b.ttile_b);
+    if (e == cudaSuccess && nchunks > 0)
+        e = launch_pdl(scatter_kernel, dim3(nchunks), dim3(kChunk), 0, s, b.topk_idx, T, E, k, b.chunk_hist,
+                       b.perm_tok, b.pos);
+    return e;
 }
 
 }  // namespace moe
