@@ -308,8 +308,9 @@ static int forward_int4(moe_plan_t *p, int T, const uint16_t *x, const float *lo
     const int A = T * k;
     const int bn = pick_bn(T, k, E);
     mark(0);
-    cudaError_t e = launch_route_permute(logits, b, T, E, k, bn, bn, s);
+    cudaError_t e = launch_route(logits, T, E, k, b.topk_idx, b.topk_w, s);
     mark(1);
+    if (e == cudaSuccess) e = launch_permute_any(b, T, E, k, bn, bn, s);
     mark(2);
     if (e != cudaSuccess) return fail_cuda(p, e);
     uint16_t *xp = reinterpret_cast<uint16_t *>(ws + L.act);
@@ -406,8 +407,9 @@ int moe_forward(moe_plan_t *p, int32_t T, const uint16_t *x, const float *logits
     const int bn_a = pick_bn(T, k, E), bn_b = bn_a;
 
     mark(0);
-    cudaError_t e = launch_route_permute(logits, b, T, E, k, bn_a, bn_b, s);
+    cudaError_t e = launch_route(logits, T, E, k, b.topk_idx, b.topk_w, s);
     mark(1);
+    if (e == cudaSuccess) e = launch_permute_any(b, T, E, k, bn_a, bn_b, s);
     mark(2);
     if (e != cudaSuccess) return fail_cuda(p, e);
 

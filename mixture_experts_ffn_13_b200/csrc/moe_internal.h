@@ -34,7 +34,9 @@ struct RouteBufs {
 cudaError_t launch_route(const float *logits, int T, int E, int k, int32_t *topk_idx, float *topk_w,
                          cudaStream_t s);
 cudaError_t launch_permute(const RouteBufs &b, int T, int E, int k, int bn_a, int bn_b, cudaStream_t s);
-// Route + permute: one fused single-block kernel for small batches, else the two launches above.
+// Permutation: one single-block kernel for small batches, else the three launches above.
+cudaError_t launch_permute_any(const RouteBufs &b, int T, int E, int k, int bn_a, int bn_b, cudaStream_t s);
+// Router followed by launch_permute_any, and the number of kernels the pair launches.
 cudaError_t launch_route_permute(const float *logits, const RouteBufs &b, int T, int E, int k, int bn_a, int bn_b,
                                  cudaStream_t s);
 int route_permute_launches(int T, int E, int k);

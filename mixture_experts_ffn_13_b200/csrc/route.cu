@@ -224,43 +224,37 @@ __global__ void __launch_bounds__(kChunk) scatter_kernel(const int32_t *__restri
     }
 }
 
-// Small batches: route and permute in one block of 1024 threads.  Routing as above (warp w
-// takes tokens w, w+32, ...); each assignment sets bit t of its expert's token bitmap
-// (E x ceil(T/32) words in shared memory).  The row of assignment (t, e) is then
-// offsets[e] + (tokens below t that chose e) = a per-(expert, word) prefix of bit counts plus
-// the popcount of the bits below t in t's word, which is the (expert, token) order without a
-// sort or a serial pass.
-template <int EPL>
-__global__ void __launch_bounds__(1024) route_permute_small_kernel(
-    const float *__restrict__ logits, int T, int E, int k, int32_t *__restrict__ topk_idx,
-    float *__restrict__ topk_w, int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
-    int32_t *__restrict__ perm_tok, int32_t *__restrict__ pos, int bn_a, int32_t *__restrict__ ttile_a, int bn_b,
-    int32_t *__restrict__ ttile_b)
+// Small batches: the whole permutation in one block of 1024 threads (after the router).  Each
+// assignment sets bit t of its expert's token bitmap (E x ceil(T/32) words in shared memory);
+// the row of assignment (t, e) is then offsets[e] + (tokens below t that chose e) = a
+// per-(expert, word) prefix of bit counts plus the popcount of the bits below t in t's word --
+// the (expert, token) order without a sort or a serial pass.
+__global__ void __launch_bounds__(1024) permute_small_kernel(const int32_t *__restrict__ topk_idx, int T, int E,
+                                                             int k, int32_t *__restrict__ counts,
+                                                             int32_t *__restrict__ offsets,
+                                                             int32_t *__restrict__ perm_tok, int32_t *__restrict__ pos,
+                                                             int bn_a, int32_t *__restrict__ ttile_a, int bn_b,
+                                                             int32_t *__restrict__ ttile_b)
 {
     extern __shared__ int sm[];
     const int W = (T + 31) >> 5;
-    int *s_scr = sm;                                      // 33
-    int *s_cnt = s_scr + 64;                              // E
+    int *s_scr = sm;                                           // 33
+    int *s_cnt = s_scr + 64;                                   // E
     uint32_t *mask = reinterpret_cast<uint32_t *>(s_cnt + E);  // E * W
     int *pre = reinterpret_cast<int *>(mask + (size_t)E * W);  // E * W
-    int *s_idx = pre + (size_t)E * W;                     // T * k
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    int *s_idx = pre + (size_t)E * W;                          // T * k
+    const int tid = threadIdx.x;
     griddep_wait();
     griddep_launch_dependents();
     for (int i = tid; i < E; i += 1024) s_cnt[i] = 0;
     for (int i = tid; i < E * W; i += 1024) mask[i] = 0;
     __syncthreads();
-    for (int t = warp; t < T; t += 32) {
-        int e;
-        float w;
-        route_one<EPL>(logits + (size_t)t * E, E, k, lane, &e, &w);
-        if (lane < k) {
-            topk_idx[(size_t)t * k + lane] = e;
-            topk_w[(size_t)t * k + lane] = w;
-            s_idx[t * k + lane] = e;
-            atomicOr(&mask[e * W + (t >> 5)], 1u << (t & 31));
-            atomicAdd(&s_cnt[e], 1);
-        }
+    for (int i = tid; i < T * k; i += 1024) {
+        const int e = __ldg(topk_idx + i);
+        const int t = i / k;
+        s_idx[i] = e;
+        atomicOr(&mask[e * W + (t >> 5)], 1u << (t & 31));
+        atomicAdd(&s_cnt[e], 1);
     }
     __syncthreads();
     const int c = tid < E ? s_cnt[tid] : 0;
@@ -304,31 +298,27 @@ size_t small_route_smem(int T, int E, int k)
 cudaError_t launch_route_permute(const float *logits, const RouteBufs &b, int T, int E, int k, int bn_a, int bn_b,
                                  cudaStream_t s)
 {
+    cudaError_t e = launch_route(logits, T, E, k, b.topk_idx, b.topk_w, s);
+    if (e != cudaSuccess) return e;
+    return launch_permute_any(b, T, E, k, bn_a, bn_b, s);
+}
+
+cudaError_t launch_permute_any(const RouteBufs &b, int T, int E, int k, int bn_a, int bn_b, cudaStream_t s)
+{
+    cudaError_t e;
     const size_t smem = small_route_smem(T, E, k);
-    if (T < 1 || T > 2048 || smem > 160 * 1024) {
-        cudaError_t e = launch_route(logits, T, E, k, b.topk_idx, b.topk_w, s);
-        if (e != cudaSuccess) return e;
-        return launch_permute(b, T, E, k, bn_a, bn_b, s);
-    }
-    const int epl = (E + 31) / 32;
-    auto go = [&](auto kern) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        return launch_pdl(kern, dim3(1), dim3(1024), smem, s, logits, T, E, k, b.topk_idx, b.topk_w, b.counts,
-                          b.offsets, b.perm_tok, b.pos, bn_a, b.ttile_a, bn_b, b.ttile_b);
-    };
-    if (epl <= 1) return go(route_permute_small_kernel<1>);
-    if (epl <= 2) return go(route_permute_small_kernel<2>);
-    if (epl <= 4) return go(route_permute_small_kernel<4>);
-    if (epl <= 8) return go(route_permute_small_kernel<8>);
-    if (epl <= 16) return go(route_permute_small_kernel<16>);
-    return go(route_permute_small_kernel<32>);
+    if (T < 1 || T > 4096 || smem > 160 * 1024) return launch_permute(b, T, E, k, bn_a, bn_b, s);
+    e = cudaFuncSetAttribute(permute_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(permute_small_kernel, dim3(1), dim3(1024), smem, s, b.topk_idx, T, E, k, b.counts, b.offsets,
+                      b.perm_tok, b.pos, bn_a, b.ttile_a, bn_b, b.ttile_b);
 }
 
 int route_permute_launches(int T, int E, int k)
 {
-    if (T < 1 || T > 2048 || small_route_smem(T, E, k) > 160 * 1024) return (T > 0 ? 1 : 0) + (T > 0 ? 3 : 1);
-    return 1;
+    if (T < 1) return 1;
+    if (T > 4096 || small_route_smem(T, E, k) > 160 * 1024) return 4;
+    return 2;
 }
 
 cudaError_t launch_route(const float *logits, int T, int E, int k, int32_t *topk_idx, float *topk_w,
