@@ -15,13 +15,16 @@
 //    cost nothing and hot experts get many token tiles.
 //  * Warp roles: warp 0 issues TMA loads of 128-byte-wide K slices (weights with an
 //    evict-first L2 hint, activations evict-last) into an NS-deep ring of shared-memory
-//    stages; warp 1 issues tcgen05.mma (E4M3 x E4M3 -> F32) from one thread; warps 2-5 are
-//    the epilogue.
+//    stages; warp 1 issues tcgen05.mma (E4M3 x E4M3 -> F32) from one thread; the remaining
+//    EW warps are the epilogue (EW/4 warps per 32-lane TMEM quarter, each owning a slice of
+//    the BN token columns so the fp32 accumulators stay in registers).
 //  * Sub-channel promotion: the scales change every 512 elements of K for both operands, so
 //    each 512-block gets its own TMEM accumulator slot (a ring of slots covering all 512
 //    TMEM columns).  The epilogue reads a finished slot, multiplies it by
 //    s_w[row, kb] * s_x[token, kb] and adds it into fp32 registers, then frees the slot, so
-//    the MMAs of the next blocks overlap the promotion of the previous ones.
+//    the MMAs of the next blocks overlap the promotion of the previous ones.  The tile's
+//    activation scales s_x[row0 .. row0+BN, :] are staged in shared memory once per tile
+//    (double-buffered across tiles) and the weight scales are prefetched a block ahead.
 //  * gate|up: two weight tiles per stage share one activation tile; the epilogue computes
 //    h = silu(G) * U in fp32 and stores it.  down: one weight tile; y is stored in fp32.
 #include "moe_internal.h"
@@ -29,42 +32,51 @@
 #include "launch.cuh"
 #include "sm100.cuh"
 
-#include <algorithm>
-
 namespace moe {
 
 namespace {
 
 constexpr int kKC = 128;     // K elements (bytes) per pipeline stage = one 128-byte swizzle row
 constexpr int kStagesPerBlock = kBlockK / kKC;
-constexpr int kSmemBudget = 200 * 1024;
+constexpr int kMaxKb = 32;   // activation-scale staging holds up to 32 blocks (K <= 16384)
+constexpr int kSmemLimit = 227 * 1024;
 
-template <int BN, bool GATEUP>
+template <int BN, bool GATEUP, int EW>
 struct Fp8Cfg {
     static constexpr int NA = GATEUP ? 2 : 1;
     static constexpr int A_BYTES = kTileM * kKC;
     static constexpr int B_BYTES = BN * kKC;
     static constexpr int STAGE_BYTES = NA * A_BYTES + B_BYTES;
-    static constexpr int NS = (kSmemBudget / STAGE_BYTES) < 16 ? (kSmemBudget / STAGE_BYTES) : 16;
     static constexpr int SLOT_COLS = NA * BN;
     static constexpr int NSLOT = 512 / SLOT_COLS;
-    static constexpr int EPI_WARPS = 4;
-    static constexpr int THREADS = 64 + 32 * EPI_WARPS;
-    static constexpr int BAR_BYTES = 8 * (2 * NS + 2 * NSLOT) + 16;
-    static constexpr int SMEM = 1024 + NS * STAGE_BYTES + BAR_BYTES;
+    static constexpr int EPI_WARPS = EW;
+    static constexpr int PARTS = EW / 4;           // epilogue warps per TMEM lane quarter
+    static constexpr int CPW = BN / PARTS;         // token columns per epilogue thread
+    static constexpr int THREADS = 64 + 32 * EW;
+    static constexpr int SX_BYTES = 2 * BN * kMaxKb * 4;
+    static constexpr int BAR_BYTES = 8 * (2 * 16 + 2 * NSLOT) + 16;
+    static constexpr int FIXED = 1024 + SX_BYTES + BAR_BYTES;
+    static constexpr int NS_FIT = (kSmemLimit - FIXED) / STAGE_BYTES;
+    static constexpr int NS = NS_FIT < 16 ? NS_FIT : 16;
+    static constexpr int SMEM = FIXED + NS * STAGE_BYTES;
     static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "stage tiles must stay 1024-byte aligned");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M=128 is a multiple of 16 in [16, 256]");
-    static_assert(NSLOT >= 1, "TMEM slots");
+    static_assert(EW % 4 == 0 && CPW % 16 == 0, "epilogue split");
+    static_assert(NSLOT >= 1 && NS >= 2, "pipeline");
 };
 
-template <int BN, bool GATEUP>
-__global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP>::THREADS, 1)
+// Named barrier among the EW epilogue warps (ids 2..2+EW-1); barrier 0 is __syncthreads.
+__device__ __forceinline__ void epi_sync(int nthreads) { asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory"); }
+
+template <int BN, bool GATEUP, int EW>
+__global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
     gemm_fp8_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmArgs args)
 {
-    using C = Fp8Cfg<BN, GATEUP>;
+    using C = Fp8Cfg<BN, GATEUP, EW>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::NS * C::STAGE_BYTES);
+    float *sxbuf = reinterpret_cast<float *>(smem + C::NS * C::STAGE_BYTES);  // [2][BN * kMaxKb]
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::NS * C::STAGE_BYTES + C::SX_BYTES);
     uint64_t *empty = full + C::NS;
     uint64_t *accf = empty + C::NS;
     uint64_t *acce = accf + C::NSLOT;
@@ -104,9 +116,8 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP>::THREADS, 1)
     griddep_wait();
     griddep_launch_dependents();
 
-    const int tot0 = __ldg(args.ttile + args.E) * (args.seg[0].N / kTileM);
-    const int tot1 = args.nseg > 1 ? ((args.T + BN - 1) / BN) * (args.seg[1].N / kTileM) : 0;
-    const int total = tot0 + tot1;
+    int tot0;
+    const int total = total_tiles(args, BN, &tot0);
     int *status = args.status;
     const uint64_t tmo = args.timeout_ns;
 
@@ -172,34 +183,51 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP>::THREADS, 1)
         }
     } else {
         // ------------------------------ epilogue ----------------------------------
-        const int q = warp & 3;  // TMEM lanes 32q..32q+31 are reachable from this warp
-        const int r = q * 32 + lane;
+        const int ew = warp - 2;
+        const int q = warp & 3;               // TMEM lanes 32q..32q+31 are reachable from this warp
+        const int cbase = (ew >> 2) * C::CPW; // this warp's first token column
+        const int r = q * 32 + lane;          // weight row within the tile
+        const int etid = ew * 32 + lane;      // index among the epilogue threads
         uint32_t ai = 0;
-        for (int w = blockIdx.x; w < total; w += gridDim.x) {
+        int ti = 0;
+        for (int w = blockIdx.x; w < total; w += gridDim.x, ++ti) {
             const TileInfo tl = decode_tile<BN>(args, w, tot0);
             const GemmSeg &sg = args.seg[tl.seg];
             const int K = sg.K;
             const int nkb = (K + kBlockK - 1) / kBlockK;
+            // stage s_x[row0 + c, kb] (rows past the segment read its last row; unused)
+            float *sxs = sxbuf + (ti & 1) * (BN * kMaxKb);
+            for (int i = etid; i < BN * nkb; i += 32 * EW) {
+                const int c = i / nkb, kb = i - c * nkb;
+                const int row = min(tl.row0 + c, sg.rows - 1);
+                sxs[kb * BN + c] = __ldg(sg.sx + (size_t)row * nkb + kb);
+            }
+            epi_sync(32 * EW);
             const float *sw0 = static_cast<const float *>(sg.sw0) + (size_t)(tl.wrow + r) * nkb;
             const float *sw1 = GATEUP ? static_cast<const float *>(sg.sw1) + (size_t)(tl.wrow + r) * nkb : nullptr;
-            float acc0[BN], acc1[GATEUP ? BN : 1];
+            float acc0[C::CPW], acc1[GATEUP ? C::CPW : 1];
 #pragma unroll
-            for (int c = 0; c < BN; ++c) acc0[c] = 0.0f;
+            for (int c = 0; c < C::CPW; ++c) acc0[c] = 0.0f;
             if constexpr (GATEUP) {
 #pragma unroll
-                for (int c = 0; c < BN; ++c) acc1[c] = 0.0f;
+                for (int c = 0; c < C::CPW; ++c) acc1[c] = 0.0f;
             }
+            float s0n = __ldg(sw0), s1n = GATEUP ? __ldg(sw1) : 0.0f;
             for (int kb = 0; kb < nkb; ++kb, ++ai) {
                 const int slot = ai % C::NSLOT;
                 const uint32_t aph = (ai / C::NSLOT) & 1;
-                const float s0 = __ldg(sw0 + kb);
-                const float s1 = GATEUP ? __ldg(sw1 + kb) : 0.0f;
+                const float s0 = s0n, s1 = s1n;
+                if (kb + 1 < nkb) {
+                    s0n = __ldg(sw0 + kb + 1);
+                    if (GATEUP) s1n = __ldg(sw1 + kb + 1);
+                }
                 const bool ok = mbar_wait(&accf[slot], aph, abort_flag, status, tmo);
                 if (!__all_sync(0xffffffffu, ok)) goto done;
                 tc_fence_after();
-                const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + slot * C::SLOT_COLS;
+                const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + slot * C::SLOT_COLS + cbase;
+                const float *sxk = sxs + kb * BN + cbase;
 #pragma unroll
-                for (int c0 = 0; c0 < BN; c0 += 16) {
+                for (int c0 = 0; c0 < C::CPW; c0 += 16) {
                     float v[16], u[16];
                     tmem_ld16(tb + c0, v);
                     if constexpr (GATEUP) {
@@ -210,8 +238,7 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP>::THREADS, 1)
                     }
 #pragma unroll
                     for (int c = 0; c < 16; ++c) {
-                        const int row = min(tl.row0 + c0 + c, sg.rows - 1);
-                        const float sx = __ldg(sg.sx + (size_t)row * nkb + kb);
+                        const float sx = sxk[c0 + c];
                         acc0[c0 + c] = fmaf(v[c], s0 * sx, acc0[c0 + c]);
                         if constexpr (GATEUP) acc1[c0 + c] = fmaf(u[c], s1 * sx, acc1[c0 + c]);
                     }
@@ -223,14 +250,14 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP>::THREADS, 1)
             float *out = static_cast<float *>(sg.out);
             const int n = tl.nt * kTileM + r;
 #pragma unroll
-            for (int c = 0; c < BN; ++c) {
-                if (c < tl.nrows) {
+            for (int c = 0; c < C::CPW; ++c) {
+                if (cbase + c < tl.nrows) {
                     float v;
                     if constexpr (GATEUP)
                         v = silu_mul(acc0[c], acc1[c]);
                     else
                         v = acc0[c];
-                    out[(size_t)(tl.row0 + c) * sg.N + n] = v;
+                    out[(size_t)(tl.row0 + cbase + c) * sg.N + n] = v;
                 }
             }
         }
@@ -245,11 +272,11 @@ done:
     }
 }
 
-template <int BN, bool GATEUP>
+template <int BN, bool GATEUP, int EW>
 cudaError_t launch_t(const GemmMaps &maps, const GemmArgs &args, int num_sms, cudaStream_t s)
 {
-    using C = Fp8Cfg<BN, GATEUP>;
-    auto kern = gemm_fp8_kernel<BN, GATEUP>;
+    using C = Fp8Cfg<BN, GATEUP, EW>;
+    auto kern = gemm_fp8_kernel<BN, GATEUP, EW>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     return launch_pdl(kern, dim3(num_sms), dim3(C::THREADS), C::SMEM, s, maps, args);
@@ -260,16 +287,20 @@ cudaError_t launch_t(const GemmMaps &maps, const GemmArgs &args, int num_sms, cu
 cudaError_t launch_gemm_fp8(bool gateup, int bn, const GemmMaps &maps, const GemmArgs &args, int num_sms,
                             cudaStream_t s)
 {
+    if (args.seg[0].K > kMaxKb * kBlockK || (args.nseg > 1 && args.seg[1].K > kMaxKb * kBlockK))
+        return cudaErrorInvalidValue;
     if (gateup) {
         switch (bn) {
-            case 32: return launch_t<32, true>(maps, args, num_sms, s);
-            case 64: return launch_t<64, true>(maps, args, num_sms, s);
+            case 32: return launch_t<32, true, 4>(maps, args, num_sms, s);
+            case 64: return launch_t<64, true, 8>(maps, args, num_sms, s);
+            case 128: return launch_t<128, true, 16>(maps, args, num_sms, s);
             default: return cudaErrorInvalidValue;
         }
     }
     switch (bn) {
-        case 32: return launch_t<32, false>(maps, args, num_sms, s);
-        case 64: return launch_t<64, false>(maps, args, num_sms, s);
+        case 32: return launch_t<32, false, 4>(maps, args, num_sms, s);
+        case 64: return launch_t<64, false, 8>(maps, args, num_sms, s);
+        case 128: return launch_t<128, false, 8>(maps, args, num_sms, s);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -16,7 +16,8 @@
 //  * warp 1 issues tcgen05.mma.kind::f16 (BF16 x BF16 -> F32) from one thread: 4 MMAs of
 //    K = 16 per stage per matrix; each 128-element K group (2 stages) accumulates into its own
 //    TMEM slot, because the weight scale changes per (row, group);
-//  * warps 6-9 promote each finished group, acc += D_g * s[row, g] in fp32 registers, and at
+//  * warps 6-13 (two per TMEM lane quarter, each owning half of the token columns) promote
+//    each finished group, acc += D_g * s[row, g] in fp32 registers, and at
 //    the end of the tile write gate|up h = silu(G) * U rounded to bf16 (the 4-bit layer keeps
 //    activations in bf16) or down y in fp32.
 // Multiplying the exact integers on the tensor cores and applying the bf16 scale to fp32
@@ -36,11 +37,12 @@ namespace {
 constexpr int kKE = 64;                // K elements per stage (one 128-byte bf16 swizzle row)
 constexpr int kRawRow = kKE / 2;       // raw bytes per weight row per stage
 constexpr int kConvWarps = 4;
-constexpr int kEpiWarps = 4;
-constexpr int kThreads = 32 * (2 + kConvWarps + kEpiWarps);
 
 template <int BN, bool GATEUP>
 struct I4Cfg {
+    static constexpr int EW = 8;                            // epilogue warps (2 per TMEM quarter)
+    static constexpr int CPW = BN / (EW / 4);               // token columns per epilogue thread
+    static constexpr int THREADS = 32 * (2 + kConvWarps + EW);
     static constexpr int NA = GATEUP ? 2 : 1;
     static constexpr int RAW_BYTES = kTileM * kRawRow;      // 4 KB per matrix
     static constexpr int A_BYTES = kTileM * kKE * 2;        // 16 KB per matrix
@@ -88,7 +90,7 @@ __device__ __forceinline__ uint4 unpack8(uint32_t w)
 }
 
 template <int BN, bool GATEUP>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
     gemm_int4_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmArgs args)
 {
     using C = I4Cfg<BN, GATEUP>;
@@ -117,7 +119,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int s = 0; s < C::NSLOT; ++s) {
             mbar_init(&accf[s], 1);
-            mbar_init(&acce[s], kEpiWarps);
+            mbar_init(&acce[s], C::EW);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -238,7 +240,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------ epilogue ----------------------------------
-        const int q = warp & 3;
+        const int q = warp & 3;                                   // TMEM lane quarter
+        const int cbase = ((warp - 2 - kConvWarps) >> 2) * C::CPW;  // first token column
         const int r = q * 32 + lane;
         uint32_t ai = 0;
         for (int w = blockIdx.x; w < total; w += gridDim.x) {
@@ -248,23 +251,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             const __nv_bfloat16 *sw0 = static_cast<const __nv_bfloat16 *>(sg.sw0) + (size_t)(tl.wrow + r) * ngrp;
             const __nv_bfloat16 *sw1 =
                 GATEUP ? static_cast<const __nv_bfloat16 *>(sg.sw1) + (size_t)(tl.wrow + r) * ngrp : nullptr;
-            float acc0[BN], acc1[GATEUP ? BN : 1];
+            float acc0[C::CPW], acc1[GATEUP ? C::CPW : 1];
 #pragma unroll
-            for (int c = 0; c < BN; ++c) acc0[c] = 0.0f;
+            for (int c = 0; c < C::CPW; ++c) acc0[c] = 0.0f;
             if constexpr (GATEUP) {
 #pragma unroll
-                for (int c = 0; c < BN; ++c) acc1[c] = 0.0f;
+                for (int c = 0; c < C::CPW; ++c) acc1[c] = 0.0f;
             }
+            float s0n = __bfloat162float(sw0[0]), s1n = GATEUP ? __bfloat162float(sw1[0]) : 0.0f;
             for (int g = 0; g < ngrp; ++g, ++ai) {
                 const int slot = ai % C::NSLOT;
-                const float s0 = __bfloat162float(sw0[g]);
-                const float s1 = GATEUP ? __bfloat162float(sw1[g]) : 0.0f;
+                const float s0 = s0n, s1 = s1n;
+                if (g + 1 < ngrp) {
+                    s0n = __bfloat162float(sw0[g + 1]);
+                    if (GATEUP) s1n = __bfloat162float(sw1[g + 1]);
+                }
                 const bool ok = mbar_wait(&accf[slot], (ai / C::NSLOT) & 1, abort_flag, status, tmo);
                 if (!__all_sync(0xffffffffu, ok)) goto done;
                 tc_fence_after();
-                const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + slot * C::SLOT_COLS;
+                const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + slot * C::SLOT_COLS + cbase;
 #pragma unroll
-                for (int c0 = 0; c0 < BN; c0 += 16) {
+                for (int c0 = 0; c0 < C::CPW; c0 += 16) {
                     float v[16], u[16];
                     tmem_ld16(tb + c0, v);
                     if constexpr (GATEUP) {
@@ -285,9 +292,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const int n = tl.nt * kTileM + r;
 #pragma unroll
-            for (int c = 0; c < BN; ++c) {
-                if (c < tl.nrows) {
-                    const size_t o = (size_t)(tl.row0 + c) * sg.N + n;
+            for (int c = 0; c < C::CPW; ++c) {
+                if (cbase + c < tl.nrows) {
+                    const size_t o = (size_t)(tl.row0 + cbase + c) * sg.N + n;
                     if constexpr (GATEUP)
                         static_cast<__nv_bfloat16 *>(sg.out)[o] = __float2bfloat16_rn(silu_mul(acc0[c], acc1[c]));
                     else
@@ -313,7 +320,7 @@ cudaError_t launch_t(const GemmMaps &maps, const GemmArgs &args, int num_sms, cu
     auto kern = gemm_int4_kernel<BN, GATEUP>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
-    return launch_pdl(kern, dim3(num_sms), dim3(kThreads), C::SMEM, s, maps, args);
+    return launch_pdl(kern, dim3(num_sms), dim3(C::THREADS), C::SMEM, s, maps, args);
 }
 
 }  // namespace
