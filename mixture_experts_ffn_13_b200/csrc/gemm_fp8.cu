@@ -145,10 +145,13 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
     } else if (warp == 1) {
         // ------------------------------ MMA issuer --------------------------------
         if (lane == 0) {
-            constexpr uint32_t kIdesc = instr_desc(kTileM, BN, 0, 0);
             uint32_t it = 0, ai = 0;
             for (int w = blockIdx.x; w < total; w += gridDim.x) {
                 const TileInfo tl = decode_tile<BN>(args, w, tot0);
+                // MMA N = the tile's valid rows rounded up to 16: a group's last, partial
+                // token tile costs no tensor-core work for the rows it does not have
+                const int n_mma = min(BN, (tl.nrows + 15) & ~15);
+                const uint32_t kIdesc = instr_desc(kTileM, n_mma, 0, 0);
                 const int K = args.seg[tl.seg].K;
                 const int nkc = K / kKC;
                 const int nkb = (K + kBlockK - 1) / kBlockK;
@@ -293,7 +296,7 @@ cudaError_t launch_gemm_fp8(bool gateup, int bn, const GemmMaps &maps, const Gem
         switch (bn) {
             case 32: return launch_t<32, true, 4>(maps, args, num_sms, s);
             case 64: return launch_t<64, true, 8>(maps, args, num_sms, s);
-            case 128: return launch_t<128, true, 16>(maps, args, num_sms, s);
+            case 128: return launch_t<128, true, 8>(maps, args, num_sms, s);
             default: return cudaErrorInvalidValue;
         }
     }

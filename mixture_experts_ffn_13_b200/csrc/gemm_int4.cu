@@ -11,8 +11,9 @@
 //  * warps 2-5 (one thread per weight row) turn each raw tile into the integers q as bf16
 //    (exact: |q| <= 8) in the 128-byte-swizzled K-major layout the MMA reads: flip each
 //    nibble's sign bit, place it in the mantissa of the bf16 value 128 (so it reads
-//    128 + q + 8), subtract 136, store 16 bytes per 8 values at the swizzled chunk; the first
-//    of these warps also loads the stage's activation tile (bf16, TMA);
+//    128 + q + 8), subtract 136, store 16 bytes per 8 values at the swizzled chunk; the
+//    activation tiles (bf16) come by TMA through their own ring, issued by warp 0 with the
+//    raw weights, so they arrive as far ahead as the weights do;
 //  * warp 1 issues tcgen05.mma.kind::f16 (BF16 x BF16 -> F32) from one thread: 4 MMAs of
 //    K = 16 per stage per matrix; each 128-element K group (2 stages) accumulates into its own
 //    TMEM slot, because the weight scale changes per (row, group);
@@ -47,14 +48,14 @@ struct I4Cfg {
     static constexpr int RAW_BYTES = kTileM * kRawRow;      // 4 KB per matrix
     static constexpr int A_BYTES = kTileM * kKE * 2;        // 16 KB per matrix
     static constexpr int B_BYTES = BN * kKE * 2;
-    static constexpr int NR = 8;                            // raw stages
-    static constexpr int MSTAGE = NA * A_BYTES + B_BYTES;
-    static constexpr int NM = GATEUP ? 3 : 4;               // MMA stages
+    static constexpr int NR = GATEUP ? 6 : 8;               // raw weight + activation stages
+    static constexpr int MSTAGE = NA * A_BYTES;             // converted weight stage
+    static constexpr int NM = GATEUP ? 3 : 4;               // converted stages
     static constexpr int SLOT_COLS = NA * BN;               // one 128-element K group
     static constexpr int NSLOT = 512 / SLOT_COLS;
     static constexpr int STAGES_PER_GROUP = kGroupK / kKE;  // 2
-    static constexpr int BAR_BYTES = 8 * (2 * NR + 2 * NM + 2 * NSLOT) + 16;
-    static constexpr int SMEM = 1024 + NM * MSTAGE + NR * NA * RAW_BYTES + BAR_BYTES;
+    static constexpr int BAR_BYTES = 8 * (4 * NR + 2 * NM + 2 * NSLOT) + 16;
+    static constexpr int SMEM = 1024 + NM * MSTAGE + NR * B_BYTES + NR * NA * RAW_BYTES + BAR_BYTES;
     static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "1024-byte aligned tiles");
     static_assert(SMEM <= 227 * 1024, "shared memory");
 };
@@ -96,11 +97,14 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
     using C = I4Cfg<BN, GATEUP>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *mst = smem;                                   // NM MMA stages [A0 | A1 | B]
-    uint8_t *raw = smem + C::NM * C::MSTAGE;               // NR raw stages [raw0 | raw1]
+    uint8_t *mst = smem;                                   // NM converted stages [A0 | A1]
+    uint8_t *bst = smem + C::NM * C::MSTAGE;               // NR activation stages
+    uint8_t *raw = bst + C::NR * C::B_BYTES;               // NR raw stages [raw0 | raw1]
     uint64_t *rfull = reinterpret_cast<uint64_t *>(raw + C::NR * C::NA * C::RAW_BYTES);
     uint64_t *rempty = rfull + C::NR;
-    uint64_t *mfull = rempty + C::NR;
+    uint64_t *bfull = rempty + C::NR;
+    uint64_t *bempty = bfull + C::NR;
+    uint64_t *mfull = bempty + C::NR;
     uint64_t *mempty = mfull + C::NM;
     uint64_t *accf = mempty + C::NM;
     uint64_t *acce = accf + C::NSLOT;
@@ -112,9 +116,11 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
         for (int s = 0; s < C::NR; ++s) {
             mbar_init(&rfull[s], 1);
             mbar_init(&rempty[s], kConvWarps);
+            mbar_init(&bfull[s], 1);
+            mbar_init(&bempty[s], 1);
         }
         for (int s = 0; s < C::NM; ++s) {
-            mbar_init(&mfull[s], kConvWarps + 1);
+            mbar_init(&mfull[s], kConvWarps);
             mbar_init(&mempty[s], 1);
         }
         for (int s = 0; s < C::NSLOT; ++s) {
@@ -143,9 +149,10 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
     const uint64_t tmo = args.timeout_ns;
 
     if (warp == 0) {
-        // ------------------------------ raw weight producer -----------------------
+        // --------------------- raw weight + activation producer ---------------------
         if (lane == 0) {
             const uint64_t pol_w = l2_policy_evict_first();
+            const uint64_t pol_x = l2_policy_evict_last();
             uint32_t it = 0;
             for (int w = blockIdx.x; w < total; w += gridDim.x) {
                 const TileInfo tl = decode_tile<BN>(args, w, tot0);
@@ -159,16 +166,20 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
                     tma_load_2d_hint(rs, &maps.a0[tl.seg], &rfull[s], kc * kRawRow, tl.wrow, pol_w);
                     if (GATEUP)
                         tma_load_2d_hint(rs + C::RAW_BYTES, &maps.a1[tl.seg], &rfull[s], kc * kRawRow, tl.wrow, pol_w);
+                    if (!mbar_wait(&bempty[s], ph ^ 1, abort_flag, status, tmo)) goto done;
+                    mbar_arrive_expect_tx(&bfull[s], C::B_BYTES);
+                    tma_load_2d_hint(bst + s * C::B_BYTES, &maps.b[tl.seg], &bfull[s], kc * kKE, tl.row0, pol_x);
                 }
             }
         }
     } else if (warp == 1) {
         // ------------------------------ MMA issuer --------------------------------
         if (lane == 0) {
-            constexpr uint32_t kIdesc = instr_desc(kTileM, BN, 1, 1);
             uint32_t it = 0, ai = 0;
             for (int w = blockIdx.x; w < total; w += gridDim.x) {
                 const TileInfo tl = decode_tile<BN>(args, w, tot0);
+                const int n_mma = min(BN, (tl.nrows + 15) & ~15);  // partial tiles: no work on absent rows
+                const uint32_t kIdesc = instr_desc(kTileM, n_mma, 1, 1);
                 const int ngrp = args.seg[tl.seg].K / kGroupK;
                 for (int g = 0; g < ngrp; ++g, ++ai) {
                     const int slot = ai % C::NSLOT;
@@ -178,12 +189,14 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
                     const uint32_t d1 = d0 + BN;
                     for (int sk = 0; sk < C::STAGES_PER_GROUP; ++sk, ++it) {
                         const int s = it % C::NM;
+                        const int bs = it % C::NR;
                         if (!mbar_wait(&mfull[s], (it / C::NM) & 1, abort_flag, status, tmo)) goto done;
+                        if (!mbar_wait(&bfull[bs], (it / C::NR) & 1, abort_flag, status, tmo)) goto done;
                         tc_fence_after();
                         uint8_t *st = mst + s * C::MSTAGE;
                         const uint64_t da0 = smem_desc_sw128(st);
                         const uint64_t da1 = smem_desc_sw128(st + C::A_BYTES);
-                        const uint64_t db = smem_desc_sw128(st + C::NA * C::A_BYTES);
+                        const uint64_t db = smem_desc_sw128(bst + bs * C::B_BYTES);
 #pragma unroll
                         for (int kk = 0; kk < kKE / 16; ++kk) {
                             const uint32_t acc = (sk > 0 || kk > 0) ? 1u : 0u;
@@ -191,6 +204,7 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
                             if (GATEUP) mma_bf16(d1, da1 + 2 * kk, db + 2 * kk, kIdesc, acc);
                         }
                         mma_commit(&mempty[s]);
+                        mma_commit(&bempty[bs]);
                     }
                     mma_commit(&accf[slot]);
                 }
@@ -211,11 +225,6 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
                 bool ok = mbar_wait(&mempty[ms_i], ((it / C::NM) & 1) ^ 1, abort_flag, status, tmo);
                 if (!__all_sync(0xffffffffu, ok)) goto done;
                 uint8_t *st = mst + ms_i * C::MSTAGE;
-                if (cw == 0 && lane == 0) {
-                    mbar_arrive_expect_tx(&mfull[ms_i], C::B_BYTES);
-                    tma_load_2d_hint(st + C::NA * C::A_BYTES, &maps.b[tl.seg], &mfull[ms_i], kc * kKE, tl.row0,
-                                     l2_policy_evict_last());
-                }
                 ok = mbar_wait(&rfull[rs_i], (it / C::NR) & 1, abort_flag, status, tmo);
                 if (!__all_sync(0xffffffffu, ok)) goto done;
                 const uint8_t *rs = raw + rs_i * C::NA * C::RAW_BYTES;

@@ -106,11 +106,15 @@ int fail_cuda(moe_plan_t *p, cudaError_t e)
     return MOE_ERR_CUDA;
 }
 
-// Tile size along the token dimension for a given token count per group.
-int pick_bn(int T, int k, int E)
+// Tile size along the token dimension from the mean rows per expert group: decode-sized
+// groups take 32-row tiles; larger groups take wider tiles so each weight tile staged in
+// shared memory feeds more MMA work (the 4-bit kernel stops at 64).
+int pick_bn(int T, int k, int E, bool fp8)
 {
     const long avg = ((long)T * k + E - 1) / E;
-    return avg > 48 ? 64 : 32;
+    if (avg <= 48) return 32;
+    if (avg <= 96 || !fp8) return 64;
+    return 128;
 }
 
 }  // namespace
@@ -284,7 +288,7 @@ int moe_route(moe_plan_t *p, int32_t T, const float *logits, int32_t *topk_idx, 
     b.offsets = offsets;
     b.perm_tok = perm_tok;
     cudaStream_t s = (cudaStream_t)stream;
-    const int bn = pick_bn(T, d.k, d.E);
+    const int bn = pick_bn(T, d.k, d.E, d.wfmt == MOE_W_FP8_SC512);
     p->launches = 0;
     cudaError_t e = launch_route_permute(logits, b, T, d.E, d.k, bn, bn, s);
     p->launches = route_permute_launches(T, d.E, d.k);
@@ -306,7 +310,7 @@ static int forward_int4(moe_plan_t *p, int T, const uint16_t *x, const float *lo
     const int H = d.H, I = d.I, Is = d.I_shared, k = d.k, E = d.E;
     const bool shared = Is > 0;
     const int A = T * k;
-    const int bn = pick_bn(T, k, E);
+    const int bn = pick_bn(T, k, E, false);
     mark(0);
     cudaError_t e = launch_route(logits, T, E, k, b.topk_idx, b.topk_w, s);
     mark(1);
@@ -404,7 +408,7 @@ int moe_forward(moe_plan_t *p, int32_t T, const uint16_t *x, const float *logits
     const RouteBufs b = route_bufs(L, ws);
     const int H = d.H, I = d.I, Is = d.I_shared, k = d.k, E = d.E;
     const int A = T * k;
-    const int bn_a = pick_bn(T, k, E), bn_b = bn_a;
+    const int bn_a = pick_bn(T, k, E, true), bn_b = bn_a;
 
     mark(0);
     cudaError_t e = launch_route(logits, T, E, k, b.topk_idx, b.topk_w, s);
