@@ -193,19 +193,53 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
         const int etid = ew * 32 + lane;      // index among the epilogue threads
         uint32_t ai = 0;
         int ti = 0;
+        // The tile's activation scales s_x[row0 + c, kb] live in shared memory (two buffers,
+        // alternating by tile).  The next tile's values are loaded into registers while the
+        // current tile is promoted, and stored at the end of it, so no tile waits on them.
+        constexpr int NPF = (BN * kMaxKb) / (32 * EW);
+        float pf[NPF];
+        auto load_sx = [&](const TileInfo &t) {
+            const GemmSeg &g = args.seg[t.seg];
+            const int nk = (g.K + kBlockK - 1) / kBlockK;
+#pragma unroll
+            for (int j = 0; j < NPF; ++j) {
+                const int i = etid + j * 32 * EW;
+                if (i < BN * nk) {
+                    const int c = i / nk, kb = i - c * nk;
+                    const int row = min(t.row0 + c, g.rows - 1);
+                    pf[j] = __ldg(g.sx + (size_t)row * nk + kb);
+                }
+            }
+        };
+        auto store_sx = [&](const TileInfo &t, float *dst) {
+            const int nk = (args.seg[t.seg].K + kBlockK - 1) / kBlockK;
+#pragma unroll
+            for (int j = 0; j < NPF; ++j) {
+                const int i = etid + j * 32 * EW;
+                if (i < BN * nk) {
+                    const int c = i / nk, kb = i - c * nk;
+                    dst[kb * BN + c] = pf[j];
+                }
+            }
+        };
+        if ((int)blockIdx.x < total) {
+            const TileInfo t0 = decode_tile<BN>(args, blockIdx.x, tot0);
+            load_sx(t0);
+            store_sx(t0, sxbuf);
+        }
+        epi_sync(32 * EW);
         for (int w = blockIdx.x; w < total; w += gridDim.x, ++ti) {
             const TileInfo tl = decode_tile<BN>(args, w, tot0);
             const GemmSeg &sg = args.seg[tl.seg];
             const int K = sg.K;
             const int nkb = (K + kBlockK - 1) / kBlockK;
-            // stage s_x[row0 + c, kb] (rows past the segment read its last row; unused)
-            float *sxs = sxbuf + (ti & 1) * (BN * kMaxKb);
-            for (int i = etid; i < BN * nkb; i += 32 * EW) {
-                const int c = i / nkb, kb = i - c * nkb;
-                const int row = min(tl.row0 + c, sg.rows - 1);
-                sxs[kb * BN + c] = __ldg(sg.sx + (size_t)row * nkb + kb);
+            const float *sxs = sxbuf + (ti & 1) * (BN * kMaxKb);
+            const int wn = w + gridDim.x;
+            TileInfo tn;
+            if (wn < total) {
+                tn = decode_tile<BN>(args, wn, tot0);
+                load_sx(tn);
             }
-            epi_sync(32 * EW);
             const float *sw0 = static_cast<const float *>(sg.sw0) + (size_t)(tl.wrow + r) * nkb;
             const float *sw1 = GATEUP ? static_cast<const float *>(sg.sw1) + (size_t)(tl.wrow + r) * nkb : nullptr;
             float acc0[C::CPW], acc1[GATEUP ? C::CPW : 1];
@@ -263,6 +297,8 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
                     out[(size_t)(tl.row0 + cbase + c) * sg.N + n] = v;
                 }
             }
+            if (wn < total) store_sx(tn, sxbuf + ((ti + 1) & 1) * (BN * kMaxKb));
+            epi_sync(32 * EW);
         }
     }
 done:
@@ -296,7 +332,6 @@ cudaError_t launch_gemm_fp8(bool gateup, int bn, const GemmMaps &maps, const Gem
         switch (bn) {
             case 32: return launch_t<32, true, 4>(maps, args, num_sms, s);
             case 64: return launch_t<64, true, 8>(maps, args, num_sms, s);
-            case 128: return launch_t<128, true, 8>(maps, args, num_sms, s);
             default: return cudaErrorInvalidValue;
         }
     }

@@ -6,9 +6,11 @@
 // can use them; on consumer GPUs that decompress-then-FMA runs on the CUDA cores with the
 // tensor cores idle.  Here the decompression feeds the tensor cores instead, and keeps the
 // weights exact:
-//  * warp 0 streams raw int4 weight tiles (128 rows x 32 bytes = 64 K-elements per matrix) by
-//    TMA into a deep ring of raw stages (evict-first);
-//  * warps 2-5 (one thread per weight row) turn each raw tile into the integers q as bf16
+//  * warp 0 streams raw int4 weight tiles (128 rows x 128 bytes = 256 K-elements per matrix,
+//    128-byte swizzle; narrower boxes make the TMA issue-bound) by TMA into a ring of raw stages
+//    (evict-first);
+//  * warps 2-5 (one thread per weight row) turn each raw tile, 64 K-elements at a time, into
+//    the integers q as bf16
 //    (exact: |q| <= 8) in the 128-byte-swizzled K-major layout the MMA reads: flip each
 //    nibble's sign bit, place it in the mantissa of the bf16 value 128 (so it reads
 //    128 + q + 8), subtract 136, store 16 bytes per 8 values at the swizzled chunk; the
@@ -35,8 +37,9 @@ namespace moe {
 
 namespace {
 
-constexpr int kKE = 64;                // K elements per stage (one 128-byte bf16 swizzle row)
-constexpr int kRawRow = kKE / 2;       // raw bytes per weight row per stage
+constexpr int kKE = 64;                // K elements per MMA stage (one 128-byte bf16 swizzle row)
+constexpr int kRawKE = 256;            // K elements per raw weight stage (128 bytes per row)
+constexpr int kSubs = kRawKE / kKE;    // MMA stages per raw stage
 constexpr int kConvWarps = 4;
 
 template <int BN, bool GATEUP>
@@ -45,17 +48,18 @@ struct I4Cfg {
     static constexpr int CPW = BN / (EW / 4);               // token columns per epilogue thread
     static constexpr int THREADS = 32 * (2 + kConvWarps + EW);
     static constexpr int NA = GATEUP ? 2 : 1;
-    static constexpr int RAW_BYTES = kTileM * kRawRow;      // 4 KB per matrix
+    static constexpr int RAW_BYTES = kTileM * (kRawKE / 2);  // 16 KB per matrix
     static constexpr int A_BYTES = kTileM * kKE * 2;        // 16 KB per matrix
     static constexpr int B_BYTES = BN * kKE * 2;
-    static constexpr int NR = GATEUP ? 6 : 8;               // raw weight + activation stages
+    static constexpr int NR = GATEUP ? 2 : 4;               // raw weight stages (256 K each)
+    static constexpr int NB = GATEUP ? 6 : 8;               // activation stages (64 K each)
     static constexpr int MSTAGE = NA * A_BYTES;             // converted weight stage
     static constexpr int NM = GATEUP ? 3 : 4;               // converted stages
     static constexpr int SLOT_COLS = NA * BN;               // one 128-element K group
     static constexpr int NSLOT = 512 / SLOT_COLS;
     static constexpr int STAGES_PER_GROUP = kGroupK / kKE;  // 2
-    static constexpr int BAR_BYTES = 8 * (4 * NR + 2 * NM + 2 * NSLOT) + 16;
-    static constexpr int SMEM = 1024 + NM * MSTAGE + NR * B_BYTES + NR * NA * RAW_BYTES + BAR_BYTES;
+    static constexpr int BAR_BYTES = 8 * (2 * NR + 2 * NB + 2 * NM + 2 * NSLOT) + 16;
+    static constexpr int SMEM = 1024 + NM * MSTAGE + NB * B_BYTES + NR * NA * RAW_BYTES + BAR_BYTES;
     static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "1024-byte aligned tiles");
     static_assert(SMEM <= 227 * 1024, "shared memory");
 };
@@ -98,13 +102,13 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *mst = smem;                                   // NM converted stages [A0 | A1]
-    uint8_t *bst = smem + C::NM * C::MSTAGE;               // NR activation stages
-    uint8_t *raw = bst + C::NR * C::B_BYTES;               // NR raw stages [raw0 | raw1]
-    uint64_t *rfull = reinterpret_cast<uint64_t *>(raw + C::NR * C::NA * C::RAW_BYTES);
+    uint8_t *raw = smem + C::NM * C::MSTAGE;               // NR raw stages [raw0 | raw1]
+    uint8_t *bst = raw + C::NR * C::NA * C::RAW_BYTES;     // NB activation stages
+    uint64_t *rfull = reinterpret_cast<uint64_t *>(bst + C::NB * C::B_BYTES);
     uint64_t *rempty = rfull + C::NR;
     uint64_t *bfull = rempty + C::NR;
-    uint64_t *bempty = bfull + C::NR;
-    uint64_t *mfull = bempty + C::NR;
+    uint64_t *bempty = bfull + C::NB;
+    uint64_t *mfull = bempty + C::NB;
     uint64_t *mempty = mfull + C::NM;
     uint64_t *accf = mempty + C::NM;
     uint64_t *acce = accf + C::NSLOT;
@@ -116,6 +120,8 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
         for (int s = 0; s < C::NR; ++s) {
             mbar_init(&rfull[s], 1);
             mbar_init(&rempty[s], kConvWarps);
+        }
+        for (int s = 0; s < C::NB; ++s) {
             mbar_init(&bfull[s], 1);
             mbar_init(&bempty[s], 1);
         }
@@ -153,22 +159,27 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
         if (lane == 0) {
             const uint64_t pol_w = l2_policy_evict_first();
             const uint64_t pol_x = l2_policy_evict_last();
-            uint32_t it = 0;
+            uint32_t it = 0, rt = 0;  // MMA-stage and raw-stage counters
             for (int w = blockIdx.x; w < total; w += gridDim.x) {
                 const TileInfo tl = decode_tile<BN>(args, w, tot0);
                 const int nkc = args.seg[tl.seg].K / kKE;
                 for (int kc = 0; kc < nkc; ++kc, ++it) {
-                    const int s = it % C::NR;
-                    const uint32_t ph = (it / C::NR) & 1;
-                    if (!mbar_wait(&rempty[s], ph ^ 1, abort_flag, status, tmo)) goto done;
-                    uint8_t *rs = raw + s * C::NA * C::RAW_BYTES;
-                    mbar_arrive_expect_tx(&rfull[s], C::NA * C::RAW_BYTES);
-                    tma_load_2d_hint(rs, &maps.a0[tl.seg], &rfull[s], kc * kRawRow, tl.wrow, pol_w);
-                    if (GATEUP)
-                        tma_load_2d_hint(rs + C::RAW_BYTES, &maps.a1[tl.seg], &rfull[s], kc * kRawRow, tl.wrow, pol_w);
-                    if (!mbar_wait(&bempty[s], ph ^ 1, abort_flag, status, tmo)) goto done;
-                    mbar_arrive_expect_tx(&bfull[s], C::B_BYTES);
-                    tma_load_2d_hint(bst + s * C::B_BYTES, &maps.b[tl.seg], &bfull[s], kc * kKE, tl.row0, pol_x);
+                    if (kc % kSubs == 0) {
+                        // raw weights for the next 256 K-elements (the last stage of a K that is
+                        // not a multiple of 256 reads zeros past the end)
+                        const int s = rt % C::NR;
+                        if (!mbar_wait(&rempty[s], ((rt / C::NR) & 1) ^ 1, abort_flag, status, tmo)) goto done;
+                        uint8_t *rs = raw + s * C::NA * C::RAW_BYTES;
+                        mbar_arrive_expect_tx(&rfull[s], C::NA * C::RAW_BYTES);
+                        const int x = (kc / kSubs) * (kRawKE / 2);
+                        tma_load_2d_hint(rs, &maps.a0[tl.seg], &rfull[s], x, tl.wrow, pol_w);
+                        if (GATEUP) tma_load_2d_hint(rs + C::RAW_BYTES, &maps.a1[tl.seg], &rfull[s], x, tl.wrow, pol_w);
+                        ++rt;
+                    }
+                    const int b = it % C::NB;
+                    if (!mbar_wait(&bempty[b], ((it / C::NB) & 1) ^ 1, abort_flag, status, tmo)) goto done;
+                    mbar_arrive_expect_tx(&bfull[b], C::B_BYTES);
+                    tma_load_2d_hint(bst + b * C::B_BYTES, &maps.b[tl.seg], &bfull[b], kc * kKE, tl.row0, pol_x);
                 }
             }
         }
@@ -189,9 +200,9 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
                     const uint32_t d1 = d0 + BN;
                     for (int sk = 0; sk < C::STAGES_PER_GROUP; ++sk, ++it) {
                         const int s = it % C::NM;
-                        const int bs = it % C::NR;
+                        const int bs = it % C::NB;
                         if (!mbar_wait(&mfull[s], (it / C::NM) & 1, abort_flag, status, tmo)) goto done;
-                        if (!mbar_wait(&bfull[bs], (it / C::NR) & 1, abort_flag, status, tmo)) goto done;
+                        if (!mbar_wait(&bfull[bs], (it / C::NB) & 1, abort_flag, status, tmo)) goto done;
                         tc_fence_after();
                         uint8_t *st = mst + s * C::MSTAGE;
                         const uint64_t da0 = smem_desc_sw128(st);
@@ -214,24 +225,29 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
         // ------------------------------ dequantisers ------------------------------
         const int cw = warp - 2;
         const int r = cw * 32 + lane;  // weight row of the tile handled by this thread
-        uint32_t it = 0;
+        uint32_t it = 0, rt = 0;
         for (int w = blockIdx.x; w < total; w += gridDim.x) {
             const TileInfo tl = decode_tile<BN>(args, w, tot0);
             const GemmSeg &sg = args.seg[tl.seg];
             const int nkc = sg.K / kKE;
             for (int kc = 0; kc < nkc; ++kc, ++it) {
-                const int rs_i = it % C::NR;
+                const int sub = kc % kSubs;
+                const int rs_i = rt % C::NR;
                 const int ms_i = it % C::NM;
-                bool ok = mbar_wait(&mempty[ms_i], ((it / C::NM) & 1) ^ 1, abort_flag, status, tmo);
+                bool ok = true;
+                if (sub == 0) ok = mbar_wait(&rfull[rs_i], (rt / C::NR) & 1, abort_flag, status, tmo);
+                if (!__all_sync(0xffffffffu, ok)) goto done;
+                ok = mbar_wait(&mempty[ms_i], ((it / C::NM) & 1) ^ 1, abort_flag, status, tmo);
                 if (!__all_sync(0xffffffffu, ok)) goto done;
                 uint8_t *st = mst + ms_i * C::MSTAGE;
-                ok = mbar_wait(&rfull[rs_i], (it / C::NR) & 1, abort_flag, status, tmo);
-                if (!__all_sync(0xffffffffu, ok)) goto done;
-                const uint8_t *rs = raw + rs_i * C::NA * C::RAW_BYTES;
+                const uint8_t *rs = raw + rs_i * C::NA * C::RAW_BYTES + r * 128;
+                // this sub-stage's 32 raw bytes are 16-byte chunks 2*sub and 2*sub+1 of the row,
+                // stored by the 128-byte swizzle at chunk positions (c ^ (r & 7))
+                const int c0 = ((2 * sub) ^ (r & 7)) << 4, c1 = ((2 * sub + 1) ^ (r & 7)) << 4;
 #pragma unroll
                 for (int m = 0; m < C::NA; ++m) {
-                    const uint4 *src = reinterpret_cast<const uint4 *>(rs + m * C::RAW_BYTES + r * kRawRow);
-                    const uint4 q0 = src[0], q1 = src[1];
+                    const uint4 q0 = *reinterpret_cast<const uint4 *>(rs + m * C::RAW_BYTES + c0);
+                    const uint4 q1 = *reinterpret_cast<const uint4 *>(rs + m * C::RAW_BYTES + c1);
                     uint8_t *dst = st + m * C::A_BYTES + r * 128;
                     const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
@@ -241,10 +257,12 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
                 // make the generic-proxy shared-memory writes visible to the tensor core
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
+                const bool raw_done = (sub == kSubs - 1) || (kc == nkc - 1);
                 if (lane == 0) {
-                    mbar_arrive(&rempty[rs_i]);
                     mbar_arrive(&mfull[ms_i]);
+                    if (raw_done) mbar_arrive(&rempty[rs_i]);
                 }
+                if (raw_done) ++rt;
             }
         }
     } else {

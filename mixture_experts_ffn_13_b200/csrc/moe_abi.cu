@@ -339,13 +339,13 @@ static int forward_int4(moe_plan_t *p, int T, const uint16_t *x, const float *lo
     ag.status = p->d_status;
     ag.timeout_ns = kDefaultTimeoutNs;
     ag.seg[0] = GemmSeg{I, H, A, w->s_gate, w->s_up, nullptr, h};
-    int rc = encode_map_2d(&mg.a0[0], w->w_gate, U8, 1, H / 2, (uint64_t)E * I, 32, 128, false);
-    rc |= encode_map_2d(&mg.a1[0], w->w_up, U8, 1, H / 2, (uint64_t)E * I, 32, 128, false);
+    int rc = encode_map_2d(&mg.a0[0], w->w_gate, U8, 1, H / 2, (uint64_t)E * I, 128, 128, true);
+    rc |= encode_map_2d(&mg.a1[0], w->w_up, U8, 1, H / 2, (uint64_t)E * I, 128, 128, true);
     rc |= encode_map_2d(&mg.b[0], xp, BF, 2, H, A, 64, bn, true);
     if (shared) {
         ag.seg[1] = GemmSeg{Is, H, T, w->ss_gate, w->ss_up, nullptr, h_sh};
-        rc |= encode_map_2d(&mg.a0[1], w->ws_gate, U8, 1, H / 2, Is, 32, 128, false);
-        rc |= encode_map_2d(&mg.a1[1], w->ws_up, U8, 1, H / 2, Is, 32, 128, false);
+        rc |= encode_map_2d(&mg.a0[1], w->ws_gate, U8, 1, H / 2, Is, 128, 128, true);
+        rc |= encode_map_2d(&mg.a1[1], w->ws_up, U8, 1, H / 2, Is, 128, 128, true);
         rc |= encode_map_2d(&mg.b[1], xp_sh, BF, 2, H, T, 64, bn, true);
     }
     if (rc) return MOE_ERR_CUDA;
@@ -358,11 +358,11 @@ static int forward_int4(moe_plan_t *p, int T, const uint16_t *x, const float *lo
     GemmArgs ad = ag;
     ad.ttile = b.ttile_b;
     ad.seg[0] = GemmSeg{H, I, A, w->s_down, nullptr, nullptr, y};
-    rc = encode_map_2d(&md.a0[0], w->w_down, U8, 1, I / 2, (uint64_t)E * H, 32, 128, false);
+    rc = encode_map_2d(&md.a0[0], w->w_down, U8, 1, I / 2, (uint64_t)E * H, 128, 128, true);
     rc |= encode_map_2d(&md.b[0], h, BF, 2, I, A, 64, bn, true);
     if (shared) {
         ad.seg[1] = GemmSeg{H, Is, T, w->ss_down, nullptr, nullptr, y_sh};
-        rc |= encode_map_2d(&md.a0[1], w->ws_down, U8, 1, Is / 2, H, 32, 128, false);
+        rc |= encode_map_2d(&md.a0[1], w->ws_down, U8, 1, Is / 2, H, 128, 128, true);
         rc |= encode_map_2d(&md.b[1], h_sh, BF, 2, Is, T, 64, bn, true);
     }
     if (rc) return MOE_ERR_CUDA;
@@ -408,7 +408,8 @@ int moe_forward(moe_plan_t *p, int32_t T, const uint16_t *x, const float *logits
     const RouteBufs b = route_bufs(L, ws);
     const int H = d.H, I = d.I, Is = d.I_shared, k = d.k, E = d.E;
     const int A = T * k;
-    const int bn_a = pick_bn(T, k, E, true), bn_b = bn_a;
+    const int bn_b = pick_bn(T, k, E, true);
+    const int bn_a = bn_b > 64 ? 64 : bn_b;  // gate|up holds two accumulators per column
 
     mark(0);
     cudaError_t e = launch_route(logits, T, E, k, b.topk_idx, b.topk_w, s);
