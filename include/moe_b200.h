@@ -95,7 +95,7 @@ typedef struct moe_plan_s moe_plan_t; /* opaque; owned by the library until moe_
 /* Validate the dimensions, choose tile shapes and report the workspace size the later calls
  * need for any T <= T_max.  Launches no kernel.  Allocates one small device status word on
  * the current device (the plan is bound to that device).
- * Supported: 1 <= E <= 1024; 1 <= k <= min(E, 32); H, I, I_shared multiples of 128;
+ * Supported: 1 <= E <= 1024; 1 <= k <= min(E, 32); H, I, I_shared multiples of 128, <= 8192;
  * 1 <= T_max <= 2^20.  Returns MOE_ERR_INVALID_ARG for NULL outputs or non-positive sizes,
  * MOE_ERR_UNSUPPORTED for shapes outside that set. */
 MOE_API int moe_plan(const moe_dims *dims, moe_plan_t **out_plan, size_t *workspace_bytes);

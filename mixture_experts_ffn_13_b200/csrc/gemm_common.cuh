@@ -19,8 +19,10 @@ struct TileInfo {
 // Work item w -> tile.  Routed items come first: group g owns items
 // [ttile[g]*nT, ttile[g+1]*nT), laid out n-tile major so consecutive items reuse the same
 // weight tile across the group's token tiles.  Shared-expert items follow.
+// `stt` is a shared-memory copy of a.ttile (E+1 entries), so the binary search costs shared
+// loads only; a chain of dependent global loads per tile would stall the TMA producer.
 template <int BN>
-__device__ __forceinline__ TileInfo decode_tile(const GemmArgs &a, int w, int tot0)
+__device__ __forceinline__ TileInfo decode_tile(const GemmArgs &a, const int *stt, int w, int tot0)
 {
     TileInfo t;
     if (w < tot0) {
@@ -28,14 +30,14 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs &a, int w, int to
         int lo = 0, hi = a.E - 1;
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
-            if (__ldg(a.ttile + mid) * nT <= w)
+            if (stt[mid] * nT <= w)
                 lo = mid;
             else
                 hi = mid - 1;
         }
         const int g = lo;
-        const int t0 = __ldg(a.ttile + g);
-        const int ntt = __ldg(a.ttile + g + 1) - t0;
+        const int t0 = stt[g];
+        const int ntt = stt[g + 1] - t0;
         const int local = w - t0 * nT;
         const int nt = local / ntt;
         const int tt = local - nt * ntt;
@@ -58,6 +60,13 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs &a, int w, int to
         t.wrow = nt * kTileM;
     }
     return t;
+}
+
+// Copy a.ttile into shared memory (all threads of the CTA take part; call after griddep_wait).
+__device__ __forceinline__ void load_ttile(const GemmArgs &a, int *stt)
+{
+    for (int i = threadIdx.x; i <= a.E; i += blockDim.x) stt[i] = __ldg(a.ttile + i);
+    __syncthreads();
 }
 
 __device__ __forceinline__ int total_tiles(const GemmArgs &a, int BN, int *tot0)

@@ -38,7 +38,7 @@ namespace {
 
 constexpr int kKC = 128;     // K elements (bytes) per pipeline stage = one 128-byte swizzle row
 constexpr int kStagesPerBlock = kBlockK / kKC;
-constexpr int kMaxKb = 32;   // activation-scale staging holds up to 32 blocks (K <= 16384)
+constexpr int kMaxKb = 16;   // activation-scale staging holds up to 16 blocks (K <= 8192)
 constexpr int kSmemLimit = 227 * 1024;
 
 template <int BN, bool GATEUP, int EW>
@@ -54,8 +54,9 @@ struct Fp8Cfg {
     static constexpr int CPW = BN / PARTS;         // token columns per epilogue thread
     static constexpr int THREADS = 64 + 32 * EW;
     static constexpr int SX_BYTES = 2 * BN * kMaxKb * 4;
+    static constexpr int TT_BYTES = (4 * (kMaxE + 1) + 15) & ~15;  // keeps the mbarriers 8-byte aligned
     static constexpr int BAR_BYTES = 8 * (2 * 16 + 2 * NSLOT) + 16;
-    static constexpr int FIXED = 1024 + SX_BYTES + BAR_BYTES;
+    static constexpr int FIXED = 1024 + SX_BYTES + TT_BYTES + BAR_BYTES;
     static constexpr int NS_FIT = (kSmemLimit - FIXED) / STAGE_BYTES;
     static constexpr int NS = NS_FIT < 16 ? NS_FIT : 16;
     static constexpr int SMEM = FIXED + NS * STAGE_BYTES;
@@ -63,6 +64,7 @@ struct Fp8Cfg {
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M=128 is a multiple of 16 in [16, 256]");
     static_assert(EW % 4 == 0 && CPW % 16 == 0, "epilogue split");
     static_assert(NSLOT >= 1 && NS >= 2, "pipeline");
+    static_assert((NS * STAGE_BYTES + SX_BYTES + TT_BYTES) % 16 == 0, "mbarriers must be 8-byte aligned");
 };
 
 // Named barrier among the EW epilogue warps (ids 2..2+EW-1); barrier 0 is __syncthreads.
@@ -76,7 +78,8 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float *sxbuf = reinterpret_cast<float *>(smem + C::NS * C::STAGE_BYTES);  // [2][BN * kMaxKb]
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::NS * C::STAGE_BYTES + C::SX_BYTES);
+    int *stt = reinterpret_cast<int *>(smem + C::NS * C::STAGE_BYTES + C::SX_BYTES);  // [E + 1]
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::NS * C::STAGE_BYTES + C::SX_BYTES + C::TT_BYTES);
     uint64_t *empty = full + C::NS;
     uint64_t *accf = empty + C::NS;
     uint64_t *acce = accf + C::NSLOT;
@@ -115,6 +118,7 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
     // prefixes are read only after it has completed
     griddep_wait();
     griddep_launch_dependents();
+    load_ttile(args, stt);
 
     int tot0;
     const int total = total_tiles(args, BN, &tot0);
@@ -128,7 +132,7 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
             const uint64_t pol_x = l2_policy_evict_last();
             uint32_t it = 0;
             for (int w = blockIdx.x; w < total; w += gridDim.x) {
-                const TileInfo tl = decode_tile<BN>(args, w, tot0);
+                const TileInfo tl = decode_tile<BN>(args, stt, w, tot0);
                 const int nkc = args.seg[tl.seg].K / kKC;
                 for (int kc = 0; kc < nkc; ++kc, ++it) {
                     const int s = it % C::NS;
@@ -147,7 +151,7 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
         if (lane == 0) {
             uint32_t it = 0, ai = 0;
             for (int w = blockIdx.x; w < total; w += gridDim.x) {
-                const TileInfo tl = decode_tile<BN>(args, w, tot0);
+                const TileInfo tl = decode_tile<BN>(args, stt, w, tot0);
                 // MMA N = the tile's valid rows rounded up to 16: a group's last, partial
                 // token tile costs no tensor-core work for the rows it does not have
                 const int n_mma = min(BN, (tl.nrows + 15) & ~15);
@@ -223,13 +227,13 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
             }
         };
         if ((int)blockIdx.x < total) {
-            const TileInfo t0 = decode_tile<BN>(args, blockIdx.x, tot0);
+            const TileInfo t0 = decode_tile<BN>(args, stt, blockIdx.x, tot0);
             load_sx(t0);
             store_sx(t0, sxbuf);
         }
         epi_sync(32 * EW);
         for (int w = blockIdx.x; w < total; w += gridDim.x, ++ti) {
-            const TileInfo tl = decode_tile<BN>(args, w, tot0);
+            const TileInfo tl = decode_tile<BN>(args, stt, w, tot0);
             const GemmSeg &sg = args.seg[tl.seg];
             const int K = sg.K;
             const int nkb = (K + kBlockK - 1) / kBlockK;
@@ -237,7 +241,7 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
             const int wn = w + gridDim.x;
             TileInfo tn;
             if (wn < total) {
-                tn = decode_tile<BN>(args, wn, tot0);
+                tn = decode_tile<BN>(args, stt, wn, tot0);
                 load_sx(tn);
             }
             const float *sw0 = static_cast<const float *>(sg.sw0) + (size_t)(tl.wrow + r) * nkb;

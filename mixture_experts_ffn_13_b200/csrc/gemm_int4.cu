@@ -8,7 +8,8 @@
 // weights exact:
 //  * warp 0 streams raw int4 weight tiles (128 rows x 128 bytes = 256 K-elements per matrix,
 //    128-byte swizzle; narrower boxes make the TMA issue-bound) by TMA into a ring of raw stages
-//    (evict-first);
+//    (evict-first), and keeps an L2 prefetch of the raw tiles kPrefetch stages further ahead,
+//    so the number of DRAM requests in flight does not depend on the shared-memory ring;
 //  * warps 2-5 (one thread per weight row) turn each raw tile, 64 K-elements at a time, into
 //    the integers q as bf16
 //    (exact: |q| <= 8) in the 128-byte-swizzled K-major layout the MMA reads: flip each
@@ -41,6 +42,7 @@ constexpr int kKE = 64;                // K elements per MMA stage (one 128-byte
 constexpr int kRawKE = 256;            // K elements per raw weight stage (128 bytes per row)
 constexpr int kSubs = kRawKE / kKE;    // MMA stages per raw stage
 constexpr int kConvWarps = 4;
+constexpr int kPrefetch = 8;           // raw stages prefetched into L2 ahead of the loads
 
 template <int BN, bool GATEUP>
 struct I4Cfg {
@@ -58,10 +60,13 @@ struct I4Cfg {
     static constexpr int SLOT_COLS = NA * BN;               // one 128-element K group
     static constexpr int NSLOT = 512 / SLOT_COLS;
     static constexpr int STAGES_PER_GROUP = kGroupK / kKE;  // 2
+    static constexpr int TT_BYTES = (4 * (kMaxE + 1) + 15) & ~15;  // keeps the mbarriers 8-byte aligned
     static constexpr int BAR_BYTES = 8 * (2 * NR + 2 * NB + 2 * NM + 2 * NSLOT) + 16;
-    static constexpr int SMEM = 1024 + NM * MSTAGE + NB * B_BYTES + NR * NA * RAW_BYTES + BAR_BYTES;
+    static constexpr int SMEM = 1024 + NM * MSTAGE + NB * B_BYTES + NR * NA * RAW_BYTES + TT_BYTES + BAR_BYTES;
     static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "1024-byte aligned tiles");
     static_assert(SMEM <= 227 * 1024, "shared memory");
+    static_assert((NM * MSTAGE + NR * NA * RAW_BYTES + NB * B_BYTES + TT_BYTES) % 16 == 0,
+                  "mbarriers must be 8-byte aligned");
 };
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
@@ -104,7 +109,8 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
     uint8_t *mst = smem;                                   // NM converted stages [A0 | A1]
     uint8_t *raw = smem + C::NM * C::MSTAGE;               // NR raw stages [raw0 | raw1]
     uint8_t *bst = raw + C::NR * C::NA * C::RAW_BYTES;     // NB activation stages
-    uint64_t *rfull = reinterpret_cast<uint64_t *>(bst + C::NB * C::B_BYTES);
+    int *stt = reinterpret_cast<int *>(bst + C::NB * C::B_BYTES);  // [E + 1]
+    uint64_t *rfull = reinterpret_cast<uint64_t *>(bst + C::NB * C::B_BYTES + C::TT_BYTES);
     uint64_t *rempty = rfull + C::NR;
     uint64_t *bfull = rempty + C::NR;
     uint64_t *bempty = bfull + C::NB;
@@ -148,6 +154,7 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
     // prefixes are read only after it has completed
     griddep_wait();
     griddep_launch_dependents();
+    load_ttile(args, stt);
 
     int tot0;
     const int total = total_tiles(args, BN, &tot0);
@@ -160,11 +167,29 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
             const uint64_t pol_w = l2_policy_evict_first();
             const uint64_t pol_x = l2_policy_evict_last();
             uint32_t it = 0, rt = 0;  // MMA-stage and raw-stage counters
+            // L2 prefetch cursor: raw stage (pw tile, pk index) runs kPrefetch raw stages ahead
+            // of the shared-memory loads, across tile boundaries
+            int pw = blockIdx.x, pk = 0;
+            TileInfo pt;
+            if (pw < total) pt = decode_tile<BN>(args, stt, pw, tot0);
+            auto prefetch_next = [&]() {
+                if (pw >= total) return;
+                const int x = pk * (kRawKE / 2);
+                tma_prefetch_l2_2d(&maps.a0[pt.seg], x, pt.wrow);
+                if (GATEUP) tma_prefetch_l2_2d(&maps.a1[pt.seg], x, pt.wrow);
+                if (++pk * kRawKE >= args.seg[pt.seg].K) {
+                    pk = 0;
+                    pw += gridDim.x;
+                    if (pw < total) pt = decode_tile<BN>(args, stt, pw, tot0);
+                }
+            };
+            for (int i = 0; i < kPrefetch; ++i) prefetch_next();
             for (int w = blockIdx.x; w < total; w += gridDim.x) {
-                const TileInfo tl = decode_tile<BN>(args, w, tot0);
+                const TileInfo tl = decode_tile<BN>(args, stt, w, tot0);
                 const int nkc = args.seg[tl.seg].K / kKE;
                 for (int kc = 0; kc < nkc; ++kc, ++it) {
                     if (kc % kSubs == 0) {
+                        prefetch_next();
                         // raw weights for the next 256 K-elements (the last stage of a K that is
                         // not a multiple of 256 reads zeros past the end)
                         const int s = rt % C::NR;
@@ -188,7 +213,7 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
         if (lane == 0) {
             uint32_t it = 0, ai = 0;
             for (int w = blockIdx.x; w < total; w += gridDim.x) {
-                const TileInfo tl = decode_tile<BN>(args, w, tot0);
+                const TileInfo tl = decode_tile<BN>(args, stt, w, tot0);
                 const int n_mma = min(BN, (tl.nrows + 15) & ~15);  // partial tiles: no work on absent rows
                 const uint32_t kIdesc = instr_desc(kTileM, n_mma, 1, 1);
                 const int ngrp = args.seg[tl.seg].K / kGroupK;
@@ -227,7 +252,7 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
         const int r = cw * 32 + lane;  // weight row of the tile handled by this thread
         uint32_t it = 0, rt = 0;
         for (int w = blockIdx.x; w < total; w += gridDim.x) {
-            const TileInfo tl = decode_tile<BN>(args, w, tot0);
+            const TileInfo tl = decode_tile<BN>(args, stt, w, tot0);
             const GemmSeg &sg = args.seg[tl.seg];
             const int nkc = sg.K / kKE;
             for (int kc = 0; kc < nkc; ++kc, ++it) {
@@ -272,7 +297,7 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
         const int r = q * 32 + lane;
         uint32_t ai = 0;
         for (int w = blockIdx.x; w < total; w += gridDim.x) {
-            const TileInfo tl = decode_tile<BN>(args, w, tot0);
+            const TileInfo tl = decode_tile<BN>(args, stt, w, tot0);
             const GemmSeg &sg = args.seg[tl.seg];
             const int ngrp = sg.K / kGroupK;
             const __nv_bfloat16 *sw0 = static_cast<const __nv_bfloat16 *>(sg.sw0) + (size_t)(tl.wrow + r) * ngrp;

@@ -165,6 +165,7 @@ int moe_plan(const moe_dims *dims, moe_plan_t **out_plan, size_t *workspace_byte
     if (d.k > d.E) return MOE_ERR_INVALID_ARG;
     if (d.E > kMaxE || d.k > kMaxK || d.T_max > (1 << 20)) return MOE_ERR_UNSUPPORTED;
     if (d.H % 128 || d.I % 128 || d.I_shared % 128) return MOE_ERR_UNSUPPORTED;
+    if (d.H > 8192 || d.I > 8192 || d.I_shared > 8192) return MOE_ERR_UNSUPPORTED;
     // 32-bit row arithmetic inside the kernels
     if ((long long)d.E * std::max(d.I, d.H) >= (1ll << 31) ||
         (long long)d.T_max * (d.k + 1) * std::max(d.I, d.H) >= (1ll << 40))
