@@ -75,6 +75,9 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
     gemm_fp8_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmArgs args)
 {
     using C = Fp8Cfg<BN, GATEUP, EW>;
+    // Wide token tiles stage the tile's activation scales in shared memory; narrow (decode)
+    // tiles read them straight from L2 in the promotion loop, which measured faster there.
+    constexpr bool kStageSx = BN >= 64;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float *sxbuf = reinterpret_cast<float *>(smem + C::NS * C::STAGE_BYTES);  // [2][BN * kMaxKb]
@@ -152,9 +155,10 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
             uint32_t it = 0, ai = 0;
             for (int w = blockIdx.x; w < total; w += gridDim.x) {
                 const TileInfo tl = decode_tile<BN>(args, stt, w, tot0);
-                // MMA N = the tile's valid rows rounded up to 16: a group's last, partial
-                // token tile costs no tensor-core work for the rows it does not have
-                const int n_mma = min(BN, (tl.nrows + 15) & ~15);
+                // MMA N = the tile's valid rows rounded up to 16 for wide tiles (a group's last,
+                // partial token tile costs no tensor-core work for absent rows); narrow
+                // decode tiles keep N = BN, which measured faster
+                const int n_mma = kStageSx ? min(BN, (tl.nrows + 15) & ~15) : BN;
                 const uint32_t kIdesc = instr_desc(kTileM, n_mma, 0, 0);
                 const int K = args.seg[tl.seg].K;
                 const int nkc = K / kKC;
@@ -226,12 +230,14 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
                 }
             }
         };
-        if ((int)blockIdx.x < total) {
-            const TileInfo t0 = decode_tile<BN>(args, stt, blockIdx.x, tot0);
-            load_sx(t0);
-            store_sx(t0, sxbuf);
+        if constexpr (kStageSx) {
+            if ((int)blockIdx.x < total) {
+                const TileInfo t0 = decode_tile<BN>(args, stt, blockIdx.x, tot0);
+                load_sx(t0);
+                store_sx(t0, sxbuf);
+            }
+            epi_sync(32 * EW);
         }
-        epi_sync(32 * EW);
         for (int w = blockIdx.x; w < total; w += gridDim.x, ++ti) {
             const TileInfo tl = decode_tile<BN>(args, stt, w, tot0);
             const GemmSeg &sg = args.seg[tl.seg];
@@ -240,7 +246,7 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
             const float *sxs = sxbuf + (ti & 1) * (BN * kMaxKb);
             const int wn = w + gridDim.x;
             TileInfo tn;
-            if (wn < total) {
+            if (kStageSx && wn < total) {
                 tn = decode_tile<BN>(args, stt, wn, tot0);
                 load_sx(tn);
             }
@@ -279,7 +285,13 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
                     }
 #pragma unroll
                     for (int c = 0; c < 16; ++c) {
-                        const float sx = sxk[c0 + c];
+                        float sx;
+                        if constexpr (kStageSx) {
+                            sx = sxk[c0 + c];
+                        } else {
+                            const int row = min(tl.row0 + cbase + c0 + c, sg.rows - 1);
+                            sx = __ldg(sg.sx + (size_t)row * nkb + kb);
+                        }
                         acc0[c0 + c] = fmaf(v[c], s0 * sx, acc0[c0 + c]);
                         if constexpr (GATEUP) acc1[c0 + c] = fmaf(u[c], s1 * sx, acc1[c0 + c]);
                     }
@@ -301,8 +313,10 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
                     out[(size_t)(tl.row0 + cbase + c) * sg.N + n] = v;
                 }
             }
-            if (wn < total) store_sx(tn, sxbuf + ((ti + 1) & 1) * (BN * kMaxKb));
-            epi_sync(32 * EW);
+            if constexpr (kStageSx) {
+                if (wn < total) store_sx(tn, sxbuf + ((ti + 1) & 1) * (BN * kMaxKb));
+                epi_sync(32 * EW);
+            }
         }
     }
 done:
