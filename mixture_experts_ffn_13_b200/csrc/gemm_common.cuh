@@ -19,25 +19,27 @@ struct TileInfo {
 // Work item w -> tile.  Routed items come first: group g owns items
 // [ttile[g]*nT, ttile[g+1]*nT), laid out n-tile major so consecutive items reuse the same
 // weight tile across the group's token tiles.  Shared-expert items follow.
-// `stt` is a shared-memory copy of a.ttile (E+1 entries), so the binary search costs shared
-// loads only; a chain of dependent global loads per tile would stall the TMA producer.
-template <int BN>
+// `stt` is a.ttile itself (read through the read-only cache) or a shared-memory copy of it
+// (E+1 entries; SMEM_TT), which keeps the binary search off global memory for kernels whose
+// tiles are short enough for its latency to show.
+template <int BN, bool SMEM_TT = false>
 __device__ __forceinline__ TileInfo decode_tile(const GemmArgs &a, const int *stt, int w, int tot0)
 {
+    auto tt = [&](int i) { return SMEM_TT ? stt[i] : __ldg(stt + i); };
     TileInfo t;
     if (w < tot0) {
         const int nT = a.seg[0].N / kTileM;
         int lo = 0, hi = a.E - 1;
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
-            if (stt[mid] * nT <= w)
+            if (tt(mid) * nT <= w)
                 lo = mid;
             else
                 hi = mid - 1;
         }
         const int g = lo;
-        const int t0 = stt[g];
-        const int ntt = stt[g + 1] - t0;
+        const int t0 = tt(g);
+        const int ntt = tt(g + 1) - t0;
         const int local = w - t0 * nT;
         const int nt = local / ntt;
         const int tt = local - nt * ntt;

@@ -53,12 +53,18 @@ struct Fp8Cfg {
     static constexpr int PARTS = EW / 4;           // epilogue warps per TMEM lane quarter
     static constexpr int CPW = BN / PARTS;         // token columns per epilogue thread
     static constexpr int THREADS = 64 + 32 * EW;
-    static constexpr int SX_BYTES = 2 * BN * kMaxKb * 4;
-    static constexpr int TT_BYTES = (4 * (kMaxE + 1) + 15) & ~15;  // keeps the mbarriers 8-byte aligned
+    // Wide tiles (BN >= 64) stage activation scales and the tile-prefix table in shared
+    // memory; narrow (decode) tiles do not, and keep shared memory under 200 KB so that L1,
+    // which serves their scale loads, stays large.
+    static constexpr bool WIDE = BN >= 64;
+    static constexpr int SX_BYTES = WIDE ? 2 * BN * kMaxKb * 4 : 0;
+    static constexpr int TT_BYTES = WIDE ? (4 * (kMaxE + 1) + 15) & ~15 : 0;  // keeps the mbarriers 8-byte aligned
     static constexpr int BAR_BYTES = 8 * (2 * 16 + 2 * NSLOT) + 16;
     static constexpr int FIXED = 1024 + SX_BYTES + TT_BYTES + BAR_BYTES;
     static constexpr int NS_FIT = (kSmemLimit - FIXED) / STAGE_BYTES;
-    static constexpr int NS = NS_FIT < 16 ? NS_FIT : 16;
+    static constexpr int NS_NARROW = (200 * 1024) / STAGE_BYTES;
+    static constexpr int NS_CAP = WIDE ? NS_FIT : (NS_NARROW < NS_FIT ? NS_NARROW : NS_FIT);
+    static constexpr int NS = NS_CAP < 16 ? NS_CAP : 16;
     static constexpr int SMEM = FIXED + NS * STAGE_BYTES;
     static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "stage tiles must stay 1024-byte aligned");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M=128 is a multiple of 16 in [16, 256]");
@@ -77,7 +83,7 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
     using C = Fp8Cfg<BN, GATEUP, EW>;
     // Wide token tiles stage the tile's activation scales in shared memory; narrow (decode)
     // tiles read them straight from L2 in the promotion loop, which measured faster there.
-    constexpr bool kStageSx = BN >= 64;
+    constexpr bool kStageSx = C::WIDE;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float *sxbuf = reinterpret_cast<float *>(smem + C::NS * C::STAGE_BYTES);  // [2][BN * kMaxKb]
@@ -121,7 +127,8 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
     // prefixes are read only after it has completed
     griddep_wait();
     griddep_launch_dependents();
-    load_ttile(args, stt);
+    if constexpr (kStageSx) load_ttile(args, stt);
+    const int *ttab = kStageSx ? stt : args.ttile;
 
     int tot0;
     const int total = total_tiles(args, BN, &tot0);
@@ -135,7 +142,7 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
             const uint64_t pol_x = l2_policy_evict_last();
             uint32_t it = 0;
             for (int w = blockIdx.x; w < total; w += gridDim.x) {
-                const TileInfo tl = decode_tile<BN>(args, stt, w, tot0);
+                const TileInfo tl = decode_tile<BN, kStageSx>(args, ttab, w, tot0);
                 const int nkc = args.seg[tl.seg].K / kKC;
                 for (int kc = 0; kc < nkc; ++kc, ++it) {
                     const int s = it % C::NS;
@@ -154,7 +161,7 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
         if (lane == 0) {
             uint32_t it = 0, ai = 0;
             for (int w = blockIdx.x; w < total; w += gridDim.x) {
-                const TileInfo tl = decode_tile<BN>(args, stt, w, tot0);
+                const TileInfo tl = decode_tile<BN, kStageSx>(args, ttab, w, tot0);
                 // MMA N = the tile's valid rows rounded up to 16 for wide tiles (a group's last,
                 // partial token tile costs no tensor-core work for absent rows); narrow
                 // decode tiles keep N = BN, which measured faster
@@ -232,14 +239,14 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
         };
         if constexpr (kStageSx) {
             if ((int)blockIdx.x < total) {
-                const TileInfo t0 = decode_tile<BN>(args, stt, blockIdx.x, tot0);
+                const TileInfo t0 = decode_tile<BN, kStageSx>(args, ttab, blockIdx.x, tot0);
                 load_sx(t0);
                 store_sx(t0, sxbuf);
             }
             epi_sync(32 * EW);
         }
         for (int w = blockIdx.x; w < total; w += gridDim.x, ++ti) {
-            const TileInfo tl = decode_tile<BN>(args, stt, w, tot0);
+            const TileInfo tl = decode_tile<BN, kStageSx>(args, ttab, w, tot0);
             const GemmSeg &sg = args.seg[tl.seg];
             const int K = sg.K;
             const int nkb = (K + kBlockK - 1) / kBlockK;
@@ -247,7 +254,7 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
             const int wn = w + gridDim.x;
             TileInfo tn;
             if (kStageSx && wn < total) {
-                tn = decode_tile<BN>(args, stt, wn, tot0);
+                tn = decode_tile<BN, kStageSx>(args, ttab, wn, tot0);
                 load_sx(tn);
             }
             const float *sw0 = static_cast<const float *>(sg.sw0) + (size_t)(tl.wrow + r) * nkb;
@@ -259,14 +266,25 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
 #pragma unroll
                 for (int c = 0; c < C::CPW; ++c) acc1[c] = 0.0f;
             }
-            float s0n = __ldg(sw0), s1n = GATEUP ? __ldg(sw1) : 0.0f;
+            float s0n = 0.0f, s1n = 0.0f;
+            if constexpr (kStageSx) {
+                s0n = __ldg(sw0);
+                if (GATEUP) s1n = __ldg(sw1);
+            }
             for (int kb = 0; kb < nkb; ++kb, ++ai) {
                 const int slot = ai % C::NSLOT;
                 const uint32_t aph = (ai / C::NSLOT) & 1;
-                const float s0 = s0n, s1 = s1n;
-                if (kb + 1 < nkb) {
-                    s0n = __ldg(sw0 + kb + 1);
-                    if (GATEUP) s1n = __ldg(sw1 + kb + 1);
+                float s0, s1;
+                if constexpr (kStageSx) {  // wide tiles: weight scales prefetched a block ahead
+                    s0 = s0n;
+                    s1 = s1n;
+                    if (kb + 1 < nkb) {
+                        s0n = __ldg(sw0 + kb + 1);
+                        if (GATEUP) s1n = __ldg(sw1 + kb + 1);
+                    }
+                } else {
+                    s0 = __ldg(sw0 + kb);
+                    s1 = GATEUP ? __ldg(sw1 + kb) : 0.0f;
                 }
                 const bool ok = mbar_wait(&accf[slot], aph, abort_flag, status, tmo);
                 if (!__all_sync(0xffffffffu, ok)) goto done;

@@ -171,7 +171,7 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
             // of the shared-memory loads, across tile boundaries
             int pw = blockIdx.x, pk = 0;
             TileInfo pt;
-            if (pw < total) pt = decode_tile<BN>(args, stt, pw, tot0);
+            if (pw < total) pt = decode_tile<BN, true>(args, stt, pw, tot0);
             auto prefetch_next = [&]() {
                 if (pw >= total) return;
                 const int x = pk * (kRawKE / 2);
@@ -180,12 +180,12 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
                 if (++pk * kRawKE >= args.seg[pt.seg].K) {
                     pk = 0;
                     pw += gridDim.x;
-                    if (pw < total) pt = decode_tile<BN>(args, stt, pw, tot0);
+                    if (pw < total) pt = decode_tile<BN, true>(args, stt, pw, tot0);
                 }
             };
             for (int i = 0; i < kPrefetch; ++i) prefetch_next();
             for (int w = blockIdx.x; w < total; w += gridDim.x) {
-                const TileInfo tl = decode_tile<BN>(args, stt, w, tot0);
+                const TileInfo tl = decode_tile<BN, true>(args, stt, w, tot0);
                 const int nkc = args.seg[tl.seg].K / kKE;
                 for (int kc = 0; kc < nkc; ++kc, ++it) {
                     if (kc % kSubs == 0) {
@@ -213,7 +213,7 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
         if (lane == 0) {
             uint32_t it = 0, ai = 0;
             for (int w = blockIdx.x; w < total; w += gridDim.x) {
-                const TileInfo tl = decode_tile<BN>(args, stt, w, tot0);
+                const TileInfo tl = decode_tile<BN, true>(args, stt, w, tot0);
                 const int n_mma = min(BN, (tl.nrows + 15) & ~15);  // partial tiles: no work on absent rows
                 const uint32_t kIdesc = instr_desc(kTileM, n_mma, 1, 1);
                 const int ngrp = args.seg[tl.seg].K / kGroupK;
@@ -252,7 +252,7 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
         const int r = cw * 32 + lane;  // weight row of the tile handled by this thread
         uint32_t it = 0, rt = 0;
         for (int w = blockIdx.x; w < total; w += gridDim.x) {
-            const TileInfo tl = decode_tile<BN>(args, stt, w, tot0);
+            const TileInfo tl = decode_tile<BN, true>(args, stt, w, tot0);
             const GemmSeg &sg = args.seg[tl.seg];
             const int nkc = sg.K / kKE;
             for (int kc = 0; kc < nkc; ++kc, ++it) {
@@ -297,7 +297,7 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
         const int r = q * 32 + lane;
         uint32_t ai = 0;
         for (int w = blockIdx.x; w < total; w += gridDim.x) {
-            const TileInfo tl = decode_tile<BN>(args, stt, w, tot0);
+            const TileInfo tl = decode_tile<BN, true>(args, stt, w, tot0);
             const GemmSeg &sg = args.seg[tl.seg];
             const int ngrp = sg.K / kGroupK;
             const __nv_bfloat16 *sw0 = static_cast<const __nv_bfloat16 *>(sg.sw0) + (size_t)(tl.wrow + r) * ngrp;
