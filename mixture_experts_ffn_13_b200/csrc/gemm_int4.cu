@@ -53,10 +53,14 @@ struct I4Cfg {
     static constexpr int RAW_BYTES = kTileM * (kRawKE / 2);  // 16 KB per matrix
     static constexpr int A_BYTES = kTileM * kKE * 2;        // 16 KB per matrix
     static constexpr int B_BYTES = BN * kKE * 2;
-    static constexpr int NR = GATEUP ? 2 : 4;               // raw weight stages (256 K each)
-    static constexpr int NB = GATEUP ? 6 : 8;               // activation stages (64 K each)
+    // The activation ring is the deepest: every 64-K stage waits for its activation tile's
+    // L2 round trip, so its depth sets the stage rate (measured: 2 -> 6 stages more than
+    // halved the time of a no-work skeleton of this pipeline).
+    static constexpr int NR = GATEUP ? 2 : 3;               // raw weight stages (256 K each)
     static constexpr int MSTAGE = NA * A_BYTES;             // converted weight stage
-    static constexpr int NM = GATEUP ? 3 : 4;               // converted stages
+    static constexpr int NM = GATEUP ? 2 : 3;               // converted stages
+    static constexpr int NB_FIT = (215 * 1024 - NM * MSTAGE - NR * NA * RAW_BYTES) / B_BYTES;
+    static constexpr int NB = NB_FIT < 12 ? NB_FIT : 12;     // activation stages (64 K each)
     static constexpr int SLOT_COLS = NA * BN;               // one 128-element K group
     static constexpr int NSLOT = 512 / SLOT_COLS;
     static constexpr int STAGES_PER_GROUP = kGroupK / kKE;  // 2
@@ -384,12 +388,14 @@ cudaError_t launch_gemm_int4(bool gateup, int bn, const GemmMaps &maps, const Ge
         switch (bn) {
             case 32: return launch_t<32, true>(maps, args, num_sms, s);
             case 64: return launch_t<64, true>(maps, args, num_sms, s);
+            case 96: return launch_t<96, true>(maps, args, num_sms, s);
             default: return cudaErrorInvalidValue;
         }
     }
     switch (bn) {
         case 32: return launch_t<32, false>(maps, args, num_sms, s);
         case 64: return launch_t<64, false>(maps, args, num_sms, s);
+        case 96: return launch_t<96, false>(maps, args, num_sms, s);
         default: return cudaErrorInvalidValue;
     }
 }

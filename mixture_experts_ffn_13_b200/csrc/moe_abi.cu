@@ -112,9 +112,9 @@ int fail_cuda(moe_plan_t *p, cudaError_t e)
 int pick_bn(int T, int k, int E, bool fp8)
 {
     const long avg = ((long)T * k + E - 1) / E;
-    if (avg <= 48) return 32;
-    if (avg <= 96 || !fp8) return 64;
-    return 128;
+    if (avg <= 48) return fp8 || avg <= 24 ? 32 : 64;
+    if (!fp8) return 96;  // 4-bit: one tile per group up to ~1.5x the mean (dequant is per tile)
+    return avg <= 96 ? 64 : 128;
 }
 
 }  // namespace
