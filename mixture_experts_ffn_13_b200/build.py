@@ -13,7 +13,8 @@ BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libmoe_b200.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 
-SOURCES = ["moe_abi.cu", "route.cu", "route_static.cu", "quant.cu", "combine.cu", "gemm_fp8.cu", "gemm_int4.cu"]
+SOURCES = ["moe_abi.cu", "route.cu", "route_static.cu", "quant.cu", "combine.cu", "gemm_fp8.cu", "gemm_int4.cu",
+           "testing.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-I" + INCLUDE]
@@ -27,7 +28,8 @@ def _nvcc() -> str:
 
 
 def _deps_mtime() -> float:
-    files = [os.path.join(CSRC, f) for f in os.listdir(CSRC)] + [os.path.join(INCLUDE, "moe_b200.h")]
+    files = [os.path.join(CSRC, f) for f in os.listdir(CSRC)] + \
+        [os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE)]
     return max(os.path.getmtime(f) for f in files)
 
 
