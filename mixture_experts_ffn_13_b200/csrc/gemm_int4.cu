@@ -1,5 +1,5 @@
-// gemm_int4.cu -- steps A4/A5 for 4-bit expert weights: persistent grouped GEMMs that
-// dequantise int4 weights into shared memory and run bf16 x bf16 -> fp32 tcgen05 MMAs.
+// gemm_int4.cu -- steps A4/A5 for 4-bit expert weights: persistent grouped GEMMs that unpack
+// int4 weights into tensor memory and run bf16 x bf16 -> fp32 tcgen05 MMAs.
 //
 // Page "Flash-Next 在 GPU 上到底在算什麼", section "① 專家 FFN" (and its NVIDIA table): expert
 // weights are stored in 4/8 bits and must be decompressed to 16-bit before the tensor units
@@ -7,23 +7,22 @@
 // tensor cores idle.  Here the decompression feeds the tensor cores instead, and keeps the
 // weights exact:
 //  * warp 0 streams raw int4 weight tiles (128 rows x 128 bytes = 256 K-elements per matrix,
-//    128-byte swizzle; narrower boxes make the TMA issue-bound) by TMA into a ring of raw stages
-//    (evict-first), and keeps an L2 prefetch of the raw tiles kPrefetch stages further ahead,
-//    so the number of DRAM requests in flight does not depend on the shared-memory ring;
-//  * warps 2-5 (one thread per weight row) turn each raw tile, 64 K-elements at a time, into
-//    the integers q as bf16
-//    (exact: |q| <= 8) in the 128-byte-swizzled K-major layout the MMA reads: flip each
-//    nibble's sign bit, place it in the mantissa of the bf16 value 128 (so it reads
-//    128 + q + 8), subtract 136, store 16 bytes per 8 values at the swizzled chunk; the
-//    activation tiles (bf16) come by TMA through their own ring, issued by warp 0 with the
-//    raw weights, so they arrive as far ahead as the weights do;
-//  * warp 1 issues tcgen05.mma.kind::f16 (BF16 x BF16 -> F32) from one thread: 4 MMAs of
-//    K = 16 per stage per matrix; each 128-element K group (2 stages) accumulates into its own
-//    TMEM slot, because the weight scale changes per (row, group);
-//  * warps 6-13 (two per TMEM lane quarter, each owning half of the token columns) promote
-//    each finished group, acc += D_g * s[row, g] in fp32 registers, and at
-//    the end of the tile write gate|up h = silu(G) * U rounded to bf16 (the 4-bit layer keeps
-//    activations in bf16) or down y in fp32.
+//    128-byte swizzle; narrower boxes make the TMA issue-bound) by TMA into a ring of raw
+//    stages (evict-first), keeps an L2 prefetch of the raw tiles kPrefetch stages further
+//    ahead, and streams the bf16 activation tiles through their own ring;
+//  * warps 2-5 (one thread per weight row, 64 K-elements at a time) turn the nibbles into the
+//    integers q as bf16 (exact: |q| <= 8): flip each nibble's sign bit, place it in the
+//    mantissa of the bf16 value 128 (so it reads 128 + q + 8), subtract 136.  The result goes
+//    to TENSOR memory with tcgen05.st (rows in lanes, two bf16 per 32-bit column): staging
+//    the 4x-expanded weights in shared memory instead costs a write and a tensor-core read of
+//    them per stage, which made the kernel shared-memory-bandwidth bound;
+//  * warp 1 issues tcgen05.mma.kind::f16 (A from tensor memory, B from shared memory) from one
+//    thread: 4 MMAs of K = 16 per stage per matrix; each 128-element K group (2 stages)
+//    accumulates into its own TMEM slot, because the weight scale changes per (row, group);
+//  * warps 6-13 (two per TMEM lane quarter, each owning half of the token columns) promote each
+//    finished group, acc += D_g * s[row, g] in fp32 registers, and at the end of the tile write
+//    gate|up h = silu(G) * U rounded to bf16 (the 4-bit layer keeps activations in bf16) or
+//    down y in fp32.
 // Multiplying the exact integers on the tensor cores and applying the bf16 scale to fp32
 // partial sums reproduces sum_i x_i * q_i * s_i up to fp32 rounding; rounding q * s to bf16
 // before the MMA would not (that costs ~2^-9 relative per weight and fails the layer's
@@ -51,26 +50,25 @@ struct I4Cfg {
     static constexpr int THREADS = 32 * (2 + kConvWarps + EW);
     static constexpr int NA = GATEUP ? 2 : 1;
     static constexpr int RAW_BYTES = kTileM * (kRawKE / 2);  // 16 KB per matrix
-    static constexpr int A_BYTES = kTileM * kKE * 2;        // 16 KB per matrix
     static constexpr int B_BYTES = BN * kKE * 2;
-    // The activation ring is the deepest: every 64-K stage waits for its activation tile's
-    // L2 round trip, so its depth sets the stage rate (measured: 2 -> 6 stages more than
-    // halved the time of a no-work skeleton of this pipeline).
-    static constexpr int NR = GATEUP ? 2 : 3;               // raw weight stages (256 K each)
-    static constexpr int MSTAGE = NA * A_BYTES;             // converted weight stage
-    static constexpr int NM = GATEUP ? 2 : 3;               // converted stages
-    static constexpr int NB_FIT = (215 * 1024 - NM * MSTAGE - NR * NA * RAW_BYTES) / B_BYTES;
-    static constexpr int NB = NB_FIT < 12 ? NB_FIT : 12;     // activation stages (64 K each)
+    // Converted weights live in tensor memory: NM stages x NA matrices x 32 columns (64 bf16
+    // per row).  The accumulator slots take the remaining columns.
+    static constexpr int NM = GATEUP ? 2 : 3;
+    static constexpr int A_COLS = 32;
+    static constexpr int A_TMEM = NM * NA * A_COLS;
     static constexpr int SLOT_COLS = NA * BN;               // one 128-element K group
-    static constexpr int NSLOT = 512 / SLOT_COLS;
+    static constexpr int NSLOT = (512 - A_TMEM) / SLOT_COLS;
     static constexpr int STAGES_PER_GROUP = kGroupK / kKE;  // 2
+    static constexpr int NR = GATEUP ? 3 : 5;               // raw weight stages (256 K each)
+    static constexpr int NB_FIT = (212 * 1024 - NR * NA * RAW_BYTES) / B_BYTES;
+    static constexpr int NB = NB_FIT < 12 ? NB_FIT : 12;     // activation stages (64 K each)
     static constexpr int TT_BYTES = (4 * (kMaxE + 1) + 15) & ~15;  // keeps the mbarriers 8-byte aligned
     static constexpr int BAR_BYTES = 8 * (2 * NR + 2 * NB + 2 * NM + 2 * NSLOT) + 16;
-    static constexpr int SMEM = 1024 + NM * MSTAGE + NB * B_BYTES + NR * NA * RAW_BYTES + TT_BYTES + BAR_BYTES;
-    static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "1024-byte aligned tiles");
+    static constexpr int SMEM = 1024 + NB * B_BYTES + NR * NA * RAW_BYTES + TT_BYTES + BAR_BYTES;
+    static_assert(B_BYTES % 1024 == 0, "1024-byte aligned tiles");
+    static_assert(NSLOT >= 2, "TMEM slots");
     static_assert(SMEM <= 227 * 1024, "shared memory");
-    static_assert((NM * MSTAGE + NR * NA * RAW_BYTES + NB * B_BYTES + TT_BYTES) % 16 == 0,
-                  "mbarriers must be 8-byte aligned");
+    static_assert((NR * NA * RAW_BYTES + NB * B_BYTES + TT_BYTES) % 16 == 0, "mbarriers must be 8-byte aligned");
 };
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
@@ -110,8 +108,7 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
     using C = I4Cfg<BN, GATEUP>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *mst = smem;                                   // NM converted stages [A0 | A1]
-    uint8_t *raw = smem + C::NM * C::MSTAGE;               // NR raw stages [raw0 | raw1]
+    uint8_t *raw = smem;                                   // NR raw stages [raw0 | raw1]
     uint8_t *bst = raw + C::NR * C::NA * C::RAW_BYTES;     // NB activation stages
     int *stt = reinterpret_cast<int *>(bst + C::NB * C::B_BYTES);  // [E + 1]
     uint64_t *rfull = reinterpret_cast<uint64_t *>(bst + C::NB * C::B_BYTES + C::TT_BYTES);
@@ -225,7 +222,7 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
                     const int slot = ai % C::NSLOT;
                     if (!mbar_wait(&acce[slot], ((ai / C::NSLOT) & 1) ^ 1, abort_flag, status, tmo)) goto done;
                     tc_fence_after();
-                    const uint32_t d0 = tmem_base + slot * C::SLOT_COLS;
+                    const uint32_t d0 = tmem_base + C::A_TMEM + slot * C::SLOT_COLS;
                     const uint32_t d1 = d0 + BN;
                     for (int sk = 0; sk < C::STAGES_PER_GROUP; ++sk, ++it) {
                         const int s = it % C::NM;
@@ -233,15 +230,14 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
                         if (!mbar_wait(&mfull[s], (it / C::NM) & 1, abort_flag, status, tmo)) goto done;
                         if (!mbar_wait(&bfull[bs], (it / C::NB) & 1, abort_flag, status, tmo)) goto done;
                         tc_fence_after();
-                        uint8_t *st = mst + s * C::MSTAGE;
-                        const uint64_t da0 = smem_desc_sw128(st);
-                        const uint64_t da1 = smem_desc_sw128(st + C::A_BYTES);
+                        const uint32_t a0 = tmem_base + s * C::NA * C::A_COLS;
+                        const uint32_t a1 = a0 + C::A_COLS;
                         const uint64_t db = smem_desc_sw128(bst + bs * C::B_BYTES);
 #pragma unroll
                         for (int kk = 0; kk < kKE / 16; ++kk) {
                             const uint32_t acc = (sk > 0 || kk > 0) ? 1u : 0u;
-                            mma_bf16(d0, da0 + 2 * kk, db + 2 * kk, kIdesc, acc);
-                            if (GATEUP) mma_bf16(d1, da1 + 2 * kk, db + 2 * kk, kIdesc, acc);
+                            mma_bf16_ts(d0, a0 + 8 * kk, db + 2 * kk, kIdesc, acc);
+                            if (GATEUP) mma_bf16_ts(d1, a1 + 8 * kk, db + 2 * kk, kIdesc, acc);
                         }
                         mma_commit(&mempty[s]);
                         mma_commit(&bempty[bs]);
@@ -252,8 +248,8 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
         }
     } else if (warp < 2 + kConvWarps) {
         // ------------------------------ dequantisers ------------------------------
-        const int cw = warp - 2;
-        const int r = cw * 32 + lane;  // weight row of the tile handled by this thread
+        const int q = warp & 3;        // TMEM lane quarter reachable from this warp
+        const int r = q * 32 + lane;   // weight row of the tile handled by this thread
         uint32_t it = 0, rt = 0;
         for (int w = blockIdx.x; w < total; w += gridDim.x) {
             const TileInfo tl = decode_tile<BN, true>(args, stt, w, tot0);
@@ -268,23 +264,30 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
                 if (!__all_sync(0xffffffffu, ok)) goto done;
                 ok = mbar_wait(&mempty[ms_i], ((it / C::NM) & 1) ^ 1, abort_flag, status, tmo);
                 if (!__all_sync(0xffffffffu, ok)) goto done;
-                uint8_t *st = mst + ms_i * C::MSTAGE;
+                tc_fence_after();
                 const uint8_t *rs = raw + rs_i * C::NA * C::RAW_BYTES + r * 128;
                 // this sub-stage's 32 raw bytes are 16-byte chunks 2*sub and 2*sub+1 of the row,
                 // stored by the 128-byte swizzle at chunk positions (c ^ (r & 7))
                 const int c0 = ((2 * sub) ^ (r & 7)) << 4, c1 = ((2 * sub + 1) ^ (r & 7)) << 4;
+                const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + ms_i * C::NA * C::A_COLS;
 #pragma unroll
                 for (int m = 0; m < C::NA; ++m) {
                     const uint4 q0 = *reinterpret_cast<const uint4 *>(rs + m * C::RAW_BYTES + c0);
                     const uint4 q1 = *reinterpret_cast<const uint4 *>(rs + m * C::RAW_BYTES + c1);
-                    uint8_t *dst = st + m * C::A_BYTES + r * 128;
                     const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+                    uint32_t v[32];
 #pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        *reinterpret_cast<uint4 *>(dst + ((j ^ (r & 7)) << 4)) = unpack8(words[j]);
+                    for (int j = 0; j < 8; ++j) {
+                        const uint4 u = unpack8(words[j]);
+                        v[4 * j] = u.x;
+                        v[4 * j + 1] = u.y;
+                        v[4 * j + 2] = u.z;
+                        v[4 * j + 3] = u.w;
+                    }
+                    tmem_st32(ta + m * C::A_COLS, v);  // row r: 64 bf16 = 32 packed columns
                 }
-                // make the generic-proxy shared-memory writes visible to the tensor core
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                tmem_wait_st();
+                tc_fence_before();
                 __syncwarp();
                 const bool raw_done = (sub == kSubs - 1) || (kc == nkc - 1);
                 if (lane == 0) {
@@ -325,7 +328,7 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
                 const bool ok = mbar_wait(&accf[slot], (ai / C::NSLOT) & 1, abort_flag, status, tmo);
                 if (!__all_sync(0xffffffffu, ok)) goto done;
                 tc_fence_after();
-                const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + slot * C::SLOT_COLS + cbase;
+                const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + C::A_TMEM + slot * C::SLOT_COLS + cbase;
 #pragma unroll
                 for (int c0 = 0; c0 < C::CPW; c0 += 16) {
                     float v[16], u[16];
