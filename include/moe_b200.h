@@ -100,6 +100,17 @@ typedef struct moe_plan_s moe_plan_t; /* opaque; owned by the library until moe_
  * MOE_ERR_UNSUPPORTED for shapes outside that set. */
 MOE_API int moe_plan(const moe_dims *dims, moe_plan_t **out_plan, size_t *workspace_bytes);
 
+/* Router logits, the dense 16-bit layer that feeds step A1 (page "Flash-Next 在 GPU 上到底在算
+ * 什麼", section "② 密集 16-bit 層": the router runs in 16 bits on the tensor cores):
+ *   logits[T, E] (fp32, out) = x[T, H] (bf16) . w_router[E, H]^T (bf16, row-major [out, in]),
+ * accumulated in fp32 on tcgen05 tensor cores.  Uses the plan's H and E; needs no workspace;
+ * 0 <= T <= T_max.  The result can be passed to moe_route / moe_forward.  All pointers are
+ * device pointers, 16-byte aligned, caller-owned.  Returns MOE_ERR_INVALID_ARG for a NULL plan,
+ * T outside [0, T_max], NULL or misaligned buffers (T > 0); MOE_ERR_CUDA if the launch fails;
+ * a device-side wait that runs out sets the plan's status (moe_get_status). */
+MOE_API int moe_router_logits(moe_plan_t *plan, int32_t T, const uint16_t *x_bf16, const uint16_t *w_router_bf16,
+                              float *logits, moe_stream_t stream);
+
 /* Route and permute only (steps A1 and A3), for inspection and parity checks.
  *   logits   [T, E] fp32 (finite values; the caller guarantees it)
  *   topk_idx [T, k] int32 out: experts by (logit desc, index asc)

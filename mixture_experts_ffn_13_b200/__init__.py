@@ -25,7 +25,7 @@ ERRORS = {-1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED", -3: "MOE_ERR_WOR
           -4: "MOE_ERR_CUDA", -5: "MOE_ERR_DEVICE_TIMEOUT", -6: "MOE_ERR_BOUNDS"}
 EXPORTS = ("moe_plan", "moe_route", "moe_forward", "moe_get_status", "moe_last_cuda_error",
            "moe_destroy", "moe_strerror", "moe_profile_enable", "moe_profile_read",
-           "moe_profile_stage_name", "moe_launch_count", "moe_route_static")
+           "moe_profile_stage_name", "moe_launch_count", "moe_route_static", "moe_router_logits")
 STAGES = ("route", "permute", "quant_x", "gemm_gateup", "quant_h", "gemm_down", "combine")
 
 
@@ -84,6 +84,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             L.moe_profile_stage_name.restype = ctypes.c_char_p
             L.moe_launch_count.argtypes = [P]
             L.moe_launch_count.restype = ctypes.c_int
+            L.moe_router_logits.argtypes = [P, I32, P, P, P, P]
+            L.moe_router_logits.restype = ctypes.c_int
             L.moe_route_static.argtypes = [I32, I32, I32, P, P, P, P, P, P, P]
             L.moe_route_static.restype = ctypes.c_int
             _lib = L
@@ -200,6 +202,22 @@ def moe_route(plan: Plan, logits: torch.Tensor, workspace: torch.Tensor, out: di
                                   _ptr(out["counts"]), _ptr(out["offsets"]), _ptr(out["perm_tok"]),
                                   _ptr(workspace), workspace.numel(), _stream(stream))
     _check(rc, "moe_route", plan.handle)
+    return out
+
+
+def moe_router_logits(plan: Plan, x: torch.Tensor, w_router: torch.Tensor, out: torch.Tensor | None = None,
+                      stream=None) -> torch.Tensor:
+    """Router logits [T, E] fp32 = x [T, H] bf16 . w_router [E, H]^T bf16, on the tensor cores."""
+    d = plan.dims
+    T = x.shape[0]
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.shape[1] != d.H:
+        raise ValueError("x must be bf16 [T, H]")
+    if w_router.dtype != torch.bfloat16 or tuple(w_router.shape) != (d.E, d.H):
+        raise ValueError("w_router must be bf16 [E, H]")
+    if out is None:
+        out = torch.empty((T, d.E), dtype=torch.float32, device=x.device)
+    rc = load_library().moe_router_logits(plan.handle, T, _ptr(x), _ptr(w_router), _ptr(out), _stream(stream))
+    _check(rc, "moe_router_logits", plan.handle)
     return out
 
 

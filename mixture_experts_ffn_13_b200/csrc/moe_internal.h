@@ -95,6 +95,10 @@ cudaError_t launch_gemm_fp8(bool gateup, int bn, const GemmMaps &maps, const Gem
 cudaError_t launch_gemm_int4(bool gateup, int bn, const GemmMaps &maps, const GemmArgs &args,
                              int num_sms, cudaStream_t s);
 
+// Router logits: logits[T, E] = x[T, H] . W[E, H]^T (bf16 in, fp32 out) on the tensor cores.
+cudaError_t launch_router_gemm(const uint16_t *x, const uint16_t *w, float *logits, int T, int H, int E, int *status,
+                               int num_sms, cudaStream_t s);
+
 // Tensor-map encoding through the driver entry point (host).
 int encode_map_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, int elem_bytes,
                   uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_outer, bool swizzle128);

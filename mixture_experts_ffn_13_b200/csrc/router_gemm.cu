@@ -1,0 +1,196 @@
+// router_gemm.cu -- the router's logits, the dense 16-bit layer that feeds step A1:
+// logits[T, E] = x[T, H] . W_router[E, H]^T, bf16 inputs, fp32 accumulation and output.
+//
+// Page "Flash-Next 在 GPU 上到底在算什麼", section "② 密集 16-bit 層": the router is one of the
+// small dense layers every token passes through; it stays in 16 bits and runs on the tensor
+// cores.  Page "把 397B MoE 榨進 TPU7x", section "數值驗證": the gating path is checked against a
+// high-precision reference because small drifts can reorder the top-k.
+//
+// Design (B200): the same operand roles as the expert GEMMs -- the MMA's 128-row M side is a
+// tile of router weight rows (experts), the N side a BN-token tile -- with a persistent grid
+// over (expert tile, token tile) pairs, warp 0 issuing TMA loads of 64-element K slices
+// (128-byte swizzle) into an NS-deep ring, warp 1 issuing tcgen05.mma.kind::f16 from one
+// thread into one of two TMEM accumulators, and warps 2-5 writing the finished tile as fp32
+// (lane = expert, consecutive lanes store consecutive logits of one token).
+#include "gemm_common.cuh"
+#include "launch.cuh"
+#include "sm100.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kRKE = 64;  // K elements per stage (128 bytes of bf16)
+
+template <int BN>
+struct RCfg {
+    static constexpr int A_BYTES = kTileM * kRKE * 2;  // 16 KB
+    static constexpr int B_BYTES = BN * kRKE * 2;
+    static constexpr int STAGE = A_BYTES + B_BYTES;
+    static constexpr int NS = (200 * 1024) / STAGE < 12 ? (200 * 1024) / STAGE : 12;
+    static constexpr int THREADS = 64 + 128;
+    static constexpr int SMEM = 1024 + NS * STAGE + 8 * (2 * NS + 4) + 16;
+    static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "1024-byte aligned tiles");
+};
+
+struct RouterArgs {
+    int T, H, E;
+    float *logits;
+    int *status;
+    uint64_t timeout_ns;
+};
+
+template <int BN>
+__global__ void __launch_bounds__(RCfg<BN>::THREADS, 1)
+    router_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
+                       const __grid_constant__ RouterArgs a)
+{
+    using C = RCfg<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::NS * C::STAGE);
+    uint64_t *empty = full + C::NS;
+    uint64_t *accf = empty + C::NS;  // 2
+    uint64_t *acce = accf + 2;       // 2
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(acce + 2);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::NS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&accf[s], 1);
+            mbar_init(&acce[s], 4);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&map_w);
+        tma_prefetch_desc(&map_x);
+    }
+    constexpr int kCols = 2 * BN < 32 ? 32 : 2 * BN;
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, kCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+    griddep_wait();
+    griddep_launch_dependents();
+
+    const int net = (a.E + kTileM - 1) / kTileM;  // the last expert tile may be partial
+    const int ntt = (a.T + BN - 1) / BN;
+    const int total = net * ntt;
+    const int nkc = a.H / kRKE;
+    if (warp == 0) {
+        if (lane == 0) {
+            const uint64_t pol_x = l2_policy_evict_last();
+            uint32_t it = 0;
+            for (int w = blockIdx.x; w < total; w += gridDim.x) {
+                const int et = w % net, tt = w / net;  // consecutive tiles share the token tile
+                for (int kc = 0; kc < nkc; ++kc, ++it) {
+                    const int s = it % C::NS;
+                    if (!mbar_wait(&empty[s], ((it / C::NS) & 1) ^ 1, abort_flag, a.status, a.timeout_ns)) goto done;
+                    uint8_t *st = smem + s * C::STAGE;
+                    mbar_arrive_expect_tx(&full[s], C::STAGE);
+                    tma_load_2d(st, &map_w, &full[s], kc * kRKE, et * kTileM);
+                    tma_load_2d_hint(st + C::A_BYTES, &map_x, &full[s], kc * kRKE, tt * BN, pol_x);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t kIdesc = instr_desc(kTileM, BN, 1, 1);
+            uint32_t it = 0, ti = 0;
+            for (int w = blockIdx.x; w < total; w += gridDim.x, ++ti) {
+                const int slot = ti & 1;
+                if (!mbar_wait(&acce[slot], ((ti >> 1) & 1) ^ 1, abort_flag, a.status, a.timeout_ns)) goto done;
+                tc_fence_after();
+                const uint32_t d = tmem_base + slot * BN;
+                for (int kc = 0; kc < nkc; ++kc, ++it) {
+                    const int s = it % C::NS;
+                    if (!mbar_wait(&full[s], (it / C::NS) & 1, abort_flag, a.status, a.timeout_ns)) goto done;
+                    tc_fence_after();
+                    uint8_t *st = smem + s * C::STAGE;
+                    const uint64_t da = smem_desc_sw128(st), db = smem_desc_sw128(st + C::A_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < kRKE / 16; ++kk)
+                        mma_bf16(d, da + 2 * kk, db + 2 * kk, kIdesc, (kc > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(&empty[s]);
+                }
+                mma_commit(&accf[slot]);
+            }
+        }
+    } else {
+        const int q = warp & 3;
+        const int e_in = q * 32 + lane;
+        uint32_t ti = 0;
+        for (int w = blockIdx.x; w < total; w += gridDim.x, ++ti) {
+            const int et = w % net, tt = w / net;
+            const int slot = ti & 1;
+            const bool ok = mbar_wait(&accf[slot], (ti >> 1) & 1, abort_flag, a.status, a.timeout_ns);
+            if (!__all_sync(0xffffffffu, ok)) goto done;
+            tc_fence_after();
+            const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + slot * BN;
+            const int e = et * kTileM + e_in;
+            const int t0 = tt * BN;
+#pragma unroll
+            for (int c0 = 0; c0 < BN; c0 += 16) {
+                float v[16];
+                tmem_ld16(tb + c0, v);
+                tmem_wait_ld(v);
+#pragma unroll
+                for (int c = 0; c < 16; ++c)
+                    if (t0 + c0 + c < a.T && e < a.E) a.logits[(size_t)(t0 + c0 + c) * a.E + e] = v[c];
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acce[slot]);
+        }
+    }
+done:
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kCols);
+    }
+}
+
+template <int BN>
+cudaError_t launch_rt(const CUtensorMap &mw, const CUtensorMap &mx, const RouterArgs &a, int num_sms, cudaStream_t s)
+{
+    using C = RCfg<BN>;
+    auto kern = router_gemm_kernel<BN>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    const int tiles = ((a.E + kTileM - 1) / kTileM) * ((a.T + BN - 1) / BN);
+    const int grid = tiles < num_sms ? tiles : num_sms;
+    return launch_pdl(kern, dim3(grid), dim3(C::THREADS), C::SMEM, s, mw, mx, a);
+}
+
+}  // namespace
+
+// Router logits for T tokens (H a multiple of 64; any E -- a partial last expert tile reads
+// zeros past row E and stores nothing there).  The token tile is 64 rows for batches of at
+// least 256 tokens and 32 below.
+cudaError_t launch_router_gemm(const uint16_t *x, const uint16_t *w, float *logits, int T, int H, int E, int *status,
+                               int num_sms, cudaStream_t s)
+{
+    if (T <= 0) return cudaSuccess;
+    const int bn = T >= 256 ? 64 : 32;
+    CUtensorMap mw, mx;
+    int rc = encode_map_2d(&mw, w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, E, kRKE, kTileM, true);
+    rc |= encode_map_2d(&mx, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, T, kRKE, bn, true);
+    if (rc) return cudaErrorInvalidValue;
+    RouterArgs a{T, H, E, logits, status, kDefaultTimeoutNs};
+    return bn == 64 ? launch_rt<64>(mw, mx, a, num_sms, s) : launch_rt<32>(mw, mx, a, num_sms, s);
+}
+
+}  // namespace moe

@@ -60,7 +60,7 @@ PROFILE_CONFIGS = {
 
 # tensor ids for the per-tensor generators
 _TID = {"x": 1, "logits": 2, "bias": 3, "rank": 4, "w_gate": 5, "w_up": 6, "w_down": 7,
-        "ws_gate": 8, "ws_up": 9, "ws_down": 10}
+        "ws_gate": 8, "ws_up": 9, "ws_down": 10, "w_router": 11}
 
 
 def _gen(seed: int, tid: int, device) -> torch.Generator:
@@ -142,6 +142,18 @@ def make_layer(name_or_cfg, device="cpu", **overrides) -> dict:
         out["ws_up"], out["ss_up"] = _weights(seed, _TID["ws_up"], (1, Is, H), H, wfmt, device)
         out["ws_down"], out["ss_down"] = _weights(seed, _TID["ws_down"], (1, H, Is), Is, wfmt, device)
     return out
+
+
+def make_router(name_or_cfg, device="cpu", **overrides) -> torch.Tensor:
+    """Router weights W_router [E, H] ~ N(0, 1/H), bf16 (so x . W_router^T ~ N(0, 1))."""
+    if isinstance(name_or_cfg, str):
+        cfg = dict(CONFIGS[name_or_cfg] if name_or_cfg in CONFIGS else PROFILE_CONFIGS[name_or_cfg])
+    else:
+        cfg = dict(name_or_cfg)
+    cfg.update(overrides)
+    g = _gen(cfg["seed"], _TID["w_router"], device)
+    w = torch.randn((cfg["E"], cfg["H"]), generator=g, device=device) / math.sqrt(cfg["H"])
+    return w.to(torch.bfloat16)
 
 
 def to_numpy(layer: dict) -> dict:

@@ -61,6 +61,7 @@ def lib():
             L.orc_double_to_bf16.restype = ctypes.c_uint16
             L.orc_double_to_bf16.argtypes = [ctypes.c_double]
             L.orc_route.argtypes = [I, I, I, P, P, P]
+            L.orc_router_logits.argtypes = [I, I, I, P, P, P, P]
             L.orc_permute.argtypes = [I, I, I, P, P, P, P, P]
             L.orc_quant_row_fp8.argtypes = [I, P, P, P]
             L.orc_quant_rows_bf16.argtypes = [I, I, P, P, P]
@@ -115,6 +116,20 @@ def route(logits: np.ndarray, k: int):
     if rc != 0:
         raise ValueError("oracle route: bad arguments")
     return idx, w
+
+
+def router_logits(x_bits: np.ndarray, w_bits: np.ndarray):
+    """Router logits in fp64 from bf16 x [T,H] and W [E,H] (bit patterns) ->
+    (logits float64 [T,E], bound float64 [T,E] = sum |x_i w_i|)."""
+    x_bits, w_bits = _c(x_bits, np.uint16), _c(w_bits, np.uint16)
+    T, H = x_bits.shape
+    E = w_bits.shape[0]
+    lg = np.empty((T, E), np.float64)
+    bd = np.empty((T, E), np.float64)
+    rc = lib().orc_router_logits(T, H, E, _p(x_bits), _p(w_bits), _p(lg), _p(bd))
+    if rc != 0:
+        raise ValueError("oracle router: bad arguments")
+    return lg, bd
 
 
 def permute(topk_idx: np.ndarray, E: int):

@@ -215,6 +215,31 @@ int orc_route(int T, int E, int k, const float *logits, int32_t *topk_idx, doubl
 }
 
 /* ------------------------------------------------------------------------------------ */
+/* router logits -- [P5] ② (the router is a dense 16-bit layer): logits = x . W_r^T       */
+/* ------------------------------------------------------------------------------------ */
+
+/* logits[t, e] = sum_i x[t, i] * w[e, i] with bf16 inputs, in fp64 (each product of two bf16
+ * values is exact; the sum of H of them is exact to ~1e-16 relative).  bound[t, e] (optional)
+ * receives sum_i |x[t, i] * w[e, i]|, the scale of the rounding error any other summation
+ * order can make. */
+int orc_router_logits(int T, int H, int E, const uint16_t *x, const uint16_t *w, double *logits, double *bound)
+{
+    if (T < 0 || H < 1 || E < 1) return -1;
+    for (int t = 0; t < T; ++t)
+        for (int e = 0; e < E; ++e) {
+            double acc = 0.0, mag = 0.0;
+            for (int i = 0; i < H; ++i) {
+                double p = orc_bf16_to_double(x[(size_t)t * H + i]) * orc_bf16_to_double(w[(size_t)e * H + i]);
+                acc += p;
+                mag += fabs(p);
+            }
+            logits[(size_t)t * E + e] = acc;
+            if (bound) bound[(size_t)t * E + e] = mag;
+        }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------------------ */
 /* A3: permute -- [P2] contiguous per-expert groups, packed (expert, token) sort key; R4  */
 /* ------------------------------------------------------------------------------------ */
 

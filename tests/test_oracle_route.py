@@ -110,3 +110,21 @@ def test_permute_matches_lexsort(orc):
     order = np.lexsort((t_flat, e_flat))  # primary key expert, then token
     assert np.array_equal(perm, t_flat[order])
     assert np.array_equal(np.bincount(e_flat, minlength=E), counts)
+
+
+def test_router_logits_against_exact_sums(orc):
+    """bf16 x bf16 products are exact in fp64; the oracle's logits equal an exact-rational sum."""
+    import torch
+    from fractions import Fraction
+    g = torch.Generator().manual_seed(11)
+    x = torch.randn(3, 64, generator=g).to(torch.bfloat16)
+    w = torch.randn(5, 64, generator=g).to(torch.bfloat16)
+    xb = x.view(torch.int16).numpy().view(np.uint16)
+    wb = w.view(torch.int16).numpy().view(np.uint16)
+    lg, bd = orc.router_logits(xb, wb)
+    xf, wf = x.double().numpy(), w.double().numpy()
+    for t in range(3):
+        for e in range(5):
+            exact = sum(Fraction(float(a)) * Fraction(float(b)) for a, b in zip(xf[t], wf[e]))
+            assert abs(Fraction(lg[t, e]) - exact) <= Fraction(1, 2 ** 40) * (1 + abs(exact))
+            assert bd[t, e] == np.abs(xf[t] * wf[e]).sum()
