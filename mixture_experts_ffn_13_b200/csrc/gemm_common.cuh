@@ -18,17 +18,19 @@ struct TileInfo {
 
 // Work item w -> tile.  Routed items come first: group g owns items
 // [ttile[g]*nT, ttile[g+1]*nT), laid out n-tile major so consecutive items reuse the same
-// weight tile across the group's token tiles.  Shared-expert items follow.
+// weight tile across the group's token tiles.  Shared-expert items follow.  RT is the number
+// of output features (weight rows of one matrix) a tile covers: 128, or 64 when a 128-row
+// MMA tile holds 64 gate rows and the matching 64 up rows.
 // `stt` is a.ttile itself (read through the read-only cache) or a shared-memory copy of it
 // (E+1 entries; SMEM_TT), which keeps the binary search off global memory for kernels whose
 // tiles are short enough for its latency to show.
-template <int BN, bool SMEM_TT = false>
+template <int BN, bool SMEM_TT = false, int RT = kTileM>
 __device__ __forceinline__ TileInfo decode_tile(const GemmArgs &a, const int *stt, int w, int tot0)
 {
     auto tt = [&](int i) { return SMEM_TT ? stt[i] : __ldg(stt + i); };
     TileInfo t;
     if (w < tot0) {
-        const int nT = a.seg[0].N / kTileM;
+        const int nT = a.seg[0].N / RT;
         int lo = 0, hi = a.E - 1;
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
@@ -49,7 +51,7 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs &a, const int *st
         t.nt = nt;
         t.row0 = rbeg;
         t.nrows = min(BN, rend - rbeg);
-        t.wrow = g * a.seg[0].N + nt * kTileM;
+        t.wrow = g * a.seg[0].N + nt * RT;
     } else {
         const int ww = w - tot0;
         const int ntt = (a.T + BN - 1) / BN;
@@ -59,7 +61,7 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs &a, const int *st
         t.nt = nt;
         t.row0 = tt * BN;
         t.nrows = min(BN, a.T - t.row0);
-        t.wrow = nt * kTileM;
+        t.wrow = nt * RT;
     }
     return t;
 }
@@ -71,13 +73,16 @@ __device__ __forceinline__ void load_ttile(const GemmArgs &a, int *stt)
     __syncthreads();
 }
 
-__device__ __forceinline__ int total_tiles(const GemmArgs &a, int BN, int *tot0)
+__device__ __forceinline__ int total_tiles(const GemmArgs &a, int BN, int *tot0, int RT = kTileM)
 {
-    *tot0 = __ldg(a.ttile + a.E) * (a.seg[0].N / kTileM);
-    const int tot1 = a.nseg > 1 ? ((a.T + BN - 1) / BN) * (a.seg[1].N / kTileM) : 0;
+    *tot0 = __ldg(a.ttile + a.E) * (a.seg[0].N / RT);
+    const int tot1 = a.nseg > 1 ? ((a.T + BN - 1) / BN) * (a.seg[1].N / RT) : 0;
     return *tot0 + tot1;
 }
 
-__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
+// silu(g) * u = g / (1 + e^-g) * u with the hardware exponential and approximate division
+// (a few ulp in fp32, far below the accumulation's own rounding).  For g below about -88 the
+// denominator overflows to infinity and the approximate quotient is the exact limit 0.
+__device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
 
 }  // namespace moe

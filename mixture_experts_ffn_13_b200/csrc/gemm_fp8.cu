@@ -25,8 +25,19 @@
 //    the MMAs of the next blocks overlap the promotion of the previous ones.  The tile's
 //    activation scales s_x[row0 .. row0+BN, :] are staged in shared memory once per tile
 //    (double-buffered across tiles) and the weight scales are prefetched a block ahead.
-//  * gate|up: two weight tiles per stage share one activation tile; the epilogue computes
-//    h = silu(G) * U in fp32 and stores it.  down: one weight tile; y is stored in fp32.
+//  * gate|up, paired form (narrow token tiles): two 128-row weight tiles per stage (gate and
+//    up) share one activation tile and accumulate into two TMEM regions; the epilogue computes
+//    h = silu(G) * U in fp32 and stores it.
+//  * gate|up, interleaved form (token tiles of up to 192 rows): one 128-row weight tile holds 64
+//    gate rows and the matching 64 up rows, 16 of each per 32-lane TMEM quarter (gate rows at
+//    lanes 0-15, up rows at lanes 16-31), so one MMA per K step covers both and each thread's
+//    partner (lane ^ 16) holds the other projection of the same feature for the SwiGLU.  Each
+//    weight byte then meets up to 192 tokens per pass through shared memory, which is what
+//    bounds the narrow forms at prefill sizes (shared-memory bandwidth, not HBM).
+//  * down: one weight tile; y is stored in fp32.
+//  * Wide token tiles load activations in 64-row boxes, only as many as the tile has rows, and
+//    size the MMA's N to the tile's valid rows rounded up to 16.  The producer warp issues a
+//    stage's copies from separate lanes, one copy each.
 #include "moe_internal.h"
 #include "gemm_common.cuh"
 #include "launch.cuh"
@@ -41,11 +52,26 @@ constexpr int kStagesPerBlock = kBlockK / kKC;
 constexpr int kMaxKb = 16;   // activation-scale staging holds up to 16 blocks (K <= 8192)
 constexpr int kSmemLimit = 227 * 1024;
 
-template <int BN, bool GATEUP, int EW>
+// Activation boxes: narrow tiles load BN rows in one box; wide tiles load 64-row boxes.
+template <int BN>
+struct BoxOf {
+    static constexpr int ROWS = BN >= 64 ? 64 : BN;
+    static constexpr int BYTES = ROWS * kKC;
+};
+
+enum { kModeDown = 0, kModePair = 1, kModeInterleaved = 2 };
+
+template <int BN, int MODE, int EW>
 struct Fp8Cfg {
-    static constexpr int NA = GATEUP ? 2 : 1;
+    static constexpr bool GATEUP = MODE != kModeDown;
+    static constexpr bool PAIR = MODE == kModePair;
+    static constexpr bool ILV = MODE == kModeInterleaved;
+    static constexpr int RT = ILV ? kTileM / 2 : kTileM;  // output features per tile
+    static constexpr int NA = PAIR ? 2 : 1;
     static constexpr int A_BYTES = kTileM * kKC;
-    static constexpr int B_BYTES = BN * kKC;
+    // activation rows a stage holds: wide tiles round up to whole 64-row boxes
+    static constexpr int B_ROWS = BN >= 64 ? (BN + 63) / 64 * 64 : BN;
+    static constexpr int B_BYTES = B_ROWS * kKC;
     static constexpr int STAGE_BYTES = NA * A_BYTES + B_BYTES;
     static constexpr int SLOT_COLS = NA * BN;
     static constexpr int NSLOT = 512 / SLOT_COLS;
@@ -55,9 +81,11 @@ struct Fp8Cfg {
     static constexpr int THREADS = 64 + 32 * EW;
     // Wide tiles (BN >= 64) stage activation scales and the tile-prefix table in shared
     // memory; narrow (decode) tiles do not, and keep shared memory under 200 KB so that L1,
-    // which serves their scale loads, stays large.
+    // which serves their scale loads, stays large.  Tiles up to 128 rows double-buffer the
+    // scales across tiles; wider tiles keep one buffer so that five stages still fit.
     static constexpr bool WIDE = BN >= 64;
-    static constexpr int SX_BYTES = WIDE ? 2 * BN * kMaxKb * 4 : 0;
+    static constexpr int SX_BUFS = BN > 128 ? 1 : 2;
+    static constexpr int SX_BYTES = WIDE ? SX_BUFS * BN * kMaxKb * 4 : 0;
     static constexpr int TT_BYTES = WIDE ? (4 * (kMaxE + 1) + 15) & ~15 : 0;  // keeps the mbarriers 8-byte aligned
     static constexpr int BAR_BYTES = 8 * (2 * 16 + 2 * NSLOT) + 16;
     static constexpr int FIXED = 1024 + SX_BYTES + TT_BYTES + BAR_BYTES;
@@ -69,6 +97,7 @@ struct Fp8Cfg {
     static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "stage tiles must stay 1024-byte aligned");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M=128 is a multiple of 16 in [16, 256]");
     static_assert(EW % 4 == 0 && CPW % 16 == 0, "epilogue split");
+    static_assert(!ILV || CPW % 2 == 0, "interleaved stores pair columns");
     static_assert(NSLOT >= 1 && NS >= 2, "pipeline");
     static_assert((NS * STAGE_BYTES + SX_BYTES + TT_BYTES) % 16 == 0, "mbarriers must be 8-byte aligned");
 };
@@ -76,17 +105,20 @@ struct Fp8Cfg {
 // Named barrier among the EW epilogue warps (ids 2..2+EW-1); barrier 0 is __syncthreads.
 __device__ __forceinline__ void epi_sync(int nthreads) { asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory"); }
 
-template <int BN, bool GATEUP, int EW>
-__global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
+template <int BN, int MODE, int EW>
+__global__ void __launch_bounds__(Fp8Cfg<BN, MODE, EW>::THREADS, 1)
     gemm_fp8_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmArgs args)
 {
-    using C = Fp8Cfg<BN, GATEUP, EW>;
+    using C = Fp8Cfg<BN, MODE, EW>;
+    constexpr bool GATEUP = C::GATEUP;
+    constexpr int RT = C::RT;
+    constexpr int kBoxRows = BoxOf<BN>::ROWS, kBoxB = BoxOf<BN>::BYTES;
     // Wide token tiles stage the tile's activation scales in shared memory; narrow (decode)
     // tiles read them straight from L2 in the promotion loop, which measured faster there.
     constexpr bool kStageSx = C::WIDE;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float *sxbuf = reinterpret_cast<float *>(smem + C::NS * C::STAGE_BYTES);  // [2][BN * kMaxKb]
+    float *sxbuf = reinterpret_cast<float *>(smem + C::NS * C::STAGE_BYTES);  // [SX_BUFS][BN * kMaxKb]
     int *stt = reinterpret_cast<int *>(smem + C::NS * C::STAGE_BYTES + C::SX_BYTES);  // [E + 1]
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::NS * C::STAGE_BYTES + C::SX_BYTES + C::TT_BYTES);
     uint64_t *empty = full + C::NS;
@@ -131,29 +163,70 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
     const int *ttab = kStageSx ? stt : args.ttile;
 
     int tot0;
-    const int total = total_tiles(args, BN, &tot0);
+    const int total = total_tiles(args, BN, &tot0, RT);
     int *status = args.status;
     const uint64_t tmo = args.timeout_ns;
 
     if (warp == 0) {
         // ------------------------------ TMA producer ------------------------------
-        if (lane == 0) {
-            const uint64_t pol_w = l2_policy_evict_first();
-            const uint64_t pol_x = l2_policy_evict_last();
-            uint32_t it = 0;
-            for (int w = blockIdx.x; w < total; w += gridDim.x) {
-                const TileInfo tl = decode_tile<BN, kStageSx>(args, ttab, w, tot0);
-                const int nkc = args.seg[tl.seg].K / kKC;
-                for (int kc = 0; kc < nkc; ++kc, ++it) {
-                    const int s = it % C::NS;
-                    const uint32_t ph = (it / C::NS) & 1;
-                    if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, status, tmo)) goto done;
-                    uint8_t *st = smem + s * C::STAGE_BYTES;
-                    mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
-                    tma_load_2d_hint(st, &maps.a0[tl.seg], &full[s], kc * kKC, tl.wrow, pol_w);
-                    if (GATEUP) tma_load_2d_hint(st + C::A_BYTES, &maps.a1[tl.seg], &full[s], kc * kKC, tl.wrow, pol_w);
-                    tma_load_2d_hint(st + C::NA * C::A_BYTES, &maps.b[tl.seg], &full[s], kc * kKC, tl.row0, pol_x);
+        // Wide tiles: lane 0 claims a free stage and posts its byte count; then each lane
+        // issues at most one of the stage's TMA copies, so a stage of several boxes is issued
+        // in parallel rather than one copy after another.  Narrow tiles (two copies a stage)
+        // run the producer on lane 0 alone, which measured faster there.
+        if (!C::WIDE && lane != 0) goto done;
+        const uint64_t pol_w = l2_policy_evict_first();
+        const uint64_t pol_x = l2_policy_evict_last();
+        uint32_t it = 0;
+        for (int w = blockIdx.x; w < total; w += gridDim.x) {
+            const TileInfo tl = decode_tile<BN, kStageSx, RT>(args, ttab, w, tot0);
+            const GemmSeg &sg = args.seg[tl.seg];
+            const int nkc = sg.K / kKC;
+            // activation boxes: the whole BN-row tile for narrow tiles, else 64-row boxes up to
+            // the tile's valid rows
+            const int nbox = C::WIDE ? (tl.nrows + kBoxRows - 1) / kBoxRows : 1;
+            // weight copies: the paired form loads two 128-row tiles; the interleaved form one
+            // 4-D box or eight 16-row boxes
+            const int nwa = C::ILV ? (sg.ilv4d ? 1 : 8) : C::NA;
+            const uint32_t tx = C::NA * C::A_BYTES + nbox * kBoxB;
+            for (int kc = 0; kc < nkc; ++kc, ++it) {
+                const int s = it % C::NS;
+                const uint32_t ph = (it / C::NS) & 1;
+                bool ok = true;
+                if (lane == 0) {
+                    ok = mbar_wait(&empty[s], ph ^ 1, abort_flag, status, tmo);
+                    if (ok) mbar_arrive_expect_tx(&full[s], tx);
                 }
+                if constexpr (C::WIDE) ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) goto done;
+                uint8_t *st = smem + s * C::STAGE_BYTES;
+                const int x = kc * kKC;
+                if constexpr (!C::WIDE) {
+                    tma_load_2d_hint(st, &maps.a0[tl.seg], &full[s], x, tl.wrow, pol_w);
+                    if (C::PAIR) tma_load_2d_hint(st + C::A_BYTES, &maps.a1[tl.seg], &full[s], x, tl.wrow, pol_w);
+                    tma_load_2d_hint(st + C::NA * C::A_BYTES, &maps.b[tl.seg], &full[s], x, tl.row0, pol_x);
+                    continue;
+                }
+                if (lane < nwa) {
+                    if constexpr (C::ILV) {
+                        if (sg.ilv4d) {
+                            tma_load_4d_hint(st, &maps.a0[tl.seg], &full[s], x, 0, 0, tl.wrow >> 4, pol_w);
+                        } else {
+                            // lane 2q loads gate rows wrow+16q.. to tile rows 32q.., lane 2q+1 the
+                            // matching up rows to tile rows 32q+16..
+                            const int q = lane >> 1, u = lane & 1;
+                            tma_load_2d_hint(st + q * 4096 + u * 2048, u ? &maps.a1[tl.seg] : &maps.a0[tl.seg],
+                                             &full[s], x, tl.wrow + 16 * q, pol_w);
+                        }
+                    } else {
+                        tma_load_2d_hint(st + lane * C::A_BYTES, lane ? &maps.a1[tl.seg] : &maps.a0[tl.seg],
+                                         &full[s], x, tl.wrow, pol_w);
+                    }
+                } else if (lane < nwa + nbox) {
+                    const int j = lane - nwa;
+                    tma_load_2d_hint(st + C::NA * C::A_BYTES + j * kBoxB, &maps.b[tl.seg], &full[s], x,
+                                     tl.row0 + j * kBoxRows, pol_x);
+                }
+                __syncwarp();
             }
         }
     } else if (warp == 1) {
@@ -161,7 +234,7 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
         if (lane == 0) {
             uint32_t it = 0, ai = 0;
             for (int w = blockIdx.x; w < total; w += gridDim.x) {
-                const TileInfo tl = decode_tile<BN, kStageSx>(args, ttab, w, tot0);
+                const TileInfo tl = decode_tile<BN, kStageSx, RT>(args, ttab, w, tot0);
                 // MMA N = the tile's valid rows rounded up to 16 for wide tiles (a group's last,
                 // partial token tile costs no tensor-core work for absent rows); narrow
                 // decode tiles keep N = BN, which measured faster
@@ -191,7 +264,7 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
                         for (int kk = 0; kk < kKC / 32; ++kk) {
                             const uint32_t acc = (kc > kb * kStagesPerBlock || kk > 0) ? 1u : 0u;
                             mma_f8(d0, da0 + 2 * kk, db + 2 * kk, kIdesc, acc);
-                            if (GATEUP) mma_f8(d1, da1 + 2 * kk, db + 2 * kk, kIdesc, acc);
+                            if (C::PAIR) mma_f8(d1, da1 + 2 * kk, db + 2 * kk, kIdesc, acc);
                         }
                         mma_commit(&empty[s]);
                     }
@@ -204,14 +277,17 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
         const int ew = warp - 2;
         const int q = warp & 3;               // TMEM lanes 32q..32q+31 are reachable from this warp
         const int cbase = (ew >> 2) * C::CPW; // this warp's first token column
-        const int r = q * 32 + lane;          // weight row within the tile
+        // weight row of this thread's TMEM lane: tile row q*32+lane, or for the interleaved
+        // form feature 16q + (lane & 15) of the tile, gate for lanes < 16 and up above
+        bool is_up = C::ILV && lane >= 16;  // refined per segment below (up rows may come first)
+        const int r = C::ILV ? q * 16 + (lane & 15) : q * 32 + lane;
         const int etid = ew * 32 + lane;      // index among the epilogue threads
         uint32_t ai = 0;
         int ti = 0;
         // The tile's activation scales s_x[row0 + c, kb] live in shared memory (two buffers,
         // alternating by tile).  The next tile's values are loaded into registers while the
         // current tile is promoted, and stored at the end of it, so no tile waits on them.
-        constexpr int NPF = (BN * kMaxKb) / (32 * EW);
+        constexpr int NPF = C::SX_BUFS == 2 ? (BN * kMaxKb) / (32 * EW) : 1;
         float pf[NPF];
         auto load_sx = [&](const TileInfo &t) {
             const GemmSeg &g = args.seg[t.seg];
@@ -237,39 +313,51 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
                 }
             }
         };
-        if constexpr (kStageSx) {
+        constexpr bool kSxDouble = kStageSx && C::SX_BUFS == 2;
+        if constexpr (kSxDouble) {
             if ((int)blockIdx.x < total) {
-                const TileInfo t0 = decode_tile<BN, kStageSx>(args, ttab, blockIdx.x, tot0);
+                const TileInfo t0 = decode_tile<BN, kStageSx, RT>(args, ttab, blockIdx.x, tot0);
                 load_sx(t0);
                 store_sx(t0, sxbuf);
             }
             epi_sync(32 * EW);
         }
         for (int w = blockIdx.x; w < total; w += gridDim.x, ++ti) {
-            const TileInfo tl = decode_tile<BN, kStageSx>(args, ttab, w, tot0);
+            const TileInfo tl = decode_tile<BN, kStageSx, RT>(args, ttab, w, tot0);
             const GemmSeg &sg = args.seg[tl.seg];
             const int K = sg.K;
             const int nkb = (K + kBlockK - 1) / kBlockK;
-            const float *sxs = sxbuf + (ti & 1) * (BN * kMaxKb);
+            if constexpr (C::ILV) is_up = (lane >= 16) != (sg.ilv4d && sg.up_lo);
+            const float *sxs = sxbuf + (kSxDouble ? (ti & 1) * (BN * kMaxKb) : 0);
             const int wn = w + gridDim.x;
             TileInfo tn;
-            if (kStageSx && wn < total) {
-                tn = decode_tile<BN, kStageSx>(args, ttab, wn, tot0);
+            if constexpr (kStageSx && !kSxDouble) {  // one buffer: copy this tile's scales now
+                for (int i = etid; i < BN * nkb; i += 32 * EW) {
+                    const int c = i / nkb, kb = i - c * nkb;
+                    const int row = min(tl.row0 + c, sg.rows - 1);
+                    sxbuf[kb * BN + c] = __ldg(sg.sx + (size_t)row * nkb + kb);
+                }
+                epi_sync(32 * EW);
+            }
+            if (kSxDouble && wn < total) {
+                tn = decode_tile<BN, kStageSx, RT>(args, ttab, wn, tot0);
                 load_sx(tn);
             }
-            const float *sw0 = static_cast<const float *>(sg.sw0) + (size_t)(tl.wrow + r) * nkb;
-            const float *sw1 = GATEUP ? static_cast<const float *>(sg.sw1) + (size_t)(tl.wrow + r) * nkb : nullptr;
-            float acc0[C::CPW], acc1[GATEUP ? C::CPW : 1];
+            // the interleaved form reads gate scales on lanes < 16 and up scales above; the
+            // paired form reads both
+            const float *sw0 = static_cast<const float *>(is_up ? sg.sw1 : sg.sw0) + (size_t)(tl.wrow + r) * nkb;
+            const float *sw1 = C::PAIR ? static_cast<const float *>(sg.sw1) + (size_t)(tl.wrow + r) * nkb : nullptr;
+            float acc0[C::CPW], acc1[C::PAIR ? C::CPW : 1];
 #pragma unroll
             for (int c = 0; c < C::CPW; ++c) acc0[c] = 0.0f;
-            if constexpr (GATEUP) {
+            if constexpr (C::PAIR) {
 #pragma unroll
                 for (int c = 0; c < C::CPW; ++c) acc1[c] = 0.0f;
             }
             float s0n = 0.0f, s1n = 0.0f;
             if constexpr (kStageSx) {
                 s0n = __ldg(sw0);
-                if (GATEUP) s1n = __ldg(sw1);
+                if (C::PAIR) s1n = __ldg(sw1);
             }
             for (int kb = 0; kb < nkb; ++kb, ++ai) {
                 const int slot = ai % C::NSLOT;
@@ -280,11 +368,11 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
                     s1 = s1n;
                     if (kb + 1 < nkb) {
                         s0n = __ldg(sw0 + kb + 1);
-                        if (GATEUP) s1n = __ldg(sw1 + kb + 1);
+                        if (C::PAIR) s1n = __ldg(sw1 + kb + 1);
                     }
                 } else {
                     s0 = __ldg(sw0 + kb);
-                    s1 = GATEUP ? __ldg(sw1 + kb) : 0.0f;
+                    s1 = C::PAIR ? __ldg(sw1 + kb) : 0.0f;
                 }
                 const bool ok = mbar_wait(&accf[slot], aph, abort_flag, status, tmo);
                 if (!__all_sync(0xffffffffu, ok)) goto done;
@@ -295,7 +383,7 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
                 for (int c0 = 0; c0 < C::CPW; c0 += 16) {
                     float v[16], u[16];
                     tmem_ld16(tb + c0, v);
-                    if constexpr (GATEUP) {
+                    if constexpr (C::PAIR) {
                         tmem_ld16(tb + BN + c0, u);
                         tmem_wait_ld2(v, u);
                     } else {
@@ -311,7 +399,7 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
                             sx = __ldg(sg.sx + (size_t)row * nkb + kb);
                         }
                         acc0[c0 + c] = fmaf(v[c], s0 * sx, acc0[c0 + c]);
-                        if constexpr (GATEUP) acc1[c0 + c] = fmaf(u[c], s1 * sx, acc1[c0 + c]);
+                        if constexpr (C::PAIR) acc1[c0 + c] = fmaf(u[c], s1 * sx, acc1[c0 + c]);
                     }
                 }
                 tc_fence_before();
@@ -319,21 +407,38 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, GATEUP, EW>::THREADS, 1)
                 if (lane == 0) mbar_arrive(&acce[slot]);
             }
             float *out = static_cast<float *>(sg.out);
-            const int n = tl.nt * kTileM + r;
+            const int n = tl.nt * RT + r;
+            if constexpr (C::ILV) {
+                // partner lane (lane ^ 16) holds the other projection of feature n.  Of each
+                // column pair the lower lane (odd = 0) finishes the even column and the upper lane
+                // the odd one; each sends its partner the value for the partner's column.
+                const bool odd = lane >= 16;
+                float *orow = out + (size_t)(tl.row0 + cbase + (odd ? 1 : 0)) * sg.N + n;
 #pragma unroll
-            for (int c = 0; c < C::CPW; ++c) {
-                if (cbase + c < tl.nrows) {
-                    float v;
-                    if constexpr (GATEUP)
-                        v = silu_mul(acc0[c], acc1[c]);
-                    else
-                        v = acc0[c];
-                    out[(size_t)(tl.row0 + cbase + c) * sg.N + n] = v;
+                for (int c = 0; c < C::CPW; c += 2) {
+                    const float other = __shfl_xor_sync(0xffffffffu, odd ? acc0[c] : acc0[c + 1], 16);
+                    const float mine = odd ? acc0[c + 1] : acc0[c];
+                    const float v = is_up ? silu_mul(other, mine) : silu_mul(mine, other);
+                    if (cbase + c + (odd ? 1 : 0) < tl.nrows) orow[(size_t)c * sg.N] = v;
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < C::CPW; ++c) {
+                    if (cbase + c < tl.nrows) {
+                        float v;
+                        if constexpr (C::PAIR)
+                            v = silu_mul(acc0[c], acc1[c]);
+                        else
+                            v = acc0[c];
+                        out[(size_t)(tl.row0 + cbase + c) * sg.N + n] = v;
+                    }
                 }
             }
-            if constexpr (kStageSx) {
+            if constexpr (kSxDouble) {
                 if (wn < total) store_sx(tn, sxbuf + ((ti + 1) & 1) * (BN * kMaxKb));
                 epi_sync(32 * EW);
+            } else if constexpr (kStageSx) {
+                epi_sync(32 * EW);  // every thread is done with the buffer before it is refilled
             }
         }
     }
@@ -347,11 +452,11 @@ done:
     }
 }
 
-template <int BN, bool GATEUP, int EW>
+template <int BN, int MODE, int EW>
 cudaError_t launch_t(const GemmMaps &maps, const GemmArgs &args, int num_sms, cudaStream_t s)
 {
-    using C = Fp8Cfg<BN, GATEUP, EW>;
-    auto kern = gemm_fp8_kernel<BN, GATEUP, EW>;
+    using C = Fp8Cfg<BN, MODE, EW>;
+    auto kern = gemm_fp8_kernel<BN, MODE, EW>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     return launch_pdl(kern, dim3(num_sms), dim3(C::THREADS), C::SMEM, s, maps, args);
@@ -366,15 +471,20 @@ cudaError_t launch_gemm_fp8(bool gateup, int bn, const GemmMaps &maps, const Gem
         return cudaErrorInvalidValue;
     if (gateup) {
         switch (bn) {
-            case 32: return launch_t<32, true, 4>(maps, args, num_sms, s);
-            case 64: return launch_t<64, true, 8>(maps, args, num_sms, s);
+            case 32: return launch_t<32, kModePair, 4>(maps, args, num_sms, s);
+            case 64: return launch_t<64, kModePair, 8>(maps, args, num_sms, s);
+            case 128: return launch_t<128, kModeInterleaved, 8>(maps, args, num_sms, s);
+            case 160: return launch_t<160, kModeInterleaved, 8>(maps, args, num_sms, s);
+            case 192: return launch_t<192, kModeInterleaved, 12>(maps, args, num_sms, s);
             default: return cudaErrorInvalidValue;
         }
     }
     switch (bn) {
-        case 32: return launch_t<32, false, 4>(maps, args, num_sms, s);
-        case 64: return launch_t<64, false, 8>(maps, args, num_sms, s);
-        case 128: return launch_t<128, false, 8>(maps, args, num_sms, s);
+        case 32: return launch_t<32, kModeDown, 4>(maps, args, num_sms, s);
+        case 64: return launch_t<64, kModeDown, 8>(maps, args, num_sms, s);
+        case 128: return launch_t<128, kModeDown, 8>(maps, args, num_sms, s);
+        case 160: return launch_t<160, kModeDown, 8>(maps, args, num_sms, s);
+        case 192: return launch_t<192, kModeDown, 12>(maps, args, num_sms, s);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -114,7 +114,7 @@ int pick_bn(int T, int k, int E, bool fp8)
     const long avg = ((long)T * k + E - 1) / E;
     if (avg <= 48) return fp8 || avg <= 24 ? 32 : 64;
     if (!fp8) return 96;  // 4-bit: one tile per group up to ~1.5x the mean (dequant is per tile)
-    return avg <= 96 ? 64 : 128;
+    return avg <= 96 ? 64 : 192;  // 192: one pass over each weight tile for groups up to 192 rows
 }
 
 }  // namespace
@@ -133,6 +133,26 @@ int encode_map_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype,
                                 swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int encode_map_gateup_ilv(CUtensorMap *map, const void *gate, const void *up, uint64_t K, uint64_t rows, int *up_lo)
+{
+    std::call_once(g_encode_once, load_encode);
+    if (!g_encode) return MOE_ERR_CUDA;
+    const uintptr_t g = reinterpret_cast<uintptr_t>(gate), u = reinterpret_cast<uintptr_t>(up);
+    const bool lo_up = u < g;
+    const uintptr_t base = lo_up ? u : g, dist = lo_up ? g - u : u - g;
+    if (dist == 0 || dist % 16 || dist >= (uint64_t(1) << 40) || rows % 64 || K % 16) return MOE_ERR_UNSUPPORTED;
+    const cuuint64_t dims[4] = {K, 16, 2, rows / 16};
+    const cuuint64_t strides[3] = {K, dist, 16 * K};
+    const cuuint32_t box[4] = {128, 16, 2, 4};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, reinterpret_cast<void *>(base), dims, strides,
+                                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return MOE_ERR_UNSUPPORTED;
+    *up_lo = lo_up ? 1 : 0;
+    return MOE_OK;
 }
 
 }  // namespace moe
@@ -426,7 +446,12 @@ int moe_forward(moe_plan_t *p, int32_t T, const uint16_t *x, const float *logits
     const int H = d.H, I = d.I, Is = d.I_shared, k = d.k, E = d.E;
     const int A = T * k;
     const int bn_b = pick_bn(T, k, E, true);
-    const int bn_a = bn_b > 64 ? 64 : bn_b;  // gate|up holds two accumulators per column
+    // gate|up: narrow tiles pair the gate and up tiles (two accumulators per column); 192-row
+    // tiles interleave 64 gate and 64 up rows in one 128-row MMA tile
+    const int bn_a = bn_b;
+    const bool ilv = bn_a > 64;
+    const uint32_t wbox = ilv ? 16 : 128;  // weight rows per TMA box (2-D maps)
+    const uint32_t kXBox = bn_a < 64 ? bn_a : 64;  // activation rows per TMA box
 
     mark(0);
     cudaError_t e = launch_route(logits, T, E, k, b.topk_idx, b.topk_w, s);
@@ -464,14 +489,23 @@ int moe_forward(moe_plan_t *p, int32_t T, const uint16_t *x, const float *logits
     ag.status = p->d_status;
     ag.timeout_ns = kDefaultTimeoutNs;
     ag.seg[0] = GemmSeg{I, H, A, w->s_gate, w->s_up, sx, h};
-    rc = encode_map_2d(&mg.a0[0], w->w_gate, U8, 1, H, (uint64_t)E * I, 128, 128, true);
-    rc |= encode_map_2d(&mg.a1[0], w->w_up, U8, 1, H, (uint64_t)E * I, 128, 128, true);
-    rc |= encode_map_2d(&mg.b[0], xq, U8, 1, H, A, 128, bn_a, true);
+    // interleaved tiles load gate and up rows with one 4-D map where the two weight arrays'
+    // distance allows it, else with 16-row boxes of two 2-D maps
+    auto gateup_maps = [&](GemmSeg &sg, CUtensorMap &m0, CUtensorMap &m1, const void *wg, const void *wu,
+                           uint64_t rows) {
+        if (ilv && encode_map_gateup_ilv(&m0, wg, wu, H, rows, &sg.up_lo) == MOE_OK) {
+            sg.ilv4d = 1;
+            return 0;
+        }
+        return encode_map_2d(&m0, wg, U8, 1, H, rows, 128, wbox, true) |
+               encode_map_2d(&m1, wu, U8, 1, H, rows, 128, wbox, true);
+    };
+    rc = gateup_maps(ag.seg[0], mg.a0[0], mg.a1[0], w->w_gate, w->w_up, (uint64_t)E * I);
+    rc |= encode_map_2d(&mg.b[0], xq, U8, 1, H, A, 128, kXBox, true);
     if (shared) {
         ag.seg[1] = GemmSeg{Is, H, T, w->ss_gate, w->ss_up, sx_sh, h_sh};
-        rc |= encode_map_2d(&mg.a0[1], w->ws_gate, U8, 1, H, Is, 128, 128, true);
-        rc |= encode_map_2d(&mg.a1[1], w->ws_up, U8, 1, H, Is, 128, 128, true);
-        rc |= encode_map_2d(&mg.b[1], xq_sh, U8, 1, H, T, 128, bn_a, true);
+        rc |= gateup_maps(ag.seg[1], mg.a0[1], mg.a1[1], w->ws_gate, w->ws_up, (uint64_t)Is);
+        rc |= encode_map_2d(&mg.b[1], xq_sh, U8, 1, H, T, 128, kXBox, true);
     }
     if (rc) return MOE_ERR_CUDA;
     e = launch_gemm_fp8(true, bn_a, mg, ag, p->num_sms, s);
@@ -489,12 +523,13 @@ int moe_forward(moe_plan_t *p, int32_t T, const uint16_t *x, const float *logits
     GemmArgs ad = ag;
     ad.ttile = b.ttile_b;
     ad.seg[0] = GemmSeg{H, I, A, w->s_down, nullptr, sh, y};
+    const uint32_t kHBox = bn_b < 64 ? bn_b : 64;
     rc = encode_map_2d(&md.a0[0], w->w_down, U8, 1, I, (uint64_t)E * H, 128, 128, true);
-    rc |= encode_map_2d(&md.b[0], hq, U8, 1, I, A, 128, bn_b, true);
+    rc |= encode_map_2d(&md.b[0], hq, U8, 1, I, A, 128, kHBox, true);
     if (shared) {
         ad.seg[1] = GemmSeg{H, Is, T, w->ss_down, nullptr, sh_sh, y_sh};
         rc |= encode_map_2d(&md.a0[1], w->ws_down, U8, 1, Is, H, 128, 128, true);
-        rc |= encode_map_2d(&md.b[1], hq_sh, U8, 1, Is, T, 128, bn_b, true);
+        rc |= encode_map_2d(&md.b[1], hq_sh, U8, 1, Is, T, 128, kHBox, true);
     }
     if (rc) return MOE_ERR_CUDA;
     e = launch_gemm_fp8(false, bn_b, md, ad, p->num_sms, s);

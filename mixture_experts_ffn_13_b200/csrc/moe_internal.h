@@ -70,6 +70,8 @@ struct GemmSeg {
     const void *sw1;  // scales of the second weight matrix (up), gate|up only
     const float *sx;  // activation scales [rows, ceil(K/512)] (FP8 only)
     void *out;        // gate|up: h [rows, N]; down: y [rows, N]
+    int ilv4d;        // interleaved gate|up: a0 is one 4-D map that loads 16 gate + 16 up rows per quarter
+    int up_lo;        // interleaved gate|up: the up rows come first in each 32-row quarter
 };
 
 struct GemmArgs {
@@ -102,5 +104,11 @@ cudaError_t launch_router_gemm(const uint16_t *x, const uint16_t *w, float *logi
 // Tensor-map encoding through the driver entry point (host).
 int encode_map_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, int elem_bytes,
                   uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_outer, bool swizzle128);
+// One 4-D map over two byte matrices gate, up [rows, K] (rows a multiple of 16) whose box of
+// (128 bytes, 16 rows, 2 matrices, 4 row groups) lands in shared memory as 128 rows ordered
+// [16 rows of the lower-addressed matrix, the same 16 rows of the other] x 4.  Sets *up_lo
+// when the up matrix has the lower address.  Returns non-zero when the two matrices are too
+// far apart (or misaligned) for one map.
+int encode_map_gateup_ilv(CUtensorMap *map, const void *gate, const void *up, uint64_t K, uint64_t rows, int *up_lo);
 
 }  // namespace moe

@@ -114,6 +114,17 @@ __device__ __forceinline__ void tma_load_2d_hint(void *dst, const CUtensorMap *m
         : "memory");
 }
 
+// 4D tiled load with an L2 hint: the box at (c0 = innermost, c1, c2, c3).
+__device__ __forceinline__ void tma_load_4d_hint(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1,
+                                                 int c2, int c3, uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2], %7;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "l"(policy)
+        : "memory");
+}
+
 // Bring the box at (x, y) of a tensor map into L2 without writing shared memory (used to keep
 // more DRAM requests in flight than the shared-memory ring can hold).
 __device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *map, int x, int y)
