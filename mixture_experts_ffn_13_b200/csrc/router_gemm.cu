@@ -27,7 +27,7 @@ struct RCfg {
     static constexpr int A_BYTES = kTileM * kRKE * 2;  // 16 KB
     static constexpr int B_BYTES = BN * kRKE * 2;
     static constexpr int STAGE = A_BYTES + B_BYTES;
-    static constexpr int NS = (200 * 1024) / STAGE < 12 ? (200 * 1024) / STAGE : 12;
+    static constexpr int NS = (208 * 1024) / STAGE < 12 ? (208 * 1024) / STAGE : 12;
     static constexpr int THREADS = 64 + 128;
     static constexpr int SMEM = 1024 + NS * STAGE + 8 * (2 * NS + 4) + 16;
     static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "1024-byte aligned tiles");
@@ -178,19 +178,28 @@ cudaError_t launch_rt(const CUtensorMap &mw, const CUtensorMap &mx, const Router
 }  // namespace
 
 // Router logits for T tokens (H a multiple of 64; any E -- a partial last expert tile reads
-// zeros past row E and stores nothing there).  The token tile is 64 rows for batches of at
-// least 256 tokens and 32 below.
+// zeros past row E and stores nothing there).  The token tile is the widest of 16..256 rows
+// that still gives about 0.8 work items per SM: wide tiles read each router-weight byte for
+// more tokens, narrow ones spread small batches over more SMs.
 cudaError_t launch_router_gemm(const uint16_t *x, const uint16_t *w, float *logits, int T, int H, int E, int *status,
                                int num_sms, cudaStream_t s)
 {
     if (T <= 0) return cudaSuccess;
-    const int bn = T >= 256 ? 64 : 32;
+    const long net = (E + kTileM - 1) / kTileM;
+    int bn = 256;
+    while (bn > 16 && net * ((T + bn - 1) / bn) < (long)num_sms * 4 / 5) bn >>= 1;
     CUtensorMap mw, mx;
     int rc = encode_map_2d(&mw, w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, E, kRKE, kTileM, true);
     rc |= encode_map_2d(&mx, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, T, kRKE, bn, true);
     if (rc) return cudaErrorInvalidValue;
     RouterArgs a{T, H, E, logits, status, kDefaultTimeoutNs};
-    return bn == 64 ? launch_rt<64>(mw, mx, a, num_sms, s) : launch_rt<32>(mw, mx, a, num_sms, s);
+    switch (bn) {
+        case 256: return launch_rt<256>(mw, mx, a, num_sms, s);
+        case 128: return launch_rt<128>(mw, mx, a, num_sms, s);
+        case 64: return launch_rt<64>(mw, mx, a, num_sms, s);
+        case 32: return launch_rt<32>(mw, mx, a, num_sms, s);
+        default: return launch_rt<16>(mw, mx, a, num_sms, s);
+    }
 }
 
 }  // namespace moe
