@@ -27,12 +27,13 @@ METRIC = "MoE-layer tokens/s; % HBM roofline (decode) / % FP8 tensor peak (prefi
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM traffic of the gate|up GEMM per algorithmic byte, from one ncu capture
-# (dram__bytes_read.sum + dram__bytes_write.sum) of the decode-shaped profiling workload
-# (profiles/gemm_fp8_profile-decode_full.md), scaled to a decode launch by its algorithmic
-# bytes, with the hash of the kernel source it was taken on; null once the source changes.
-TRAFFIC = {"decode": {"kernel": "gemm_gateup", "ratio": (552.47872e6 + 4.306944e6) / 557973504.0,
-                      "src_sha": "d2072a50228e4526"}}
+# DRAM traffic of the gate|up GEMM per algorithmic byte: one ncu capture of
+# dram__bytes_read.sum + dram__bytes_write.sum for the gate|up launch of the decode-shaped
+# profiling workload (moe_synth "profile-decode": 552,472,064 + 3,480,320 bytes against
+# 549,519,360 algorithmic), scaled to a decode launch by its algorithmic bytes.  Stored with
+# the hash of the kernel source it was taken on; the figure is null once that source changes.
+TRAFFIC = {"decode": {"kernel": "gemm_gateup", "ratio": (552472064 + 3480320) / 549519360,
+                      "src_sha": "566b989ae73b3fca"}}
 
 
 def parse():
