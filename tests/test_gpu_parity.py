@@ -108,7 +108,36 @@ SMALL_FP8 = [
     dict(T=200, H=768, E=8, I=640, k=3, Is=0, seed=23, bias="zipf"),       # partial K blocks, >1 token tile
     dict(T=130, H=512, E=2, I=128, k=1, Is=512, seed=24, bias=None),       # groups of ~65 rows
     dict(T=64, H=1536, E=64, I=256, k=8, Is=0, seed=25, bias="zipf"),      # empty experts
+    # > 96 rows per group: 192-row token tiles, interleaved gate/up rows, 64-row activation boxes
+    dict(T=700, H=512, E=8, I=384, k=2, Is=128, seed=26, bias="normal"),   # groups above and below 192
+    dict(T=500, H=1024, E=4, I=256, k=2, Is=0, seed=27, bias="zipf"),      # one group of several tiles
+    dict(T=600, H=640, E=6, I=256, k=2, Is=256, seed=28, bias=None),       # partial 512-block of H
 ]
+
+
+def _up_below_gate(layer, g, u):
+    """Re-home two weight arrays in one buffer with the up array first (lower address)."""
+    wg, wu = layer[g], layer[u]
+    buf = torch.empty(wg.numel() + wu.numel(), dtype=wg.dtype, device=wg.device)
+    buf[: wu.numel()].copy_(wu.reshape(-1))
+    buf[wu.numel():].copy_(wg.reshape(-1))
+    layer[u] = buf[: wu.numel()].view(wu.shape)
+    layer[g] = buf[wu.numel():].view(wg.shape)
+
+
+def test_layer_fp8_wide_tiles_up_array_first():
+    """Interleaved gate/up tiles when the up weights sit below the gate weights in memory (the
+    4-D tensor map then orders each quarter up-first)."""
+    cfg = dict(T=400, H=512, E=4, I=128, k=2, Is=256, seed=29, bias=None, wfmt="fp8")
+    layer = moe_synth.make_layer(cfg, device="cuda")
+    _up_below_gate(layer, "w_gate", "w_up")
+    _up_below_gate(layer, "ws_gate", "ws_up")
+    assert layer["w_up"].data_ptr() < layer["w_gate"].data_ptr()
+    m = moe.MoELayer(layer)
+    out = m(layer["x"], layer["logits"])
+    assert moe.moe_get_status(m.plan) == 0
+    want, _, amb = oracle.layer(moe_synth.to_numpy(layer), ambiguity=True)
+    check_out(out, want, "layer (up first)", amb)
 
 
 @pytest.mark.parametrize("cfg", SMALL_FP8, ids=lambda c: f"T{c['T']}-H{c['H']}-E{c['E']}-I{c['I']}-k{c['k']}-Is{c['Is']}")
@@ -181,3 +210,36 @@ def _sampled_parity(name, n_sample=12):
 @pytest.mark.parametrize("name", ["tiny", "decode", "prefill", "skewed", "int4"])
 def test_layer_configs_sampled(name):
     _sampled_parity(name)
+
+
+def test_forward_replays_in_cuda_graph():
+    """moe_forward is stream-ordered and allocates nothing, so it can be captured in a CUDA
+    graph (its programmatic-dependent launches become graph edges); replays match the eager
+    call bit for bit, also after new inputs are copied into the captured buffers."""
+    cfg = dict(T=96, H=512, E=16, I=256, k=4, Is=128, seed=30, bias=None, wfmt="fp8")
+    layer = moe_synth.make_layer(cfg, device="cuda")
+    m = moe.MoELayer(layer)
+    x = layer["x"].clone()
+    logits = layer["logits"].clone()
+    ref = m(x, logits)
+    torch.cuda.synchronize()
+    out = torch.empty_like(ref)
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    with torch.cuda.graph(g, stream=side):
+        moe.moe_forward(m.plan, x, logits, m.weights, m.workspace, out=out)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
+    # new inputs through the same captured buffers
+    layer2 = moe_synth.make_layer(dict(cfg, seed=31), device="cuda")
+    x.copy_(layer2["x"])
+    logits.copy_(layer2["logits"])
+    g.replay()
+    torch.cuda.synchronize()
+    assert moe.moe_get_status(m.plan) == 0
+    L2 = moe_synth.to_numpy(layer)
+    L2["x"] = moe_synth.to_numpy(layer2)["x"]
+    L2["logits"] = layer2["logits"].cpu().numpy()
+    want, _, amb = oracle.layer(L2, ambiguity=True)
+    check_out(out, want, "graph replay", amb)
