@@ -306,30 +306,55 @@ def run_ours(args, ws, rank, local, cfg_name):
     prof_ms = sum(a.elapsed_time(b) for a, b in ev)
     moe.moe_profile_enable(m.plan, False)
 
-    # end to end through the public API with host buffers: H2D of x and logits from pinned
-    # memory, the layer, D2H of the output, every step inside the timed region
+    # end to end through the public API with host buffers: every step copies its x and logits
+    # from pinned host memory and reads its output back.  Copies run on their own streams,
+    # double-buffered, so step i+1's upload and step i-1's read-back overlap step i's layer
+    # (the copy engines and the SMs work at once); events order each buffer's reuse.  No L2
+    # flush here: every step streams the expert weights (far larger than L2) from HBM.
     xh = x.cpu().pin_memory()
     lh = logits.cpu().pin_memory()
-    oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    xd, ld = torch.empty_like(x), torch.empty_like(logits)
-    for _ in range(max(1, args.warmup)):
-        xd.copy_(xh, non_blocking=True)
-        ld.copy_(lh, non_blocking=True)
-        m(xd, ld, out=out)
-        oh.copy_(out, non_blocking=True)
+    oh = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    xd = [torch.empty_like(x) for _ in range(2)]
+    ld = [torch.empty_like(logits) for _ in range(2)]
+    od = [torch.empty_like(out) for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def e2e_run(n):
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        s_in.wait_event(t0)
+        for i in range(n):
+            b = i % 2
+            if i >= 2:
+                s_in.wait_event(ev_done[b])   # the layer two steps back has read xd[b], ld[b]
+            with torch.cuda.stream(s_in):
+                xd[b].copy_(xh, non_blocking=True)
+                ld[b].copy_(lh, non_blocking=True)
+            ev_in[b].record(s_in)
+            stream.wait_event(ev_in[b])
+            if i >= 2:
+                stream.wait_event(ev_out[b])  # od[b] has been read back
+            m(xd[b], ld[b], out=od[b], stream=stream)
+            ev_done[b].record(stream)
+            s_out.wait_event(ev_done[b])
+            with torch.cuda.stream(s_out):
+                oh[b].copy_(od[b], non_blocking=True)
+            ev_out[b].record(s_out)
+        for b in range(min(n, 2)):
+            stream.wait_event(ev_out[b])
+        t1.record(stream)
+        return t0, t1
+
+    e2e_run(max(2, args.warmup))
     torch.cuda.synchronize()
-    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     barrier(ws)
-    for i in range(args.steps):
-        flush.zero_()
-        e2e_ev[i][0].record(stream)
-        xd.copy_(xh, non_blocking=True)
-        ld.copy_(lh, non_blocking=True)
-        m(xd, ld, out=out)
-        oh.copy_(out, non_blocking=True)
-        e2e_ev[i][1].record(stream)
+    t0, t1 = e2e_run(args.steps)
     torch.cuda.synchronize()
     barrier(ws)
+    e2e_ev = [(t0, t1)]
     e2e_ms = max_over_ranks(ws, sum(a.elapsed_time(b) for a, b in e2e_ev))
 
     r = m.route(logits)
@@ -364,7 +389,10 @@ def run_ours(args, ws, rank, local, cfg_name):
         "stages_ms": mean_stage,
         "ms_per_step_with_stage_events": prof_ms / args.steps,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": x.numel() * 2 + logits.numel() * 4,
-                "d2h_bytes_per_step": out.numel() * 2},
+                "d2h_bytes_per_step": out.numel() * 2,
+                "copies": "pinned host buffers, H2D and D2H on their own streams, double-buffered "
+                          "across steps (overlapping the layer)",
+                "l2": "not flushed: every step streams the expert weights (far larger than L2)"},
         "gpu_launches": launches,
         "clocks": clk,
     }
