@@ -74,9 +74,12 @@ def dist_setup(args):
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if ws > 1:
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:  # host-only ranks (the multi-process tests): the same plumbing over gloo
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return ws, rank, local
@@ -93,9 +96,16 @@ def max_over_ranks(ws, v):
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_throughput(ws, tokens_per_rank_step, steps, max_ms):
+    """Whole-job tokens/s of ws independent replicas, each doing `steps` steps of
+    `tokens_per_rank_step` tokens, timed as the slowest rank's total device time."""
+    return ws * tokens_per_rank_step * steps / (max_ms / 1e3)
 
 
 class ClockSampler:
@@ -362,8 +372,8 @@ def run_ours(args, ws, rank, local, cfg_name):
     alg = algorithmic(cfg, counts)
     pk, pk_src = peaks()
     T = cfg["T"]
-    value = ws * T * args.steps / (total_ms / 1e3)
-    e2e_value = ws * T * args.steps / (e2e_ms / 1e3)
+    value = replica_throughput(ws, T, args.steps, total_ms)
+    e2e_value = replica_throughput(ws, T, args.steps, e2e_ms)
     ms_step = total_ms / args.steps
     mean_stage = {k: v / args.steps for k, v in stage_ms.items()}
     dom = max(("gemm_gateup", "gemm_down"), key=lambda s: mean_stage[s])
