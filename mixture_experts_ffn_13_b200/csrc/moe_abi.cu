@@ -513,8 +513,7 @@ int moe_forward(moe_plan_t *p, int32_t T, const uint16_t *x, const float *logits
     if (e != cudaSuccess) return fail_cuda(p, e);
 
     // quantise h per (row, 512-block)
-    e = launch_quant_rows_fp8(h, A, I, hq, sh, s);
-    if (e == cudaSuccess && shared) e = launch_quant_rows_fp8(h_sh, T, Is, hq_sh, sh_sh, s);
+    e = launch_quant_rows_fp8(h, A, I, hq, sh, shared ? h_sh : nullptr, T, Is, hq_sh, sh_sh, s);
     mark(5);
     if (e != cudaSuccess) return fail_cuda(p, e);
 
@@ -540,7 +539,7 @@ int moe_forward(moe_plan_t *p, int32_t T, const uint16_t *x, const float *logits
     e = launch_combine(y, y_sh, b.pos, b.topk_w, T, H, k, out, s);
     mark(7);
     if (e != cudaSuccess) return fail_cuda(p, e);
-    p->launches = route_permute_launches(T, E, k) + 1 + 1 + (shared ? 2 : 1) + 1 + 1;
+    p->launches = route_permute_launches(T, E, k) + 1 + 1 + 1 + 1 + 1;
     p->prof_recorded = p->prof;
     return MOE_OK;
 }

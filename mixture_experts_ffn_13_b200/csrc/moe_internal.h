@@ -48,7 +48,10 @@ int route_permute_launches(int T, int E, int k);
 cudaError_t launch_quant_x_fp8(const uint16_t *x, int T, int H, int k, const int32_t *pos, uint8_t *xq,
                                float *sx, uint8_t *xq_shared, float *sx_shared, cudaStream_t s);
 // FP8: quantise fp32 rows (h) per 512-block.
-cudaError_t launch_quant_rows_fp8(const float *h, int R, int K, uint8_t *q, float *sq, cudaStream_t s);
+// h -> e4m3 per (row, 512-block) for two row segments in one launch (segment 1 skipped when
+// h1 is null or R1 == 0).
+cudaError_t launch_quant_rows_fp8(const float *h, int R, int K, uint8_t *q, float *sq, const float *h1, int R1,
+                                  int K1, uint8_t *q1, float *sq1, cudaStream_t s);
 // int4 layers: copy bf16 token rows into the permuted rows (and the shared rows).
 cudaError_t launch_gather_x_bf16(const uint16_t *x, int T, int H, int k, const int32_t *pos, uint16_t *xp,
                                  uint16_t *xp_shared, cudaStream_t s);

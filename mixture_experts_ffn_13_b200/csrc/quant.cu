@@ -95,15 +95,30 @@ __global__ void __launch_bounds__(256) quant_x_fp8_kernel(const uint16_t *__rest
 }
 
 // One warp per (row, 512-block), 8 warps per block: fp32 rows -> e4m3 rows + scales.
-__global__ void __launch_bounds__(256) quant_rows_fp8_kernel(const float *__restrict__ h, int R, int K,
-                                                             uint8_t *__restrict__ q, float *__restrict__ sq)
+struct RowsSeg {
+    const float *h;
+    int R, K;
+    uint8_t *q;
+    float *sq;
+};
+
+// Two row segments (the routed h and the shared expert's h) in one launch: warps
+// [0, R0*nb0) quantise segment 0, the next R1*nb1 warps segment 1.
+__global__ void __launch_bounds__(256) quant_rows_fp8_kernel(RowsSeg s0, RowsSeg s1)
 {
     griddep_wait();
     griddep_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    long wid = (long)blockIdx.x * 8 + warp;
+    const long n0 = (long)s0.R * ((s0.K + kBlockK - 1) / kBlockK);
+    const RowsSeg &sg = wid < n0 ? s0 : s1;
+    if (wid >= n0) wid -= n0;
+    const float *h = sg.h;
+    const int K = sg.K;
+    uint8_t *q = sg.q;
+    float *sq = sg.sq;
     const int nb = (K + kBlockK - 1) / kBlockK;
-    const long wid = (long)blockIdx.x * 8 + warp;
-    if (wid >= (long)R * nb) return;
+    if (wid >= (long)sg.R * nb) return;
     const int r = (int)(wid / nb);
     const int kb = (int)(wid - (long)r * nb);
     const int i0 = kb * kBlockK + lane * 16;
@@ -157,11 +172,13 @@ cudaError_t launch_quant_x_fp8(const uint16_t *x, int T, int H, int k, const int
                       xq_shared, sx_shared);
 }
 
-cudaError_t launch_quant_rows_fp8(const float *h, int R, int K, uint8_t *q, float *sq, cudaStream_t s)
+cudaError_t launch_quant_rows_fp8(const float *h, int R, int K, uint8_t *q, float *sq, const float *h1, int R1,
+                                  int K1, uint8_t *q1, float *sq1, cudaStream_t s)
 {
-    if (R <= 0) return cudaSuccess;
-    const long warps = (long)R * ((K + kBlockK - 1) / kBlockK);
-    return launch_pdl(quant_rows_fp8_kernel, dim3((unsigned)((warps + 7) / 8)), dim3(256), 0, s, h, R, K, q, sq);
+    const RowsSeg a{h, R > 0 ? R : 0, K, q, sq}, b{h1, h1 && R1 > 0 ? R1 : 0, K1, q1, sq1};
+    const long warps = (long)a.R * ((a.K + kBlockK - 1) / kBlockK) + (long)b.R * ((b.K + kBlockK - 1) / kBlockK);
+    if (warps == 0) return cudaSuccess;
+    return launch_pdl(quant_rows_fp8_kernel, dim3((unsigned)((warps + 7) / 8)), dim3(256), 0, s, a, b);
 }
 
 cudaError_t launch_gather_x_bf16(const uint16_t *x, int T, int H, int k, const int32_t *pos, uint16_t *xp,

@@ -139,6 +139,49 @@ __device__ int block_exclusive_scan(int v, int *scratch /* 33 ints */, int *tota
     return res;
 }
 
+// The same over 64-bit values: the small-batch permutation scans three packed 21-bit counters
+// at once (there T*k <= 4096*32 = 2^17, so each field's block total stays below 2^21 and no
+// carry crosses into the next field).
+__device__ unsigned long long block_exclusive_scan64(unsigned long long v, unsigned long long *scratch /* 33 */,
+                                                     unsigned long long *total)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    unsigned long long incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const unsigned long long o = __shfl_up_sync(kFull, incl, off);
+        if (lane >= off) incl += o;
+    }
+    if (lane == 31) scratch[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const unsigned long long w = (lane < (int)(blockDim.x >> 5)) ? scratch[lane] : 0ull;
+        unsigned long long wi = w;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const unsigned long long o = __shfl_up_sync(kFull, wi, off);
+            if (lane >= off) wi += o;
+        }
+        scratch[lane] = wi - w;
+        if (lane == 31) scratch[32] = wi;
+    }
+    __syncthreads();
+    const unsigned long long res = scratch[warp] + incl - v;
+    *total = scratch[32];
+    __syncthreads();
+    return res;
+}
+
+// Counts of one expert packed for one scan: rows, token tiles of width bn_a, of width bn_b.
+constexpr int kPackBits = 21;
+constexpr unsigned long long kPackMask = (1ull << kPackBits) - 1;
+__device__ __forceinline__ unsigned long long pack3(int c, int bn_a, int bn_b)
+{
+    return (unsigned long long)c | ((unsigned long long)((c + bn_a - 1) / bn_a) << kPackBits) |
+           ((unsigned long long)((c + bn_b - 1) / bn_b) << (2 * kPackBits));
+}
+__device__ __forceinline__ int field(unsigned long long v, int i) { return (int)((v >> (i * kPackBits)) & kPackMask); }
+
 // One block of 1024 threads, thread e owns expert e:
 //   counts[e] = sum over chunks; offsets = exclusive scan of counts;
 //   chunk_hist[c, e] <- offsets[e] + assignments to e in chunks < c  (the chunk's base row);
@@ -238,8 +281,8 @@ __global__ void __launch_bounds__(1024) permute_small_kernel(const int32_t *__re
 {
     extern __shared__ int sm[];
     const int W = (T + 31) >> 5;
-    int *s_scr = sm;                                           // 33
-    int *s_cnt = s_scr + 64;                                   // E
+    int *s_scr = sm;                                           // 33 x 64-bit
+    int *s_cnt = s_scr + 68;                                   // E
     uint32_t *mask = reinterpret_cast<uint32_t *>(s_cnt + E);  // E * W
     int *pre = reinterpret_cast<int *>(mask + (size_t)E * W);  // E * W
     int *s_idx = pre + (size_t)E * W;                          // T * k
@@ -258,24 +301,26 @@ __global__ void __launch_bounds__(1024) permute_small_kernel(const int32_t *__re
     }
     __syncthreads();
     const int c = tid < E ? s_cnt[tid] : 0;
-    int total;
-    const int off = block_exclusive_scan(c, s_scr, &total);
+    unsigned long long tot;
+    const unsigned long long o3 = block_exclusive_scan64(tid < E ? pack3(c, bn_a, bn_b) : 0ull,
+                                                         reinterpret_cast<unsigned long long *>(s_scr), &tot);
     if (tid < E) {
+        const int off = field(o3, 0);
         counts[tid] = c;
         offsets[tid] = off;
+        ttile_a[tid] = field(o3, 1);
+        ttile_b[tid] = field(o3, 2);
         int run = off;
         for (int w = 0; w < W; ++w) {
             pre[tid * W + w] = run;
             run += __popc(mask[tid * W + w]);
         }
     }
-    if (tid == 0) offsets[E] = total;
-    const int oa = block_exclusive_scan(tid < E ? (c + bn_a - 1) / bn_a : 0, s_scr, &total);
-    if (tid < E) ttile_a[tid] = oa;
-    if (tid == 0) ttile_a[E] = total;
-    const int ob = block_exclusive_scan(tid < E ? (c + bn_b - 1) / bn_b : 0, s_scr, &total);
-    if (tid < E) ttile_b[tid] = ob;
-    if (tid == 0) ttile_b[E] = total;
+    if (tid == 0) {
+        offsets[E] = field(tot, 0);
+        ttile_a[E] = field(tot, 1);
+        ttile_b[E] = field(tot, 2);
+    }
     __syncthreads();
     for (int i = tid; i < T * k; i += 1024) {
         const int t = i / k;
@@ -290,7 +335,7 @@ __global__ void __launch_bounds__(1024) permute_small_kernel(const int32_t *__re
 size_t small_route_smem(int T, int E, int k)
 {
     const size_t W = ((size_t)T + 31) / 32;
-    return 4 * (64 + (size_t)E + 2 * (size_t)E * W + (size_t)T * k);
+    return 4 * (68 + (size_t)E + 2 * (size_t)E * W + (size_t)T * k);
 }
 
 }  // namespace
