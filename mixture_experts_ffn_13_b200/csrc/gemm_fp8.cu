@@ -80,8 +80,8 @@ struct Fp8Cfg {
     static constexpr int CPW = BN / PARTS;         // token columns per epilogue thread
     static constexpr int THREADS = 64 + 32 * EW;
     // Wide tiles (BN >= 64) stage activation scales and the tile-prefix table in shared
-    // memory; narrow (decode) tiles do not, and keep shared memory under 200 KB so that L1,
-    // which serves their scale loads, stays large.  Tiles up to 128 rows double-buffer the
+    // memory; narrow (decode) tiles do not, and keep the whole block within 196 KB of shared
+    // memory so that the carve-out leaves ~60 KB of L1 for their inline scale loads.  Tiles up to 128 rows double-buffer the
     // scales across tiles; wider tiles keep one buffer so that five stages still fit.
     static constexpr bool WIDE = BN >= 64;
     static constexpr int SX_BUFS = BN > 128 ? 1 : 2;
@@ -90,7 +90,7 @@ struct Fp8Cfg {
     static constexpr int BAR_BYTES = 8 * (2 * 16 + 2 * NSLOT) + 16;
     static constexpr int FIXED = 1024 + SX_BYTES + TT_BYTES + BAR_BYTES;
     static constexpr int NS_FIT = (kSmemLimit - FIXED) / STAGE_BYTES;
-    static constexpr int NS_NARROW = (200 * 1024) / STAGE_BYTES;
+    static constexpr int NS_NARROW = (196 * 1024 - FIXED) / STAGE_BYTES;
     static constexpr int NS_CAP = WIDE ? NS_FIT : (NS_NARROW < NS_FIT ? NS_NARROW : NS_FIT);
     static constexpr int NS = NS_CAP < 16 ? NS_CAP : 16;
     static constexpr int SMEM = FIXED + NS * STAGE_BYTES;

@@ -54,7 +54,11 @@ CASES = {
     "decode": moe_synth.CONFIGS["decode"],
     "int4": moe_synth.CONFIGS["int4"],
     # ragged token tile, two expert tiles with the second partial, H of 12 K slices
+    # (small batches like this one and the three above take the cluster split-K form)
     "ragged": dict(T=300, H=768, E=200, I=128, k=6, Is=0, wfmt="fp8", seed=60, bias=None),
+    # enough token tiles that every SM gets whole tiles: the one-CTA-per-tile form, again with
+    # a partial second expert tile
+    "persistent": dict(T=4096, H=256, E=200, I=128, k=6, Is=0, wfmt="fp8", seed=61, bias=None),
 }
 
 
