@@ -21,10 +21,12 @@
  *     index in the low nibble, [out, in/2] bytes; one bf16 scale per (row, 128-element
  *     K group); activations stay bf16 (h is rounded to bf16).
  *
- * Pointer conventions.  Every buffer passed to moe_route / moe_forward is DEVICE memory that
- * the caller allocates and owns; the library keeps no pointer to it after the call returns.
- * All calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream) and
- * never synchronise the host, except moe_get_status.  Rows are contiguous (stride = row
+ * Pointer conventions.  Every buffer passed to moe_router_logits / moe_route / moe_forward is
+ * DEVICE memory that the caller allocates and owns; the library keeps no pointer to it after
+ * the call returns.  All calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ * default stream) and never synchronise the host, except moe_get_status.  moe_forward
+ * allocates nothing and only enqueues kernels on `stream`, so a call can be captured into a
+ * CUDA graph and replayed (inputs updated in place between replays).  Rows are contiguous (stride = row
  * length).  Every pointer must be 16-byte aligned.  bf16 values are passed as uint16 bit
  * patterns.
  *

@@ -22,9 +22,10 @@
 //    each 512-block gets its own TMEM accumulator slot (a ring of slots covering all 512
 //    TMEM columns).  The epilogue reads a finished slot, multiplies it by
 //    s_w[row, kb] * s_x[token, kb] and adds it into fp32 registers, then frees the slot, so
-//    the MMAs of the next blocks overlap the promotion of the previous ones.  The tile's
-//    activation scales s_x[row0 .. row0+BN, :] are staged in shared memory once per tile
-//    (double-buffered across tiles) and the weight scales are prefetched a block ahead.
+//    the MMAs of the next blocks overlap the promotion of the previous ones.  Wide tiles stage
+//    the tile's activation scales s_x[row0 .. row0+BN, :] in shared memory once per tile
+//    (double-buffered across tiles up to 128 rows, one buffer above) and prefetch the weight
+//    scales a block ahead; narrow tiles read both through L1 in the promotion loop.
 //  * gate|up, paired form (narrow token tiles): two 128-row weight tiles per stage (gate and
 //    up) share one activation tile and accumulate into two TMEM regions; the epilogue computes
 //    h = silu(G) * U in fp32 and stores it.
@@ -33,7 +34,9 @@
 //    lanes 0-15, up rows at lanes 16-31), so one MMA per K step covers both and each thread's
 //    partner (lane ^ 16) holds the other projection of the same feature for the SwiGLU.  Each
 //    weight byte then meets up to 192 tokens per pass through shared memory, which is what
-//    bounds the narrow forms at prefill sizes (shared-memory bandwidth, not HBM).
+//    bounds the narrow forms at prefill sizes (shared-memory bandwidth, not HBM).  The whole
+//    interleaved weight tile is one 4-D TMA box: (128 K bytes, 16 rows, {gate, up}, 4 row
+//    groups), the {gate, up} dimension's stride being the distance between the two arrays.
 //  * down: one weight tile; y is stored in fp32.
 //  * Wide token tiles load activations in 64-row boxes, only as many as the tile has rows, and
 //    size the MMA's N to the tile's valid rows rounded up to 16.  The producer warp issues a

@@ -9,7 +9,9 @@
 // 路由与专家内核": tokens are collected into contiguous per-expert groups, ordered by a packed
 // (expert, token) key.  Here that order is produced without a sort: a per-chunk histogram,
 // one prefix sum over (expert, chunk), and an in-order scatter inside each chunk, so the
-// result is deterministic and equal to sorting by (expert, token).
+// result is deterministic and equal to sorting by (expert, token).  Batches of up to 4096
+// tokens (token bitmaps within 160 KB of shared memory) permute in one block instead: per-expert
+// token bitmaps, one packed scan, and popcount ranks.
 #include "launch.cuh"
 #include "moe_internal.h"
 
