@@ -113,6 +113,15 @@ MOE_API int moe_plan(const moe_dims *dims, moe_plan_t **out_plan, size_t *worksp
 MOE_API int moe_router_logits(moe_plan_t *plan, int32_t T, const uint16_t *x_bf16, const uint16_t *w_router_bf16,
                               float *logits, moe_stream_t stream);
 
+/* Router logits and step A1 from hidden states (the pages' router as one dense 16-bit layer
+ * followed by the softmax top-k, page "Flash-Next 在 GPU 上到底在算什麼", section "② 密集 16-bit
+ * 層"): logits as moe_router_logits ([T, E] fp32, written), then topk_idx [T, k] int32 and
+ * topk_w [T, k] fp32 with the conventions of moe_route, by the route kernel on those logits
+ * (two launches, the second overlapping the first's tail).  Device pointers, 16-byte aligned,
+ * caller-owned; 0 <= T <= T_max; no workspace.  Errors as moe_router_logits. */
+MOE_API int moe_router_topk(moe_plan_t *plan, int32_t T, const uint16_t *x_bf16, const uint16_t *w_router_bf16,
+                            float *logits, int32_t *topk_idx, float *topk_w, moe_stream_t stream);
+
 /* Route and permute only (steps A1 and A3), for inspection and parity checks.
  *   logits   [T, E] fp32 (finite values; the caller guarantees it)
  *   topk_idx [T, k] int32 out: experts by (logit desc, index asc)

@@ -25,7 +25,8 @@ ERRORS = {-1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED", -3: "MOE_ERR_WOR
           -4: "MOE_ERR_CUDA", -5: "MOE_ERR_DEVICE_TIMEOUT", -6: "MOE_ERR_BOUNDS"}
 EXPORTS = ("moe_plan", "moe_route", "moe_forward", "moe_get_status", "moe_last_cuda_error",
            "moe_destroy", "moe_strerror", "moe_profile_enable", "moe_profile_read",
-           "moe_profile_stage_name", "moe_launch_count", "moe_route_static", "moe_router_logits")
+           "moe_profile_stage_name", "moe_launch_count", "moe_route_static", "moe_router_logits",
+           "moe_router_topk")
 STAGES = ("route", "permute", "quant_x", "gemm_gateup", "quant_h", "gemm_down", "combine")
 
 
@@ -86,6 +87,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             L.moe_launch_count.restype = ctypes.c_int
             L.moe_router_logits.argtypes = [P, I32, P, P, P, P]
             L.moe_router_logits.restype = ctypes.c_int
+            L.moe_router_topk.argtypes = [P, I32, P, P, P, P, P, P]
+            L.moe_router_topk.restype = ctypes.c_int
             L.moe_route_static.argtypes = [I32, I32, I32, P, P, P, P, P, P, P]
             L.moe_route_static.restype = ctypes.c_int
             _lib = L
@@ -218,6 +221,27 @@ def moe_router_logits(plan: Plan, x: torch.Tensor, w_router: torch.Tensor, out: 
         out = torch.empty((T, d.E), dtype=torch.float32, device=x.device)
     rc = load_library().moe_router_logits(plan.handle, T, _ptr(x), _ptr(w_router), _ptr(out), _stream(stream))
     _check(rc, "moe_router_logits", plan.handle)
+    return out
+
+
+def moe_router_topk(plan: Plan, x: torch.Tensor, w_router: torch.Tensor, out: dict | None = None,
+                    stream=None) -> dict:
+    """Router logits and their softmax top-k from hidden states: dict(logits [T, E] fp32,
+    topk_idx [T, k] int32, topk_w [T, k] fp32)."""
+    d = plan.dims
+    T = x.shape[0]
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.shape[1] != d.H:
+        raise ValueError("x must be bf16 [T, H]")
+    if w_router.dtype != torch.bfloat16 or tuple(w_router.shape) != (d.E, d.H):
+        raise ValueError("w_router must be bf16 [E, H]")
+    dev = x.device
+    if out is None:
+        out = dict(logits=torch.empty((T, d.E), dtype=torch.float32, device=dev),
+                   topk_idx=torch.empty((T, d.k), dtype=torch.int32, device=dev),
+                   topk_w=torch.empty((T, d.k), dtype=torch.float32, device=dev))
+    rc = load_library().moe_router_topk(plan.handle, T, _ptr(x), _ptr(w_router), _ptr(out["logits"]),
+                                        _ptr(out["topk_idx"]), _ptr(out["topk_w"]), _stream(stream))
+    _check(rc, "moe_router_topk", plan.handle)
     return out
 
 

@@ -305,6 +305,23 @@ int moe_router_logits(moe_plan_t *p, int32_t T, const uint16_t *x, const uint16_
     return MOE_OK;
 }
 
+int moe_router_topk(moe_plan_t *p, int32_t T, const uint16_t *x, const uint16_t *w_router, float *logits,
+                    int32_t *topk_idx, float *topk_w, moe_stream_t stream)
+{
+    if (!p) return MOE_ERR_INVALID_ARG;
+    if (T < 0 || T > p->d.T_max) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!x || !w_router || !logits || !topk_idx || !topk_w)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w_router) || !aligned16(logits) || !aligned16(topk_idx) || !aligned16(topk_w))
+        return MOE_ERR_INVALID_ARG;
+    p->launches = 0;
+    if (T == 0) return MOE_OK;
+    const cudaError_t e = launch_router_topk(x, w_router, logits, topk_idx, topk_w, T, p->d.H, p->d.E, p->d.k,
+                                             p->d_status, p->num_sms, (cudaStream_t)stream);
+    if (e != cudaSuccess) return fail_cuda(p, e);
+    p->launches = 2;
+    return MOE_OK;
+}
+
 int moe_route(moe_plan_t *p, int32_t T, const float *logits, int32_t *topk_idx, float *topk_w, int32_t *counts,
               int32_t *offsets, int32_t *perm_tok, void *workspace, size_t ws_bytes, moe_stream_t stream)
 {

@@ -100,6 +100,10 @@ cudaError_t launch_gemm_fp8(bool gateup, int bn, const GemmMaps &maps, const Gem
 cudaError_t launch_gemm_int4(bool gateup, int bn, const GemmMaps &maps, const GemmArgs &args,
                              int num_sms, cudaStream_t s);
 
+// Router logits [T, E] (written) and their softmax top-k (step A1): the router GEMM, then the
+// route kernel.
+cudaError_t launch_router_topk(const uint16_t *x, const uint16_t *w, float *logits, int32_t *topk_idx, float *topk_w,
+                               int T, int H, int E, int k, int *status, int num_sms, cudaStream_t s);
 // Router logits: logits[T, E] = x[T, H] . W[E, H]^T (bf16 in, fp32 out) on the tensor cores.
 cudaError_t launch_router_gemm(const uint16_t *x, const uint16_t *w, float *logits, int T, int H, int E, int *status,
                                int num_sms, cudaStream_t s);

@@ -447,3 +447,18 @@ cudaError_t launch_router_gemm(const uint16_t *x, const uint16_t *w, float *logi
 }
 
 }  // namespace moe
+
+namespace moe {
+
+// Router logits, then the route kernel's softmax top-k on them (PDL-chained, so the route
+// kernel's prologue overlaps the GEMM's tail).
+cudaError_t launch_router_topk(const uint16_t *x, const uint16_t *w, float *logits, int32_t *topk_idx, float *topk_w,
+                               int T, int H, int E, int k, int *status, int num_sms, cudaStream_t s)
+{
+    if (T <= 0) return cudaSuccess;
+    cudaError_t e = launch_router_gemm(x, w, logits, T, H, E, status, num_sms, s);
+    if (e != cudaSuccess) return e;
+    return launch_route(logits, T, E, k, topk_idx, topk_w, s);
+}
+
+}  // namespace moe

@@ -112,3 +112,31 @@ def test_router_then_layer_decode():
     L["logits"] = exact.astype(np.float32)  # the oracle routes on the exact logits
     want, _, amb = oracle.layer(L, sel, ambiguity=True)
     check_out(out[torch.from_numpy(sel).long().cuda()], want, "router + layer", amb)
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode", "int4", "ragged", "persistent", "e1024", "fallback"])
+def test_router_topk_selects_what_route_selects(name):
+    """moe_router_topk: logits within the fp32 bound of the exact sums, and the selection (and
+    its weights) identical to the oracle's top-k of those same fp32 logits."""
+    cfg = dict(EXTRA[name]) if name in EXTRA else dict(CASES[name], I=128, Is=0)
+    T, H, E, k = cfg["T"], cfg["H"], cfg["E"], cfg["k"]
+    x = moe_synth.make_layer(dict(cfg, I=128, Is=0), device="cuda")["x"]
+    w = moe_synth.make_router(cfg, device="cuda")
+    plan = moe.Plan(T, H, E, 128, k, 0, cfg["wfmt"])
+    r = moe.moe_router_topk(plan, x, w)
+    torch.cuda.synchronize()
+    assert moe.moe_get_status(plan) == 0
+    want, bound = oracle.router_logits(_bits(x), _bits(w))
+    got = r["logits"].cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(got - want) <= _rel(H) * bound)
+    idx, wts = oracle.route(r["logits"].cpu().numpy(), k)
+    assert np.array_equal(r["topk_idx"].cpu().numpy(), idx)
+    assert np.allclose(r["topk_w"].cpu().numpy(), wts, rtol=2e-6, atol=1e-7)
+
+
+EXTRA = {
+    # the largest expert count (32 logits per lane in the warp top-k)
+    "e1024": dict(T=96, H=512, E=1024, I=128, k=8, Is=0, wfmt="fp8", seed=62, bias=None),
+    # a prefill-sized batch of a small layer (one-CTA-per-tile router GEMM)
+    "fallback": dict(T=8192, H=256, E=200, I=128, k=6, Is=0, wfmt="fp8", seed=63, bias=None),
+}
