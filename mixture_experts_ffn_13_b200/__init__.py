@@ -26,7 +26,7 @@ ERRORS = {-1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED", -3: "MOE_ERR_WOR
 EXPORTS = ("moe_plan", "moe_route", "moe_forward", "moe_get_status", "moe_last_cuda_error",
            "moe_destroy", "moe_strerror", "moe_profile_enable", "moe_profile_read",
            "moe_profile_stage_name", "moe_launch_count", "moe_route_static", "moe_router_logits",
-           "moe_router_topk")
+           "moe_router_topk", "moe_forward_x")
 STAGES = ("route", "permute", "quant_x", "gemm_gateup", "quant_h", "gemm_down", "combine")
 
 
@@ -89,6 +89,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             L.moe_router_logits.restype = ctypes.c_int
             L.moe_router_topk.argtypes = [P, I32, P, P, P, P, P, P]
             L.moe_router_topk.restype = ctypes.c_int
+            L.moe_forward_x.argtypes = [P, I32, P, P, ctypes.POINTER(moe_weights), P, P, SZ, P]
+            L.moe_forward_x.restype = ctypes.c_int
             L.moe_route_static.argtypes = [I32, I32, I32, P, P, P, P, P, P, P]
             L.moe_route_static.restype = ctypes.c_int
             _lib = L
@@ -280,6 +282,24 @@ def moe_forward(plan: Plan, x: torch.Tensor, logits: torch.Tensor, weights: dict
     rc = load_library().moe_forward(plan.handle, T, _ptr(x), _ptr(logits), ctypes.byref(W), _ptr(out),
                                     _ptr(workspace), workspace.numel(), _stream(stream))
     _check(rc, "moe_forward", plan.handle)
+    return out
+
+
+def moe_forward_x(plan: Plan, x: torch.Tensor, w_router: torch.Tensor, weights: dict, workspace: torch.Tensor,
+                  out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """The whole layer from hidden states and router weights: out[T, H] bf16."""
+    d = plan.dims
+    T = x.shape[0]
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.shape[1] != d.H:
+        raise ValueError("x must be bf16 [T, H]")
+    if w_router.dtype != torch.bfloat16 or tuple(w_router.shape) != (d.E, d.H):
+        raise ValueError("w_router must be bf16 [E, H]")
+    if out is None:
+        out = torch.empty((T, d.H), dtype=torch.bfloat16, device=x.device)
+    W = _weights_struct(weights)
+    rc = load_library().moe_forward_x(plan.handle, T, _ptr(x), _ptr(w_router), ctypes.byref(W), _ptr(out),
+                                      _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(rc, "moe_forward_x", plan.handle)
     return out
 
 

@@ -38,6 +38,7 @@ struct Layout {
     size_t h, h_sh;              // gate|up output, routed / shared
     size_t hq, hq_sh, sh, sh_sh; // quantised h (FP8)
     size_t y;                    // down output rows (routed then shared), fp32
+    size_t lg;                   // router logits [T, E] fp32 (moe_forward_x)
     size_t total;
 };
 
@@ -82,6 +83,7 @@ Layout make_layout(const moe_dims &d)
         L.hq = L.hq_sh = L.sh = L.sh_sh = 0;
     }
     L.y = take(R * H * 4);
+    L.lg = take(Tm * E * 4);
     L.total = o;
     return L;
 }
@@ -431,6 +433,20 @@ static int forward_int4(moe_plan_t *p, int T, const uint16_t *x, const float *lo
     return MOE_OK;
 }
 
+// Weight pointers present (the shared expert's when I_shared > 0) and 16-byte aligned.
+static int check_weights(const moe_plan_t *p, const moe_weights *w)
+{
+    if (!w->w_gate || !w->w_up || !w->w_down || !w->s_gate || !w->s_up || !w->s_down) return MOE_ERR_INVALID_ARG;
+    if (p->d.I_shared > 0 &&
+        (!w->ws_gate || !w->ws_up || !w->ws_down || !w->ss_gate || !w->ss_up || !w->ss_down))
+        return MOE_ERR_INVALID_ARG;
+    const void *ptrs[] = {w->w_gate, w->w_up, w->w_down, w->s_gate, w->s_up, w->s_down,
+                          w->ws_gate, w->ws_up, w->ws_down, w->ss_gate, w->ss_up, w->ss_down};
+    for (const void *q : ptrs)
+        if (!aligned16(q)) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
 int moe_forward(moe_plan_t *p, int32_t T, const uint16_t *x, const float *logits, const moe_weights *w,
                 uint16_t *out, void *workspace, size_t ws_bytes, moe_stream_t stream)
 {
@@ -438,12 +454,9 @@ int moe_forward(moe_plan_t *p, int32_t T, const uint16_t *x, const float *logits
     const moe_dims &d = p->d;
     if (T < 0 || T > d.T_max) return MOE_ERR_INVALID_ARG;
     if (T > 0 && (!x || !logits || !out)) return MOE_ERR_INVALID_ARG;
-    if (!w->w_gate || !w->w_up || !w->w_down || !w->s_gate || !w->s_up || !w->s_down) return MOE_ERR_INVALID_ARG;
     const bool shared = d.I_shared > 0;
-    if (shared && (!w->ws_gate || !w->ws_up || !w->ws_down || !w->ss_gate || !w->ss_up || !w->ss_down))
-        return MOE_ERR_INVALID_ARG;
-    const void *ptrs[] = {x, logits, out, w->w_gate, w->w_up, w->w_down, w->s_gate, w->s_up, w->s_down,
-                          w->ws_gate, w->ws_up, w->ws_down, w->ss_gate, w->ss_up, w->ss_down};
+    if (check_weights(p, w) != MOE_OK) return MOE_ERR_INVALID_ARG;
+    const void *ptrs[] = {x, logits, out};
     for (const void *q : ptrs)
         if (!aligned16(q)) return MOE_ERR_INVALID_ARG;
     int rc = check_ws(p, workspace, ws_bytes);
@@ -560,5 +573,29 @@ int moe_forward(moe_plan_t *p, int32_t T, const uint16_t *x, const float *logits
     p->prof_recorded = p->prof;
     return MOE_OK;
 }
+
+int moe_forward_x(moe_plan_t *p, int32_t T, const uint16_t *x, const uint16_t *w_router, const moe_weights *w,
+                  uint16_t *out, void *workspace, size_t ws_bytes, moe_stream_t stream)
+{
+    if (!p || !w) return MOE_ERR_INVALID_ARG;
+    const moe_dims &d = p->d;
+    if (T < 0 || T > d.T_max) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!x || !w_router || !out)) return MOE_ERR_INVALID_ARG;
+    if (check_weights(p, w) != MOE_OK) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w_router) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+    int rc = check_ws(p, workspace, ws_bytes);
+    if (rc) return rc;
+    p->launches = 0;
+    if (T == 0) return MOE_OK;
+    const Layout L = make_layout(d);
+    float *lg = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + L.lg);
+    const cudaError_t e =
+        launch_router_gemm(x, w_router, lg, T, d.H, d.E, p->d_status, p->num_sms, (cudaStream_t)stream);
+    if (e != cudaSuccess) return fail_cuda(p, e);
+    rc = moe_forward(p, T, x, lg, w, out, workspace, ws_bytes, stream);
+    if (rc == MOE_OK) p->launches += 1;
+    return rc;
+}
+
 
 }  // extern "C"

@@ -140,3 +140,42 @@ EXTRA = {
     # a prefill-sized batch of a small layer (one-CTA-per-tile router GEMM)
     "fallback": dict(T=8192, H=256, E=200, I=128, k=6, Is=0, wfmt="fp8", seed=63, bias=None),
 }
+
+
+@pytest.mark.parametrize("name", ["decode", "int4", "tiny"])
+def test_forward_x_equals_router_then_forward(name):
+    """moe_forward_x (hidden states + router weights) is bit-identical to moe_router_logits
+    followed by moe_forward on those logits, and matches the oracle on clear tokens."""
+    cfg = moe_synth.CONFIGS[name]
+    layer = moe_synth.make_layer(name, device="cuda")
+    w = moe_synth.make_router(cfg, device="cuda")
+    m = moe.MoELayer(layer)
+    got = moe.moe_forward_x(m.plan, layer["x"], w, m.weights, m.workspace)
+    torch.cuda.synchronize()
+    assert moe.moe_get_status(m.plan) == 0
+    assert moe.moe_launch_count(m.plan) >= 7
+    lg = moe.moe_router_logits(m.plan, layer["x"], w)
+    ref = m(layer["x"], lg)
+    torch.cuda.synchronize()
+    assert torch.equal(got, ref)
+    exact, _ = oracle.router_logits(_bits(layer["x"]), _bits(w))
+    clear, _ = _clear_tokens(lg.cpu().numpy().astype(np.float64), exact, cfg["k"])
+    sel = np.nonzero(clear)[0][::37][:8].astype(np.int32)
+    L = moe_synth.to_numpy(layer)
+    L["logits"] = exact.astype(np.float32)
+    want, _, amb = oracle.layer(L, sel, ambiguity=True)
+    check_out(got[torch.from_numpy(sel).long().cuda()], want, "forward_x", amb)
+
+
+def test_forward_x_argument_errors_launch_nothing():
+    cfg = dict(T=16, H=512, E=8, I=256, k=2, Is=0, seed=64, bias=None, wfmt="fp8")
+    layer = moe_synth.make_layer(cfg, device="cuda")
+    m = moe.MoELayer(layer)
+    w = moe_synth.make_router(cfg, device="cuda")
+    with pytest.raises(moe.MoEError) as ei:  # workspace one byte short
+        moe.moe_forward_x(m.plan, layer["x"], w, m.weights, m.workspace[: m.plan.workspace_bytes - 1])
+    assert ei.value.code == -3 and moe.moe_launch_count(m.plan) == 0
+    bad = dict(m.weights)
+    bad["w_down"] = None
+    with pytest.raises((moe.MoEError, TypeError, AttributeError)):
+        moe.moe_forward_x(m.plan, layer["x"], w, bad, m.workspace)
