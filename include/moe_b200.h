@@ -160,7 +160,8 @@ MOE_API int moe_forward(moe_plan_t *plan, int32_t T, const uint16_t *x_bf16, con
 /* The whole layer from hidden states: the router logits x . W_router^T (as moe_router_logits,
  * written into the workspace) and then exactly the work of moe_forward on them.  w_router is
  * bf16 [E, H] (device, 16-byte aligned).  Same workspace (moe_plan's size covers the logits),
- * outputs and errors as moe_forward; no argument error launches anything. */
+ * outputs and errors as moe_forward; no argument error launches anything.  (The logits share
+ * the workspace bytes of the down projection's output, which is written only after routing.) */
 MOE_API int moe_forward_x(moe_plan_t *plan, int32_t T, const uint16_t *x_bf16, const uint16_t *w_router_bf16,
                           const moe_weights *weights, uint16_t *out_bf16, void *workspace, size_t workspace_bytes,
                           moe_stream_t stream);

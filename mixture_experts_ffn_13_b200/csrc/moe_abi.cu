@@ -38,7 +38,7 @@ struct Layout {
     size_t h, h_sh;              // gate|up output, routed / shared
     size_t hq, hq_sh, sh, sh_sh; // quantised h (FP8)
     size_t y;                    // down output rows (routed then shared), fp32
-    size_t lg;                   // router logits [T, E] fp32 (moe_forward_x)
+    size_t lg;                   // router logits [T, E] fp32 (moe_forward_x): inside y when they fit
     size_t total;
 };
 
@@ -83,7 +83,10 @@ Layout make_layout(const moe_dims &d)
         L.hq = L.hq_sh = L.sh = L.sh_sh = 0;
     }
     L.y = take(R * H * 4);
-    L.lg = take(Tm * E * 4);
+    // moe_forward_x's logits are read only by the route kernel, the first kernel of the
+    // forward, and y is written by the down GEMM later on the same stream, so they share y's
+    // bytes unless they do not fit there
+    L.lg = Tm * E <= R * H ? L.y : take(Tm * E * 4);
     L.total = o;
     return L;
 }
