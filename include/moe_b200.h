@@ -187,7 +187,7 @@ MOE_API int moe_profile_enable(moe_plan_t *plan, int enable);
 MOE_API int moe_profile_read(moe_plan_t *plan, float *ms, int max_stages);
 MOE_API const char *moe_profile_stage_name(int stage);
 
-/* Number of kernels the last moe_route / moe_forward call on this plan launched. */
+/* Number of kernels the last router / route / forward call on this plan launched. */
 MOE_API int moe_launch_count(const moe_plan_t *plan);
 
 /* A static, human-readable name of a status code. */
