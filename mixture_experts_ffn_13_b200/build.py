@@ -33,10 +33,26 @@ def _deps_mtime() -> float:
     return max(os.path.getmtime(f) for f in files)
 
 
+def _fresh() -> bool:
+    return os.path.exists(LIB) and os.path.getmtime(LIB) >= _deps_mtime()
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile every .cu under csrc/ and link libmoe_b200.so; returns the library path."""
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= _deps_mtime():
+    """Compile every .cu under csrc/ and link libmoe_b200.so; returns the library path.
+    Concurrent callers (one process per GPU, parallel test workers) serialise on a lock file;
+    whoever gets it second finds the library fresh and returns."""
+    if not force and _fresh():
         return LIB
+    import fcntl
+    os.makedirs(BUILD, exist_ok=True)
+    with open(os.path.join(BUILD, ".lock"), "w") as lk:
+        fcntl.flock(lk, fcntl.LOCK_EX)
+        if not force and _fresh():
+            return LIB
+        return _build_locked(verbose)
+
+
+def _build_locked(verbose: bool) -> str:
     nvcc = _nvcc()
     os.makedirs(BUILD, exist_ok=True)
     extra = os.environ.get("MOE_NVCC_FLAGS", "").split()
