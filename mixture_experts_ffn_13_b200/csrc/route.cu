@@ -285,8 +285,10 @@ __global__ void __launch_bounds__(1024) permute_small_kernel(const int32_t *__re
     const int W = (T + 31) >> 5;
     int *s_scr = sm;                                           // 33 x 64-bit
     int *s_cnt = s_scr + 68;                                   // E
-    uint32_t *mask = reinterpret_cast<uint32_t *>(s_cnt + E);  // E * W
-    int *pre = reinterpret_cast<int *>(mask + (size_t)E * W);  // E * W
+    // word-major [W][E]: in the per-expert prefix pass thread e walks its column, so the 32
+    // lanes of a warp touch 32 consecutive words (no bank conflicts)
+    uint32_t *mask = reinterpret_cast<uint32_t *>(s_cnt + E);  // W * E
+    int *pre = reinterpret_cast<int *>(mask + (size_t)E * W);  // W * E
     int *s_idx = pre + (size_t)E * W;                          // T * k
     const int tid = threadIdx.x;
     griddep_wait();
@@ -298,7 +300,7 @@ __global__ void __launch_bounds__(1024) permute_small_kernel(const int32_t *__re
         const int e = __ldg(topk_idx + i);
         const int t = i / k;
         s_idx[i] = e;
-        atomicOr(&mask[e * W + (t >> 5)], 1u << (t & 31));
+        atomicOr(&mask[(t >> 5) * E + e], 1u << (t & 31));
         atomicAdd(&s_cnt[e], 1);
     }
     __syncthreads();
@@ -314,8 +316,8 @@ __global__ void __launch_bounds__(1024) permute_small_kernel(const int32_t *__re
         ttile_b[tid] = field(o3, 2);
         int run = off;
         for (int w = 0; w < W; ++w) {
-            pre[tid * W + w] = run;
-            run += __popc(mask[tid * W + w]);
+            pre[w * E + tid] = run;
+            run += __popc(mask[w * E + tid]);
         }
     }
     if (tid == 0) {
@@ -328,7 +330,7 @@ __global__ void __launch_bounds__(1024) permute_small_kernel(const int32_t *__re
         const int t = i / k;
         const int e = s_idx[i];
         const int w = t >> 5;
-        const int r = pre[e * W + w] + __popc(mask[e * W + w] & ((1u << (t & 31)) - 1u));
+        const int r = pre[w * E + e] + __popc(mask[w * E + e] & ((1u << (t & 31)) - 1u));
         perm_tok[r] = t;
         pos[i] = r;
     }
