@@ -14,21 +14,31 @@ namespace moe {
 
 namespace {
 
-// grid (T, ceil(H/1024)), 256 threads: each thread owns 4 consecutive hidden features.
+// grid (T, ceil(H/1024)), 256 threads: each thread owns 4 consecutive hidden features.  The
+// token's k (row, weight) pairs are staged in shared memory once per block, so the k row loads
+// of a thread do not each wait behind a load of their row index.
 __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ y, const float *__restrict__ ysh,
                                                       const int32_t *__restrict__ pos,
                                                       const float *__restrict__ topk_w, int H, int k,
                                                       uint16_t *__restrict__ out)
 {
+    __shared__ int s_row[kMaxK];
+    __shared__ float s_w[kMaxK];
     griddep_wait();
     griddep_launch_dependents();
     const int t = blockIdx.x;
+    if (threadIdx.x < k) {
+        s_row[threadIdx.x] = __ldg(pos + (size_t)t * k + threadIdx.x);
+        s_w[threadIdx.x] = __ldg(topk_w + (size_t)t * k + threadIdx.x);
+    }
+    __syncthreads();
     const int c = blockIdx.y * blockDim.x + threadIdx.x;  // float4 index within the row
     if (c >= H / 4) return;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
     for (int j = 0; j < k; ++j) {
-        const int r = __ldg(pos + (size_t)t * k + j);
-        const float w = __ldg(topk_w + (size_t)t * k + j);
+        const int r = s_row[j];
+        const float w = s_w[j];
         const float4 v = __ldg(reinterpret_cast<const float4 *>(y + (size_t)r * H) + c);
         acc.x = fmaf(w, v.x, acc.x);
         acc.y = fmaf(w, v.y, acc.y);
