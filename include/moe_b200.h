@@ -65,7 +65,8 @@ enum moe_status {
     MOE_ERR_WORKSPACE = -3,      /* workspace NULL or smaller than moe_plan reported */
     MOE_ERR_CUDA = -4,           /* a CUDA runtime call or kernel launch failed */
     MOE_ERR_DEVICE_TIMEOUT = -5, /* a bounded device-side wait gave up (from moe_get_status) */
-    MOE_ERR_BOUNDS = -6          /* a device-side index check failed (from moe_get_status) */
+    MOE_ERR_BOUNDS = -6          /* a checked-mode device check failed: a non-finite router logit or a
+                                    permuted row index out of range (from moe_get_status) */
 };
 
 typedef struct {
@@ -186,6 +187,14 @@ MOE_API void moe_destroy(moe_plan_t *plan);
 MOE_API int moe_profile_enable(moe_plan_t *plan, int enable);
 MOE_API int moe_profile_read(moe_plan_t *plan, float *ms, int max_stages);
 MOE_API const char *moe_profile_stage_name(int stage);
+
+/* Checked mode (off by default): with enable != 0, later moe_route / moe_forward /
+ * moe_forward_x calls on this plan also verify on the device that every router logit is
+ * finite (non-finite logits are caller error) and that every permuted row index the combine
+ * reads is in range; a failed check records MOE_ERR_BOUNDS in the plan's status word
+ * (moe_get_status) and the outputs of that call are unspecified.  Costs one extra read of the
+ * logits.  Returns MOE_OK or MOE_ERR_INVALID_ARG (NULL plan). */
+MOE_API int moe_set_checked(moe_plan_t *plan, int enable);
 
 /* Number of kernels the last router / route / forward call on this plan launched. */
 MOE_API int moe_launch_count(const moe_plan_t *plan);

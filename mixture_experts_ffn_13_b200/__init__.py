@@ -26,7 +26,7 @@ ERRORS = {-1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED", -3: "MOE_ERR_WOR
 EXPORTS = ("moe_plan", "moe_route", "moe_forward", "moe_get_status", "moe_last_cuda_error",
            "moe_destroy", "moe_strerror", "moe_profile_enable", "moe_profile_read",
            "moe_profile_stage_name", "moe_launch_count", "moe_route_static", "moe_router_logits",
-           "moe_router_topk", "moe_forward_x")
+           "moe_router_topk", "moe_forward_x", "moe_set_checked")
 STAGES = ("route", "permute", "quant_x", "gemm_gateup", "quant_h", "gemm_down", "combine")
 
 
@@ -91,6 +91,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             L.moe_router_topk.restype = ctypes.c_int
             L.moe_forward_x.argtypes = [P, I32, P, P, ctypes.POINTER(moe_weights), P, P, SZ, P]
             L.moe_forward_x.restype = ctypes.c_int
+            L.moe_set_checked.argtypes = [P, ctypes.c_int]
+            L.moe_set_checked.restype = ctypes.c_int
             L.moe_route_static.argtypes = [I32, I32, I32, P, P, P, P, P, P, P]
             L.moe_route_static.restype = ctypes.c_int
             _lib = L
@@ -177,6 +179,12 @@ def moe_profile_read(plan: Plan) -> dict:
     if n < 0:
         _check(n, "moe_profile_read", plan.handle)
     return {STAGES[i]: float(buf[i]) for i in range(n)}
+
+
+def moe_set_checked(plan: Plan, enable: bool = True):
+    """Checked mode: device-side checks of the router logits (finite) and permuted row indices;
+    a failure shows as MOE_ERR_BOUNDS from moe_get_status."""
+    _check(load_library().moe_set_checked(plan.handle, 1 if enable else 0), "moe_set_checked")
 
 
 def moe_launch_count(plan: Plan) -> int:

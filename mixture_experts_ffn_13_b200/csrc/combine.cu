@@ -17,10 +17,12 @@ namespace {
 // grid (T, ceil(H/1024)), 256 threads: each thread owns 4 consecutive hidden features.  The
 // token's k (row, weight) pairs are staged in shared memory once per block, so the k row loads
 // of a thread do not each wait behind a load of their row index.
+// With `check` set (checked mode), a permuted row index outside [0, rows) records
+// MOE_ERR_BOUNDS in *check and the token's output is left unspecified (the row is not read).
 __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ y, const float *__restrict__ ysh,
                                                       const int32_t *__restrict__ pos,
                                                       const float *__restrict__ topk_w, int H, int k,
-                                                      uint16_t *__restrict__ out)
+                                                      uint16_t *__restrict__ out, int rows, int *check)
 {
     __shared__ int s_row[kMaxK];
     __shared__ float s_w[kMaxK];
@@ -28,7 +30,12 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
     griddep_launch_dependents();
     const int t = blockIdx.x;
     if (threadIdx.x < k) {
-        s_row[threadIdx.x] = __ldg(pos + (size_t)t * k + threadIdx.x);
+        int r = __ldg(pos + (size_t)t * k + threadIdx.x);
+        if (check && (r < 0 || r >= rows)) {
+            atomicCAS(check, 0, MOE_ERR_BOUNDS);
+            r = 0;
+        }
+        s_row[threadIdx.x] = r;
         s_w[threadIdx.x] = __ldg(topk_w + (size_t)t * k + threadIdx.x);
     }
     __syncthreads();
@@ -63,11 +70,11 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
 }  // namespace
 
 cudaError_t launch_combine(const float *y, const float *y_shared, const int32_t *pos, const float *topk_w, int T,
-                           int H, int k, uint16_t *out, cudaStream_t s)
+                           int H, int k, uint16_t *out, cudaStream_t s, int *check)
 {
     if (T <= 0) return cudaSuccess;
     return launch_pdl(combine_kernel, dim3(T, (H / 4 + 255) / 256), dim3(256), 0, s, y, y_shared, pos, topk_w, H, k,
-                      out);
+                      out, T * k, check);
 }
 
 }  // namespace moe

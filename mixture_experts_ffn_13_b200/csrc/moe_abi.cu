@@ -16,6 +16,7 @@ struct moe_plan_s {
     int last_cuda_error;
     size_t ws_bytes;
     int launches;             // kernels launched by the last route/forward call
+    bool checked = false;     // checked mode (moe_set_checked): device-side argument checks
     bool prof;                // stage events enabled
     bool prof_recorded;       // the last forward recorded them
     cudaEvent_t ev[8];        // stage boundaries 0..7
@@ -228,6 +229,13 @@ const char *moe_profile_stage_name(int i) { return (i >= 0 && i < 7) ? kStageNam
 
 int moe_launch_count(const moe_plan_t *p) { return p ? p->launches : 0; }
 
+int moe_set_checked(moe_plan_t *p, int enable)
+{
+    if (!p) return MOE_ERR_INVALID_ARG;
+    p->checked = enable != 0;
+    return MOE_OK;
+}
+
 int moe_profile_enable(moe_plan_t *p, int enable)
 {
     if (!p) return MOE_ERR_INVALID_ARG;
@@ -349,7 +357,7 @@ int moe_route(moe_plan_t *p, int32_t T, const float *logits, int32_t *topk_idx, 
     cudaStream_t s = (cudaStream_t)stream;
     const int bn = pick_bn(T, d.k, d.E, d.wfmt == MOE_W_FP8_SC512);
     p->launches = 0;
-    cudaError_t e = launch_route_permute(logits, b, T, d.E, d.k, bn, bn, s);
+    cudaError_t e = launch_route_permute(logits, b, T, d.E, d.k, bn, bn, s, p->checked ? p->d_status : nullptr);
     p->launches = route_permute_launches(T, d.E, d.k);
     return e == cudaSuccess ? MOE_OK : fail_cuda(p, e);
 }
@@ -371,7 +379,8 @@ static int forward_int4(moe_plan_t *p, int T, const uint16_t *x, const float *lo
     const int A = T * k;
     const int bn = pick_bn(T, k, E, false);
     mark(0);
-    cudaError_t e = launch_route(logits, T, E, k, b.topk_idx, b.topk_w, s);
+    int *chk = p->checked ? p->d_status : nullptr;
+    cudaError_t e = launch_route(logits, T, E, k, b.topk_idx, b.topk_w, s, chk);
     mark(1);
     if (e == cudaSuccess) e = launch_permute_any(b, T, E, k, bn, bn, s);
     mark(2);
@@ -428,7 +437,7 @@ static int forward_int4(moe_plan_t *p, int T, const uint16_t *x, const float *lo
     e = launch_gemm_int4(false, bn, md, ad, p->num_sms, s);
     mark(6);
     if (e != cudaSuccess) return fail_cuda(p, e);
-    e = launch_combine(y, y_sh, b.pos, b.topk_w, T, H, k, out, s);
+    e = launch_combine(y, y_sh, b.pos, b.topk_w, T, H, k, out, s, chk);
     mark(7);
     if (e != cudaSuccess) return fail_cuda(p, e);
     p->launches = route_permute_launches(T, E, k) + 1 + 1 + 1 + 1;
@@ -487,7 +496,8 @@ int moe_forward(moe_plan_t *p, int32_t T, const uint16_t *x, const float *logits
     const uint32_t kXBox = bn_a < 64 ? bn_a : 64;  // activation rows per TMA box
 
     mark(0);
-    cudaError_t e = launch_route(logits, T, E, k, b.topk_idx, b.topk_w, s);
+    int *chk = p->checked ? p->d_status : nullptr;
+    cudaError_t e = launch_route(logits, T, E, k, b.topk_idx, b.topk_w, s, chk);
     mark(1);
     if (e == cudaSuccess) e = launch_permute_any(b, T, E, k, bn_a, bn_b, s);
     mark(2);
@@ -569,7 +579,7 @@ int moe_forward(moe_plan_t *p, int32_t T, const uint16_t *x, const float *logits
     if (e != cudaSuccess) return fail_cuda(p, e);
 
     // A6: combine
-    e = launch_combine(y, y_sh, b.pos, b.topk_w, T, H, k, out, s);
+    e = launch_combine(y, y_sh, b.pos, b.topk_w, T, H, k, out, s, chk);
     mark(7);
     if (e != cudaSuccess) return fail_cuda(p, e);
     p->launches = route_permute_launches(T, E, k) + 1 + 1 + 1 + 1 + 1;

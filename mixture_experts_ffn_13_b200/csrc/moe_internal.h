@@ -31,14 +31,15 @@ struct RouteBufs {
     int32_t *ttile_b;     // [E + 1] token-tile prefix for the down GEMM tile size
 };
 
+// check != nullptr (checked mode): non-finite logits record MOE_ERR_BOUNDS in *check.
 cudaError_t launch_route(const float *logits, int T, int E, int k, int32_t *topk_idx, float *topk_w,
-                         cudaStream_t s);
+                         cudaStream_t s, int *check = nullptr);
 cudaError_t launch_permute(const RouteBufs &b, int T, int E, int k, int bn_a, int bn_b, cudaStream_t s);
 // Permutation: one single-block kernel for small batches, else the three launches above.
 cudaError_t launch_permute_any(const RouteBufs &b, int T, int E, int k, int bn_a, int bn_b, cudaStream_t s);
 // Router followed by launch_permute_any, and the number of kernels the pair launches.
 cudaError_t launch_route_permute(const float *logits, const RouteBufs &b, int T, int E, int k, int bn_a, int bn_b,
-                                 cudaStream_t s);
+                                 cudaStream_t s, int *check = nullptr);
 int route_permute_launches(int T, int E, int k);
 
 // ---- activation quantisation and gathers (quant.cu) --------------------------------------
@@ -58,8 +59,10 @@ cudaError_t launch_gather_x_bf16(const uint16_t *x, int T, int H, int k, const i
 
 // ---- combine (combine.cu) ----------------------------------------------------------------
 
+// check != nullptr (checked mode): a permuted row index outside [0, T*k) records
+// MOE_ERR_BOUNDS in *check.
 cudaError_t launch_combine(const float *y, const float *y_shared, const int32_t *pos, const float *topk_w,
-                           int T, int H, int k, uint16_t *out, cudaStream_t s);
+                           int T, int H, int k, uint16_t *out, cudaStream_t s, int *check = nullptr);
 
 // ---- grouped GEMMs (gemm_fp8.cu, gemm_int4.cu) -------------------------------------------
 

@@ -36,7 +36,8 @@ __device__ __forceinline__ void route_one(const float *__restrict__ L, int E, in
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
         const int e = lane + 32 * i;
-        v[i] = (e < E) ? __ldg(L + e) : -INFINITY;
+        const float l = (e < E) ? __ldg(L + e) : -INFINITY;
+        v[i] = (l != l) ? -INFINITY : l;  // NaN (caller error) ranks lowest: indices stay valid
         if (e >= E) taken |= 1u << i;
     }
     float sel_v = 0.0f;
@@ -76,15 +77,23 @@ __device__ __forceinline__ void route_one(const float *__restrict__ L, int E, in
 }
 
 // One warp per token.
+// With `check` set (checked mode), a token whose logits are not all finite records
+// MOE_ERR_BOUNDS in *check; selection then proceeds as usual (its result is unspecified).
 template <int EPL>
 __global__ void __launch_bounds__(256) route_kernel(const float *__restrict__ logits, int T, int E, int k,
-                                                    int32_t *__restrict__ topk_idx, float *__restrict__ topk_w)
+                                                    int32_t *__restrict__ topk_idx, float *__restrict__ topk_w,
+                                                    int *check)
 {
     griddep_wait();
     griddep_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t = blockIdx.x * 8 + warp;
     if (t >= T) return;
+    if (check) {
+        bool bad = false;
+        for (int e = lane; e < E; e += 32) bad |= !isfinite(__ldg(logits + (size_t)t * E + e));
+        if (__any_sync(kFull, bad) && lane == 0) atomicCAS(check, 0, MOE_ERR_BOUNDS);
+    }
     int e;
     float w;
     route_one<EPL>(logits + (size_t)t * E, E, k, lane, &e, &w);
@@ -345,9 +354,9 @@ size_t small_route_smem(int T, int E, int k)
 }  // namespace
 
 cudaError_t launch_route_permute(const float *logits, const RouteBufs &b, int T, int E, int k, int bn_a, int bn_b,
-                                 cudaStream_t s)
+                                 cudaStream_t s, int *check)
 {
-    cudaError_t e = launch_route(logits, T, E, k, b.topk_idx, b.topk_w, s);
+    cudaError_t e = launch_route(logits, T, E, k, b.topk_idx, b.topk_w, s, check);
     if (e != cudaSuccess) return e;
     return launch_permute_any(b, T, E, k, bn_a, bn_b, s);
 }
@@ -371,12 +380,12 @@ int route_permute_launches(int T, int E, int k)
 }
 
 cudaError_t launch_route(const float *logits, int T, int E, int k, int32_t *topk_idx, float *topk_w,
-                         cudaStream_t s)
+                         cudaStream_t s, int *check)
 {
     if (T <= 0) return cudaSuccess;
     const dim3 grid((T + 7) / 8), block(256);
     const int epl = (E + 31) / 32;
-    auto go = [&](auto kern) { return launch_pdl(kern, grid, block, 0, s, logits, T, E, k, topk_idx, topk_w); };
+    auto go = [&](auto kern) { return launch_pdl(kern, grid, block, 0, s, logits, T, E, k, topk_idx, topk_w, check); };
     if (epl <= 1) return go(route_kernel<1>);
     if (epl <= 2) return go(route_kernel<2>);
     if (epl <= 4) return go(route_kernel<4>);

@@ -102,3 +102,30 @@ def test_bounded_wait_gives_up_and_reports():
     assert L.moe_test_bounded_wait(status.data_ptr(), 0, stream) == -1
     # the device still runs the layer correctly afterwards
     _layer_parity(dict(T=16, H=512, E=8, I=256, k=2, Is=0, seed=0, bias=None, wfmt="fp8"))
+
+
+def test_checked_mode_reports_non_finite_logits():
+    """Checked mode: a NaN or infinite router logit is reported as MOE_ERR_BOUNDS through the
+    status word (for moe_route and moe_forward); unchecked, nothing is reported; finite logits
+    pass; the plan keeps working afterwards."""
+    cfg = dict(T=40, H=512, E=16, I=128, k=4, Is=128, seed=65, bias=None, wfmt="fp8")
+    layer = moe_synth.make_layer(cfg, device="cuda")
+    m = moe.MoELayer(layer)
+    bad = layer["logits"].clone()
+    bad[7, 3] = float("nan")
+    bad[20, 0] = float("inf")
+    bad[31, :] = float("nan")                        # a whole row: selection still stays in range
+    m(layer["x"], bad)                               # unchecked: no device check
+    assert moe.moe_get_status(m.plan) == 0
+    moe.moe_set_checked(m.plan, True)
+    m(layer["x"], layer["logits"])                   # checked, finite logits: passes
+    assert moe.moe_get_status(m.plan) == 0
+    m(layer["x"], bad)
+    assert moe.moe_get_status(m.plan) == -6          # MOE_ERR_BOUNDS, then the word is cleared
+    m.route(bad)
+    assert moe.moe_get_status(m.plan) == -6
+    out = m(layer["x"], layer["logits"])             # still correct afterwards
+    assert moe.moe_get_status(m.plan) == 0
+    want, _, amb = oracle.layer(moe_synth.to_numpy(layer), ambiguity=True)
+    check_out(out, want, "checked mode", amb)
+    moe.moe_set_checked(m.plan, False)
