@@ -51,6 +51,7 @@ int main(void)
     CHECK(moe_router_topk(NULL, 1, NULL, NULL, NULL, NULL, NULL, NULL) == MOE_ERR_INVALID_ARG);
     CHECK(moe_route(NULL, 1, NULL, NULL, NULL, NULL, NULL, NULL, NULL, 0, NULL) == MOE_ERR_INVALID_ARG);
     CHECK(moe_launch_count(NULL) == 0);
+    CHECK(moe_set_checked(NULL, 1) == MOE_ERR_INVALID_ARG);
     moe_destroy(NULL); /* accepted */
     /* static routing beyond its fixed scratch: rejected before any device work */
     CHECK(moe_route_static(1 << 18, 512, 10, NULL, NULL, NULL, NULL, NULL, NULL, NULL) != MOE_OK);
