@@ -408,6 +408,12 @@ def run_ours(args, ws, rank, local, cfg_name):
                    "peak": tpk, "unit": "TFLOP/s", "frac": alg["flops_" + dom] / (mean_stage[dom] / 1e3) / 1e12 / tpk,
                    "layer_achieved": alg["flops"] / (ms_step / 1e3) / 1e12,
                    "layer_frac": alg["flops"] / (ms_step / 1e3) / 1e12 / tpk, "peak_source": tpk_src},
+        # the layer's binding roofline: the slower of streaming its algorithmic bytes at the
+        # measured HBM bandwidth and running its FLOPs at the tensor peak above
+        "binding_roofline": {"t_hbm_ms": alg["layer"] / (pk["hbm_gbs"] * 1e9) * 1e3,
+                             "t_tensor_ms": alg["flops"] / (tpk * 1e12) * 1e3,
+                             "bound": "hbm" if alg["layer"] / pk["hbm_gbs"] >= alg["flops"] / (tpk * 1e3) else "tensor",
+                             "frac": max(alg["layer"] / (pk["hbm_gbs"] * 1e9), alg["flops"] / (tpk * 1e12)) * 1e3 / ms_step},
         "stages_ms": mean_stage,
         "ms_per_step_with_stage_events": prof_ms / args.steps,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": x.numel() * 2 + logits.numel() * 4,
