@@ -112,6 +112,8 @@ SMALL_FP8 = [
     dict(T=700, H=512, E=8, I=384, k=2, Is=128, seed=26, bias="normal"),   # groups above and below 192
     dict(T=500, H=1024, E=4, I=256, k=2, Is=0, seed=27, bias="zipf"),      # one group of several tiles
     dict(T=600, H=640, E=6, I=256, k=2, Is=256, seed=28, bias=None),       # partial 512-block of H
+    # more than 4096 tokens: the histogram -> scan -> scatter permutation, every output checked
+    dict(T=4500, H=256, E=8, I=128, k=2, Is=128, seed=40, bias="normal"),
 ]
 
 
@@ -173,6 +175,8 @@ SMALL_INT4 = [
     dict(T=37, H=512, E=8, I=384, k=3, Is=256, seed=42, bias="normal"),   # shared expert, ragged groups
     dict(T=200, H=1024, E=4, I=256, k=2, Is=0, seed=43, bias="zipf"),     # 64-row token tiles, several per group
     dict(T=3, H=128, E=16, I=128, k=4, Is=128, seed=44, bias=None),       # mostly empty experts
+    # more than 4096 tokens (multi-kernel permutation), groups of many 96-row token tiles
+    dict(T=4500, H=256, E=8, I=128, k=2, Is=0, seed=45, bias="zipf"),
 ]
 
 
