@@ -17,11 +17,16 @@ Recipe (every tensor has its own seeded torch generator on the chosen device):
              codes = e4m3(W/s) by torch's float8_e4m3fn conversion (round to nearest even);
       - int4: one bf16 scale per (row, 128-element K group), s = bf16(amax/7) (1 when 0),
              q = clamp(round_half_even(W/s), -7, 7), two's-complement nibbles, the even K
-             index in the low nibble.
+             index in the low nibble;
+      - MXFP4: one E8M0 byte per (row, 32-element K block) holding the exponent
+             x = floor(log2(amax)) - 2 (the largest E2M1 power of two is 2^2; 0 when
+             amax = 0), stored as x + 127; each element is W / 2^x rounded to the nearest
+             E2M1 value (ties to the even code, magnitudes above 6 saturate to 6), the
+             even K index in the low nibble.
 Shapes follow the pages' models: a Qwen3.5-397B-shaped layer (512 experts x 1024, top-10,
 one shared expert of 1024, hidden 4096) at decode and prefill sizes; a DeepSeek-R1-shaped
 layer (hidden 7168, 256 experts x 2048, top-8, shared 2048) with skewed routing; a 4-bit
-128-expert layer; and a tiny layer for the oracle.
+128-expert layer (int4, and the same shape with MXFP4 weights); and a tiny layer for the oracle.
 """
 from __future__ import annotations
 
@@ -45,6 +50,8 @@ CONFIGS = {
                             "2048, FP8 e4m3 sc512, Zipf-skewed routing"),
     "int4": dict(T=1024, H=4096, E=128, I=1536, k=8, Is=0, wfmt="int4", seed=4, bias=None,
                  workload="4-bit-weight MoE T=1024 H=4096 E=128 I=1536 top-8, int4 g128 bf16"),
+    "mxfp4": dict(T=1024, H=4096, E=128, I=1536, k=8, Is=0, wfmt="mxfp4", seed=8, bias=None,
+                  workload="MXFP4-weight MoE T=1024 H=4096 E=128 I=1536 top-8, e2m1 + E8M0/32, bf16"),
 }
 
 # Smaller layers with the same per-expert shapes, for profiler captures (weights still far
@@ -56,6 +63,8 @@ PROFILE_CONFIGS = {
                             workload="prefill-shaped MoE T=1024 H=4096 E=64 I=1024 top-10 + shared 1024, FP8"),
     "profile-int4": dict(T=128, H=4096, E=16, I=1536, k=8, Is=0, wfmt="int4", seed=7, bias=None,
                          workload="4-bit MoE T=128 H=4096 E=16 I=1536 top-8, int4 g128"),
+    "profile-mxfp4": dict(T=128, H=4096, E=16, I=1536, k=8, Is=0, wfmt="mxfp4", seed=9, bias=None,
+                          workload="MXFP4 MoE T=128 H=4096 E=16 I=1536 top-8, e2m1 + E8M0/32"),
 }
 
 # tensor ids for the per-tensor generators
@@ -97,6 +106,34 @@ def _quant_int4(w: torch.Tensor):
     return packed.contiguous(), s.contiguous()
 
 
+# E2M1 magnitude code of 2 * |value| for the representable magnitudes 0, 0.5, ..., 6
+_E2M1_CODE_OF_2V = {0: 0, 1: 1, 2: 2, 3: 3, 4: 4, 6: 5, 8: 6, 12: 7}
+
+
+def _quant_mxfp4(w: torch.Tensor):
+    """W [..., N, K] fp32 -> (packed uint8 [..., N, K/2], E8M0 scales uint8 [..., N, K/32])."""
+    K = w.shape[-1]
+    assert K % 32 == 0
+    blk = w.reshape(*w.shape[:-1], K // 32, 32).double()
+    amax = blk.abs().amax(dim=-1)
+    _, e = torch.frexp(amax)  # amax = m * 2^e, m in [0.5, 1): floor(log2(amax)) = e - 1
+    xexp = torch.where(amax == 0, torch.zeros_like(e), e - 1 - 2).clamp(-127, 127)
+    v = blk / torch.pow(2.0, xexp.double()).unsqueeze(-1)  # exact: a power of two
+    a = v.abs()
+    step = torch.where(a < 2, 0.5, torch.where(a < 4, 1.0, 2.0))
+    q2 = (torch.round(a / step) * step).clamp(max=6.0) * 2  # 2|q| in {0, 1, 2, 3, 4, 6, 8, 12}
+    lut = torch.zeros(13, dtype=torch.int16, device=w.device)
+    for k2, c in _E2M1_CODE_OF_2V.items():
+        lut[k2] = c
+    mag = lut[q2.long()]
+    nib = torch.where((v < 0) & (mag > 0), mag | 8, mag).reshape(*w.shape[:-1], K)
+    packed = (nib[..., 0::2] | (nib[..., 1::2] << 4)).to(torch.uint8)
+    return packed.contiguous(), (xexp + 127).to(torch.uint8).contiguous()
+
+
+_QUANT = {"fp8": _quant_fp8, "int4": _quant_int4, "mxfp4": _quant_mxfp4}
+
+
 def _weights(seed, tid, shape, fan_in, wfmt, device, chunk_elems=1 << 28):
     """Draw W ~ N(0, 1/fan_in) of `shape` [E, N, K] in expert chunks and quantise."""
     E, N, K = shape
@@ -107,7 +144,7 @@ def _weights(seed, tid, shape, fan_in, wfmt, device, chunk_elems=1 << 28):
         e1 = min(E, e0 + per)
         w = torch.randn((e1 - e0, N, K), generator=g, device=device, dtype=torch.float32)
         w.mul_(1.0 / math.sqrt(fan_in))
-        q, s = _quant_fp8(w) if wfmt == "fp8" else _quant_int4(w)
+        q, s = _QUANT[wfmt](w)
         qs.append(q)
         ss.append(s)
         del w

@@ -24,6 +24,8 @@ _lib = None
 
 FP8_SC512 = 1
 INT4_G128 = 2
+MXFP4_G32 = 3
+_WFMT = {"fp8": FP8_SC512, "int4": INT4_G128, "mxfp4": MXFP4_G32}
 
 
 class Dims(ctypes.Structure):
@@ -58,6 +60,10 @@ def lib():
             L.orc_e4m3_encode.restype = ctypes.c_uint8
             L.orc_e4m3_encode.argtypes = [ctypes.c_float]
             L.orc_e4m3_encode_n.argtypes = [I, P, P]
+            L.orc_e2m1_decode.restype = ctypes.c_double
+            L.orc_e2m1_decode.argtypes = [I]
+            L.orc_e8m0_decode.restype = ctypes.c_double
+            L.orc_e8m0_decode.argtypes = [ctypes.c_uint8]
             L.orc_double_to_bf16.restype = ctypes.c_uint16
             L.orc_double_to_bf16.argtypes = [ctypes.c_double]
             L.orc_route.argtypes = [I, I, I, P, P, P]
@@ -67,6 +73,7 @@ def lib():
             L.orc_quant_rows_bf16.argtypes = [I, I, P, P, P]
             L.orc_expert_fp8_row.argtypes = [I, I] + [P] * 10
             L.orc_expert_int4_row.argtypes = [I, I] + [P] * 9
+            L.orc_expert_w4_row.argtypes = [I, I, I] + [P] * 9
             L.orc_layer.argtypes = [ctypes.POINTER(Dims), ctypes.POINTER(Weights), P, P, I, P, P, P, P, I]
             _lib = L
     return _lib
@@ -96,6 +103,14 @@ def e4m3_encode(x) -> np.ndarray:
     q = np.empty(x.shape, np.uint8)
     lib().orc_e4m3_encode_n(x.size, _p(x), _p(q))
     return q
+
+
+def e2m1_decode(nib: int) -> float:
+    return lib().orc_e2m1_decode(int(nib))
+
+
+def e8m0_decode(code: int) -> float:
+    return lib().orc_e8m0_decode(int(code))
 
 
 def double_to_bf16(x: float) -> int:
@@ -197,6 +212,20 @@ def expert_int4_row(x_bits, wg, sg, wu, su, wd, sd):
     return y, h
 
 
+def expert_mxfp4_row(x_bits, wg, sg, wu, su, wd, sd):
+    """One MXFP4 expert on one bf16 row -> (y float64 [H], h float64 [I], bf16-rounded)."""
+    x_bits = _c(x_bits, np.uint16)
+    wg, wu, wd = _c(wg, np.uint8), _c(wu, np.uint8), _c(wd, np.uint8)
+    sg, su, sd = _c(sg, np.uint8), _c(su, np.uint8), _c(sd, np.uint8)
+    I = wg.shape[0]
+    H = x_bits.shape[0]
+    y = np.empty(H, np.float64)
+    h = np.empty(I, np.float64)
+    lib().orc_expert_w4_row(MXFP4_G32, H, I, _p(x_bits), _p(wg), _p(sg), _p(wu), _p(su), _p(wd),
+                            _p(sd), _p(y), _p(h))
+    return y, h
+
+
 # --------------------------------------------------------------------------------------
 # the layer
 # --------------------------------------------------------------------------------------
@@ -209,7 +238,7 @@ def layer(layer_np: dict, tokens=None, nthreads: int | None = None, ambiguity: b
     ``layer_np`` holds numpy arrays with the keys of ``moe_synth`` (x as bf16 bit patterns).
     """
     d = layer_np["dims"]
-    wfmt = FP8_SC512 if d["wfmt"] == "fp8" else INT4_G128
+    wfmt = _WFMT[d["wfmt"]]
     dims = Dims(d["T"], d["H"], d["E"], d["I"], d["k"], d["Is"], wfmt)
     keep = {}
 
@@ -221,7 +250,7 @@ def layer(layer_np: dict, tokens=None, nthreads: int | None = None, ambiguity: b
         keep[name] = a
         return _p(a)
 
-    sdt = np.float32 if wfmt == FP8_SC512 else np.uint16
+    sdt = {FP8_SC512: np.float32, INT4_G128: np.uint16, MXFP4_G32: np.uint8}[wfmt]
     W = Weights(arr("w_gate", np.uint8), arr("w_up", np.uint8), arr("w_down", np.uint8),
                 arr("s_gate", sdt), arr("s_up", sdt), arr("s_down", sdt),
                 arr("ws_gate", np.uint8), arr("ws_up", np.uint8), arr("ws_down", np.uint8),

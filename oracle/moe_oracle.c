@@ -41,6 +41,13 @@
  *         round-to-nearest-even, finite values beyond 448 saturate to 448.
  *  R14    int4 weights are symmetric two's-complement nibbles, the even K index in the
  *         low nibble; the weight is q * s with one bf16 s per (row, 128-element K group).
+ *  R20    MXFP4 weights ([P4] same section: MXFP4 spends 4.25 bits per number, i.e. one
+ *         8-bit scale per 32 four-bit values) follow the OCP Microscaling format: each
+ *         nibble is an E2M1 value (S.EE.M, bias 1, exponent field 0 = 0.M, no inf/NaN,
+ *         largest 6), the even K index in the low nibble; each (row, 32-element K block)
+ *         has one E8M0 byte c, the scale 2^(c-127) (c = 255 is NaN).  The weight is
+ *         e2m1 * 2^(c-127); activations and h stay bf16 as in R11 (the same page calls
+ *         4-bit activations far harder than 4-bit weights).
  *
  * Every sum below is written out in the order the definition states; nothing is blocked,
  * fused or reordered beyond it.  Build: gcc -O2 -fno-fast-math -ffp-contract=off.
@@ -53,15 +60,17 @@
 
 #define ORC_FP8_SC512 1
 #define ORC_INT4_G128 2
+#define ORC_MXFP4_G32 3
 
 typedef struct {
     int T, H, E, I, k, Is; /* Is = 0: no shared expert */
-    int wfmt;              /* ORC_FP8_SC512 or ORC_INT4_G128 */
+    int wfmt;              /* ORC_FP8_SC512, ORC_INT4_G128 or ORC_MXFP4_G32 */
 } orc_dims;
 
 typedef struct {
     /* FP8: codes [E,I,H], [E,I,H], [E,H,I]; scales fp32 [E,I,nb(H)], [E,I,nb(H)], [E,H,nb(I)]
-     * int4: packed bytes [E,I,H/2], [E,I,H/2], [E,H,I/2]; scales bf16 [E,I,H/128] ... */
+     * int4: packed bytes [E,I,H/2], [E,I,H/2], [E,H,I/2]; scales bf16 [E,I,H/128] ...
+     * MXFP4: packed bytes as int4; scales E8M0 bytes [E,I,H/32], [E,I,H/32], [E,H,I/32] */
     const uint8_t *w_gate, *w_up, *w_down;
     const void *s_gate, *s_up, *s_down;
     /* shared expert, same formats with E = 1 and I -> Is (NULL when Is == 0) */
@@ -127,6 +136,24 @@ uint8_t orc_e4m3_encode(float xf)
 void orc_e4m3_encode_n(int n, const float *x, uint8_t *q)
 {
     for (int i = 0; i < n; ++i) q[i] = orc_e4m3_encode(x[i]);
+}
+
+/* E2M1 decode from the format definition (R20): S.EE.M, exponent bias 1; exponent field 0
+ * holds 0.M (so 0 or 0.5); field E >= 1 holds 1.M x 2^(E-1). */
+double orc_e2m1_decode(int nib)
+{
+    int sign = (nib >> 3) & 1;
+    int e = (nib >> 1) & 3;
+    int m = nib & 1;
+    double v = (e == 0) ? 0.5 * (double)m : ldexp(1.0 + 0.5 * (double)m, e - 1);
+    return sign ? -v : v;
+}
+
+/* E8M0 decode (R20): the byte is a biased exponent, 2^(c-127); 255 is NaN. */
+double orc_e8m0_decode(uint8_t c)
+{
+    if (c == 255) return NAN;
+    return ldexp(1.0, (int)c - 127);
 }
 
 double orc_bf16_to_double(uint16_t b)
@@ -322,10 +349,13 @@ void orc_quant_row_fp8(int K, const float *x, uint8_t *q, float *s)
 /* ------------------------------------------------------------------------------------ */
 
 static double orc_dec_tab[256];
+static double orc_e2m1_tab[16], orc_e8m0_tab[256]; /* memoised R20 decodes */
 static pthread_once_t orc_tab_once = PTHREAD_ONCE_INIT;
 static void orc_tab_init(void)
 {
     for (int c = 0; c < 256; ++c) orc_dec_tab[c] = orc_e4m3_decode((uint8_t)c);
+    for (int c = 0; c < 16; ++c) orc_e2m1_tab[c] = orc_e2m1_decode(c);
+    for (int c = 0; c < 256; ++c) orc_e8m0_tab[c] = orc_e8m0_decode((uint8_t)c);
 }
 
 /* y[n] = sum_kb sx[kb] * sw[n,kb] * sum_{i in kb} dec(qx[i]) * dec(qw[n,i]),  n < N.
@@ -417,7 +447,8 @@ static void orc_expert_fp8(int H, int I, const uint8_t *qx, const float *sx, con
 }
 
 /* ------------------------------------------------------------------------------------ */
-/* int4 experts -- [P5] ① (4-bit weights dequantised to 16-bit, then multiply-add); R11, R14 */
+/* 4-bit experts -- [P5] ① (4-bit weights dequantised to 16-bit, then multiply-add);        */
+/* R11, R14 (int4), R20 (MXFP4)                                                         */
 /* ------------------------------------------------------------------------------------ */
 
 static int orc_nib(const uint8_t *packed_row, int i)
@@ -427,26 +458,47 @@ static int orc_nib(const uint8_t *packed_row, int i)
     return v >= 8 ? v - 16 : v;
 }
 
-/* y[n] = sum_i a[i] * (q[n,i] * s[n, i/128])  with a in fp64 (bf16 values, exact). */
-static void orc_proj_int4(int N, int K, const double *a, const uint8_t *qw, const uint16_t *sw,
-                          double *y)
+/* The raw nibble (0..15) of element i of a packed row. */
+static int orc_nib_raw(const uint8_t *packed_row, int i)
 {
-    int ng = K / 128;
+    int b = packed_row[i >> 1];
+    return (i & 1) ? (b >> 4) : (b & 0xF);
+}
+
+/* Weight [n, i] of a 4-bit [N, K] matrix: int4 q * s (R14) or e2m1 * 2^(c-127) (R20). */
+static double orc_w4(int wfmt, int K, const uint8_t *qw, const void *sw, int n, int i)
+{
+    const uint8_t *row = qw + (size_t)n * (K / 2);
+    if (wfmt == ORC_MXFP4_G32) {
+        const uint8_t *sc = (const uint8_t *)sw;
+        return orc_e2m1_tab[orc_nib_raw(row, i)] * orc_e8m0_tab[sc[(size_t)n * (K / 32) + i / 32]];
+    }
+    const uint16_t *sc = (const uint16_t *)sw;
+    return (double)orc_nib(row, i) * orc_bf16_to_double(sc[(size_t)n * (K / 128) + i / 128]);
+}
+
+/* The scale array of expert e of a 4-bit [E, N, K] weight set. */
+static const void *orc_w4_scales(int wfmt, const void *sw, size_t e, int N, int K)
+{
+    if (wfmt == ORC_MXFP4_G32) return (const uint8_t *)sw + e * (size_t)N * (size_t)(K / 32);
+    return (const uint16_t *)sw + e * (size_t)N * (size_t)(K / 128);
+}
+
+/* y[n] = sum_i a[i] * W[n, i]  with a in fp64 (bf16 values, exact). */
+static void orc_proj_w4(int wfmt, int N, int K, const double *a, const uint8_t *qw, const void *sw,
+                        double *y)
+{
     for (int n = 0; n < N; ++n) {
-        const uint8_t *row = qw + (size_t)n * (K / 2);
         double acc = 0.0;
-        for (int i = 0; i < K; ++i) {
-            double w = (double)orc_nib(row, i) * orc_bf16_to_double(sw[(size_t)n * ng + i / 128]);
-            acc += a[i] * w;
-        }
+        for (int i = 0; i < K; ++i) acc += a[i] * orc_w4(wfmt, K, qw, sw, n, i);
         y[n] = acc;
     }
 }
 
 /* R10a for 4-bit layers: h is rounded to bf16, so an h within ORC_AMBIG_REL of a bf16
  * rounding midpoint may round either way; env[n] gets |h_alt - h| * |W[n, i]| for each such i. */
-static void orc_h_ambiguity_bf16(int H, int I, const double *hx, const uint8_t *wd,
-                                 const uint16_t *sd, double *env)
+static void orc_h_ambiguity_bf16(int wfmt, int H, int I, const double *hx, const uint8_t *wd,
+                                 const void *sd, double *env)
 {
     for (int i = 0; i < I; ++i) {
         double a = fabs(hx[i]);
@@ -457,33 +509,29 @@ static void orc_h_ambiguity_bf16(int H, int I, const double *hx, const uint8_t *
         double quantum = ldexp(1.0, lead - 7);
         double frac = a / quantum - floor(a / quantum); /* position between two bf16 values */
         if (fabs(frac - 0.5) * quantum > ORC_AMBIG_REL * a) continue;
-        for (int n = 0; n < H; ++n) {
-            const uint8_t *row = wd + (size_t)n * (I / 2);
-            double wv = (double)orc_nib(row, i) * orc_bf16_to_double(sd[(size_t)n * (I / 128) + i / 128]);
-            env[n] += quantum * fabs(wv);
-        }
+        for (int n = 0; n < H; ++n) env[n] += quantum * fabs(orc_w4(wfmt, I, wd, sd, n, i));
     }
 }
 
-static void orc_expert_int4(int H, int I, const double *x, const uint8_t *wg, const uint16_t *sg,
-                            const uint8_t *wu, const uint16_t *su, const uint8_t *wd,
-                            const uint16_t *sd, double *y, double *h_out, double *env)
+static void orc_expert_w4(int wfmt, int H, int I, const double *x, const uint8_t *wg, const void *sg,
+                          const uint8_t *wu, const void *su, const uint8_t *wd, const void *sd,
+                          double *y, double *h_out, double *env)
 {
     double *G = (double *)malloc(sizeof(double) * (size_t)I);
     double *U = (double *)malloc(sizeof(double) * (size_t)I);
     double *hx = (double *)malloc(sizeof(double) * (size_t)I);
     double *h = (double *)malloc(sizeof(double) * (size_t)I);
-    orc_proj_int4(I, H, x, wg, sg, G);
-    orc_proj_int4(I, H, x, wu, su, U);
+    orc_proj_w4(wfmt, I, H, x, wg, sg, G);
+    orc_proj_w4(wfmt, I, H, x, wu, su, U);
     for (int n = 0; n < I; ++n) {
         hx[n] = orc_silu(G[n]) * U[n];
         h[n] = orc_bf16_to_double(orc_double_to_bf16(hx[n]));
     }
     if (h_out) memcpy(h_out, h, sizeof(double) * (size_t)I);
-    orc_proj_int4(H, I, h, wd, sd, y);
+    orc_proj_w4(wfmt, H, I, h, wd, sd, y);
     if (env) {
         for (int n = 0; n < H; ++n) env[n] = 0.0;
-        orc_h_ambiguity_bf16(H, I, hx, wd, sd, env);
+        orc_h_ambiguity_bf16(wfmt, H, I, hx, wd, sd, env);
     }
     free(G);
     free(U);
@@ -555,21 +603,19 @@ static void orc_layer_token(const orc_dims *d, const orc_weights *w, const uint1
     } else {
         double *xd = (double *)malloc(sizeof(double) * (size_t)H);
         for (int i = 0; i < H; ++i) xd[i] = orc_bf16_to_double(xrow[i]);
-        const uint16_t *sg = (const uint16_t *)w->s_gate, *su = (const uint16_t *)w->s_up,
-                       *sd = (const uint16_t *)w->s_down;
+        const int f = d->wfmt;
         for (int j = 0; j < k; ++j) {
             size_t e = (size_t)idx[j];
-            orc_expert_int4(H, I, xd, w->w_gate + e * I * (H / 2), sg + e * I * (H / 128),
-                            w->w_up + e * I * (H / 2), su + e * I * (H / 128),
-                            w->w_down + e * H * (I / 2), sd + e * H * (I / 128), y, NULL, env);
+            orc_expert_w4(f, H, I, xd, w->w_gate + e * I * (H / 2), orc_w4_scales(f, w->s_gate, e, I, H),
+                          w->w_up + e * I * (H / 2), orc_w4_scales(f, w->s_up, e, I, H),
+                          w->w_down + e * H * (I / 2), orc_w4_scales(f, w->s_down, e, H, I), y, NULL, env);
             for (int n = 0; n < H; ++n) out[n] += p[j] * y[n];
             if (amb)
                 for (int n = 0; n < H; ++n) amb[n] += p[j] * env[n];
         }
         if (Is > 0) {
-            orc_expert_int4(H, Is, xd, w->ws_gate, (const uint16_t *)w->ss_gate, w->ws_up,
-                            (const uint16_t *)w->ss_up, w->ws_down, (const uint16_t *)w->ss_down,
-                            y, NULL, env);
+            orc_expert_w4(f, H, Is, xd, w->ws_gate, w->ss_gate, w->ws_up, w->ss_up, w->ws_down,
+                          w->ss_down, y, NULL, env);
             for (int n = 0; n < H; ++n) out[n] += y[n];
             if (amb)
                 for (int n = 0; n < H; ++n) amb[n] += env[n];
@@ -611,8 +657,8 @@ int orc_layer(const orc_dims *d, const orc_weights *w, const uint16_t *x, const 
               int nthreads)
 {
     if (d->E < 1 || d->k < 1 || d->k > d->E || d->H < 1 || d->I < 1 || d->Is < 0) return -1;
-    if (d->wfmt == ORC_INT4_G128 && (d->H % 128 || d->I % 128 || d->Is % 128)) return -1;
-    if (d->wfmt != ORC_FP8_SC512 && d->wfmt != ORC_INT4_G128) return -1;
+    if (d->wfmt != ORC_FP8_SC512 && d->wfmt != ORC_INT4_G128 && d->wfmt != ORC_MXFP4_G32) return -1;
+    if (d->wfmt != ORC_FP8_SC512 && (d->H % 128 || d->I % 128 || d->Is % 128)) return -1;
     for (int i = 0; i < n_sel; ++i)
         if (sel[i] < 0 || sel[i] >= d->T) return -1;
     pthread_once(&orc_tab_once, orc_tab_init);
@@ -663,13 +709,23 @@ void orc_expert_fp8_row(int H, int I, const uint8_t *qx, const float *sx, const 
     orc_expert_fp8(H, I, qx, sx, wg, sg, wu, su, wd, sd, y, h, NULL);
 }
 
+/* One 4-bit expert (int4 or MXFP4) on one bf16 row: y (H values) and h (I values,
+ * bf16-rounded). */
+void orc_expert_w4_row(int wfmt, int H, int I, const uint16_t *x, const uint8_t *wg, const void *sg,
+                       const uint8_t *wu, const void *su, const uint8_t *wd, const void *sd, double *y,
+                       double *h)
+{
+    pthread_once(&orc_tab_once, orc_tab_init);
+    double *xd = (double *)malloc(sizeof(double) * (size_t)H);
+    for (int i = 0; i < H; ++i) xd[i] = orc_bf16_to_double(x[i]);
+    orc_expert_w4(wfmt, H, I, xd, wg, sg, wu, su, wd, sd, y, h, NULL);
+    free(xd);
+}
+
 /* One int4 expert on one bf16 row: y (H values) and h (I values, bf16-rounded). */
 void orc_expert_int4_row(int H, int I, const uint16_t *x, const uint8_t *wg, const uint16_t *sg,
                          const uint8_t *wu, const uint16_t *su, const uint8_t *wd,
                          const uint16_t *sd, double *y, double *h)
 {
-    double *xd = (double *)malloc(sizeof(double) * (size_t)H);
-    for (int i = 0; i < H; ++i) xd[i] = orc_bf16_to_double(x[i]);
-    orc_expert_int4(H, I, xd, wg, sg, wu, su, wd, sd, y, h, NULL);
-    free(xd);
+    orc_expert_w4_row(ORC_INT4_G128, H, I, x, wg, sg, wu, su, wd, sd, y, h);
 }

@@ -21,3 +21,9 @@ def test_layer_and_router_are_reproducible():
 def test_int4_layer_is_reproducible():
     cfg = dict(T=8, H=256, E=3, I=128, k=2, Is=0, seed=5, bias=None, wfmt="int4")
     assert _same(moe_synth.make_layer(cfg), moe_synth.make_layer(cfg))
+
+
+def test_mxfp4_layer_is_reproducible():
+    cfg = dict(T=8, H=256, E=3, I=128, k=2, Is=128, seed=5, bias=None, wfmt="mxfp4")
+    assert _same(moe_synth.make_layer(cfg), moe_synth.make_layer(cfg))
+    assert not _same(moe_synth.make_layer(cfg), moe_synth.make_layer(dict(cfg, seed=6)))
