@@ -20,6 +20,14 @@
  *   MOE_W_INT4_G128: symmetric int4, two's-complement nibbles, two per byte with the even K
  *     index in the low nibble, [out, in/2] bytes; one bf16 scale per (row, 128-element
  *     K group); activations stay bf16 (h is rounded to bf16).
+ *   MOE_W_MXFP4_G32: OCP Microscaling FP4 (page "设计 AI 芯片的硬件与软件", section "数值格式，
+ *     或如何制造便宜的脉动阵列": 4-bit values plus an 8-bit scale per 32, 4.25 bits per number).
+ *     E2M1 nibbles (sign, 2 exponent bits with bias 1, 1 mantissa bit: magnitudes 0, 0.5, 1,
+ *     1.5, 2, 3, 4, 6), two per byte with the even K index in the low nibble, [out, in/2]
+ *     bytes; one E8M0 byte c per (row, 32-element K block), the scale 2^(c-127).  The weight
+ *     e2m1 * 2^(c-127) is formed exactly for c in 2..252 (other codes are outside the
+ *     supported domain: the product may flush to zero or overflow).  Activations stay bf16
+ *     (h is rounded to bf16), as for int4.
  *
  * Pointer conventions.  Every buffer passed to moe_router_logits / moe_route / moe_forward is
  * DEVICE memory that the caller allocates and owns; the library keeps no pointer to it after
@@ -55,7 +63,8 @@ typedef struct CUstream_st *moe_stream_t; /* the same type as cudaStream_t */
 
 enum moe_wfmt {
     MOE_W_FP8_SC512 = 1, /* e4m3 weights + fp32 scale per (row, 512-block of K) */
-    MOE_W_INT4_G128 = 2  /* int4 weights + bf16 scale per (row, 128-group of K) */
+    MOE_W_INT4_G128 = 2, /* int4 weights + bf16 scale per (row, 128-group of K) */
+    MOE_W_MXFP4_G32 = 3  /* E2M1 weights + E8M0 scale per (row, 32-block of K) */
 };
 
 enum moe_status {
@@ -84,6 +93,8 @@ typedef struct {
  *         s_gate, s_up [E, I, ceil(H/512)] fp32; s_down [E, H, ceil(I/512)] fp32.
  *   int4: w_gate, w_up [E, I, H/2] bytes; w_down [E, H, I/2] bytes;
  *         s_gate, s_up [E, I, H/128] bf16; s_down [E, H, I/128] bf16.
+ *   MXFP4: w_* as int4 (E2M1 nibbles); s_gate, s_up [E, I, H/32] bytes; s_down [E, H, I/32]
+ *         bytes (E8M0).
  *   ws_* / ss_*: the shared expert in the same format with E = 1 and I -> I_shared; NULL when
  *   I_shared == 0. */
 typedef struct {

@@ -20,6 +20,8 @@ LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 
 MOE_W_FP8_SC512 = 1
 MOE_W_INT4_G128 = 2
+MOE_W_MXFP4_G32 = 3
+_WFMT = {"fp8": MOE_W_FP8_SC512, "int4": MOE_W_INT4_G128, "mxfp4": MOE_W_MXFP4_G32}
 MOE_OK = 0
 ERRORS = {-1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED", -3: "MOE_ERR_WORKSPACE",
           -4: "MOE_ERR_CUDA", -5: "MOE_ERR_DEVICE_TIMEOUT", -6: "MOE_ERR_BOUNDS"}
@@ -132,9 +134,11 @@ class Plan:
 
     def __init__(self, T_max, H, E, I, k, I_shared=0, wfmt="fp8"):
         L = load_library()
-        fmt = MOE_W_FP8_SC512 if wfmt in ("fp8", MOE_W_FP8_SC512) else MOE_W_INT4_G128
+        if wfmt not in _WFMT and wfmt not in _WFMT.values():
+            raise ValueError(f"unknown weight format {wfmt!r}")
+        fmt = _WFMT.get(wfmt, wfmt)
         self.dims = moe_dims(T_max, H, E, I, k, I_shared, fmt)
-        self.wfmt = "fp8" if fmt == MOE_W_FP8_SC512 else "int4"
+        self.wfmt = next(n for n, v in _WFMT.items() if v == fmt)
         h = ctypes.c_void_p()
         ws = ctypes.c_size_t()
         _check(L.moe_plan(ctypes.byref(self.dims), ctypes.byref(h), ctypes.byref(ws)), "moe_plan")

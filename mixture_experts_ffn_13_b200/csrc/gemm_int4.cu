@@ -1,5 +1,5 @@
 // gemm_int4.cu -- steps A4/A5 for 4-bit expert weights: persistent grouped GEMMs that unpack
-// int4 weights into tensor memory and run bf16 x bf16 -> fp32 tcgen05 MMAs.
+// int4 or MXFP4 weights into tensor memory and run bf16 x bf16 -> fp32 tcgen05 MMAs.
 //
 // Page "Flash-Next 在 GPU 上到底在算什麼", section "① 專家 FFN" (and its NVIDIA table): expert
 // weights are stored in 4/8 bits and must be decompressed to 16-bit before the tensor units
@@ -27,6 +27,13 @@
 // partial sums reproduces sum_i x_i * q_i * s_i up to fp32 rounding; rounding q * s to bf16
 // before the MMA would not (that costs ~2^-9 relative per weight and fails the layer's
 // tolerance at these sizes).
+//
+// MXFP4 weights (page "设计 AI 芯片的硬件与软件", section "数值格式，或如何制造便宜的脉动阵列":
+// 4-bit values plus an 8-bit scale per 32 of them, 4.25 bits per number) use the same
+// pipeline with one change in the dequantisers and one in the MMA/epilogue split: an E2M1
+// value (at most two significant bits) times its block's power-of-two E8M0 scale is exact in
+// bf16, so the dequantisers write the scaled weights themselves, the whole K accumulates in
+// one TMEM slot, and the epilogue has no promotion to do.
 #include "gemm_common.cuh"
 #include "launch.cuh"
 #include "sm100.cuh"
@@ -82,6 +89,31 @@ __device__ __forceinline__ uint32_t bf2_bits(__nv_bfloat162 v) { return *reinter
 
 __device__ __forceinline__ __nv_bfloat162 bits_bf2(uint32_t u) { return *reinterpret_cast<__nv_bfloat162 *>(&u); }
 
+// 8 E2M1 nibbles (element 2i in the low nibble of byte i) times the block scale sc (2^x in both
+// halves), as 4 words of bf16 pairs in element order.  Each 3-bit magnitude picks the low and
+// the high byte of its bf16 value from two 8-entry byte tables with prmt (4 elements per prmt);
+// the nibble's sign bit goes to bit 7 of the high byte; one bf16 multiply by 2^x scales a
+// pair, exactly while the product stays a normal bf16 (E8M0 codes 2..252).
+__device__ __forceinline__ uint4 unpack8_fp4(uint32_t w, __nv_bfloat162 sc)
+{
+    // bf16 of the magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6: 0000 3F00 3F80 3FC0 4000 4040 4080 40C0
+    constexpr uint32_t kLo03 = 0xC0800000u, kLo47 = 0xC0804000u;  // low bytes, codes 0-3 | 4-7
+    constexpr uint32_t kHi03 = 0x3F3F3F00u, kHi47 = 0x40404040u;  // high bytes
+    const uint32_t mag = w & 0x77777777u;                          // prmt reads 4 selectors
+    const uint32_t lo_a = prmt(kLo03, kLo47, mag), hi_a = prmt(kHi03, kHi47, mag);  // elements 0-3
+    const uint32_t lo_b = prmt(kLo03, kLo47, mag >> 16), hi_b = prmt(kHi03, kHi47, mag >> 16);  // 4-7
+    const uint32_t ev = (w << 4) & 0x80808080u;  // signs of elements 0, 2, 4, 6 at bit 7 of bytes 0-3
+    const uint32_t od = w & 0x80808080u;         // signs of elements 1, 3, 5, 7
+    const uint32_t ha = hi_a | prmt(ev, od, 0x5140u), hb = hi_b | prmt(ev, od, 0x7362u);
+    const uint32_t r0 = prmt(lo_a, ha, 0x5140u), r1 = prmt(lo_a, ha, 0x7362u);
+    const uint32_t r2 = prmt(lo_b, hb, 0x5140u), r3 = prmt(lo_b, hb, 0x7362u);
+    return make_uint4(bf2_bits(__hmul2(bits_bf2(r0), sc)), bf2_bits(__hmul2(bits_bf2(r1), sc)),
+                      bf2_bits(__hmul2(bits_bf2(r2), sc)), bf2_bits(__hmul2(bits_bf2(r3), sc)));
+}
+
+// The bf16 pair (2^(c-127), 2^(c-127)) of an E8M0 code c in 1..254.
+__device__ __forceinline__ __nv_bfloat162 e8m0_pair(uint32_t c) { return bits_bf2((c << 7) | (c << 23)); }
+
 // 8 two's-complement nibbles (element 2i in the low nibble of byte i) -> the 8 integers as
 // bf16 (exact), returned as 4 words of bf16 pairs in element order.
 __device__ __forceinline__ uint4 unpack8(uint32_t w)
@@ -101,7 +133,8 @@ __device__ __forceinline__ uint4 unpack8(uint32_t w)
     return make_uint4(r[0], r[1], r[2], r[3]);
 }
 
-template <int BN, bool GATEUP>
+// MX = false: int4 weights with bf16 scales per 128-group; MX = true: MXFP4 weights.
+template <int BN, bool GATEUP, bool MX>
 __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
     gemm_int4_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmArgs args)
 {
@@ -217,14 +250,16 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
                 const TileInfo tl = decode_tile<BN, true>(args, stt, w, tot0);
                 const int n_mma = min(BN, (tl.nrows + 15) & ~15);  // partial tiles: no work on absent rows
                 const uint32_t kIdesc = instr_desc(kTileM, n_mma, 1, 1);
-                const int ngrp = args.seg[tl.seg].K / kGroupK;
+                // int4: one TMEM slot per 128-element scale group; MXFP4: one for the whole K
+                const int ngrp = MX ? 1 : args.seg[tl.seg].K / kGroupK;
+                const int spg = MX ? args.seg[tl.seg].K / kKE : C::STAGES_PER_GROUP;
                 for (int g = 0; g < ngrp; ++g, ++ai) {
                     const int slot = ai % C::NSLOT;
                     if (!mbar_wait(&acce[slot], ((ai / C::NSLOT) & 1) ^ 1, abort_flag, status, tmo)) goto done;
                     tc_fence_after();
                     const uint32_t d0 = tmem_base + C::A_TMEM + slot * C::SLOT_COLS;
                     const uint32_t d1 = d0 + BN;
-                    for (int sk = 0; sk < C::STAGES_PER_GROUP; ++sk, ++it) {
+                    for (int sk = 0; sk < spg; ++sk, ++it) {
                         const int s = it % C::NM;
                         const int bs = it % C::NB;
                         if (!mbar_wait(&mfull[s], (it / C::NM) & 1, abort_flag, status, tmo)) goto done;
@@ -251,12 +286,42 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
         const int q = warp & 3;        // TMEM lane quarter reachable from this warp
         const int r = q * 32 + lane;   // weight row of the tile handled by this thread
         uint32_t it = 0, rt = 0;
+        // MXFP4: this row's 8 E8M0 bytes (two words per matrix) of the current raw stage, and
+        // those of the next raw stage in this CTA's sequence (the next tile's first one at a
+        // tile's end), loaded a raw stage ahead so that their latency overlaps the conversion
+        uint32_t scur[C::NA][2] = {}, snxt[C::NA][2] = {};
+        auto load_scales = [&](int wi, int kr, uint32_t (&dst)[C::NA][2]) {
+            const TileInfo t = decode_tile<BN, true>(args, stt, wi, tot0);
+            const GemmSeg &s = args.seg[t.seg];
+            const int nbk = s.K / 32;              // E8M0 bytes per weight row, a multiple of 4
+            const int b0 = kr * (kRawKE / 32);     // first byte of raw stage kr: b0 + 4 <= nbk
+#pragma unroll
+            for (int m = 0; m < C::NA; ++m) {
+                const uint8_t *base = static_cast<const uint8_t *>(m == 0 ? s.sw0 : s.sw1);
+                const uint32_t *p = reinterpret_cast<const uint32_t *>(base + (size_t)(t.wrow + r) * nbk + b0);
+                dst[m][0] = __ldg(p);
+                dst[m][1] = b0 + 4 < nbk ? __ldg(p + 1) : 0u;  // a last raw stage of 128 K has 4
+            }
+        };
+        if (MX && (int)blockIdx.x < total) load_scales(blockIdx.x, 0, snxt);
         for (int w = blockIdx.x; w < total; w += gridDim.x) {
             const TileInfo tl = decode_tile<BN, true>(args, stt, w, tot0);
             const GemmSeg &sg = args.seg[tl.seg];
             const int nkc = sg.K / kKE;
             for (int kc = 0; kc < nkc; ++kc, ++it) {
                 const int sub = kc % kSubs;
+                if (MX && sub == 0) {
+#pragma unroll
+                    for (int m = 0; m < C::NA; ++m) {
+                        scur[m][0] = snxt[m][0];
+                        scur[m][1] = snxt[m][1];
+                    }
+                    const int kr = kc / kSubs;
+                    if ((kr + 1) * kRawKE < sg.K)
+                        load_scales(w, kr + 1, snxt);
+                    else if (w + (int)gridDim.x < total)
+                        load_scales(w + gridDim.x, 0, snxt);
+                }
                 const int rs_i = rt % C::NR;
                 const int ms_i = it % C::NM;
                 bool ok = true;
@@ -275,10 +340,22 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
                     const uint4 q0 = *reinterpret_cast<const uint4 *>(rs + m * C::RAW_BYTES + c0);
                     const uint4 q1 = *reinterpret_cast<const uint4 *>(rs + m * C::RAW_BYTES + c1);
                     const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+                    // MXFP4: chunk c0 is 32-block 2*sub of the raw stage, c1 block 2*sub + 1
+                    __nv_bfloat162 sca, scb;
+                    if constexpr (MX) {
+                        const uint32_t sw = (sub >> 1) ? scur[m][1] : scur[m][0];
+                        const uint32_t sh = (sub & 1) * 16;
+                        sca = e8m0_pair((sw >> sh) & 0xFFu);
+                        scb = e8m0_pair((sw >> (sh + 8)) & 0xFFu);
+                    }
                     uint32_t v[32];
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
-                        const uint4 u = unpack8(words[j]);
+                        uint4 u;
+                        if constexpr (MX)
+                            u = unpack8_fp4(words[j], j < 4 ? sca : scb);
+                        else
+                            u = unpack8(words[j]);
                         v[4 * j] = u.x;
                         v[4 * j + 1] = u.y;
                         v[4 * j + 2] = u.z;
@@ -306,10 +383,12 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
         for (int w = blockIdx.x; w < total; w += gridDim.x) {
             const TileInfo tl = decode_tile<BN, true>(args, stt, w, tot0);
             const GemmSeg &sg = args.seg[tl.seg];
-            const int ngrp = sg.K / kGroupK;
-            const __nv_bfloat16 *sw0 = static_cast<const __nv_bfloat16 *>(sg.sw0) + (size_t)(tl.wrow + r) * ngrp;
+            // MXFP4: the weights arrive scaled and the whole K sits in one slot (scale 1)
+            const int ngrp = MX ? 1 : sg.K / kGroupK;
+            const __nv_bfloat16 *sw0 =
+                MX ? nullptr : static_cast<const __nv_bfloat16 *>(sg.sw0) + (size_t)(tl.wrow + r) * ngrp;
             const __nv_bfloat16 *sw1 =
-                GATEUP ? static_cast<const __nv_bfloat16 *>(sg.sw1) + (size_t)(tl.wrow + r) * ngrp : nullptr;
+                (GATEUP && !MX) ? static_cast<const __nv_bfloat16 *>(sg.sw1) + (size_t)(tl.wrow + r) * ngrp : nullptr;
             float acc0[C::CPW], acc1[GATEUP ? C::CPW : 1];
 #pragma unroll
             for (int c = 0; c < C::CPW; ++c) acc0[c] = 0.0f;
@@ -317,13 +396,19 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
 #pragma unroll
                 for (int c = 0; c < C::CPW; ++c) acc1[c] = 0.0f;
             }
-            float s0n = __bfloat162float(sw0[0]), s1n = GATEUP ? __bfloat162float(sw1[0]) : 0.0f;
+            float s0n = 1.0f, s1n = 1.0f;
+            if constexpr (!MX) {
+                s0n = __bfloat162float(sw0[0]);
+                s1n = GATEUP ? __bfloat162float(sw1[0]) : 0.0f;
+            }
             for (int g = 0; g < ngrp; ++g, ++ai) {
                 const int slot = ai % C::NSLOT;
                 const float s0 = s0n, s1 = s1n;
-                if (g + 1 < ngrp) {
-                    s0n = __bfloat162float(sw0[g + 1]);
-                    if (GATEUP) s1n = __bfloat162float(sw1[g + 1]);
+                if constexpr (!MX) {
+                    if (g + 1 < ngrp) {
+                        s0n = __bfloat162float(sw0[g + 1]);
+                        if (GATEUP) s1n = __bfloat162float(sw1[g + 1]);
+                    }
                 }
                 const bool ok = mbar_wait(&accf[slot], (ai / C::NSLOT) & 1, abort_flag, status, tmo);
                 if (!__all_sync(0xffffffffu, ok)) goto done;
@@ -372,35 +457,42 @@ done:
     }
 }
 
-template <int BN, bool GATEUP>
+template <int BN, bool GATEUP, bool MX>
 cudaError_t launch_t(const GemmMaps &maps, const GemmArgs &args, int num_sms, cudaStream_t s)
 {
     using C = I4Cfg<BN, GATEUP>;
-    auto kern = gemm_int4_kernel<BN, GATEUP>;
+    auto kern = gemm_int4_kernel<BN, GATEUP, MX>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     return launch_pdl(kern, dim3(num_sms), dim3(C::THREADS), C::SMEM, s, maps, args);
 }
 
-}  // namespace
-
-cudaError_t launch_gemm_int4(bool gateup, int bn, const GemmMaps &maps, const GemmArgs &args, int num_sms,
-                             cudaStream_t s)
+template <bool MX>
+cudaError_t launch_fmt(bool gateup, int bn, const GemmMaps &maps, const GemmArgs &args, int num_sms, cudaStream_t s)
 {
     if (gateup) {
         switch (bn) {
-            case 32: return launch_t<32, true>(maps, args, num_sms, s);
-            case 64: return launch_t<64, true>(maps, args, num_sms, s);
-            case 96: return launch_t<96, true>(maps, args, num_sms, s);
+            case 32: return launch_t<32, true, MX>(maps, args, num_sms, s);
+            case 64: return launch_t<64, true, MX>(maps, args, num_sms, s);
+            case 96: return launch_t<96, true, MX>(maps, args, num_sms, s);
             default: return cudaErrorInvalidValue;
         }
     }
     switch (bn) {
-        case 32: return launch_t<32, false>(maps, args, num_sms, s);
-        case 64: return launch_t<64, false>(maps, args, num_sms, s);
-        case 96: return launch_t<96, false>(maps, args, num_sms, s);
+        case 32: return launch_t<32, false, MX>(maps, args, num_sms, s);
+        case 64: return launch_t<64, false, MX>(maps, args, num_sms, s);
+        case 96: return launch_t<96, false, MX>(maps, args, num_sms, s);
         default: return cudaErrorInvalidValue;
     }
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_w4(bool gateup, bool mx, int bn, const GemmMaps &maps, const GemmArgs &args, int num_sms,
+                           cudaStream_t s)
+{
+    return mx ? launch_fmt<true>(gateup, bn, maps, args, num_sms, s)
+              : launch_fmt<false>(gateup, bn, maps, args, num_sms, s);
 }
 
 }  // namespace moe

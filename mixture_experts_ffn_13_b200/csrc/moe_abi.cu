@@ -187,7 +187,8 @@ int moe_plan(const moe_dims *dims, moe_plan_t **out_plan, size_t *workspace_byte
     *out_plan = nullptr;
     const moe_dims d = *dims;
     if (d.T_max < 1 || d.H < 1 || d.E < 1 || d.I < 1 || d.k < 1 || d.I_shared < 0) return MOE_ERR_INVALID_ARG;
-    if (d.wfmt != MOE_W_FP8_SC512 && d.wfmt != MOE_W_INT4_G128) return MOE_ERR_INVALID_ARG;
+    if (d.wfmt != MOE_W_FP8_SC512 && d.wfmt != MOE_W_INT4_G128 && d.wfmt != MOE_W_MXFP4_G32)
+        return MOE_ERR_INVALID_ARG;
     if (d.k > d.E) return MOE_ERR_INVALID_ARG;
     if (d.E > kMaxE || d.k > kMaxK || d.T_max > (1 << 20)) return MOE_ERR_UNSUPPORTED;
     if (d.H % 128 || d.I % 128 || d.I_shared % 128) return MOE_ERR_UNSUPPORTED;
@@ -362,10 +363,10 @@ int moe_route(moe_plan_t *p, int32_t T, const float *logits, int32_t *topk_idx, 
     return e == cudaSuccess ? MOE_OK : fail_cuda(p, e);
 }
 
-// The 4-bit layer: route, permute, gather bf16 rows, int4 gate|up (h in bf16), int4 down,
-// combine.  Stage events: 0 route | 1 permute | 2 gather | 3 gate|up | 4 (no h quantiser) |
-// 5 down | 6 combine | 7.
-static int forward_int4(moe_plan_t *p, int T, const uint16_t *x, const float *logits, const moe_weights *w,
+// The 4-bit layer (int4 or MXFP4): route, permute, gather bf16 rows, 4-bit gate|up (h in
+// bf16), 4-bit down, combine.  Stage events: 0 route | 1 permute | 2 gather | 3 gate|up |
+// 4 (no h quantiser) | 5 down | 6 combine | 7.
+static int forward_w4(moe_plan_t *p, int T, const uint16_t *x, const float *logits, const moe_weights *w,
                         uint16_t *out, uint8_t *ws, cudaStream_t s)
 {
     const moe_dims &d = p->d;
@@ -378,6 +379,7 @@ static int forward_int4(moe_plan_t *p, int T, const uint16_t *x, const float *lo
     const bool shared = Is > 0;
     const int A = T * k;
     const int bn = pick_bn(T, k, E, false);
+    const bool mx = d.wfmt == MOE_W_MXFP4_G32;
     mark(0);
     int *chk = p->checked ? p->d_status : nullptr;
     cudaError_t e = launch_route(logits, T, E, k, b.topk_idx, b.topk_w, s, chk);
@@ -417,7 +419,7 @@ static int forward_int4(moe_plan_t *p, int T, const uint16_t *x, const float *lo
         rc |= encode_map_2d(&mg.b[1], xp_sh, BF, 2, H, T, 64, bn, true);
     }
     if (rc) return MOE_ERR_CUDA;
-    e = launch_gemm_int4(true, bn, mg, ag, p->num_sms, s);
+    e = launch_gemm_w4(true, mx, bn, mg, ag, p->num_sms, s);
     mark(4);
     mark(5);
     if (e != cudaSuccess) return fail_cuda(p, e);
@@ -434,7 +436,7 @@ static int forward_int4(moe_plan_t *p, int T, const uint16_t *x, const float *lo
         rc |= encode_map_2d(&md.b[1], h_sh, BF, 2, Is, T, 64, bn, true);
     }
     if (rc) return MOE_ERR_CUDA;
-    e = launch_gemm_int4(false, bn, md, ad, p->num_sms, s);
+    e = launch_gemm_w4(false, mx, bn, md, ad, p->num_sms, s);
     mark(6);
     if (e != cudaSuccess) return fail_cuda(p, e);
     e = launch_combine(y, y_sh, b.pos, b.topk_w, T, H, k, out, s, chk);
@@ -481,7 +483,7 @@ int moe_forward(moe_plan_t *p, int32_t T, const uint16_t *x, const float *logits
     auto mark = [&](int i) {
         if (p->prof) cudaEventRecord(p->ev[i], s);
     };
-    if (d.wfmt == MOE_W_INT4_G128) return forward_int4(p, T, x, logits, w, out, static_cast<uint8_t *>(workspace), s);
+    if (d.wfmt != MOE_W_FP8_SC512) return forward_w4(p, T, x, logits, w, out, static_cast<uint8_t *>(workspace), s);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     const Layout L = make_layout(d);
     const RouteBufs b = route_bufs(L, ws);

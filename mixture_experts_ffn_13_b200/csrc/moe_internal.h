@@ -15,6 +15,7 @@ constexpr int kMaxK = 32;     // router: one lane per selected expert
 constexpr int kChunk = 256;   // permutation: tokens per chunk (8 warps x 32)
 constexpr int kBlockK = 512;  // FP8 sub-channel block along K
 constexpr int kGroupK = 128;  // int4 scale group along K
+constexpr int kMxBlock = 32;  // MXFP4 scale block along K
 constexpr uint64_t kDefaultTimeoutNs = 1000000000ull;  // device-side waits give up after 1 s
 
 // ---- routing / permutation (route.cu) ---------------------------------------------------
@@ -99,9 +100,10 @@ struct GemmMaps {
 // FP8 grouped GEMMs.  gateup: h = silu(x Wg^T) * (x Wu^T) in fp32; down: y = h Wd^T in fp32.
 cudaError_t launch_gemm_fp8(bool gateup, int bn, const GemmMaps &maps, const GemmArgs &args, int num_sms,
                             cudaStream_t s);
-// int4 grouped GEMMs over bf16 activations: gate|up writes h as bf16, down writes y fp32.
-cudaError_t launch_gemm_int4(bool gateup, int bn, const GemmMaps &maps, const GemmArgs &args,
-                             int num_sms, cudaStream_t s);
+// 4-bit grouped GEMMs over bf16 activations (int4 with bf16 scales per 128-group, or MXFP4
+// when mx): gate|up writes h as bf16, down writes y fp32.
+cudaError_t launch_gemm_w4(bool gateup, bool mx, int bn, const GemmMaps &maps, const GemmArgs &args,
+                           int num_sms, cudaStream_t s);
 
 // Router logits [T, E] (written) and their softmax top-k (step A1): the router GEMM, then the
 // route kernel.

@@ -58,7 +58,8 @@ def _plan_rc(lib, **kw):
 @pytest.mark.parametrize("kw,code", [
     (dict(k=0), -1), (dict(k=9), -1), (dict(T_max=0), -1), (dict(H=0), -1), (dict(wfmt=7), -1),
     (dict(I_shared=-128), -1), (dict(E=2048, k=2), -2), (dict(k=33, E=64), -2), (dict(H=520), -2),
-    (dict(I=200), -2), (dict(I_shared=100), -2), (dict(wfmt=2, H=4100), -2),
+    (dict(I=200), -2), (dict(I_shared=100), -2), (dict(wfmt=2, H=4100), -2), (dict(wfmt=4), -1),
+    (dict(wfmt=3, H=4100), -2), (dict(wfmt=3, I=160), -2), (dict(wfmt=0), -1),
 ])
 def test_plan_rejects_bad_dims(lib, kw, code):
     assert _plan_rc(lib, **kw) == code
@@ -80,3 +81,8 @@ def test_binding_raises_without_library(tmp_path):
             moe.load_library(str(tmp_path / "missing.so"))
         finally:
             moe._lib = None
+
+
+def test_binding_rejects_unknown_weight_format():
+    with pytest.raises(ValueError):
+        moe.Plan(16, 512, 8, 256, 2, 0, "fp4")

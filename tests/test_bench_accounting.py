@@ -17,7 +17,7 @@ def _tensor_bytes(t):
     return t.numel() * t.element_size()
 
 
-@pytest.mark.parametrize("wfmt", ["fp8", "int4"])
+@pytest.mark.parametrize("wfmt", ["fp8", "int4", "mxfp4"])
 @pytest.mark.parametrize("Is", [0, 256])
 def test_gemm_bytes_are_the_touched_experts_tensors(wfmt, Is):
     cfg = dict(T=24, H=1024, E=8, I=384, k=2, Is=Is, seed=70, bias=None, wfmt=wfmt)

@@ -39,6 +39,8 @@ def _layer_parity(cfg):
     dict(T=64, H=256, E=1024, I=128, k=4, Is=128, seed=54, bias="zipf", wfmt="fp8"),  # the largest E
     dict(T=24, H=256, E=4, I=128, k=4, Is=0, seed=55, bias=None, wfmt="int4"),      # k = E, 4-bit
     dict(T=9, H=256, E=1, I=256, k=1, Is=128, seed=56, bias=None, wfmt="int4"),     # one 4-bit expert + shared
+    dict(T=24, H=256, E=4, I=128, k=4, Is=0, seed=59, bias=None, wfmt="mxfp4"),     # k = E, MXFP4
+    dict(T=9, H=128, E=1, I=256, k=1, Is=128, seed=60, bias=None, wfmt="mxfp4"),    # one MXFP4 expert + shared
 ], ids=lambda c: f"{c['wfmt']}-T{c['T']}-E{c['E']}-k{c['k']}-Is{c['Is']}")
 def test_degenerate_and_extreme_shapes(cfg):
     _layer_parity(cfg)
