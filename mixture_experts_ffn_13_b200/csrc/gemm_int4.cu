@@ -47,14 +47,19 @@ namespace {
 constexpr int kKE = 64;                // K elements per MMA stage (one 128-byte bf16 swizzle row)
 constexpr int kRawKE = 256;            // K elements per raw weight stage (128 bytes per row)
 constexpr int kSubs = kRawKE / kKE;    // MMA stages per raw stage
-constexpr int kConvWarps = 4;
 constexpr int kPrefetch = 8;           // raw stages prefetched into L2 ahead of the loads
 
-template <int BN, bool GATEUP>
+// Warp roles: 0 producer, 1 MMA issuer, CONV dequantisers, EW epilogue warps.  int4 keeps two
+// epilogue warps per TMEM lane quarter (each holds half the token columns' fp32 sums across
+// the scale groups); MXFP4 has no promotion, so one epilogue warp per quarter streams the
+// accumulator out, and the freed warps become a second dequantiser per quarter (each of the
+// pair converts one 32-element block of a 64-K stage).
+template <int BN, bool GATEUP, bool MX>
 struct I4Cfg {
-    static constexpr int EW = 8;                            // epilogue warps (2 per TMEM quarter)
+    static constexpr int CONV = MX ? 8 : 4;                 // dequantiser warps
+    static constexpr int EW = MX ? 4 : 8;                   // epilogue warps
     static constexpr int CPW = BN / (EW / 4);               // token columns per epilogue thread
-    static constexpr int THREADS = 32 * (2 + kConvWarps + EW);
+    static constexpr int THREADS = 32 * (2 + CONV + EW);
     static constexpr int NA = GATEUP ? 2 : 1;
     static constexpr int RAW_BYTES = kTileM * (kRawKE / 2);  // 16 KB per matrix
     static constexpr int B_BYTES = BN * kKE * 2;
@@ -74,6 +79,7 @@ struct I4Cfg {
     static constexpr int SMEM = 1024 + NB * B_BYTES + NR * NA * RAW_BYTES + TT_BYTES + BAR_BYTES;
     static_assert(B_BYTES % 1024 == 0, "1024-byte aligned tiles");
     static_assert(NSLOT >= 2, "TMEM slots");
+    static_assert(CONV % 4 == 0 && EW % 4 == 0, "whole TMEM lane quarters per role");
     static_assert(SMEM <= 227 * 1024, "shared memory");
     static_assert((NR * NA * RAW_BYTES + NB * B_BYTES + TT_BYTES) % 16 == 0, "mbarriers must be 8-byte aligned");
 };
@@ -135,10 +141,10 @@ __device__ __forceinline__ uint4 unpack8(uint32_t w)
 
 // MX = false: int4 weights with bf16 scales per 128-group; MX = true: MXFP4 weights.
 template <int BN, bool GATEUP, bool MX>
-__global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
+__global__ void __launch_bounds__(I4Cfg<BN, GATEUP, MX>::THREADS, 1)
     gemm_int4_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmArgs args)
 {
-    using C = I4Cfg<BN, GATEUP>;
+    using C = I4Cfg<BN, GATEUP, MX>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *raw = smem;                                   // NR raw stages [raw0 | raw1]
@@ -159,14 +165,14 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::NR; ++s) {
             mbar_init(&rfull[s], 1);
-            mbar_init(&rempty[s], kConvWarps);
+            mbar_init(&rempty[s], C::CONV);
         }
         for (int s = 0; s < C::NB; ++s) {
             mbar_init(&bfull[s], 1);
             mbar_init(&bempty[s], 1);
         }
         for (int s = 0; s < C::NM; ++s) {
-            mbar_init(&mfull[s], kConvWarps);
+            mbar_init(&mfull[s], C::CONV);
             mbar_init(&mempty[s], 1);
         }
         for (int s = 0; s < C::NSLOT; ++s) {
@@ -281,7 +287,7 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
                 }
             }
         }
-    } else if (warp < 2 + kConvWarps) {
+    } else if (warp < 2 + C::CONV) {
         // ------------------------------ dequantisers ------------------------------
         const int q = warp & 3;        // TMEM lane quarter reachable from this warp
         const int r = q * 32 + lane;   // weight row of the tile handled by this thread
@@ -331,37 +337,50 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
                 if (!__all_sync(0xffffffffu, ok)) goto done;
                 tc_fence_after();
                 const uint8_t *rs = raw + rs_i * C::NA * C::RAW_BYTES + r * 128;
-                // this sub-stage's 32 raw bytes are 16-byte chunks 2*sub and 2*sub+1 of the row,
-                // stored by the 128-byte swizzle at chunk positions (c ^ (r & 7))
-                const int c0 = ((2 * sub) ^ (r & 7)) << 4, c1 = ((2 * sub + 1) ^ (r & 7)) << 4;
                 const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + ms_i * C::NA * C::A_COLS;
+                if constexpr (MX) {
+                    // half hx of the stage: 16-byte chunk 2*sub + hx of the row (the 128-byte
+                    // swizzle stores chunk c at position c ^ (r & 7)) = 32-block 2*sub + hx of
+                    // the raw stage, written to TMEM columns 16*hx .. 16*hx + 15
+                    const int hx = (warp - 2) >> 2;
+                    const int cc = ((2 * sub + hx) ^ (r & 7)) << 4;
 #pragma unroll
-                for (int m = 0; m < C::NA; ++m) {
-                    const uint4 q0 = *reinterpret_cast<const uint4 *>(rs + m * C::RAW_BYTES + c0);
-                    const uint4 q1 = *reinterpret_cast<const uint4 *>(rs + m * C::RAW_BYTES + c1);
-                    const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-                    // MXFP4: chunk c0 is 32-block 2*sub of the raw stage, c1 block 2*sub + 1
-                    __nv_bfloat162 sca, scb;
-                    if constexpr (MX) {
+                    for (int m = 0; m < C::NA; ++m) {
+                        const uint4 qq = *reinterpret_cast<const uint4 *>(rs + m * C::RAW_BYTES + cc);
                         const uint32_t sw = (sub >> 1) ? scur[m][1] : scur[m][0];
-                        const uint32_t sh = (sub & 1) * 16;
-                        sca = e8m0_pair((sw >> sh) & 0xFFu);
-                        scb = e8m0_pair((sw >> (sh + 8)) & 0xFFu);
-                    }
-                    uint32_t v[32];
+                        const __nv_bfloat162 sc = e8m0_pair((sw >> ((sub & 1) * 16 + hx * 8)) & 0xFFu);
+                        const uint32_t words[4] = {qq.x, qq.y, qq.z, qq.w};
+                        uint32_t v[16];
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        uint4 u;
-                        if constexpr (MX)
-                            u = unpack8_fp4(words[j], j < 4 ? sca : scb);
-                        else
-                            u = unpack8(words[j]);
-                        v[4 * j] = u.x;
-                        v[4 * j + 1] = u.y;
-                        v[4 * j + 2] = u.z;
-                        v[4 * j + 3] = u.w;
+                        for (int j = 0; j < 4; ++j) {
+                            const uint4 u = unpack8_fp4(words[j], sc);
+                            v[4 * j] = u.x;
+                            v[4 * j + 1] = u.y;
+                            v[4 * j + 2] = u.z;
+                            v[4 * j + 3] = u.w;
+                        }
+                        tmem_st16(ta + m * C::A_COLS + 16 * hx, v);  // 32 bf16 = 16 packed columns
                     }
-                    tmem_st32(ta + m * C::A_COLS, v);  // row r: 64 bf16 = 32 packed columns
+                } else {
+                    // this sub-stage's 32 raw bytes are 16-byte chunks 2*sub and 2*sub+1 of the
+                    // row, stored by the 128-byte swizzle at chunk positions (c ^ (r & 7))
+                    const int c0 = ((2 * sub) ^ (r & 7)) << 4, c1 = ((2 * sub + 1) ^ (r & 7)) << 4;
+#pragma unroll
+                    for (int m = 0; m < C::NA; ++m) {
+                        const uint4 q0 = *reinterpret_cast<const uint4 *>(rs + m * C::RAW_BYTES + c0);
+                        const uint4 q1 = *reinterpret_cast<const uint4 *>(rs + m * C::RAW_BYTES + c1);
+                        const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+                        uint32_t v[32];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const uint4 u = unpack8(words[j]);
+                            v[4 * j] = u.x;
+                            v[4 * j + 1] = u.y;
+                            v[4 * j + 2] = u.z;
+                            v[4 * j + 3] = u.w;
+                        }
+                        tmem_st32(ta + m * C::A_COLS, v);  // row r: 64 bf16 = 32 packed columns
+                    }
                 }
                 tmem_wait_st();
                 tc_fence_before();
@@ -377,12 +396,46 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP>::THREADS, 1)
     } else {
         // ------------------------------ epilogue ----------------------------------
         const int q = warp & 3;                                   // TMEM lane quarter
-        const int cbase = ((warp - 2 - kConvWarps) >> 2) * C::CPW;  // first token column
+        const int cbase = ((warp - 2 - C::CONV) >> 2) * C::CPW;  // first token column
         const int r = q * 32 + lane;
         uint32_t ai = 0;
         for (int w = blockIdx.x; w < total; w += gridDim.x) {
             const TileInfo tl = decode_tile<BN, true>(args, stt, w, tot0);
             const GemmSeg &sg = args.seg[tl.seg];
+            if constexpr (MX) {
+                // MXFP4: the tile's whole K sits in one slot; stream it out 16 columns at a time
+                const int slot = ai % C::NSLOT;
+                const bool ok = mbar_wait(&accf[slot], (ai / C::NSLOT) & 1, abort_flag, status, tmo);
+                if (!__all_sync(0xffffffffu, ok)) goto done;
+                tc_fence_after();
+                const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + C::A_TMEM + slot * C::SLOT_COLS;
+                const int n = tl.nt * kTileM + r;
+                for (int c0 = 0; c0 < BN && c0 < tl.nrows; c0 += 16) {  // warp-uniform bounds
+                    float v[16], u[16];
+                    tmem_ld16(tb + c0, v);
+                    if constexpr (GATEUP) {
+                        tmem_ld16(tb + BN + c0, u);
+                        tmem_wait_ld2(v, u);
+                    } else {
+                        tmem_wait_ld(v);
+                    }
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        if (c0 + c < tl.nrows) {
+                            const size_t o = (size_t)(tl.row0 + c0 + c) * sg.N + n;
+                            if constexpr (GATEUP)
+                                static_cast<__nv_bfloat16 *>(sg.out)[o] = __float2bfloat16_rn(silu_mul(v[c], u[c]));
+                            else
+                                static_cast<float *>(sg.out)[o] = v[c];
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acce[slot]);
+                ++ai;
+                continue;
+            }
             // MXFP4: the weights arrive scaled and the whole K sits in one slot (scale 1)
             const int ngrp = MX ? 1 : sg.K / kGroupK;
             const __nv_bfloat16 *sw0 =
@@ -460,7 +513,7 @@ done:
 template <int BN, bool GATEUP, bool MX>
 cudaError_t launch_t(const GemmMaps &maps, const GemmArgs &args, int num_sms, cudaStream_t s)
 {
-    using C = I4Cfg<BN, GATEUP>;
+    using C = I4Cfg<BN, GATEUP, MX>;
     auto kern = gemm_int4_kernel<BN, GATEUP, MX>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
