@@ -33,7 +33,9 @@
 // pipeline with one change in the dequantisers and one in the MMA/epilogue split: an E2M1
 // value (at most two significant bits) times its block's power-of-two E8M0 scale is exact in
 // bf16, so the dequantisers write the scaled weights themselves, the whole K accumulates in
-// one TMEM slot, and the epilogue has no promotion to do.
+// one TMEM slot, and the epilogue has no promotion to do.  The warp roles shift with that:
+// warps 2-9 dequantise (two per TMEM lane quarter, one 32-element block of each 64-K stage
+// apiece) and warps 10-13 (one per quarter) stream each finished tile out.
 #include "gemm_common.cuh"
 #include "launch.cuh"
 #include "sm100.cuh"
