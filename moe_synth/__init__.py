@@ -114,11 +114,12 @@ def _quant_mxfp4(w: torch.Tensor):
     """W [..., N, K] fp32 -> (packed uint8 [..., N, K/2], E8M0 scales uint8 [..., N, K/32])."""
     K = w.shape[-1]
     assert K % 32 == 0
-    blk = w.reshape(*w.shape[:-1], K // 32, 32).double()
+    blk = w.reshape(*w.shape[:-1], K // 32, 32).float()
     amax = blk.abs().amax(dim=-1)
     _, e = torch.frexp(amax)  # amax = m * 2^e, m in [0.5, 1): floor(log2(amax)) = e - 1
     xexp = torch.where(amax == 0, torch.zeros_like(e), e - 1 - 2).clamp(-127, 127)
-    v = blk / torch.pow(2.0, xexp.double()).unsqueeze(-1)  # exact: a power of two
+    # dividing by a power of two and the rounding steps below are exact in fp32
+    v = blk / torch.pow(2.0, xexp.float()).unsqueeze(-1)
     a = v.abs()
     step = torch.where(a < 2, 0.5, torch.where(a < 4, 1.0, 2.0))
     q2 = (torch.round(a / step) * step).clamp(max=6.0) * 2  # 2|q| in {0, 1, 2, 3, 4, 6, 8, 12}
