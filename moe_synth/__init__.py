@@ -22,7 +22,11 @@ Recipe (every tensor has its own seeded torch generator on the chosen device):
              x = floor(log2(amax)) - 2 (the largest E2M1 power of two is 2^2; 0 when
              amax = 0), stored as x + 127; each element is W / 2^x rounded to the nearest
              E2M1 value (ties to the even code, magnitudes above 6 saturate to 6), the
-             even K index in the low nibble.
+             even K index in the low nibble;
+      - NVFP4: one fp32 tensor scale per expert matrix, t = amax / (448 * 6) (1 when 0);
+             one E4M3 byte per (row, 16-element K block), s = e4m3(amax_block / (6 t))
+             (torch's cast, round to nearest even, at least 2^-9; 1 for an all-zero block);
+             each element is W / (s t) rounded to the nearest E2M1 value as for MXFP4.
 Shapes follow the pages' models: a Qwen3.5-397B-shaped layer (512 experts x 1024, top-10,
 one shared expert of 1024, hidden 4096) at decode and prefill sizes; a DeepSeek-R1-shaped
 layer (hidden 7168, 256 experts x 2048, top-8, shared 2048) with skewed routing; a 4-bit
@@ -52,6 +56,9 @@ CONFIGS = {
                  workload="4-bit-weight MoE T=1024 H=4096 E=128 I=1536 top-8, int4 g128 bf16"),
     "mxfp4": dict(T=1024, H=4096, E=128, I=1536, k=8, Is=0, wfmt="mxfp4", seed=8, bias=None,
                   workload="MXFP4-weight MoE T=1024 H=4096 E=128 I=1536 top-8, e2m1 + E8M0/32, bf16"),
+    "nvfp4": dict(T=1024, H=4096, E=128, I=1536, k=8, Is=0, wfmt="nvfp4", seed=10, bias=None,
+                  workload="NVFP4-weight MoE T=1024 H=4096 E=128 I=1536 top-8, e2m1 + E4M3/16 + fp32 "
+                           "tensor scale, bf16"),
 }
 
 # Smaller layers with the same per-expert shapes, for profiler captures (weights still far
@@ -65,6 +72,8 @@ PROFILE_CONFIGS = {
                          workload="4-bit MoE T=128 H=4096 E=16 I=1536 top-8, int4 g128"),
     "profile-mxfp4": dict(T=128, H=4096, E=16, I=1536, k=8, Is=0, wfmt="mxfp4", seed=9, bias=None,
                           workload="MXFP4 MoE T=128 H=4096 E=16 I=1536 top-8, e2m1 + E8M0/32"),
+    "profile-nvfp4": dict(T=128, H=4096, E=16, I=1536, k=8, Is=0, wfmt="nvfp4", seed=11, bias=None,
+                          workload="NVFP4 MoE T=128 H=4096 E=16 I=1536 top-8, e2m1 + E4M3/16 + tensor scale"),
 }
 
 # tensor ids for the per-tensor generators
@@ -110,6 +119,20 @@ def _quant_int4(w: torch.Tensor):
 _E2M1_CODE_OF_2V = {0: 0, 1: 1, 2: 2, 3: 3, 4: 4, 6: 5, 8: 6, 12: 7}
 
 
+def _e2m1_packed(v: torch.Tensor, shape):
+    """Values v (already divided by their scales) -> nearest E2M1 nibbles (ties to the even
+    code, magnitudes above 6 saturate), packed two per byte with the even K index low."""
+    a = v.abs()
+    step = torch.where(a < 2, 0.5, torch.where(a < 4, 1.0, 2.0))
+    q2 = (torch.round(a / step) * step).clamp(max=6.0) * 2  # 2|q| in {0, 1, 2, 3, 4, 6, 8, 12}
+    lut = torch.zeros(13, dtype=torch.int16, device=v.device)
+    for k2, c in _E2M1_CODE_OF_2V.items():
+        lut[k2] = c
+    mag = lut[q2.long()]
+    nib = torch.where((v < 0) & (mag > 0), mag | 8, mag).reshape(shape)
+    return (nib[..., 0::2] | (nib[..., 1::2] << 4)).to(torch.uint8).contiguous()
+
+
 def _quant_mxfp4(w: torch.Tensor):
     """W [..., N, K] fp32 -> (packed uint8 [..., N, K/2], E8M0 scales uint8 [..., N, K/32])."""
     K = w.shape[-1]
@@ -118,21 +141,29 @@ def _quant_mxfp4(w: torch.Tensor):
     amax = blk.abs().amax(dim=-1)
     _, e = torch.frexp(amax)  # amax = m * 2^e, m in [0.5, 1): floor(log2(amax)) = e - 1
     xexp = torch.where(amax == 0, torch.zeros_like(e), e - 1 - 2).clamp(-127, 127)
-    # dividing by a power of two and the rounding steps below are exact in fp32
+    # dividing by a power of two and the rounding steps are exact in fp32
     v = blk / torch.pow(2.0, xexp.float()).unsqueeze(-1)
-    a = v.abs()
-    step = torch.where(a < 2, 0.5, torch.where(a < 4, 1.0, 2.0))
-    q2 = (torch.round(a / step) * step).clamp(max=6.0) * 2  # 2|q| in {0, 1, 2, 3, 4, 6, 8, 12}
-    lut = torch.zeros(13, dtype=torch.int16, device=w.device)
-    for k2, c in _E2M1_CODE_OF_2V.items():
-        lut[k2] = c
-    mag = lut[q2.long()]
-    nib = torch.where((v < 0) & (mag > 0), mag | 8, mag).reshape(*w.shape[:-1], K)
-    packed = (nib[..., 0::2] | (nib[..., 1::2] << 4)).to(torch.uint8)
-    return packed.contiguous(), (xexp + 127).to(torch.uint8).contiguous()
+    return _e2m1_packed(v, w.shape), (xexp + 127).to(torch.uint8).contiguous()
 
 
-_QUANT = {"fp8": _quant_fp8, "int4": _quant_int4, "mxfp4": _quant_mxfp4}
+def _quant_nvfp4(w: torch.Tensor):
+    """W [E, N, K] fp32 -> (packed uint8 [E, N, K/2], E4M3 scales uint8 [E, N, K/16],
+    tensor scales fp32 [E])."""
+    E, N, K = w.shape
+    assert K % 16 == 0
+    amax_t = w.abs().reshape(E, -1).amax(dim=1)
+    t = torch.where(amax_t == 0, torch.ones_like(amax_t), amax_t / (448.0 * 6.0))
+    blk = w.reshape(E, N, K // 16, 16).float()
+    amax = blk.abs().amax(dim=-1)
+    target = (amax / (6.0 * t.view(E, 1, 1))).clamp(min=2.0 ** -9, max=448.0)
+    s = target.to(torch.float8_e4m3fn).float()
+    s = torch.where(amax == 0, torch.ones_like(s), s)
+    v = blk / (s * t.view(E, 1, 1)).unsqueeze(-1)
+    codes = s.to(torch.float8_e4m3fn).view(torch.uint8).contiguous()
+    return _e2m1_packed(v, w.shape), codes, t.contiguous()
+
+
+_QUANT = {"fp8": _quant_fp8, "int4": _quant_int4, "mxfp4": _quant_mxfp4, "nvfp4": _quant_nvfp4}
 
 
 def _weights(seed, tid, shape, fan_in, wfmt, device, chunk_elems=1 << 28):
@@ -140,16 +171,15 @@ def _weights(seed, tid, shape, fan_in, wfmt, device, chunk_elems=1 << 28):
     E, N, K = shape
     g = _gen(seed, tid, device)
     per = max(1, chunk_elems // (N * K))
-    qs, ss = [], []
+    parts = []
     for e0 in range(0, E, per):
         e1 = min(E, e0 + per)
         w = torch.randn((e1 - e0, N, K), generator=g, device=device, dtype=torch.float32)
         w.mul_(1.0 / math.sqrt(fan_in))
-        q, s = _QUANT[wfmt](w)
-        qs.append(q)
-        ss.append(s)
+        parts.append(_QUANT[wfmt](w))
         del w
-    return torch.cat(qs, 0), torch.cat(ss, 0)
+    # (codes, scales) or, for NVFP4, (codes, scales, tensor scales)
+    return tuple(torch.cat([p[i] for p in parts], 0) for i in range(len(parts[0])))
 
 
 def make_layer(name_or_cfg, device="cpu", **overrides) -> dict:
@@ -172,13 +202,14 @@ def make_layer(name_or_cfg, device="cpu", **overrides) -> dict:
         rank = torch.randperm(E, generator=_gen(seed, _TID["rank"], device), device=device) + 1
         logits = logits + (-1.2) * torch.log(rank.to(torch.float32))
     out["logits"] = logits.contiguous()
-    out["w_gate"], out["s_gate"] = _weights(seed, _TID["w_gate"], (E, I, H), H, wfmt, device)
-    out["w_up"], out["s_up"] = _weights(seed, _TID["w_up"], (E, I, H), H, wfmt, device)
-    out["w_down"], out["s_down"] = _weights(seed, _TID["w_down"], (E, H, I), I, wfmt, device)
+    mats = [("gate", (E, I, H), H, ""), ("up", (E, I, H), H, ""), ("down", (E, H, I), I, "")]
     if Is > 0:
-        out["ws_gate"], out["ss_gate"] = _weights(seed, _TID["ws_gate"], (1, Is, H), H, wfmt, device)
-        out["ws_up"], out["ss_up"] = _weights(seed, _TID["ws_up"], (1, Is, H), H, wfmt, device)
-        out["ws_down"], out["ss_down"] = _weights(seed, _TID["ws_down"], (1, H, Is), Is, wfmt, device)
+        mats += [("gate", (1, Is, H), H, "s"), ("up", (1, Is, H), H, "s"), ("down", (1, H, Is), Is, "s")]
+    for proj, shape, fan_in, sh in mats:
+        res = _weights(seed, _TID[f"w{sh}_{proj}"], shape, fan_in, wfmt, device)
+        out[f"w{sh}_{proj}"], out[f"s{sh}_{proj}"] = res[0], res[1]
+        if len(res) > 2:
+            out[f"t{sh}_{proj}"] = res[2]
     return out
 
 
@@ -211,4 +242,4 @@ def to_numpy(layer: dict) -> dict:
 
 def weight_bytes(layer: dict) -> int:
     return sum(v.numel() * v.element_size() for key, v in layer.items()
-               if isinstance(v, torch.Tensor) and key[:2] in ("w_", "s_", "ws", "ss"))
+               if isinstance(v, torch.Tensor) and key[:2] in ("w_", "s_", "ws", "ss", "t_", "ts"))

@@ -25,7 +25,8 @@ _lib = None
 FP8_SC512 = 1
 INT4_G128 = 2
 MXFP4_G32 = 3
-_WFMT = {"fp8": FP8_SC512, "int4": INT4_G128, "mxfp4": MXFP4_G32}
+NVFP4_G16 = 4
+_WFMT = {"fp8": FP8_SC512, "int4": INT4_G128, "mxfp4": MXFP4_G32, "nvfp4": NVFP4_G16}
 
 
 class Dims(ctypes.Structure):
@@ -35,7 +36,8 @@ class Dims(ctypes.Structure):
 class Weights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "w_gate", "w_up", "w_down", "s_gate", "s_up", "s_down",
-        "ws_gate", "ws_up", "ws_down", "ss_gate", "ss_up", "ss_down")]
+        "ws_gate", "ws_up", "ws_down", "ss_gate", "ss_up", "ss_down",
+        "t_gate", "t_up", "t_down", "ts_gate", "ts_up", "ts_down")]
 
 
 def build(force: bool = False) -> str:
@@ -73,7 +75,7 @@ def lib():
             L.orc_quant_rows_bf16.argtypes = [I, I, P, P, P]
             L.orc_expert_fp8_row.argtypes = [I, I] + [P] * 10
             L.orc_expert_int4_row.argtypes = [I, I] + [P] * 9
-            L.orc_expert_w4_row.argtypes = [I, I, I] + [P] * 9
+            L.orc_expert_w4_row.argtypes = [I, I, I] + [P] * 10
             L.orc_layer.argtypes = [ctypes.POINTER(Dims), ctypes.POINTER(Weights), P, P, I, P, P, P, P, I]
             _lib = L
     return _lib
@@ -221,8 +223,9 @@ def expert_mxfp4_row(x_bits, wg, sg, wu, su, wd, sd):
     H = x_bits.shape[0]
     y = np.empty(H, np.float64)
     h = np.empty(I, np.float64)
+    ones = np.ones(3)
     lib().orc_expert_w4_row(MXFP4_G32, H, I, _p(x_bits), _p(wg), _p(sg), _p(wu), _p(su), _p(wd),
-                            _p(sd), _p(y), _p(h))
+                            _p(sd), _p(ones), _p(y), _p(h))
     return y, h
 
 
@@ -250,11 +253,13 @@ def layer(layer_np: dict, tokens=None, nthreads: int | None = None, ambiguity: b
         keep[name] = a
         return _p(a)
 
-    sdt = {FP8_SC512: np.float32, INT4_G128: np.uint16, MXFP4_G32: np.uint8}[wfmt]
+    sdt = {FP8_SC512: np.float32, INT4_G128: np.uint16, MXFP4_G32: np.uint8, NVFP4_G16: np.uint8}[wfmt]
     W = Weights(arr("w_gate", np.uint8), arr("w_up", np.uint8), arr("w_down", np.uint8),
                 arr("s_gate", sdt), arr("s_up", sdt), arr("s_down", sdt),
                 arr("ws_gate", np.uint8), arr("ws_up", np.uint8), arr("ws_down", np.uint8),
-                arr("ss_gate", sdt), arr("ss_up", sdt), arr("ss_down", sdt))
+                arr("ss_gate", sdt), arr("ss_up", sdt), arr("ss_down", sdt),
+                arr("t_gate", np.float32), arr("t_up", np.float32), arr("t_down", np.float32),
+                arr("ts_gate", np.float32), arr("ts_up", np.float32), arr("ts_down", np.float32))
     x = _c(layer_np["x"], np.uint16)
     logits = _c(layer_np["logits"], np.float32)
     if tokens is None:

@@ -18,6 +18,8 @@
  *  [P2] "TPU推理外部化全面加速：InferenceX首份第三方性能數據發布" -- section "优化 MoE 路由与
  *       专家内核": tokens are gathered into contiguous per-expert groups; the sort key packs
  *       (expert id, token index); the combine is an un-permute weighted by the top-k weights.
+ *  [P3] the NVIDIA model/hardware co-design commentary -- section "讀的時候記得這是廠商文":
+ *       NVFP4 keeps two levels of scale factors.
  *  [P4] "设计 AI 芯片的硬件与软件" -- section "数值格式，或如何制造便宜的脉动阵列": FP8 means the
  *       E4M3 and E5M2 formats; products are accumulated at higher precision.
  *  [P5] "Flash-Next 在 GPU 上到底在算什麼" -- section "① 專家 FFN": each expert computes
@@ -48,6 +50,11 @@
  *         has one E8M0 byte c, the scale 2^(c-127) (c = 255 is NaN).  The weight is
  *         e2m1 * 2^(c-127); activations and h stay bf16 as in R11 (the same page calls
  *         4-bit activations far harder than 4-bit weights).
+ *  R21    NVFP4 weights ([P3] section "讀的時候記得這是廠商文": NVFP4 reaches near-8-bit accuracy
+ *         at 4-bit speed through two levels of scale factors): E2M1 nibbles as in R20; one
+ *         E4M3 byte (R13) per (row, 16-element K block); one fp32 tensor scale per weight
+ *         matrix (per expert and projection).  The weight is e2m1 * e4m3(s) * t; activations
+ *         and h stay bf16.
  *
  * Every sum below is written out in the order the definition states; nothing is blocked,
  * fused or reordered beyond it.  Build: gcc -O2 -fno-fast-math -ffp-contract=off.
@@ -61,21 +68,26 @@
 #define ORC_FP8_SC512 1
 #define ORC_INT4_G128 2
 #define ORC_MXFP4_G32 3
+#define ORC_NVFP4_G16 4
 
 typedef struct {
     int T, H, E, I, k, Is; /* Is = 0: no shared expert */
-    int wfmt;              /* ORC_FP8_SC512, ORC_INT4_G128 or ORC_MXFP4_G32 */
+    int wfmt;              /* ORC_FP8_SC512, ORC_INT4_G128, ORC_MXFP4_G32 or ORC_NVFP4_G16 */
 } orc_dims;
 
 typedef struct {
     /* FP8: codes [E,I,H], [E,I,H], [E,H,I]; scales fp32 [E,I,nb(H)], [E,I,nb(H)], [E,H,nb(I)]
      * int4: packed bytes [E,I,H/2], [E,I,H/2], [E,H,I/2]; scales bf16 [E,I,H/128] ...
-     * MXFP4: packed bytes as int4; scales E8M0 bytes [E,I,H/32], [E,I,H/32], [E,H,I/32] */
+     * MXFP4: packed bytes as int4; scales E8M0 bytes [E,I,H/32], [E,I,H/32], [E,H,I/32]
+     * NVFP4: packed bytes as int4; scales E4M3 bytes [E,I,H/16], [E,I,H/16], [E,H,I/16] */
     const uint8_t *w_gate, *w_up, *w_down;
     const void *s_gate, *s_up, *s_down;
     /* shared expert, same formats with E = 1 and I -> Is (NULL when Is == 0) */
     const uint8_t *ws_gate, *ws_up, *ws_down;
     const void *ss_gate, *ss_up, *ss_down;
+    /* NVFP4 tensor scales: fp32 [E] per projection, [1] for the shared expert (else NULL) */
+    const float *t_gate, *t_up, *t_down;
+    const float *ts_gate, *ts_up, *ts_down;
 } orc_weights;
 
 /* ------------------------------------------------------------------------------------ */
@@ -465,10 +477,15 @@ static int orc_nib_raw(const uint8_t *packed_row, int i)
     return (i & 1) ? (b >> 4) : (b & 0xF);
 }
 
-/* Weight [n, i] of a 4-bit [N, K] matrix: int4 q * s (R14) or e2m1 * 2^(c-127) (R20). */
+/* Weight [n, i] of a 4-bit [N, K] matrix without its tensor scale: int4 q * s (R14),
+ * e2m1 * 2^(c-127) (R20) or e2m1 * e4m3(s) (R21). */
 static double orc_w4(int wfmt, int K, const uint8_t *qw, const void *sw, int n, int i)
 {
     const uint8_t *row = qw + (size_t)n * (K / 2);
+    if (wfmt == ORC_NVFP4_G16) {
+        const uint8_t *sc = (const uint8_t *)sw;
+        return orc_e2m1_tab[orc_nib_raw(row, i)] * orc_dec_tab[sc[(size_t)n * (K / 16) + i / 16]];
+    }
     if (wfmt == ORC_MXFP4_G32) {
         const uint8_t *sc = (const uint8_t *)sw;
         return orc_e2m1_tab[orc_nib_raw(row, i)] * orc_e8m0_tab[sc[(size_t)n * (K / 32) + i / 32]];
@@ -480,17 +497,19 @@ static double orc_w4(int wfmt, int K, const uint8_t *qw, const void *sw, int n, 
 /* The scale array of expert e of a 4-bit [E, N, K] weight set. */
 static const void *orc_w4_scales(int wfmt, const void *sw, size_t e, int N, int K)
 {
+    if (wfmt == ORC_NVFP4_G16) return (const uint8_t *)sw + e * (size_t)N * (size_t)(K / 16);
     if (wfmt == ORC_MXFP4_G32) return (const uint8_t *)sw + e * (size_t)N * (size_t)(K / 32);
     return (const uint16_t *)sw + e * (size_t)N * (size_t)(K / 128);
 }
 
-/* y[n] = sum_i a[i] * W[n, i]  with a in fp64 (bf16 values, exact). */
+/* y[n] = sum_i a[i] * (W[n, i] * t)  with a in fp64 (bf16 values, exact); t is the matrix's
+ * tensor scale (1 except for NVFP4).  Every product is exact in fp64. */
 static void orc_proj_w4(int wfmt, int N, int K, const double *a, const uint8_t *qw, const void *sw,
-                        double *y)
+                        double t, double *y)
 {
     for (int n = 0; n < N; ++n) {
         double acc = 0.0;
-        for (int i = 0; i < K; ++i) acc += a[i] * orc_w4(wfmt, K, qw, sw, n, i);
+        for (int i = 0; i < K; ++i) acc += a[i] * (orc_w4(wfmt, K, qw, sw, n, i) * t);
         y[n] = acc;
     }
 }
@@ -498,7 +517,7 @@ static void orc_proj_w4(int wfmt, int N, int K, const double *a, const uint8_t *
 /* R10a for 4-bit layers: h is rounded to bf16, so an h within ORC_AMBIG_REL of a bf16
  * rounding midpoint may round either way; env[n] gets |h_alt - h| * |W[n, i]| for each such i. */
 static void orc_h_ambiguity_bf16(int wfmt, int H, int I, const double *hx, const uint8_t *wd,
-                                 const void *sd, double *env)
+                                 const void *sd, double td, double *env)
 {
     for (int i = 0; i < I; ++i) {
         double a = fabs(hx[i]);
@@ -509,29 +528,30 @@ static void orc_h_ambiguity_bf16(int wfmt, int H, int I, const double *hx, const
         double quantum = ldexp(1.0, lead - 7);
         double frac = a / quantum - floor(a / quantum); /* position between two bf16 values */
         if (fabs(frac - 0.5) * quantum > ORC_AMBIG_REL * a) continue;
-        for (int n = 0; n < H; ++n) env[n] += quantum * fabs(orc_w4(wfmt, I, wd, sd, n, i));
+        for (int n = 0; n < H; ++n) env[n] += quantum * fabs(orc_w4(wfmt, I, wd, sd, n, i) * td);
     }
 }
 
+/* tg, tu, td: the three matrices' tensor scales (1 except for NVFP4). */
 static void orc_expert_w4(int wfmt, int H, int I, const double *x, const uint8_t *wg, const void *sg,
-                          const uint8_t *wu, const void *su, const uint8_t *wd, const void *sd,
-                          double *y, double *h_out, double *env)
+                          double tg, const uint8_t *wu, const void *su, double tu, const uint8_t *wd,
+                          const void *sd, double td, double *y, double *h_out, double *env)
 {
     double *G = (double *)malloc(sizeof(double) * (size_t)I);
     double *U = (double *)malloc(sizeof(double) * (size_t)I);
     double *hx = (double *)malloc(sizeof(double) * (size_t)I);
     double *h = (double *)malloc(sizeof(double) * (size_t)I);
-    orc_proj_w4(wfmt, I, H, x, wg, sg, G);
-    orc_proj_w4(wfmt, I, H, x, wu, su, U);
+    orc_proj_w4(wfmt, I, H, x, wg, sg, tg, G);
+    orc_proj_w4(wfmt, I, H, x, wu, su, tu, U);
     for (int n = 0; n < I; ++n) {
         hx[n] = orc_silu(G[n]) * U[n];
         h[n] = orc_bf16_to_double(orc_double_to_bf16(hx[n]));
     }
     if (h_out) memcpy(h_out, h, sizeof(double) * (size_t)I);
-    orc_proj_w4(wfmt, H, I, h, wd, sd, y);
+    orc_proj_w4(wfmt, H, I, h, wd, sd, td, y);
     if (env) {
         for (int n = 0; n < H; ++n) env[n] = 0.0;
-        orc_h_ambiguity_bf16(wfmt, H, I, hx, wd, sd, env);
+        orc_h_ambiguity_bf16(wfmt, H, I, hx, wd, sd, td, env);
     }
     free(G);
     free(U);
@@ -604,18 +624,22 @@ static void orc_layer_token(const orc_dims *d, const orc_weights *w, const uint1
         double *xd = (double *)malloc(sizeof(double) * (size_t)H);
         for (int i = 0; i < H; ++i) xd[i] = orc_bf16_to_double(xrow[i]);
         const int f = d->wfmt;
+        const int nv = f == ORC_NVFP4_G16;
         for (int j = 0; j < k; ++j) {
             size_t e = (size_t)idx[j];
             orc_expert_w4(f, H, I, xd, w->w_gate + e * I * (H / 2), orc_w4_scales(f, w->s_gate, e, I, H),
-                          w->w_up + e * I * (H / 2), orc_w4_scales(f, w->s_up, e, I, H),
-                          w->w_down + e * H * (I / 2), orc_w4_scales(f, w->s_down, e, H, I), y, NULL, env);
+                          nv ? (double)w->t_gate[e] : 1.0, w->w_up + e * I * (H / 2),
+                          orc_w4_scales(f, w->s_up, e, I, H), nv ? (double)w->t_up[e] : 1.0,
+                          w->w_down + e * H * (I / 2), orc_w4_scales(f, w->s_down, e, H, I),
+                          nv ? (double)w->t_down[e] : 1.0, y, NULL, env);
             for (int n = 0; n < H; ++n) out[n] += p[j] * y[n];
             if (amb)
                 for (int n = 0; n < H; ++n) amb[n] += p[j] * env[n];
         }
         if (Is > 0) {
-            orc_expert_w4(f, H, Is, xd, w->ws_gate, w->ss_gate, w->ws_up, w->ss_up, w->ws_down,
-                          w->ss_down, y, NULL, env);
+            orc_expert_w4(f, H, Is, xd, w->ws_gate, w->ss_gate, nv ? (double)w->ts_gate[0] : 1.0, w->ws_up,
+                          w->ss_up, nv ? (double)w->ts_up[0] : 1.0, w->ws_down, w->ss_down,
+                          nv ? (double)w->ts_down[0] : 1.0, y, NULL, env);
             for (int n = 0; n < H; ++n) out[n] += y[n];
             if (amb)
                 for (int n = 0; n < H; ++n) amb[n] += env[n];
@@ -657,7 +681,10 @@ int orc_layer(const orc_dims *d, const orc_weights *w, const uint16_t *x, const 
               int nthreads)
 {
     if (d->E < 1 || d->k < 1 || d->k > d->E || d->H < 1 || d->I < 1 || d->Is < 0) return -1;
-    if (d->wfmt != ORC_FP8_SC512 && d->wfmt != ORC_INT4_G128 && d->wfmt != ORC_MXFP4_G32) return -1;
+    if (d->wfmt < ORC_FP8_SC512 || d->wfmt > ORC_NVFP4_G16) return -1;
+    if (d->wfmt == ORC_NVFP4_G16 &&
+        (!w->t_gate || !w->t_up || !w->t_down || (d->Is > 0 && (!w->ts_gate || !w->ts_up || !w->ts_down))))
+        return -1;
     if (d->wfmt != ORC_FP8_SC512 && (d->H % 128 || d->I % 128 || d->Is % 128)) return -1;
     for (int i = 0; i < n_sel; ++i)
         if (sel[i] < 0 || sel[i] >= d->T) return -1;
@@ -709,16 +736,16 @@ void orc_expert_fp8_row(int H, int I, const uint8_t *qx, const float *sx, const 
     orc_expert_fp8(H, I, qx, sx, wg, sg, wu, su, wd, sd, y, h, NULL);
 }
 
-/* One 4-bit expert (int4 or MXFP4) on one bf16 row: y (H values) and h (I values,
- * bf16-rounded). */
+/* One 4-bit expert (int4, MXFP4 or NVFP4; t = the tensor scales, 1 unless NVFP4) on one bf16
+ * row: y (H values) and h (I values, bf16-rounded). */
 void orc_expert_w4_row(int wfmt, int H, int I, const uint16_t *x, const uint8_t *wg, const void *sg,
-                       const uint8_t *wu, const void *su, const uint8_t *wd, const void *sd, double *y,
-                       double *h)
+                       const uint8_t *wu, const void *su, const uint8_t *wd, const void *sd, const double *t,
+                       double *y, double *h)
 {
     pthread_once(&orc_tab_once, orc_tab_init);
     double *xd = (double *)malloc(sizeof(double) * (size_t)H);
     for (int i = 0; i < H; ++i) xd[i] = orc_bf16_to_double(x[i]);
-    orc_expert_w4(wfmt, H, I, xd, wg, sg, wu, su, wd, sd, y, h, NULL);
+    orc_expert_w4(wfmt, H, I, xd, wg, sg, t[0], wu, su, t[1], wd, sd, t[2], y, h, NULL);
     free(xd);
 }
 
@@ -727,5 +754,6 @@ void orc_expert_int4_row(int H, int I, const uint16_t *x, const uint8_t *wg, con
                          const uint8_t *wu, const uint16_t *su, const uint8_t *wd,
                          const uint16_t *sd, double *y, double *h)
 {
-    orc_expert_w4_row(ORC_INT4_G128, H, I, x, wg, sg, wu, su, wd, sd, y, h);
+    const double ones[3] = {1.0, 1.0, 1.0};
+    orc_expert_w4_row(ORC_INT4_G128, H, I, x, wg, sg, wu, su, wd, sd, ones, y, h);
 }
