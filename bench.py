@@ -179,10 +179,12 @@ def algorithmic(cfg, counts):
         gu = touched * 2 * (I * H + I * nbH * 4) + (2 * (Is * H + Is * nbH * 4) if Is else 0)
         dn = touched * (H * I + H * nbI * 4) + ((H * Is + H * nbIs * 4) if Is else 0)
     else:
-        # 4-bit weights: packed nibbles plus the scales (int4: bf16 per 128; MXFP4: one byte per 32)
-        sb = (lambda K: (K // 128) * 2) if cfg["wfmt"] == "int4" else (lambda K: K // 32)
-        gu = touched * 2 * (I * H // 2 + I * sb(H)) + (2 * (Is * H // 2 + Is * sb(H)) if Is else 0)
-        dn = touched * (H * I // 2 + H * sb(I)) + ((H * Is // 2 + H * sb(Is)) if Is else 0)
+        # 4-bit weights: packed nibbles plus the scales (int4: bf16 per 128; MXFP4: one byte per
+        # 32; NVFP4: one byte per 16 and an fp32 tensor scale per matrix)
+        sb = {"int4": lambda K: (K // 128) * 2, "mxfp4": lambda K: K // 32, "nvfp4": lambda K: K // 16}[cfg["wfmt"]]
+        ts = 4 if cfg["wfmt"] == "nvfp4" else 0
+        gu = touched * 2 * (I * H // 2 + I * sb(H) + ts) + (2 * (Is * H // 2 + Is * sb(H) + ts) if Is else 0)
+        dn = touched * (H * I // 2 + H * sb(I) + ts) + ((H * Is // 2 + H * sb(Is) + ts) if Is else 0)
     act = T * H * 2 + T * H * 2 + T * cfg["E"] * 4  # x in, out, logits
     f_gu = 2 * 2 * H * I * T * k + (2 * 2 * H * Is * T if Is else 0)
     f_dn = 2 * H * I * T * k + (2 * H * Is * T if Is else 0)

@@ -28,6 +28,11 @@
  *     e2m1 * 2^(c-127) is formed exactly for c in 2..252 (other codes are outside the
  *     supported domain: the product may flush to zero or overflow).  Activations stay bf16
  *     (h is rounded to bf16), as for int4.
+ *   MOE_W_NVFP4_G16: NVFP4 (the NVIDIA co-design commentary, section "讀的時候記得這是廠商文":
+ *     two levels of scale factors).  E2M1 nibbles as for MXFP4; one E4M3 byte per (row,
+ *     16-element K block), a positive finite value; one fp32 tensor scale per weight matrix
+ *     (per expert and projection).  The weight is e2m1 * e4m3(s) * t: the first product is
+ *     formed exactly in bf16, t multiplies the fp32 accumulator.  Activations stay bf16.
  *
  * Pointer conventions.  Every buffer passed to moe_router_logits / moe_route / moe_forward is
  * DEVICE memory that the caller allocates and owns; the library keeps no pointer to it after
@@ -64,7 +69,8 @@ typedef struct CUstream_st *moe_stream_t; /* the same type as cudaStream_t */
 enum moe_wfmt {
     MOE_W_FP8_SC512 = 1, /* e4m3 weights + fp32 scale per (row, 512-block of K) */
     MOE_W_INT4_G128 = 2, /* int4 weights + bf16 scale per (row, 128-group of K) */
-    MOE_W_MXFP4_G32 = 3  /* E2M1 weights + E8M0 scale per (row, 32-block of K) */
+    MOE_W_MXFP4_G32 = 3, /* E2M1 weights + E8M0 scale per (row, 32-block of K) */
+    MOE_W_NVFP4_G16 = 4  /* E2M1 weights + E4M3 scale per (row, 16-block of K) + fp32 per matrix */
 };
 
 enum moe_status {
@@ -95,6 +101,9 @@ typedef struct {
  *         s_gate, s_up [E, I, H/128] bf16; s_down [E, H, I/128] bf16.
  *   MXFP4: w_* as int4 (E2M1 nibbles); s_gate, s_up [E, I, H/32] bytes; s_down [E, H, I/32]
  *         bytes (E8M0).
+ *   NVFP4: w_* as int4 (E2M1 nibbles); s_gate, s_up [E, I, H/16] bytes; s_down [E, H, I/16]
+ *         bytes (E4M3); t_gate, t_up, t_down [E] fp32 tensor scales (ts_*: [1]).  The t_* and
+ *         ts_* fields are read for NVFP4 only (NULL otherwise).
  *   ws_* / ss_*: the shared expert in the same format with E = 1 and I -> I_shared; NULL when
  *   I_shared == 0. */
 typedef struct {
@@ -102,6 +111,8 @@ typedef struct {
     const void *s_gate, *s_up, *s_down;
     const void *ws_gate, *ws_up, *ws_down;
     const void *ss_gate, *ss_up, *ss_down;
+    const float *t_gate, *t_up, *t_down;
+    const float *ts_gate, *ts_up, *ts_down;
 } moe_weights;
 
 typedef struct moe_plan_s moe_plan_t; /* opaque; owned by the library until moe_destroy */

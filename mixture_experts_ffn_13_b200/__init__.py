@@ -21,7 +21,8 @@ LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 MOE_W_FP8_SC512 = 1
 MOE_W_INT4_G128 = 2
 MOE_W_MXFP4_G32 = 3
-_WFMT = {"fp8": MOE_W_FP8_SC512, "int4": MOE_W_INT4_G128, "mxfp4": MOE_W_MXFP4_G32}
+MOE_W_NVFP4_G16 = 4
+_WFMT = {"fp8": MOE_W_FP8_SC512, "int4": MOE_W_INT4_G128, "mxfp4": MOE_W_MXFP4_G32, "nvfp4": MOE_W_NVFP4_G16}
 MOE_OK = 0
 ERRORS = {-1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED", -3: "MOE_ERR_WORKSPACE",
           -4: "MOE_ERR_CUDA", -5: "MOE_ERR_DEVICE_TIMEOUT", -6: "MOE_ERR_BOUNDS"}
@@ -48,7 +49,8 @@ class moe_dims(ctypes.Structure):
 class moe_weights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "w_gate", "w_up", "w_down", "s_gate", "s_up", "s_down",
-        "ws_gate", "ws_up", "ws_down", "ss_gate", "ss_up", "ss_down")]
+        "ws_gate", "ws_up", "ws_down", "ss_gate", "ss_up", "ss_down",
+        "t_gate", "t_up", "t_down", "ts_gate", "ts_up", "ts_down")]
 
 
 _lib = None
@@ -198,7 +200,8 @@ def moe_launch_count(plan: Plan) -> int:
 def _weights_struct(w: dict) -> moe_weights:
     g = lambda n: _ptr(w.get(n))
     return moe_weights(g("w_gate"), g("w_up"), g("w_down"), g("s_gate"), g("s_up"), g("s_down"),
-                       g("ws_gate"), g("ws_up"), g("ws_down"), g("ss_gate"), g("ss_up"), g("ss_down"))
+                       g("ws_gate"), g("ws_up"), g("ws_down"), g("ss_gate"), g("ss_up"), g("ss_down"),
+                       g("t_gate"), g("t_up"), g("t_down"), g("ts_gate"), g("ts_up"), g("ts_down"))
 
 
 def moe_route(plan: Plan, logits: torch.Tensor, workspace: torch.Tensor, out: dict | None = None,
@@ -323,7 +326,7 @@ class MoELayer:
         self.dims = d
         self.plan = Plan(T_max or d["T"], d["H"], d["E"], d["I"], d["k"], d["Is"], d["wfmt"])
         self.weights = {k: v for k, v in layer.items() if isinstance(v, torch.Tensor)
-                        and k[:2] in ("w_", "s_", "ws", "ss")}
+                        and k[:2] in ("w_", "s_", "ws", "ss", "t_", "ts")}
         self.workspace = self.plan.new_workspace(layer["x"].device)
 
     def route(self, logits, stream=None):

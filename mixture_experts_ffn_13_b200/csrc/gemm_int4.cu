@@ -1,5 +1,5 @@
 // gemm_int4.cu -- steps A4/A5 for 4-bit expert weights: persistent grouped GEMMs that unpack
-// int4 or MXFP4 weights into tensor memory and run bf16 x bf16 -> fp32 tcgen05 MMAs.
+// int4, MXFP4 or NVFP4 weights into tensor memory and run bf16 x bf16 -> fp32 tcgen05 MMAs.
 //
 // Page "Flash-Next 在 GPU 上到底在算什麼", section "① 專家 FFN" (and its NVIDIA table): expert
 // weights are stored in 4/8 bits and must be decompressed to 16-bit before the tensor units
@@ -36,11 +36,19 @@
 // one TMEM slot, and the epilogue has no promotion to do.  The warp roles shift with that:
 // warps 2-9 dequantise (two per TMEM lane quarter, one 32-element block of each 64-K stage
 // apiece) and warps 10-13 (one per quarter) stream each finished tile out.
+//
+// NVFP4 weights (the NVIDIA co-design commentary, section "讀的時候記得這是廠商文": two levels
+// of scale factors) take the same path: an E2M1 value times its 16-block's E4M3 scale has at
+// most six significant bits and stays within bf16's normal range, so it too is formed exactly
+// in bf16 by the dequantisers; the matrix's fp32 tensor scale multiplies the accumulator in
+// the epilogue.
 #include "gemm_common.cuh"
 #include "launch.cuh"
 #include "sm100.cuh"
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 namespace moe {
 
@@ -56,10 +64,12 @@ constexpr int kPrefetch = 8;           // raw stages prefetched into L2 ahead of
 // the scale groups); MXFP4 has no promotion, so one epilogue warp per quarter streams the
 // accumulator out, and the freed warps become a second dequantiser per quarter (each of the
 // pair converts one 32-element block of a 64-K stage).
-template <int BN, bool GATEUP, bool MX>
+enum { kFmtInt4 = 0, kFmtMx = 1, kFmtNv = 2 };
+
+template <int BN, bool GATEUP, bool FP4>
 struct I4Cfg {
-    static constexpr int CONV = MX ? 8 : 4;                 // dequantiser warps
-    static constexpr int EW = MX ? 4 : 8;                   // epilogue warps
+    static constexpr int CONV = FP4 ? 8 : 4;                // dequantiser warps
+    static constexpr int EW = FP4 ? 4 : 8;                  // epilogue warps
     static constexpr int CPW = BN / (EW / 4);               // token columns per epilogue thread
     static constexpr int THREADS = 32 * (2 + CONV + EW);
     static constexpr int NA = GATEUP ? 2 : 1;
@@ -122,6 +132,14 @@ __device__ __forceinline__ uint4 unpack8_fp4(uint32_t w, __nv_bfloat162 sc)
 // The bf16 pair (2^(c-127), 2^(c-127)) of an E8M0 code c in 1..254.
 __device__ __forceinline__ __nv_bfloat162 e8m0_pair(uint32_t c) { return bits_bf2((c << 7) | (c << 23)); }
 
+// The bf16 pair (v, v) of the E4M3 byte c (every finite E4M3 value is exact in bf16).
+__device__ __forceinline__ __nv_bfloat162 e4m3_pair(uint32_t c)
+{
+    const __half_raw hr = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(c), __NV_E4M3);
+    const __nv_bfloat16 b = __float2bfloat16_rn(__half2float(__half(hr)));
+    return __halves2bfloat162(b, b);
+}
+
 // 8 two's-complement nibbles (element 2i in the low nibble of byte i) -> the 8 integers as
 // bf16 (exact), returned as 4 words of bf16 pairs in element order.
 __device__ __forceinline__ uint4 unpack8(uint32_t w)
@@ -141,12 +159,14 @@ __device__ __forceinline__ uint4 unpack8(uint32_t w)
     return make_uint4(r[0], r[1], r[2], r[3]);
 }
 
-// MX = false: int4 weights with bf16 scales per 128-group; MX = true: MXFP4 weights.
-template <int BN, bool GATEUP, bool MX>
-__global__ void __launch_bounds__(I4Cfg<BN, GATEUP, MX>::THREADS, 1)
+// FMT: kFmtInt4 (bf16 scales per 128-group), kFmtMx (MXFP4) or kFmtNv (NVFP4).
+template <int BN, bool GATEUP, int FMT>
+__global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1)
     gemm_int4_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmArgs args)
 {
-    using C = I4Cfg<BN, GATEUP, MX>;
+    constexpr bool FP4 = FMT != kFmtInt4;  // E2M1 elements with exact bf16 scaling (MXFP4, NVFP4)
+    constexpr bool NV = FMT == kFmtNv;
+    using C = I4Cfg<BN, GATEUP, FP4>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *raw = smem;                                   // NR raw stages [raw0 | raw1]
@@ -258,9 +278,9 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, MX>::THREADS, 1)
                 const TileInfo tl = decode_tile<BN, true>(args, stt, w, tot0);
                 const int n_mma = min(BN, (tl.nrows + 15) & ~15);  // partial tiles: no work on absent rows
                 const uint32_t kIdesc = instr_desc(kTileM, n_mma, 1, 1);
-                // int4: one TMEM slot per 128-element scale group; MXFP4: one for the whole K
-                const int ngrp = MX ? 1 : args.seg[tl.seg].K / kGroupK;
-                const int spg = MX ? args.seg[tl.seg].K / kKE : C::STAGES_PER_GROUP;
+                // int4: one TMEM slot per 128-element scale group; E2M1 formats: one for the K
+                const int ngrp = FP4 ? 1 : args.seg[tl.seg].K / kGroupK;
+                const int spg = FP4 ? args.seg[tl.seg].K / kKE : C::STAGES_PER_GROUP;
                 for (int g = 0; g < ngrp; ++g, ++ai) {
                     const int slot = ai % C::NSLOT;
                     if (!mbar_wait(&acce[slot], ((ai / C::NSLOT) & 1) ^ 1, abort_flag, status, tmo)) goto done;
@@ -294,36 +314,50 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, MX>::THREADS, 1)
         const int q = warp & 3;        // TMEM lane quarter reachable from this warp
         const int r = q * 32 + lane;   // weight row of the tile handled by this thread
         uint32_t it = 0, rt = 0;
-        // MXFP4: this row's 8 E8M0 bytes (two words per matrix) of the current raw stage, and
-        // those of the next raw stage in this CTA's sequence (the next tile's first one at a
-        // tile's end), loaded a raw stage ahead so that their latency overlaps the conversion
-        uint32_t scur[C::NA][2] = {}, snxt[C::NA][2] = {};
-        auto load_scales = [&](int wi, int kr, uint32_t (&dst)[C::NA][2]) {
+        // E2M1 formats: this row's block-scale bytes of the current raw stage (MXFP4: 8 E8M0
+        // bytes, NVFP4: 16 E4M3 bytes per matrix) and those of the next raw stage in this
+        // CTA's sequence (the next tile's first one at a tile's end), loaded a raw stage ahead
+        // so that their latency overlaps the conversion
+        constexpr int SBLK = NV ? 16 : 32;         // K elements per block scale
+        constexpr int SW = kRawKE / SBLK / 4;      // scale words per raw stage: 2 (MX), 4 (NV)
+        uint32_t scur[C::NA][SW] = {}, snxt[C::NA][SW] = {};
+        auto load_scales = [&](int wi, int kr, uint32_t (&dst)[C::NA][SW]) {
             const TileInfo t = decode_tile<BN, true>(args, stt, wi, tot0);
             const GemmSeg &s = args.seg[t.seg];
-            const int nbk = s.K / 32;              // E8M0 bytes per weight row, a multiple of 4
-            const int b0 = kr * (kRawKE / 32);     // first byte of raw stage kr: b0 + 4 <= nbk
+            const int nbk = s.K / SBLK;            // scale bytes per weight row: a multiple of 4
+                                                   // (MX) or 8 (NV), so each load is aligned
+            const int b0 = kr * (4 * SW);          // first byte of raw stage kr
+            const int half = 2 * SW;               // bytes of the first 128 K of the raw stage
 #pragma unroll
             for (int m = 0; m < C::NA; ++m) {
                 const uint8_t *base = static_cast<const uint8_t *>(m == 0 ? s.sw0 : s.sw1);
-                const uint32_t *p = reinterpret_cast<const uint32_t *>(base + (size_t)(t.wrow + r) * nbk + b0);
-                dst[m][0] = __ldg(p);
-                dst[m][1] = b0 + 4 < nbk ? __ldg(p + 1) : 0u;  // a last raw stage of 128 K has 4
+                const uint8_t *p = base + (size_t)(t.wrow + r) * nbk + b0;
+                // a last raw stage of 128 K has only its first half: b0 + half <= nbk always
+                if constexpr (NV) {
+                    const uint2 lo = __ldg(reinterpret_cast<const uint2 *>(p));
+                    const uint2 hi = b0 + half < nbk ? __ldg(reinterpret_cast<const uint2 *>(p + 8)) : make_uint2(0u, 0u);
+                    dst[m][0] = lo.x;
+                    dst[m][1] = lo.y;
+                    dst[m][SW - 2] = hi.x;
+                    dst[m][SW - 1] = hi.y;
+                } else {
+                    dst[m][0] = __ldg(reinterpret_cast<const uint32_t *>(p));
+                    dst[m][SW - 1] = b0 + half < nbk ? __ldg(reinterpret_cast<const uint32_t *>(p + 4)) : 0u;
+                }
             }
         };
-        if (MX && (int)blockIdx.x < total) load_scales(blockIdx.x, 0, snxt);
+        if (FP4 && (int)blockIdx.x < total) load_scales(blockIdx.x, 0, snxt);
         for (int w = blockIdx.x; w < total; w += gridDim.x) {
             const TileInfo tl = decode_tile<BN, true>(args, stt, w, tot0);
             const GemmSeg &sg = args.seg[tl.seg];
             const int nkc = sg.K / kKE;
             for (int kc = 0; kc < nkc; ++kc, ++it) {
                 const int sub = kc % kSubs;
-                if (MX && sub == 0) {
+                if (FP4 && sub == 0) {
 #pragma unroll
-                    for (int m = 0; m < C::NA; ++m) {
-                        scur[m][0] = snxt[m][0];
-                        scur[m][1] = snxt[m][1];
-                    }
+                    for (int m = 0; m < C::NA; ++m)
+#pragma unroll
+                        for (int j = 0; j < SW; ++j) scur[m][j] = snxt[m][j];
                     const int kr = kc / kSubs;
                     if ((kr + 1) * kRawKE < sg.K)
                         load_scales(w, kr + 1, snxt);
@@ -340,22 +374,33 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, MX>::THREADS, 1)
                 tc_fence_after();
                 const uint8_t *rs = raw + rs_i * C::NA * C::RAW_BYTES + r * 128;
                 const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + ms_i * C::NA * C::A_COLS;
-                if constexpr (MX) {
-                    // half hx of the stage: 16-byte chunk 2*sub + hx of the row (the 128-byte
-                    // swizzle stores chunk c at position c ^ (r & 7)) = 32-block 2*sub + hx of
+                if constexpr (FP4) {
+                    // half hx of the stage: 16-byte chunk ch = 2*sub + hx of the row (the 128-byte
+                    // swizzle stores chunk c at position c ^ (r & 7)), K elements 32*ch .. +31 of
                     // the raw stage, written to TMEM columns 16*hx .. 16*hx + 15
                     const int hx = (warp - 2) >> 2;
                     const int cc = ((2 * sub + hx) ^ (r & 7)) << 4;
 #pragma unroll
                     for (int m = 0; m < C::NA; ++m) {
                         const uint4 qq = *reinterpret_cast<const uint4 *>(rs + m * C::RAW_BYTES + cc);
-                        const uint32_t sw = (sub >> 1) ? scur[m][1] : scur[m][0];
-                        const __nv_bfloat162 sc = e8m0_pair((sw >> ((sub & 1) * 16 + hx * 8)) & 0xFFu);
+                        // scales of the chunk's elements 0-15 (sa) and 16-31 (sb)
+                        __nv_bfloat162 sa, sb;
+                        if constexpr (NV) {
+                            // 16-blocks 2*ch and 2*ch + 1: bytes 2*ch, 2*ch + 1 = word sub, bytes
+                            // 2*hx and 2*hx + 1 of it
+                            const uint32_t sw = sub == 0 ? scur[m][0] : sub == 1 ? scur[m][1] : sub == 2 ? scur[m][SW - 2] : scur[m][SW - 1];
+                            sa = e4m3_pair((sw >> (hx * 16)) & 0xFFu);
+                            sb = e4m3_pair((sw >> (hx * 16 + 8)) & 0xFFu);
+                        } else {
+                            // 32-block ch: byte ch = word sub >> 1, byte (sub & 1) * 2 + hx of it
+                            const uint32_t sw = (sub >> 1) ? scur[m][SW - 1] : scur[m][0];
+                            sa = sb = e8m0_pair((sw >> ((sub & 1) * 16 + hx * 8)) & 0xFFu);
+                        }
                         const uint32_t words[4] = {qq.x, qq.y, qq.z, qq.w};
                         uint32_t v[16];
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
-                            const uint4 u = unpack8_fp4(words[j], sc);
+                            const uint4 u = unpack8_fp4(words[j], j < 2 ? sa : sb);
                             v[4 * j] = u.x;
                             v[4 * j + 1] = u.y;
                             v[4 * j + 2] = u.z;
@@ -404,8 +449,15 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, MX>::THREADS, 1)
         for (int w = blockIdx.x; w < total; w += gridDim.x) {
             const TileInfo tl = decode_tile<BN, true>(args, stt, w, tot0);
             const GemmSeg &sg = args.seg[tl.seg];
-            if constexpr (MX) {
-                // MXFP4: the tile's whole K sits in one slot; stream it out 16 columns at a time
+            if constexpr (FP4) {
+                // E2M1 formats: the tile's whole K sits in one slot; stream it out 16 columns
+                // at a time (NVFP4: times the matrices' tensor scales, expert wrow / N)
+                float t0 = 1.0f, t1 = 1.0f;
+                if constexpr (NV) {
+                    const int g = tl.wrow / sg.N;
+                    t0 = __ldg(sg.ts0 + g);
+                    if (GATEUP) t1 = __ldg(sg.ts1 + g);
+                }
                 const int slot = ai % C::NSLOT;
                 const bool ok = mbar_wait(&accf[slot], (ai / C::NSLOT) & 1, abort_flag, status, tmo);
                 if (!__all_sync(0xffffffffu, ok)) goto done;
@@ -426,9 +478,10 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, MX>::THREADS, 1)
                         if (c0 + c < tl.nrows) {
                             const size_t o = (size_t)(tl.row0 + c0 + c) * sg.N + n;
                             if constexpr (GATEUP)
-                                static_cast<__nv_bfloat16 *>(sg.out)[o] = __float2bfloat16_rn(silu_mul(v[c], u[c]));
+                                static_cast<__nv_bfloat16 *>(sg.out)[o] =
+                                    __float2bfloat16_rn(NV ? silu_mul(v[c] * t0, u[c] * t1) : silu_mul(v[c], u[c]));
                             else
-                                static_cast<float *>(sg.out)[o] = v[c];
+                                static_cast<float *>(sg.out)[o] = NV ? v[c] * t0 : v[c];
                         }
                     }
                 }
@@ -438,12 +491,11 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, MX>::THREADS, 1)
                 ++ai;
                 continue;
             }
-            // MXFP4: the weights arrive scaled and the whole K sits in one slot (scale 1)
-            const int ngrp = MX ? 1 : sg.K / kGroupK;
-            const __nv_bfloat16 *sw0 =
-                MX ? nullptr : static_cast<const __nv_bfloat16 *>(sg.sw0) + (size_t)(tl.wrow + r) * ngrp;
+            // int4 only from here on (the E2M1 formats took the branch above)
+            const int ngrp = sg.K / kGroupK;
+            const __nv_bfloat16 *sw0 = static_cast<const __nv_bfloat16 *>(sg.sw0) + (size_t)(tl.wrow + r) * ngrp;
             const __nv_bfloat16 *sw1 =
-                (GATEUP && !MX) ? static_cast<const __nv_bfloat16 *>(sg.sw1) + (size_t)(tl.wrow + r) * ngrp : nullptr;
+                GATEUP ? static_cast<const __nv_bfloat16 *>(sg.sw1) + (size_t)(tl.wrow + r) * ngrp : nullptr;
             float acc0[C::CPW], acc1[GATEUP ? C::CPW : 1];
 #pragma unroll
             for (int c = 0; c < C::CPW; ++c) acc0[c] = 0.0f;
@@ -451,19 +503,13 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, MX>::THREADS, 1)
 #pragma unroll
                 for (int c = 0; c < C::CPW; ++c) acc1[c] = 0.0f;
             }
-            float s0n = 1.0f, s1n = 1.0f;
-            if constexpr (!MX) {
-                s0n = __bfloat162float(sw0[0]);
-                s1n = GATEUP ? __bfloat162float(sw1[0]) : 0.0f;
-            }
+            float s0n = __bfloat162float(sw0[0]), s1n = GATEUP ? __bfloat162float(sw1[0]) : 0.0f;
             for (int g = 0; g < ngrp; ++g, ++ai) {
                 const int slot = ai % C::NSLOT;
                 const float s0 = s0n, s1 = s1n;
-                if constexpr (!MX) {
-                    if (g + 1 < ngrp) {
-                        s0n = __bfloat162float(sw0[g + 1]);
-                        if (GATEUP) s1n = __bfloat162float(sw1[g + 1]);
-                    }
+                if (g + 1 < ngrp) {
+                    s0n = __bfloat162float(sw0[g + 1]);
+                    if (GATEUP) s1n = __bfloat162float(sw1[g + 1]);
                 }
                 const bool ok = mbar_wait(&accf[slot], (ai / C::NSLOT) & 1, abort_flag, status, tmo);
                 if (!__all_sync(0xffffffffu, ok)) goto done;
@@ -512,42 +558,46 @@ done:
     }
 }
 
-template <int BN, bool GATEUP, bool MX>
+template <int BN, bool GATEUP, int FMT>
 cudaError_t launch_t(const GemmMaps &maps, const GemmArgs &args, int num_sms, cudaStream_t s)
 {
-    using C = I4Cfg<BN, GATEUP, MX>;
-    auto kern = gemm_int4_kernel<BN, GATEUP, MX>;
+    using C = I4Cfg<BN, GATEUP, FMT != kFmtInt4>;
+    auto kern = gemm_int4_kernel<BN, GATEUP, FMT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     return launch_pdl(kern, dim3(num_sms), dim3(C::THREADS), C::SMEM, s, maps, args);
 }
 
-template <bool MX>
+template <int FMT>
 cudaError_t launch_fmt(bool gateup, int bn, const GemmMaps &maps, const GemmArgs &args, int num_sms, cudaStream_t s)
 {
     if (gateup) {
         switch (bn) {
-            case 32: return launch_t<32, true, MX>(maps, args, num_sms, s);
-            case 64: return launch_t<64, true, MX>(maps, args, num_sms, s);
-            case 96: return launch_t<96, true, MX>(maps, args, num_sms, s);
+            case 32: return launch_t<32, true, FMT>(maps, args, num_sms, s);
+            case 64: return launch_t<64, true, FMT>(maps, args, num_sms, s);
+            case 96: return launch_t<96, true, FMT>(maps, args, num_sms, s);
             default: return cudaErrorInvalidValue;
         }
     }
     switch (bn) {
-        case 32: return launch_t<32, false, MX>(maps, args, num_sms, s);
-        case 64: return launch_t<64, false, MX>(maps, args, num_sms, s);
-        case 96: return launch_t<96, false, MX>(maps, args, num_sms, s);
+        case 32: return launch_t<32, false, FMT>(maps, args, num_sms, s);
+        case 64: return launch_t<64, false, FMT>(maps, args, num_sms, s);
+        case 96: return launch_t<96, false, FMT>(maps, args, num_sms, s);
         default: return cudaErrorInvalidValue;
     }
 }
 
 }  // namespace
 
-cudaError_t launch_gemm_w4(bool gateup, bool mx, int bn, const GemmMaps &maps, const GemmArgs &args, int num_sms,
+cudaError_t launch_gemm_w4(bool gateup, int wfmt, int bn, const GemmMaps &maps, const GemmArgs &args, int num_sms,
                            cudaStream_t s)
 {
-    return mx ? launch_fmt<true>(gateup, bn, maps, args, num_sms, s)
-              : launch_fmt<false>(gateup, bn, maps, args, num_sms, s);
+    switch (wfmt) {
+        case MOE_W_INT4_G128: return launch_fmt<kFmtInt4>(gateup, bn, maps, args, num_sms, s);
+        case MOE_W_MXFP4_G32: return launch_fmt<kFmtMx>(gateup, bn, maps, args, num_sms, s);
+        case MOE_W_NVFP4_G16: return launch_fmt<kFmtNv>(gateup, bn, maps, args, num_sms, s);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace moe

@@ -187,8 +187,7 @@ int moe_plan(const moe_dims *dims, moe_plan_t **out_plan, size_t *workspace_byte
     *out_plan = nullptr;
     const moe_dims d = *dims;
     if (d.T_max < 1 || d.H < 1 || d.E < 1 || d.I < 1 || d.k < 1 || d.I_shared < 0) return MOE_ERR_INVALID_ARG;
-    if (d.wfmt != MOE_W_FP8_SC512 && d.wfmt != MOE_W_INT4_G128 && d.wfmt != MOE_W_MXFP4_G32)
-        return MOE_ERR_INVALID_ARG;
+    if (d.wfmt < MOE_W_FP8_SC512 || d.wfmt > MOE_W_NVFP4_G16) return MOE_ERR_INVALID_ARG;
     if (d.k > d.E) return MOE_ERR_INVALID_ARG;
     if (d.E > kMaxE || d.k > kMaxK || d.T_max > (1 << 20)) return MOE_ERR_UNSUPPORTED;
     if (d.H % 128 || d.I % 128 || d.I_shared % 128) return MOE_ERR_UNSUPPORTED;
@@ -363,8 +362,8 @@ int moe_route(moe_plan_t *p, int32_t T, const float *logits, int32_t *topk_idx, 
     return e == cudaSuccess ? MOE_OK : fail_cuda(p, e);
 }
 
-// The 4-bit layer (int4 or MXFP4): route, permute, gather bf16 rows, 4-bit gate|up (h in
-// bf16), 4-bit down, combine.  Stage events: 0 route | 1 permute | 2 gather | 3 gate|up |
+// The 4-bit layer (int4, MXFP4 or NVFP4): route, permute, gather bf16 rows, 4-bit gate|up
+// (h in bf16), 4-bit down, combine.  Stage events: 0 route | 1 permute | 2 gather | 3 gate|up |
 // 4 (no h quantiser) | 5 down | 6 combine | 7.
 static int forward_w4(moe_plan_t *p, int T, const uint16_t *x, const float *logits, const moe_weights *w,
                         uint16_t *out, uint8_t *ws, cudaStream_t s)
@@ -379,7 +378,6 @@ static int forward_w4(moe_plan_t *p, int T, const uint16_t *x, const float *logi
     const bool shared = Is > 0;
     const int A = T * k;
     const int bn = pick_bn(T, k, E, false);
-    const bool mx = d.wfmt == MOE_W_MXFP4_G32;
     mark(0);
     int *chk = p->checked ? p->d_status : nullptr;
     cudaError_t e = launch_route(logits, T, E, k, b.topk_idx, b.topk_w, s, chk);
@@ -409,17 +407,21 @@ static int forward_w4(moe_plan_t *p, int T, const uint16_t *x, const float *logi
     ag.status = p->d_status;
     ag.timeout_ns = kDefaultTimeoutNs;
     ag.seg[0] = GemmSeg{I, H, A, w->s_gate, w->s_up, nullptr, h};
+    ag.seg[0].ts0 = w->t_gate;
+    ag.seg[0].ts1 = w->t_up;
     int rc = encode_map_2d(&mg.a0[0], w->w_gate, U8, 1, H / 2, (uint64_t)E * I, 128, 128, true);
     rc |= encode_map_2d(&mg.a1[0], w->w_up, U8, 1, H / 2, (uint64_t)E * I, 128, 128, true);
     rc |= encode_map_2d(&mg.b[0], xp, BF, 2, H, A, 64, bn, true);
     if (shared) {
         ag.seg[1] = GemmSeg{Is, H, T, w->ss_gate, w->ss_up, nullptr, h_sh};
+        ag.seg[1].ts0 = w->ts_gate;
+        ag.seg[1].ts1 = w->ts_up;
         rc |= encode_map_2d(&mg.a0[1], w->ws_gate, U8, 1, H / 2, Is, 128, 128, true);
         rc |= encode_map_2d(&mg.a1[1], w->ws_up, U8, 1, H / 2, Is, 128, 128, true);
         rc |= encode_map_2d(&mg.b[1], xp_sh, BF, 2, H, T, 64, bn, true);
     }
     if (rc) return MOE_ERR_CUDA;
-    e = launch_gemm_w4(true, mx, bn, mg, ag, p->num_sms, s);
+    e = launch_gemm_w4(true, d.wfmt, bn, mg, ag, p->num_sms, s);
     mark(4);
     mark(5);
     if (e != cudaSuccess) return fail_cuda(p, e);
@@ -428,15 +430,17 @@ static int forward_w4(moe_plan_t *p, int T, const uint16_t *x, const float *logi
     GemmArgs ad = ag;
     ad.ttile = b.ttile_b;
     ad.seg[0] = GemmSeg{H, I, A, w->s_down, nullptr, nullptr, y};
+    ad.seg[0].ts0 = w->t_down;
     rc = encode_map_2d(&md.a0[0], w->w_down, U8, 1, I / 2, (uint64_t)E * H, 128, 128, true);
     rc |= encode_map_2d(&md.b[0], h, BF, 2, I, A, 64, bn, true);
     if (shared) {
         ad.seg[1] = GemmSeg{H, Is, T, w->ss_down, nullptr, nullptr, y_sh};
+        ad.seg[1].ts0 = w->ts_down;
         rc |= encode_map_2d(&md.a0[1], w->ws_down, U8, 1, Is / 2, H, 128, 128, true);
         rc |= encode_map_2d(&md.b[1], h_sh, BF, 2, Is, T, 64, bn, true);
     }
     if (rc) return MOE_ERR_CUDA;
-    e = launch_gemm_w4(false, mx, bn, md, ad, p->num_sms, s);
+    e = launch_gemm_w4(false, d.wfmt, bn, md, ad, p->num_sms, s);
     mark(6);
     if (e != cudaSuccess) return fail_cuda(p, e);
     e = launch_combine(y, y_sh, b.pos, b.topk_w, T, H, k, out, s, chk);
@@ -447,7 +451,8 @@ static int forward_w4(moe_plan_t *p, int T, const uint16_t *x, const float *logi
     return MOE_OK;
 }
 
-// Weight pointers present (the shared expert's when I_shared > 0) and 16-byte aligned.
+// Weight pointers present (the shared expert's when I_shared > 0, the tensor scales for NVFP4)
+// and 16-byte aligned.
 static int check_weights(const moe_plan_t *p, const moe_weights *w)
 {
     if (!w->w_gate || !w->w_up || !w->w_down || !w->s_gate || !w->s_up || !w->s_down) return MOE_ERR_INVALID_ARG;
@@ -458,6 +463,13 @@ static int check_weights(const moe_plan_t *p, const moe_weights *w)
                           w->ws_gate, w->ws_up, w->ws_down, w->ss_gate, w->ss_up, w->ss_down};
     for (const void *q : ptrs)
         if (!aligned16(q)) return MOE_ERR_INVALID_ARG;
+    if (p->d.wfmt == MOE_W_NVFP4_G16) {  // the tensor scales are read for NVFP4 only
+        if (!w->t_gate || !w->t_up || !w->t_down) return MOE_ERR_INVALID_ARG;
+        if (p->d.I_shared > 0 && (!w->ts_gate || !w->ts_up || !w->ts_down)) return MOE_ERR_INVALID_ARG;
+        const void *ts[] = {w->t_gate, w->t_up, w->t_down, w->ts_gate, w->ts_up, w->ts_down};
+        for (const void *q : ts)
+            if (!aligned16(q)) return MOE_ERR_INVALID_ARG;
+    }
     return MOE_OK;
 }
 

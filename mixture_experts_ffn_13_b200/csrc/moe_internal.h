@@ -79,6 +79,8 @@ struct GemmSeg {
     void *out;        // gate|up: h [rows, N]; down: y [rows, N]
     int ilv4d;        // interleaved gate|up: a0 is one 4-D map that loads 16 gate + 16 up rows per quarter
     int up_lo;        // interleaved gate|up: the up rows come first in each 32-row quarter
+    const float *ts0; // NVFP4: fp32 tensor scales of the first / second weight matrix, one per
+    const float *ts1; //   group (routed: [E], shared: [1]); unused otherwise
 };
 
 struct GemmArgs {
@@ -100,9 +102,9 @@ struct GemmMaps {
 // FP8 grouped GEMMs.  gateup: h = silu(x Wg^T) * (x Wu^T) in fp32; down: y = h Wd^T in fp32.
 cudaError_t launch_gemm_fp8(bool gateup, int bn, const GemmMaps &maps, const GemmArgs &args, int num_sms,
                             cudaStream_t s);
-// 4-bit grouped GEMMs over bf16 activations (int4 with bf16 scales per 128-group, or MXFP4
-// when mx): gate|up writes h as bf16, down writes y fp32.
-cudaError_t launch_gemm_w4(bool gateup, bool mx, int bn, const GemmMaps &maps, const GemmArgs &args,
+// 4-bit grouped GEMMs over bf16 activations (wfmt: MOE_W_INT4_G128, MOE_W_MXFP4_G32 or
+// MOE_W_NVFP4_G16): gate|up writes h as bf16, down writes y fp32.
+cudaError_t launch_gemm_w4(bool gateup, int wfmt, int bn, const GemmMaps &maps, const GemmArgs &args,
                            int num_sms, cudaStream_t s);
 
 // Router logits [T, E] (written) and their softmax top-k (step A1): the router GEMM, then the

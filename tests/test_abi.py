@@ -58,8 +58,8 @@ def _plan_rc(lib, **kw):
 @pytest.mark.parametrize("kw,code", [
     (dict(k=0), -1), (dict(k=9), -1), (dict(T_max=0), -1), (dict(H=0), -1), (dict(wfmt=7), -1),
     (dict(I_shared=-128), -1), (dict(E=2048, k=2), -2), (dict(k=33, E=64), -2), (dict(H=520), -2),
-    (dict(I=200), -2), (dict(I_shared=100), -2), (dict(wfmt=2, H=4100), -2), (dict(wfmt=4), -1),
-    (dict(wfmt=3, H=4100), -2), (dict(wfmt=3, I=160), -2), (dict(wfmt=0), -1),
+    (dict(I=200), -2), (dict(I_shared=100), -2), (dict(wfmt=2, H=4100), -2), (dict(wfmt=3, H=4100), -2),
+    (dict(wfmt=3, I=160), -2), (dict(wfmt=0), -1), (dict(wfmt=5), -1), (dict(wfmt=4, H=200), -2),
 ])
 def test_plan_rejects_bad_dims(lib, kw, code):
     assert _plan_rc(lib, **kw) == code

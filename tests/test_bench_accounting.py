@@ -17,7 +17,7 @@ def _tensor_bytes(t):
     return t.numel() * t.element_size()
 
 
-@pytest.mark.parametrize("wfmt", ["fp8", "int4", "mxfp4"])
+@pytest.mark.parametrize("wfmt", ["fp8", "int4", "mxfp4", "nvfp4"])
 @pytest.mark.parametrize("Is", [0, 256])
 def test_gemm_bytes_are_the_touched_experts_tensors(wfmt, Is):
     cfg = dict(T=24, H=1024, E=8, I=384, k=2, Is=Is, seed=70, bias=None, wfmt=wfmt)
@@ -25,11 +25,14 @@ def test_gemm_bytes_are_the_touched_experts_tensors(wfmt, Is):
     counts = np.array([3, 0, 5, 0, 0, 1, 2, 1])  # experts 1, 3, 4 untouched
     alg = bench.algorithmic(cfg, counts)
     touched = np.nonzero(counts)[0]
-    gu = sum(_tensor_bytes(layer[n][e]) for n in ("w_gate", "w_up", "s_gate", "s_up") for e in touched)
-    dn = sum(_tensor_bytes(layer[n][e]) for n in ("w_down", "s_down") for e in touched)
+    has = lambda n: n in layer  # NVFP4 adds the per-matrix tensor scales t_*, ts_*
+    gu = sum(_tensor_bytes(layer[n][e]) for n in ("w_gate", "w_up", "s_gate", "s_up", "t_gate", "t_up")
+             if has(n) for e in touched)
+    dn = sum(_tensor_bytes(layer[n][e]) for n in ("w_down", "s_down", "t_down") if has(n) for e in touched)
     if Is:
-        gu += sum(_tensor_bytes(layer[n]) for n in ("ws_gate", "ws_up", "ss_gate", "ss_up"))
-        dn += sum(_tensor_bytes(layer[n]) for n in ("ws_down", "ss_down"))
+        gu += sum(_tensor_bytes(layer[n]) for n in ("ws_gate", "ws_up", "ss_gate", "ss_up", "ts_gate", "ts_up")
+                  if has(n))
+        dn += sum(_tensor_bytes(layer[n]) for n in ("ws_down", "ss_down", "ts_down") if has(n))
     assert alg["touched"] == len(touched)
     assert alg["gemm_gateup"] == gu
     assert alg["gemm_down"] == dn

@@ -41,6 +41,8 @@ def _layer_parity(cfg):
     dict(T=9, H=256, E=1, I=256, k=1, Is=128, seed=56, bias=None, wfmt="int4"),     # one 4-bit expert + shared
     dict(T=24, H=256, E=4, I=128, k=4, Is=0, seed=59, bias=None, wfmt="mxfp4"),     # k = E, MXFP4
     dict(T=9, H=128, E=1, I=256, k=1, Is=128, seed=60, bias=None, wfmt="mxfp4"),    # one MXFP4 expert + shared
+    dict(T=24, H=256, E=4, I=128, k=4, Is=0, seed=61, bias=None, wfmt="nvfp4"),     # k = E, NVFP4
+    dict(T=9, H=128, E=1, I=256, k=1, Is=128, seed=62, bias=None, wfmt="nvfp4"),    # one NVFP4 expert + shared
 ], ids=lambda c: f"{c['wfmt']}-T{c['T']}-E{c['E']}-k{c['k']}-Is{c['Is']}")
 def test_degenerate_and_extreme_shapes(cfg):
     _layer_parity(cfg)
@@ -131,3 +133,17 @@ def test_checked_mode_reports_non_finite_logits():
     want, _, amb = oracle.layer(moe_synth.to_numpy(layer), ambiguity=True)
     check_out(out, want, "checked mode", amb)
     moe.moe_set_checked(m.plan, False)
+
+
+def test_nvfp4_without_tensor_scales_is_rejected():
+    """NVFP4 reads one fp32 tensor scale per weight matrix: a missing one is an argument error
+    that launches nothing."""
+    cfg = dict(T=8, H=256, E=4, I=128, k=2, Is=128, seed=63, bias=None, wfmt="nvfp4")
+    layer = moe_synth.make_layer(cfg, device="cuda")
+    m = moe.MoELayer(layer)
+    for name in ("t_down", "ts_up"):
+        w = dict(m.weights)
+        del w[name]
+        with pytest.raises(moe.MoEError) as ei:
+            moe.moe_forward(m.plan, layer["x"], layer["logits"], w, m.workspace)
+        assert ei.value.code == -1 and moe.moe_launch_count(m.plan) == 0

@@ -194,7 +194,7 @@ def test_layer_int4_small(cfg):
     assert torch.equal(out, out2)
 
 
-SMALL_MXFP4 = [
+SMALL_FP4 = [
     dict(T=16, H=256, E=4, I=128, k=2, Is=0, seed=81, bias=None),
     # K = 384 in both GEMMs: a last raw stage of 128 K (4 scale bytes per row), shared expert
     dict(T=37, H=384, E=8, I=384, k=3, Is=256, seed=82, bias="normal"),
@@ -205,15 +205,16 @@ SMALL_MXFP4 = [
 ]
 
 
-@pytest.mark.parametrize("cfg", SMALL_MXFP4, ids=lambda c: f"T{c['T']}-H{c['H']}-E{c['E']}-I{c['I']}-k{c['k']}-Is{c['Is']}")
-def test_layer_mxfp4_small(cfg):
-    cfg = dict(cfg, wfmt="mxfp4")
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
+@pytest.mark.parametrize("cfg", SMALL_FP4, ids=lambda c: f"T{c['T']}-H{c['H']}-E{c['E']}-I{c['I']}-k{c['k']}-Is{c['Is']}")
+def test_layer_fp4_small(cfg, fmt):
+    cfg = dict(cfg, wfmt=fmt)
     layer = moe_synth.make_layer(cfg, device="cuda")
     m = moe.MoELayer(layer)
     out = m(layer["x"], layer["logits"])
     assert moe.moe_get_status(m.plan) == 0
     want, _, amb = oracle.layer(moe_synth.to_numpy(layer), ambiguity=True)
-    check_out(out, want, "mxfp4 layer", amb)
+    check_out(out, want, f"{fmt} layer", amb)
     out2 = m(layer["x"], layer["logits"])
     torch.cuda.synchronize()
     assert torch.equal(out, out2)
@@ -236,7 +237,7 @@ def _sampled_parity(name, n_sample=12):
     check_route(m.plan, m.workspace, layer["logits"], cfg["k"])
 
 
-@pytest.mark.parametrize("name", ["tiny", "decode", "prefill", "skewed", "int4", "mxfp4"])
+@pytest.mark.parametrize("name", ["tiny", "decode", "prefill", "skewed", "int4", "mxfp4", "nvfp4"])
 def test_layer_configs_sampled(name):
     _sampled_parity(name)
 
