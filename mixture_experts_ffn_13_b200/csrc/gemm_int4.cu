@@ -335,7 +335,8 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
                 // a last raw stage of 128 K has only its first half: b0 + half <= nbk always
                 if constexpr (NV) {
                     const uint2 lo = __ldg(reinterpret_cast<const uint2 *>(p));
-                    const uint2 hi = b0 + half < nbk ? __ldg(reinterpret_cast<const uint2 *>(p + 8)) : make_uint2(0u, 0u);
+                    const uint2 hi =
+                        b0 + half < nbk ? __ldg(reinterpret_cast<const uint2 *>(p + 8)) : make_uint2(0u, 0u);
                     dst[m][0] = lo.x;
                     dst[m][1] = lo.y;
                     dst[m][SW - 2] = hi.x;
@@ -388,7 +389,10 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
                         if constexpr (NV) {
                             // 16-blocks 2*ch and 2*ch + 1: bytes 2*ch, 2*ch + 1 = word sub, bytes
                             // 2*hx and 2*hx + 1 of it
-                            const uint32_t sw = sub == 0 ? scur[m][0] : sub == 1 ? scur[m][1] : sub == 2 ? scur[m][SW - 2] : scur[m][SW - 1];
+                            const uint32_t sw = sub == 0   ? scur[m][0]
+                                                : sub == 1 ? scur[m][1]
+                                                : sub == 2 ? scur[m][SW - 2]
+                                                           : scur[m][SW - 1];
                             sa = e4m3_pair((sw >> (hx * 16)) & 0xFFu);
                             sb = e4m3_pair((sw >> (hx * 16 + 8)) & 0xFFu);
                         } else {
