@@ -1,7 +1,9 @@
 /* A plain C caller of the library: compiled with gcc against include/moe_b200.h and linked
  * against libmoe_b200.so.  Exercises the calls that need no GPU -- status strings, plan
  * validation of unsupported or invalid dimensions (checked before any device call), and the
- * rejection of NULL plans and oversize static routing -- and prints "c abi ok" on success. */
+ * rejection of NULL plans and oversize static routing -- prints the weight struct's layout,
+ * and prints "c abi ok" on success. */
+#include <stddef.h>
 #include <stdio.h>
 #include <string.h>
 
@@ -44,6 +46,15 @@ int main(void)
     d.k = 10;
     d.wfmt = 7; /* unknown weight format */
     CHECK(moe_plan(&d, &p, &ws) == MOE_ERR_INVALID_ARG);
+    d.H = 4000; /* the 4-bit formats need whole 128-element groups too */
+    d.wfmt = MOE_W_MXFP4_G32;
+    CHECK(moe_plan(&d, &p, &ws) == MOE_ERR_UNSUPPORTED);
+    d.wfmt = MOE_W_NVFP4_G16;
+    CHECK(moe_plan(&d, &p, &ws) == MOE_ERR_UNSUPPORTED);
+    d.H = 4096;
+    /* struct layout, compared by the test with the Python binding's ctypes mirror */
+    printf("layout moe_weights %zu %zu moe_dims %zu\n", sizeof(moe_weights), offsetof(moe_weights, t_gate),
+           sizeof(moe_dims));
 
     CHECK(moe_forward(NULL, 1, NULL, NULL, NULL, NULL, NULL, 0, NULL) == MOE_ERR_INVALID_ARG);
     CHECK(moe_forward_x(NULL, 1, NULL, NULL, NULL, NULL, NULL, 0, NULL) == MOE_ERR_INVALID_ARG);

@@ -25,3 +25,11 @@ def test_c_program_against_header_and_library(tmp_path):
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0, r.stdout + r.stderr
     assert "c abi ok" in r.stdout
+    # the Python binding's ctypes mirrors of the structs have the C layout
+    import ctypes
+    import mixture_experts_ffn_13_b200 as moe
+    line = next(ln for ln in r.stdout.splitlines() if ln.startswith("layout"))
+    _, _, w_size, t_off, _, d_size = line.split()
+    assert int(w_size) == ctypes.sizeof(moe.moe_weights)
+    assert int(t_off) == moe.moe_weights.t_gate.offset
+    assert int(d_size) == ctypes.sizeof(moe.moe_dims)
