@@ -54,31 +54,36 @@ def lib():
     with _lock:
         if _lib is None:
             build()
-            L = ctypes.CDLL(_LIB)
-            P = ctypes.c_void_p
-            I = ctypes.c_int
-            L.orc_e4m3_decode.restype = ctypes.c_double
-            L.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
-            L.orc_e4m3_encode.restype = ctypes.c_uint8
-            L.orc_e4m3_encode.argtypes = [ctypes.c_float]
-            L.orc_e4m3_encode_n.argtypes = [I, P, P]
-            L.orc_e2m1_decode.restype = ctypes.c_double
-            L.orc_e2m1_decode.argtypes = [I]
-            L.orc_e8m0_decode.restype = ctypes.c_double
-            L.orc_e8m0_decode.argtypes = [ctypes.c_uint8]
-            L.orc_double_to_bf16.restype = ctypes.c_uint16
-            L.orc_double_to_bf16.argtypes = [ctypes.c_double]
-            L.orc_route.argtypes = [I, I, I, P, P, P]
-            L.orc_router_logits.argtypes = [I, I, I, P, P, P, P]
-            L.orc_permute.argtypes = [I, I, I, P, P, P, P, P]
-            L.orc_quant_row_fp8.argtypes = [I, P, P, P]
-            L.orc_quant_rows_bf16.argtypes = [I, I, P, P, P]
-            L.orc_expert_fp8_row.argtypes = [I, I] + [P] * 10
-            L.orc_expert_int4_row.argtypes = [I, I] + [P] * 9
-            L.orc_expert_w4_row.argtypes = [I, I, I] + [P] * 10
-            L.orc_layer.argtypes = [ctypes.POINTER(Dims), ctypes.POINTER(Weights), P, P, I, P, P, P, P, I]
-            _lib = L
+            _lib = load(_LIB)
     return _lib
+
+
+def load(path: str):
+    """Open a compiled copy of moe_oracle.c and declare its entry points."""
+    L = ctypes.CDLL(path)
+    P = ctypes.c_void_p
+    I = ctypes.c_int
+    L.orc_e4m3_decode.restype = ctypes.c_double
+    L.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
+    L.orc_e4m3_encode.restype = ctypes.c_uint8
+    L.orc_e4m3_encode.argtypes = [ctypes.c_float]
+    L.orc_e4m3_encode_n.argtypes = [I, P, P]
+    L.orc_e2m1_decode.restype = ctypes.c_double
+    L.orc_e2m1_decode.argtypes = [I]
+    L.orc_e8m0_decode.restype = ctypes.c_double
+    L.orc_e8m0_decode.argtypes = [ctypes.c_uint8]
+    L.orc_double_to_bf16.restype = ctypes.c_uint16
+    L.orc_double_to_bf16.argtypes = [ctypes.c_double]
+    L.orc_route.argtypes = [I, I, I, P, P, P]
+    L.orc_router_logits.argtypes = [I, I, I, P, P, P, P]
+    L.orc_permute.argtypes = [I, I, I, P, P, P, P, P]
+    L.orc_quant_row_fp8.argtypes = [I, P, P, P]
+    L.orc_quant_rows_bf16.argtypes = [I, I, P, P, P]
+    L.orc_expert_fp8_row.argtypes = [I, I] + [P] * 10
+    L.orc_expert_int4_row.argtypes = [I, I] + [P] * 9
+    L.orc_expert_w4_row.argtypes = [I, I, I] + [P] * 10
+    L.orc_layer.argtypes = [ctypes.POINTER(Dims), ctypes.POINTER(Weights), P, P, I, P, P, P, P, I]
+    return L
 
 
 def _p(a: np.ndarray | None):
