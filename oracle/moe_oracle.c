@@ -37,6 +37,8 @@
  *  R8     the shared expert has no gate; its output is added with weight 1.
  *  R9     gate is the first projection, up the second; h = silu(G) * U.
  *  R10    h is rounded to fp32 then quantised with the R5/R6 rule per 512-block of I.
+ *  R10a   the h codes (bf16 values for 4-bit layers) that another valid fp32 evaluation of
+ *         G and U could also produce: see the rounding budget before orc_h_window.
  *  R11    4-bit layers keep activations in bf16: h is rounded to bf16 (RNE).
  *  R12    outputs are summed in fp64 here and rounded to bf16 (RNE) once.
  *  R13    e4m3 = OCP FP8 E4M3: bias 7, no infinities, max finite 448, subnormal step 2^-9,
@@ -372,59 +374,122 @@ static void orc_tab_init(void)
 
 /* y[n] = sum_kb sx[kb] * sw[n,kb] * sum_{i in kb} dec(qx[i]) * dec(qw[n,i]),  n < N.
  * The inner sum is exact in fp64 (each product of two e4m3 values has at most 8
- * significant bits and lies in [2^-18, 2^18)). */
+ * significant bits and lies in [2^-18, 2^18)).  yabs (optional) receives the running-error
+ * magnitude of that sum evaluated the way the tensor cores do (R10a): the exact products are
+ * added in chunks of 32 consecutive K elements (one MMA) into an fp32 accumulator per
+ * 512-block, and each block's sum times its two scales is added into an fp32 total.  With one
+ * rounding per addition or product, the fp32 result is within u times the sum of the
+ * magnitudes of every partial result of that order: the chunk partials of each block (scaled
+ * by the block's scales), each block's scaled sum and the running total after each block. */
 static void orc_proj_fp8(int N, int K, const uint8_t *qx, const float *sx, const uint8_t *qw,
-                         const float *sw, double *y)
+                         const float *sw, double *y, double *yabs)
 {
     int nb = (K + 511) / 512;
     for (int n = 0; n < N; ++n) {
         const uint8_t *row = qw + (size_t)n * K;
-        double acc = 0.0;
+        double acc = 0.0, mag = 0.0;
         for (int kb = 0; kb < nb; ++kb) {
             int i0 = kb * 512, i1 = (kb + 1) * 512 < K ? (kb + 1) * 512 : K;
-            double part = 0.0;
-            for (int i = i0; i < i1; ++i) part += orc_dec_tab[qx[i]] * orc_dec_tab[row[i]];
+            double part = 0.0, pmag = 0.0;
+            for (int i = i0; i < i1; ++i) {
+                part += orc_dec_tab[qx[i]] * orc_dec_tab[row[i]];
+                if ((i - i0) % 32 == 31 || i == i1 - 1) pmag += fabs(part);
+            }
             acc += (double)sx[kb] * (double)sw[(size_t)n * nb + kb] * part;
+            double sc = fabs((double)sx[kb] * (double)sw[(size_t)n * nb + kb]);
+            mag += sc * pmag + sc * fabs(part) + fabs(acc);
         }
         y[n] = acc;
+        if (yabs) yabs[n] = mag;
     }
 }
 
+static double orc_sigmoid(double z) { return 1.0 / (1.0 + exp(-z)); }
+
 static double orc_silu(double z) { return z * (1.0 / (1.0 + exp(-z))); }
 
-/* R10a -- which h codes are not unique.  The layer rounds h to fp32 before quantising it
- * (R10), and an fp32 h obtained with another (equally valid) summation order can sit on the
- * other side of an e4m3 rounding midpoint, which moves that code by one step.  A code counts
- * as ambiguous when fl32(h/s) lies within a relative distance ORC_AMBIG_REL of the midpoint
- * between its e4m3 value and the neighbour on that side; the neighbour is then an equally
- * valid result.  For each ambiguous element i the down projection can move by
- * |dec(q_alt) - dec(q)| * s * |Wd[n, i] * sd[n, block(i)]| in output n; env[n] receives the
- * sum of those bounds (the envelope of the valid outputs around y).  ORC_AMBIG_REL = 2^-16
- * bounds the relative error of an fp32 accumulation of these dot products with margin. */
-#define ORC_AMBIG_REL (1.0 / 65536.0)
+/* ---- R10a: the h codes (or bf16 values) that are not unique ------------------------------
+ *
+ * The layer holds h in fp32 and then rounds it to a coarse format (e4m3 codes per 512-block
+ * for FP8 layers, bf16 for 4-bit layers).  fp32 results of G and U obtained in any other
+ * valid summation order (R17) differ from the exact values, and where the exact h lies close
+ * to a rounding boundary of the coarse format, the other side of that boundary is an equally
+ * valid result.  The oracle bounds, per element, how far a valid fp32 h can lie from the
+ * exact one, lists every coarse value a valid h can round to, and reports for each output
+ * the largest move those alternatives allow through the down projection (the envelope).
+ *
+ * Rounding budget (a reading; the pages give none).  G and U are evaluated the way the tensor
+ * cores do: every MMA adds its chunk of exact products (32 e4m3 or 16 bf16 products) into an
+ * fp32 accumulator with one rounding, and each accumulator (a 512-block for FP8, a 128-group
+ * for int4, the whole K for the E2M1 formats) is scaled into an fp32 total with one rounding
+ * per product or addition.  The projections return the running-error magnitude M of that
+ * order (the sum of |every partial result|), and a valid fp32 G lies within
+ * ORC_ROUND * M of the exact G, ORC_ROUND = 2^-22: one rounding of at most 2^-23 relative
+ * (truncation; round-to-nearest is 2^-24), doubled.  h = silu(G) * U then moves by at most
+ *   dh = |silu'(G)| |U| dG + |silu(G)| dU + dG dU + (2^-20 + |G| 2^-23) |h|,
+ * the last term covering the fp32 exponential (its argument's rounding grows with |G|), the
+ * division, the product and the final fp32 rounding of h. */
 
-static void orc_h_ambiguity(int H, int I, const float *h, const uint8_t *qh, const float *sh,
-                            const uint8_t *wd, const float *sd, double *env)
+#define ORC_U22 (1.0 / 4194304.0)
+#define ORC_U23 (1.0 / 8388608.0)
+#define ORC_ROUND ORC_U22
+
+/* The largest distance of a valid fp32 h from the exact silu(G) * U, given the distances
+ * dG, dU of valid fp32 G, U from the exact G, U. */
+static double orc_h_window(double G, double U, double dG, double dU)
+{
+    double sg = orc_sigmoid(G);
+    double dsilu = sg * (1.0 + G * (1.0 - sg));
+    double h = G * sg * U;
+    return fabs(dsilu) * fabs(U) * dG + fabs(G * sg) * dU + dG * dU +
+           (1.0 / 1048576.0 + fabs(G) * ORC_U23) * fabs(h);
+}
+
+/* e4m3 code of the double v rounded toward -inf (dir < 0) or +inf (dir > 0) to fp32 first,
+ * so that no value of the interval it bounds escapes through that rounding. */
+static uint8_t orc_e4m3_encode_dir(double v, int dir)
+{
+    float f = (float)v;
+    if (dir > 0 && (double)f < v) f = nextafterf(f, INFINITY);
+    if (dir < 0 && (double)f > v) f = nextafterf(f, -INFINITY);
+    return orc_e4m3_encode(f);
+}
+
+/* FP8 layers.  h: the exact h rounded to fp32 as the layer holds it; dh: its window; qh, sh:
+ * the oracle's codes and scales (R10).  Per 512-block of I with scale s (amax / 448): a valid
+ * amax differs by at most the block's largest window, so a valid scale differs by at most
+ * that over amax (relative) plus one rounding; a valid h / s then lies in
+ * v +- (|v| (ds/s + 2^-22) + dh / s) around the oracle's v = h / s, and every code between
+ * the roundings of the two ends is valid (rounding is monotone).  D_i = the largest
+ * |dec(code) - dec(q_i)| * s over those codes; env[n] += D_i * |Wd[n, i] * sd[n, block(i)]|. */
+static void orc_h_ambiguity(int H, int I, const float *h, const double *dh, const uint8_t *qh,
+                            const float *sh, const uint8_t *wd, const float *sd, double *env)
 {
     int nbI = (I + 511) / 512;
-    for (int i = 0; i < I; ++i) {
-        int code = qh[i] & 0x7F;
-        float sc = sh[i / 512];
-        double a = fabs((double)(float)(h[i] / sc)); /* the value the rounding decided on */
-        double r = orc_dec_tab[code];
-        int nb_code;
-        if (a >= r)
-            nb_code = code + 1;
-        else
-            nb_code = code - 1;
-        if (nb_code < 0 || nb_code > 0x7E) continue; /* no neighbour (zero side or saturated) */
-        double rn = orc_dec_tab[nb_code];
-        double mid = 0.5 * (r + rn);
-        if (fabs(a - mid) > ORC_AMBIG_REL * a) continue;
-        double dh = fabs(rn - r) * (double)sc;
-        for (int n = 0; n < H; ++n) {
-            double wv = orc_dec_tab[wd[(size_t)n * I + i]] * (double)sd[(size_t)n * nbI + i / 512];
-            env[n] += dh * fabs(wv);
+    for (int kb = 0; kb < nbI; ++kb) {
+        int i0 = kb * 512, i1 = (kb + 1) * 512 < I ? (kb + 1) * 512 : I;
+        double amax = 0.0, dmax = 0.0;
+        for (int i = i0; i < i1; ++i) {
+            if (fabs((double)h[i]) > amax) amax = fabs((double)h[i]);
+            if (dh[i] > dmax) dmax = dh[i];
+        }
+        if (amax == 0.0 && dmax == 0.0) continue;
+        double s = (double)sh[kb];
+        double ds = amax > 0.0 ? dmax / amax + ORC_U23 : 1.0;
+        for (int i = i0; i < i1; ++i) {
+            double v = (double)h[i] / s;
+            double half = fabs(v) * (ds + ORC_U22) + dh[i] / s;
+            if (half == 0.0) continue;
+            double q = orc_dec_tab[qh[i]];
+            double lo = orc_dec_tab[orc_e4m3_encode_dir(v - half, -1)];
+            double hi = orc_dec_tab[orc_e4m3_encode_dir(v + half, +1)];
+            double D = fabs(lo - q) > fabs(hi - q) ? fabs(lo - q) : fabs(hi - q);
+            if (D == 0.0) continue;
+            D *= s;
+            for (int n = 0; n < H; ++n) {
+                double wv = orc_dec_tab[wd[(size_t)n * I + i]] * (double)sd[(size_t)n * nbI + i / 512];
+                env[n] += D * fabs(wv);
+            }
         }
     }
 }
@@ -438,21 +503,28 @@ static void orc_expert_fp8(int H, int I, const uint8_t *qx, const float *sx, con
 {
     double *G = (double *)malloc(sizeof(double) * (size_t)I);
     double *U = (double *)malloc(sizeof(double) * (size_t)I);
+    double *SG = (double *)malloc(sizeof(double) * (size_t)I);
+    double *SU = (double *)malloc(sizeof(double) * (size_t)I);
     float *h = (float *)malloc(sizeof(float) * (size_t)I);
     uint8_t *qh = (uint8_t *)malloc((size_t)I);
     float *sh = (float *)malloc(sizeof(float) * (size_t)((I + 511) / 512));
-    orc_proj_fp8(I, H, qx, sx, wg, sg, G);
-    orc_proj_fp8(I, H, qx, sx, wu, su, U);
+    orc_proj_fp8(I, H, qx, sx, wg, sg, G, SG);
+    orc_proj_fp8(I, H, qx, sx, wu, su, U, SU);
     for (int n = 0; n < I; ++n) h[n] = (float)(orc_silu(G[n]) * U[n]);
     if (h_out) memcpy(h_out, h, sizeof(float) * (size_t)I);
     orc_quant_row_fp8(I, h, qh, sh);
-    orc_proj_fp8(H, I, qh, sh, wd, sd, y);
+    orc_proj_fp8(H, I, qh, sh, wd, sd, y, NULL);
     if (env) {
+        const double c = ORC_ROUND;
+        double *dh = SG; /* reused: the window of each h */
+        for (int n = 0; n < I; ++n) dh[n] = orc_h_window(G[n], U[n], c * SG[n], c * SU[n]);
         for (int n = 0; n < H; ++n) env[n] = 0.0;
-        orc_h_ambiguity(H, I, h, qh, sh, wd, sd, env);
+        orc_h_ambiguity(H, I, h, dh, qh, sh, wd, sd, env);
     }
     free(G);
     free(U);
+    free(SG);
+    free(SU);
     free(h);
     free(qh);
     free(sh);
@@ -503,32 +575,47 @@ static const void *orc_w4_scales(int wfmt, const void *sw, size_t e, int N, int 
 }
 
 /* y[n] = sum_i a[i] * (W[n, i] * t)  with a in fp64 (bf16 values, exact); t is the matrix's
- * tensor scale (1 except for NVFP4).  Every product is exact in fp64. */
+ * tensor scale (1 except for NVFP4).  Every product is exact in fp64.  yabs (optional)
+ * receives the running-error magnitude of the tensor cores' order (R10a): chunks of 16
+ * exact products of q (int4: per 128-group, promoted by the group's scale into an fp32 total;
+ * E2M1 formats: the scaled weights over the whole K, then times t). */
 static void orc_proj_w4(int wfmt, int N, int K, const double *a, const uint8_t *qw, const void *sw,
-                        double t, double *y)
+                        double t, double *y, double *yabs)
 {
+    const int chain = wfmt == ORC_INT4_G128 ? 128 : K;
     for (int n = 0; n < N; ++n) {
-        double acc = 0.0;
-        for (int i = 0; i < K; ++i) acc += a[i] * (orc_w4(wfmt, K, qw, sw, n, i) * t);
+        double acc = 0.0, mag = 0.0, part = 0.0, tot = 0.0;
+        for (int i = 0; i < K; ++i) {
+            double pr = a[i] * (orc_w4(wfmt, K, qw, sw, n, i) * t);
+            acc += pr;
+            part += pr;
+            if (i % 16 == 15) mag += fabs(part);
+            if (i % chain == chain - 1) {  /* the chain's sum enters the total */
+                tot += part;
+                mag += fabs(part) + fabs(tot);
+                part = 0.0;
+            }
+        }
         y[n] = acc;
+        if (yabs) yabs[n] = mag;
     }
 }
 
-/* R10a for 4-bit layers: h is rounded to bf16, so an h within ORC_AMBIG_REL of a bf16
- * rounding midpoint may round either way; env[n] gets |h_alt - h| * |W[n, i]| for each such i. */
-static void orc_h_ambiguity_bf16(int wfmt, int H, int I, const double *hx, const uint8_t *wd,
-                                 const void *sd, double td, double *env)
+/* R10a for 4-bit layers: h is rounded to bf16 (R11).  A valid fp32 h lies in
+ * hx +- dh around the exact hx; every bf16 value between the roundings of the two ends is a
+ * valid result (rounding is monotone).  D_i = the largest |that value - bf16(hx_i)|;
+ * env[n] += D_i * |W[n, i] * td| (td: the down matrix's tensor scale, 1 except for NVFP4). */
+static void orc_h_ambiguity_bf16(int wfmt, int H, int I, const double *hx, const double *dh,
+                                 const uint8_t *wd, const void *sd, double td, double *env)
 {
     for (int i = 0; i < I; ++i) {
-        double a = fabs(hx[i]);
-        if (a == 0.0) continue;
-        int e2;
-        frexp(a, &e2);
-        int lead = e2 - 1 < -126 ? -126 : e2 - 1;
-        double quantum = ldexp(1.0, lead - 7);
-        double frac = a / quantum - floor(a / quantum); /* position between two bf16 values */
-        if (fabs(frac - 0.5) * quantum > ORC_AMBIG_REL * a) continue;
-        for (int n = 0; n < H; ++n) env[n] += quantum * fabs(orc_w4(wfmt, I, wd, sd, n, i) * td);
+        if (dh[i] == 0.0) continue;
+        double b = orc_bf16_to_double(orc_double_to_bf16(hx[i]));
+        double lo = orc_bf16_to_double(orc_double_to_bf16(hx[i] - dh[i]));
+        double hi = orc_bf16_to_double(orc_double_to_bf16(hx[i] + dh[i]));
+        double D = fabs(lo - b) > fabs(hi - b) ? fabs(lo - b) : fabs(hi - b);
+        if (D == 0.0) continue;
+        for (int n = 0; n < H; ++n) env[n] += D * fabs(orc_w4(wfmt, I, wd, sd, n, i) * td);
     }
 }
 
@@ -539,22 +626,29 @@ static void orc_expert_w4(int wfmt, int H, int I, const double *x, const uint8_t
 {
     double *G = (double *)malloc(sizeof(double) * (size_t)I);
     double *U = (double *)malloc(sizeof(double) * (size_t)I);
+    double *SG = (double *)malloc(sizeof(double) * (size_t)I);
+    double *SU = (double *)malloc(sizeof(double) * (size_t)I);
     double *hx = (double *)malloc(sizeof(double) * (size_t)I);
     double *h = (double *)malloc(sizeof(double) * (size_t)I);
-    orc_proj_w4(wfmt, I, H, x, wg, sg, tg, G);
-    orc_proj_w4(wfmt, I, H, x, wu, su, tu, U);
+    orc_proj_w4(wfmt, I, H, x, wg, sg, tg, G, SG);
+    orc_proj_w4(wfmt, I, H, x, wu, su, tu, U, SU);
     for (int n = 0; n < I; ++n) {
         hx[n] = orc_silu(G[n]) * U[n];
         h[n] = orc_bf16_to_double(orc_double_to_bf16(hx[n]));
     }
     if (h_out) memcpy(h_out, h, sizeof(double) * (size_t)I);
-    orc_proj_w4(wfmt, H, I, h, wd, sd, td, y);
+    orc_proj_w4(wfmt, H, I, h, wd, sd, td, y, NULL);
     if (env) {
+        const double c = ORC_ROUND;
+        double *dh = SG; /* reused: the window of each h */
+        for (int n = 0; n < I; ++n) dh[n] = orc_h_window(G[n], U[n], c * SG[n], c * SU[n]);
         for (int n = 0; n < H; ++n) env[n] = 0.0;
-        orc_h_ambiguity_bf16(wfmt, H, I, hx, wd, sd, td, env);
+        orc_h_ambiguity_bf16(wfmt, H, I, hx, dh, wd, sd, td, env);
     }
     free(G);
     free(U);
+    free(SG);
+    free(SU);
     free(hx);
     free(h);
 }

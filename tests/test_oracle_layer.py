@@ -289,10 +289,14 @@ def test_h_on_a_rounding_midpoint_reports_the_envelope(orc):
     assert np.all(amb[0, 200:] == 0) and np.all(amb[0, :200] > 0)
 
 
-def test_envelope_is_zero_off_the_midpoints(orc):
-    L = moe_synth.to_numpy(moe_synth.make_layer(SMALL[0]))
+@pytest.mark.parametrize("cfg", SMALL, ids=lambda c: f"{c['wfmt']}-T{c['T']}-H{c['H']}-I{c['I']}-Is{c['Is']}")
+def test_envelope_does_not_change_the_layer_and_stays_small(orc, cfg):
+    """Asking for the envelope leaves the outputs unchanged, and on random layers the envelope
+    is a small part of the tolerance for a typical output: only the few h values whose window
+    reaches a rounding boundary contribute, each by one step of the coarse format."""
+    L = moe_synth.to_numpy(moe_synth.make_layer(cfg))
     out, outb, amb = orc.layer(L, ambiguity=True)
     out2, _ = orc.layer(L)
     assert np.array_equal(out, out2)
-    # random data essentially never puts an h within 2^-16 of a midpoint
-    assert (amb != 0).mean() < 0.05
+    assert np.all(amb >= 0)
+    assert np.median(amb / (2e-3 + 1e-2 * np.abs(out))) < 0.05

@@ -13,6 +13,7 @@ import subprocess
 import pytest
 
 import oracle
+import test_oracle_envelope as ENV
 import test_oracle_formats as F
 import test_oracle_layer as LY
 import test_oracle_mxfp4 as MX
@@ -40,6 +41,11 @@ PINS = [
     (NV.test_nvfp4_one_hot_reads_single_weights, {}),
     (NV.test_tensor_scales_apply_to_their_own_matrices, {}),
     (LY.test_shared_expert_adds_with_weight_one, {}),
+    (LY.test_h_on_a_rounding_midpoint_reports_the_envelope, {}),
+    (ENV.test_fp8_window_follows_the_partial_sums, {}),
+    (ENV.test_bf16_h_on_a_rounding_midpoint, {"fmt": "int4"}),
+    (ENV.test_bf16_h_on_a_rounding_midpoint, {"fmt": "mxfp4"}),
+    (ENV.test_bf16_h_on_a_rounding_midpoint, {"fmt": "nvfp4"}),
     (LY.test_layer_equals_dense_masked_bruteforce, {"cfg": LY.SMALL[1]}),
     (LY.test_layer_equals_dense_masked_bruteforce, {"cfg": LY.SMALL[3]}),
 ]
@@ -70,6 +76,16 @@ MUTANTS = [
      "orc_dec_tab[sc[(size_t)n * (K / 16) + i / 32]]", 1),
     ("combine ignores the routing weights", "for (int n = 0; n < H; ++n) out[n] += p[j] * y[n];",
      "for (int n = 0; n < H; ++n) out[n] += y[n] / k;", 2),
+    ("bf16 envelope without the down matrix's tensor scale",
+     "env[n] += D * fabs(orc_w4(wfmt, I, wd, sd, n, i) * td);", "env[n] += D * fabs(orc_w4(wfmt, I, wd, sd, n, i));",
+     1),
+    ("bf16 envelope measured from the exact h", "double b = orc_bf16_to_double(orc_double_to_bf16(hx[i]));",
+     "double b = hx[i];", 1),
+    ("bf16 alternatives ignore the window above h",
+     "double hi = orc_bf16_to_double(orc_double_to_bf16(hx[i] + dh[i]));", "double hi = b;", 1),
+    ("FP8 window from the result instead of the partial sums",
+     "mag += sc * pmag + sc * fabs(part) + fabs(acc);", "mag += fabs(acc);", 1),
+    ("FP8 envelope one code step too wide", "D *= s;", "D *= 2.0 * s;", 1),
     ("shared expert weighted like a routed one", "            for (int n = 0; n < H; ++n) out[n] += y[n];\n",
      "            for (int n = 0; n < H; ++n) out[n] += p[0] * y[n];\n", 2),
 ]
