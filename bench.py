@@ -45,6 +45,9 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target oracle time for cpu_baseline")
+    ap.add_argument("--no-per-config", action="store_true", help="time the headline workload only")
+    ap.add_argument("--per-config-steps", type=int, default=10)
+    ap.add_argument("--per-config-cpu-seconds", type=float, default=3.0)
     return ap.parse_args()
 
 
@@ -256,15 +259,41 @@ def run_reference(args, ws, rank, cfg_name):
     print(json.dumps(line), flush=True)
 
 
-def run_ours(args, ws, rank, local, cfg_name):
-    import numpy as np
+def fp8_peak_tflops(dev):
+    """Dense FP8 (e4m3) tensor throughput of this GPU as cuBLAS reaches it: the best of 10
+    8192^3 torch._scaled_mm calls (e4m3 x e4m3 -> bf16).  A measured denominator for the FP8
+    tensor fraction; None if the call is unavailable."""
+    import torch
+    try:
+        n = 8192
+        a = torch.randn((n, n), device=dev).to(torch.float8_e4m3fn)
+        b = torch.randn((n, n), device=dev).to(torch.float8_e4m3fn).t()
+        one = torch.ones((), device=dev)
+        for _ in range(3):
+            torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        best = 1e9
+        for _ in range(10):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+            e1.record()
+            torch.cuda.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        del a, b
+        return 2 * n ** 3 / (best / 1e3) / 1e12
+    except Exception:
+        return None
+
+
+def measure_layer(cfg_name, steps, warmup, ws, rank, local, pk, pk_src, fp8_tf, flush, timing_barrier=True):
+    """Time `steps` moe_forward calls of one synthetic layer (L2 flushed before each, CUDA
+    events on the launching stream), then the same steps with the library's stage events for
+    the per-kernel times.  Returns the layer, its MoELayer and the measurement dict."""
     import torch
 
     import moe_synth
     import mixture_experts_ffn_13_b200 as moe
-    from mixture_experts_ffn_13_b200 import build as moe_build
 
-    moe_build.build()
     cfg = {**moe_synth.CONFIGS, **moe_synth.PROFILE_CONFIGS}[cfg_name]
     dev = torch.device("cuda", torch.cuda.current_device())
     layer = moe_synth.make_layer(cfg_name, device=dev)
@@ -272,46 +301,43 @@ def run_ours(args, ws, rank, local, cfg_name):
     x, logits = layer["x"], layer["logits"]
     out = torch.empty_like(x)
     stream = torch.cuda.current_stream()
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > 126 MB L2
-
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         m(x, logits, out=out)
     torch.cuda.synchronize()
     rc = moe.moe_get_status(m.plan)
     if rc != 0:
-        raise RuntimeError(f"device status after warm-up: {moe.moe_strerror(rc)}")
+        raise RuntimeError(f"{cfg_name}: device status after warm-up: {moe.moe_strerror(rc)}")
 
-    # pass A -- the timed region: K steps, each bracketed by CUDA events on the launching
-    # stream, L2 flushed before each step (outside the events)
     clocks = ClockSampler(local) if rank == 0 else None
     if clocks:
         clocks.start()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     launches = 0
-    barrier(ws)
+    if timing_barrier:
+        barrier(ws)
     torch.cuda.synchronize()
-    for i in range(args.steps):
+    for i in range(steps):
         flush.zero_()
         ev[i][0].record(stream)
         m(x, logits, out=out)
         ev[i][1].record(stream)
         launches += moe.moe_launch_count(m.plan)
     torch.cuda.synchronize()
-    barrier(ws)
+    if timing_barrier:
+        barrier(ws)
     step_ms = [a.elapsed_time(b) for a, b in ev]
     clk = clocks.stop() if clocks else None
     rc = moe.moe_get_status(m.plan)
     if rc != 0:
-        raise RuntimeError(f"device status after timing: {moe.moe_strerror(rc)}")
-    total_ms = max_over_ranks(ws, sum(step_ms))
+        raise RuntimeError(f"{cfg_name}: device status after timing: {moe.moe_strerror(rc)}")
+    total_ms = max_over_ranks(ws, sum(step_ms)) if timing_barrier else sum(step_ms)
 
-    # pass B -- the same K steps with the library's stage events on the same stream: per-kernel
-    # device times for the roofline of the dominant kernel (events between kernels keep the
-    # next kernel from starting early, so this pass is not the one `value` comes from)
+    # the same steps with the library's stage events on the same stream: per-kernel device
+    # times for the roofline of the dominant kernel (events between kernels keep the next
+    # kernel from starting early, so this pass is not the one the throughput comes from)
     moe.moe_profile_enable(m.plan, True)
     stage_ms = {s_: 0.0 for s_ in moe.STAGES}
-    prof_ms = 0.0
-    for i in range(args.steps):
+    for i in range(steps):
         flush.zero_()
         ev[i][0].record(stream)
         m(x, logits, out=out)
@@ -321,6 +347,73 @@ def run_ours(args, ws, rank, local, cfg_name):
     torch.cuda.synchronize()
     prof_ms = sum(a.elapsed_time(b) for a, b in ev)
     moe.moe_profile_enable(m.plan, False)
+
+    r = m.route(logits)
+    counts = r["counts"].cpu().numpy()
+    alg = algorithmic(cfg, counts)
+    T = cfg["T"]
+    ms_step = total_ms / steps
+    mean_stage = {k: v / steps for k, v in stage_ms.items()}
+    dom = max(("gemm_gateup", "gemm_down"), key=lambda s_: mean_stage[s_])
+    achieved = alg[dom] / (mean_stage[dom] / 1e3) / 1e9
+    layer_gbs = alg["layer"] / (ms_step / 1e3) / 1e9
+    if cfg["wfmt"] == "fp8":
+        if fp8_tf:
+            tpk, tpk_src = fp8_tf, "cuBLAS e4m3 8192^3 (torch._scaled_mm), measured in this run"
+        else:
+            tpk, tpk_src = 2 * pk["bf16_tflops"], f"2 x {pk_src} bf16 burst (FP8 = 2x bf16 nominal ratio)"
+    else:
+        tpk, tpk_src = pk["bf16_tflops"], f"{pk_src} bf16 burst"
+    t_hbm = alg["layer"] / (pk["hbm_gbs"] * 1e9) * 1e3
+    t_tc = alg["flops"] / (tpk * 1e12) * 1e3
+    small = sum(v for k, v in mean_stage.items() if not k.startswith("gemm_"))
+    res = {
+        "workload": cfg["workload"], "value": replica_throughput(ws, T, steps, total_ms), "unit": UNIT,
+        "ms_per_step": ms_step, "steps": steps, "warmup": warmup,
+        "experts_touched": alg["touched"], "max_tokens_per_expert": int(counts.max()),
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / pk["hbm_gbs"], "algorithmic_bytes": alg[dom],
+                     "peak_source": pk_src, "layer_achieved_gbs": layer_gbs, "layer_frac": layer_gbs / pk["hbm_gbs"]},
+        # tensor-core view of the same run: FP8 MMAs against the FP8 peak named in peak_source,
+        # the 4-bit path's bf16 MMAs against the bf16 peak
+        "tensor": {"kernel": dom, "achieved": alg["flops_" + dom] / (mean_stage[dom] / 1e3) / 1e12,
+                   "peak": tpk, "unit": "TFLOP/s",
+                   "frac": alg["flops_" + dom] / (mean_stage[dom] / 1e3) / 1e12 / tpk,
+                   "layer_achieved": alg["flops"] / (ms_step / 1e3) / 1e12,
+                   "layer_frac": alg["flops"] / (ms_step / 1e3) / 1e12 / tpk, "peak_source": tpk_src},
+        # the layer's binding roofline: the slower of streaming its algorithmic bytes at the
+        # measured HBM bandwidth and running its FLOPs at the tensor peak above
+        "binding_roofline": {"t_hbm_ms": t_hbm, "t_tensor_ms": t_tc, "bound": "hbm" if t_hbm >= t_tc else "tensor",
+                             "frac": max(t_hbm, t_tc) / ms_step},
+        "stages_ms": mean_stage,
+        "small_kernels_share": small / max(sum(mean_stage.values()), 1e-9),
+        "ms_per_step_with_stage_events": prof_ms / steps,
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    return layer, m, res, cfg
+
+
+PER_CONFIG = ("tiny", "prefill", "skewed", "int4", "mxfp4", "nvfp4")
+
+
+def run_ours(args, ws, rank, local, cfg_name):
+    import torch
+
+    import moe_synth
+    import mixture_experts_ffn_13_b200 as moe
+    from mixture_experts_ffn_13_b200 import build as moe_build
+
+    moe_build.build()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    pk, pk_src = peaks()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > 126 MB L2
+    fp8_tf = fp8_peak_tflops(dev)
+    torch.cuda.empty_cache()
+    layer, m, res, cfg = measure_layer(cfg_name, args.steps, args.warmup, ws, rank, local, pk, pk_src, fp8_tf, flush)
+    x, logits = layer["x"], layer["logits"]
+    out = torch.empty_like(x)
+    stream = torch.cuda.current_stream()
 
     # end to end through the public API with host buffers: every step copies its x and logits
     # from pinned host memory and reads its output back.  Copies run on their own streams,
@@ -370,69 +463,66 @@ def run_ours(args, ws, rank, local, cfg_name):
     t0, t1 = e2e_run(args.steps)
     torch.cuda.synchronize()
     barrier(ws)
-    e2e_ev = [(t0, t1)]
-    e2e_ms = max_over_ranks(ws, sum(a.elapsed_time(b) for a, b in e2e_ev))
+    e2e_ms = max_over_ranks(ws, t0.elapsed_time(t1))
+    e2e_value = replica_throughput(ws, cfg["T"], args.steps, e2e_ms)
 
-    r = m.route(logits)
-    counts = r["counts"].cpu().numpy()
-    alg = algorithmic(cfg, counts)
-    pk, pk_src = peaks()
-    T = cfg["T"]
-    value = replica_throughput(ws, T, args.steps, total_ms)
-    e2e_value = replica_throughput(ws, T, args.steps, e2e_ms)
-    ms_step = total_ms / args.steps
-    mean_stage = {k: v / args.steps for k, v in stage_ms.items()}
-    dom = max(("gemm_gateup", "gemm_down"), key=lambda s: mean_stage[s])
-    achieved = alg[dom] / (mean_stage[dom] / 1e3) / 1e9
+    dom = res["roofline"]["kernel"]
     tr = TRAFFIC.get(cfg_name)
     traffic = None
     if tr and tr["kernel"] == dom and tr["src_sha"] == src_sha(
             os.path.join(ROOT, "mixture_experts_ffn_13_b200", "csrc", "gemm_fp8.cu")):
-        traffic = tr["ratio"] * alg[dom]
-    layer_gbs = alg["layer"] / (ms_step / 1e3) / 1e9
-    if cfg["wfmt"] == "fp8":
-        tpk, tpk_src = 2 * pk["bf16_tflops"], f"2 x {pk_src} bf16 burst (FP8 = 2x bf16 nominal ratio)"
-    else:
-        tpk, tpk_src = pk["bf16_tflops"], f"{pk_src} bf16 burst"
+        traffic = tr["ratio"] * res["roofline"]["algorithmic_bytes"]
+    roof = dict(res["roofline"], traffic=traffic)
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "fp8_e4m3" if cfg["wfmt"] == "fp8" else "bf16", "data": "synthetic",
-        "config": {"workload": cfg["workload"], "T": T, "H": cfg["H"], "E": cfg["E"], "I": cfg["I"], "k": cfg["k"],
-                   "I_shared": cfg["Is"], "wfmt": cfg["wfmt"], "seed": cfg["seed"],
+        "metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp8_e4m3" if cfg["wfmt"] == "fp8" else "bf16", "data": "synthetic",
+        "config": {"workload": cfg["workload"], "T": cfg["T"], "H": cfg["H"], "E": cfg["E"], "I": cfg["I"],
+                   "k": cfg["k"], "I_shared": cfg["Is"], "wfmt": cfg["wfmt"], "seed": cfg["seed"],
                    "parallelism": f"replicas x{ws}", "l2": "flushed (256 MiB write) before every timed step",
-                   "experts_touched": alg["touched"], "max_tokens_per_expert": int(counts.max())},
-        "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
-                     "algorithmic_bytes": alg[dom], "peak_source": pk_src,
-                     "layer_achieved_gbs": layer_gbs, "layer_frac": layer_gbs / pk["hbm_gbs"]},
-        # tensor-core view of the same run: FP8 MMAs against 2x the measured bf16 peak (the
-        # nominal FP8/bf16 ratio), the 4-bit path's bf16 MMAs against the bf16 peak
-        "tensor": {"kernel": dom, "achieved": alg["flops_" + dom] / (mean_stage[dom] / 1e3) / 1e12,
-                   "peak": tpk, "unit": "TFLOP/s", "frac": alg["flops_" + dom] / (mean_stage[dom] / 1e3) / 1e12 / tpk,
-                   "layer_achieved": alg["flops"] / (ms_step / 1e3) / 1e12,
-                   "layer_frac": alg["flops"] / (ms_step / 1e3) / 1e12 / tpk, "peak_source": tpk_src},
-        # the layer's binding roofline: the slower of streaming its algorithmic bytes at the
-        # measured HBM bandwidth and running its FLOPs at the tensor peak above
-        "binding_roofline": {"t_hbm_ms": alg["layer"] / (pk["hbm_gbs"] * 1e9) * 1e3,
-                             "t_tensor_ms": alg["flops"] / (tpk * 1e12) * 1e3,
-                             "bound": "hbm" if alg["layer"] / pk["hbm_gbs"] >= alg["flops"] / (tpk * 1e3) else "tensor",
-                             "frac": max(alg["layer"] / (pk["hbm_gbs"] * 1e9), alg["flops"] / (tpk * 1e12)) * 1e3 / ms_step},
-        "stages_ms": mean_stage,
-        "ms_per_step_with_stage_events": prof_ms / args.steps,
+                   "experts_touched": res["experts_touched"], "max_tokens_per_expert": res["max_tokens_per_expert"]},
+        "roofline": roof,
+        "tensor": res["tensor"],
+        "binding_roofline": res["binding_roofline"],
+        "stages_ms": res["stages_ms"],
+        "small_kernels_share": res["small_kernels_share"],
+        "ms_per_step_with_stage_events": res["ms_per_step_with_stage_events"],
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": x.numel() * 2 + logits.numel() * 4,
                 "d2h_bytes_per_step": out.numel() * 2,
                 "copies": "pinned host buffers, H2D and D2H on their own streams, double-buffered "
                           "across steps (overlapping the layer)",
                 "l2": "not flushed: every step streams the expert weights (far larger than L2)"},
-        "gpu_launches": launches,
-        "clocks": clk,
+        "gpu_launches": res["gpu_launches"],
+        "clocks": res["clocks"],
+        "fp8_peak_tflops_measured": fp8_tf,
     }
+    del xd, ld, od, xh, lh, oh
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        del layer, m, flush
+        del layer, m
         torch.cuda.empty_cache()
         Lnp, _ = make_host_layer(cfg_name, dev)
         line["cpu_baseline"] = cpu_baseline(Lnp, args.cpu_seconds)
+        del Lnp
+    else:
+        del layer, m
+    # every other workload of the build, measured the same way (one GPU only: the scaling runs
+    # time the headline workload alone); each with a short oracle sample on the host cores
+    if ws == 1 and not args.no_per_config:
+        per = {}
+        for name in PER_CONFIG:
+            if name == cfg_name:
+                continue
+            torch.cuda.empty_cache()
+            lyr, mm, r_, _ = measure_layer(name, args.per_config_steps, max(3, args.warmup), ws, rank, local, pk,
+                                           pk_src, fp8_tf, flush, timing_barrier=False)
+            del lyr, mm
+            torch.cuda.empty_cache()
+            if not args.no_cpu_baseline:
+                Lnp, _ = make_host_layer(name, dev)
+                r_["cpu_baseline"] = cpu_baseline(Lnp, args.per_config_cpu_seconds)
+                del Lnp
+            per[name] = r_
+        line["per_config"] = per
     if rank == 0:
         print(json.dumps(line), flush=True)
 

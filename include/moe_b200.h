@@ -164,8 +164,11 @@ MOE_API int moe_route(moe_plan_t *plan, int32_t T, const float *logits, int32_t 
  * (held by every GPU that loads it until the process exits), so
  *   T*k + ceil(T/256)*E + 2*(E+1) <= 2^19 is required (else MOE_ERR_UNSUPPORTED, before any
  *   device work), with 1 <= k <= min(E, 32) and E <= 1024;
- *   the first call on a device looks up the array's address (cudaGetSymbolAddress, once per
- *   device, with it current) -- make that first call before any stream capture;
+ *   the first call on a device looks up the array's address (cudaGetSymbolAddress, with the
+ *   device current; again after the device's context is replaced, e.g. by cudaDeviceReset)
+ *   -- make that first call before any stream capture;
+ *   `stream` must belong to the current device (else MOE_ERR_INVALID_ARG) and the buffers must
+ *   live on it;
  *   all calls share the array: calls whose kernels may overlap on the GPU race and must be
  *   serialised by the caller.
  * Returns MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED or MOE_ERR_CUDA. */

@@ -265,9 +265,9 @@ def moe_router_topk(plan: Plan, x: torch.Tensor, w_router: torch.Tensor, out: di
 def moe_route_static(logits: torch.Tensor, k: int, out: dict | None = None, stream=None) -> dict:
     """moe_route without a plan or workspace (fixed static scratch inside the library; for
     callers that cannot allocate device memory -- see include/moe_b200.h for its limits)."""
-    T, E = logits.shape
     if logits.dtype != torch.float32 or logits.dim() != 2:
         raise ValueError("logits must be fp32 [T, E]")
+    T, E = logits.shape
     dev = logits.device
     if out is None:
         out = dict(topk_idx=torch.empty((T, k), dtype=torch.int32, device=dev),
@@ -275,9 +275,15 @@ def moe_route_static(logits: torch.Tensor, k: int, out: dict | None = None, stre
                    counts=torch.empty((E,), dtype=torch.int32, device=dev),
                    offsets=torch.empty((E + 1,), dtype=torch.int32, device=dev),
                    perm_tok=torch.empty((max(T * k, 1),), dtype=torch.int32, device=dev))
-    rc = load_library().moe_route_static(T, E, k, _ptr(logits), _ptr(out["topk_idx"]), _ptr(out["topk_w"]),
-                                         _ptr(out["counts"]), _ptr(out["offsets"]), _ptr(out["perm_tok"]),
-                                         _stream(stream))
+    if any(t.device != dev for t in out.values()):
+        raise ValueError("outputs must live on the logits' device")
+    # the library launches on the current device with that device's scratch array: make the
+    # logits' device current for the call (its default stream unless one is given)
+    with torch.cuda.device(dev):
+        s = torch.cuda.current_stream(dev) if stream is None else stream
+        rc = load_library().moe_route_static(T, E, k, _ptr(logits), _ptr(out["topk_idx"]), _ptr(out["topk_w"]),
+                                             _ptr(out["counts"]), _ptr(out["offsets"]), _ptr(out["perm_tok"]),
+                                             s.cuda_stream)
     _check(rc, "moe_route_static")
     return out
 

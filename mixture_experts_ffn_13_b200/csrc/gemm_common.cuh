@@ -80,6 +80,30 @@ __device__ __forceinline__ int total_tiles(const GemmArgs &a, int BN, int *tot0,
     return *tot0 + tot1;
 }
 
+// Down GEMM epilogue, one output value v of permuted row `row` and feature n: either the
+// stored y (plain mode) or, with the combine fused, p_hat(row) * v added into the fp32
+// accumulator row of the row's token (atomic add in L2; the summation order of a token's k+1
+// contributions is therefore unspecified).  Lanes of a warp hold consecutive n, so each add
+// instruction of a warp covers 128 contiguous bytes.
+__device__ __forceinline__ void down_out(const GemmSeg &sg, const GemmArgs &a, int row, int n, float v)
+{
+    if (!sg.accum) {
+        static_cast<float *>(sg.out)[(size_t)row * sg.N + n] = v;
+        return;
+    }
+    int t = row;
+    float w = 1.0f;
+    if (sg.tok) {
+        t = __ldg(sg.tok + row);
+        w = __ldg(sg.rw + row);
+    }
+    if (a.check && (unsigned)t >= (unsigned)a.T) {
+        atomicCAS(a.check, 0, MOE_ERR_BOUNDS);
+        return;
+    }
+    atomicAdd(sg.accum + (size_t)t * sg.N + n, w * v);
+}
+
 // silu(g) * u = g / (1 + e^-g) * u with the hardware exponential and approximate division
 // (a few ulp in fp32, far below the accumulation's own rounding).  For g below about -88 the
 // denominator overflows to infinity and the approximate quotient is the exact limit 0.

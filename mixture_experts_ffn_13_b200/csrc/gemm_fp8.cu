@@ -129,6 +129,7 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, MODE, EW>::THREADS, 1)
     uint64_t *acce = accf + C::NSLOT;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(acce + C::NSLOT);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+    uint64_t *drain_bar = reinterpret_cast<uint64_t *>(tmem_holder + 2);  // MMA drain on exit
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -140,6 +141,7 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, MODE, EW>::THREADS, 1)
             mbar_init(&accf[s], 1);
             mbar_init(&acce[s], C::EPI_WARPS);
         }
+        mbar_init(drain_bar, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -169,6 +171,7 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, MODE, EW>::THREADS, 1)
     const int total = total_tiles(args, BN, &tot0, RT);
     int *status = args.status;
     const uint64_t tmo = args.timeout_ns;
+    uint32_t issued = 0;  // producer: stages whose copies have been issued
 
     if (warp == 0) {
         // ------------------------------ TMA producer ------------------------------
@@ -201,6 +204,7 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, MODE, EW>::THREADS, 1)
                 }
                 if constexpr (C::WIDE) ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) goto done;
+                issued = it + 1;
                 uint8_t *st = smem + s * C::STAGE_BYTES;
                 const int x = kc * kKC;
                 if constexpr (!C::WIDE) {
@@ -428,12 +432,10 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, MODE, EW>::THREADS, 1)
 #pragma unroll
                 for (int c = 0; c < C::CPW; ++c) {
                     if (cbase + c < tl.nrows) {
-                        float v;
                         if constexpr (C::PAIR)
-                            v = silu_mul(acc0[c], acc1[c]);
+                            out[(size_t)(tl.row0 + cbase + c) * sg.N + n] = silu_mul(acc0[c], acc1[c]);
                         else
-                            v = acc0[c];
-                        out[(size_t)(tl.row0 + cbase + c) * sg.N + n] = v;
+                            down_out(sg, args, tl.row0 + cbase + c, n, acc0[c]);
                     }
                 }
             }
@@ -446,6 +448,12 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, MODE, EW>::THREADS, 1)
         }
     }
 done:
+    // own asynchronous work first: the producer's copies of the last NS stages have landed and
+    // the MMAs this CTA issued have completed (both already true unless a role gave up early)
+    if (warp == 0 && lane == 0)
+        for (uint32_t j = issued > (uint32_t)C::NS ? issued - C::NS : 0; j < issued; ++j)
+            mbar_wait_drain(&full[j % C::NS], (j / C::NS) & 1, tmo);
+    if (warp == 1 && lane == 0) mma_drain(drain_bar, tmo);
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {

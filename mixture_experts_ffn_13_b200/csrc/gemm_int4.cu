@@ -182,6 +182,7 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
     uint64_t *acce = accf + C::NSLOT;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(acce + C::NSLOT);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+    uint64_t *drain_bar = reinterpret_cast<uint64_t *>(tmem_holder + 2);  // MMA drain on exit
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -201,6 +202,7 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
             mbar_init(&accf[s], 1);
             mbar_init(&acce[s], C::EW);
         }
+        mbar_init(drain_bar, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -222,6 +224,7 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
     const int total = total_tiles(args, BN, &tot0);
     int *status = args.status;
     const uint64_t tmo = args.timeout_ns;
+    uint32_t issued_r = 0, issued_b = 0;  // producer: raw and activation stages issued
 
     if (warp == 0) {
         // --------------------- raw weight + activation producer ---------------------
@@ -257,6 +260,7 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
                         const int s = rt % C::NR;
                         if (!mbar_wait(&rempty[s], ((rt / C::NR) & 1) ^ 1, abort_flag, status, tmo)) goto done;
                         uint8_t *rs = raw + s * C::NA * C::RAW_BYTES;
+                        issued_r = rt + 1;
                         mbar_arrive_expect_tx(&rfull[s], C::NA * C::RAW_BYTES);
                         const int x = (kc / kSubs) * (kRawKE / 2);
                         tma_load_2d_hint(rs, &maps.a0[tl.seg], &rfull[s], x, tl.wrow, pol_w);
@@ -265,6 +269,7 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
                     }
                     const int b = it % C::NB;
                     if (!mbar_wait(&bempty[b], ((it / C::NB) & 1) ^ 1, abort_flag, status, tmo)) goto done;
+                    issued_b = it + 1;
                     mbar_arrive_expect_tx(&bfull[b], C::B_BYTES);
                     tma_load_2d_hint(bst + b * C::B_BYTES, &maps.b[tl.seg], &bfull[b], kc * kKE, tl.row0, pol_x);
                 }
@@ -485,7 +490,7 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
                                 static_cast<__nv_bfloat16 *>(sg.out)[o] =
                                     __float2bfloat16_rn(NV ? silu_mul(v[c] * t0, u[c] * t1) : silu_mul(v[c], u[c]));
                             else
-                                static_cast<float *>(sg.out)[o] = NV ? v[c] * t0 : v[c];
+                                down_out(sg, args, tl.row0 + c0 + c, n, NV ? v[c] * t0 : v[c]);
                         }
                     }
                 }
@@ -543,16 +548,25 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
 #pragma unroll
             for (int c = 0; c < C::CPW; ++c) {
                 if (cbase + c < tl.nrows) {
-                    const size_t o = (size_t)(tl.row0 + cbase + c) * sg.N + n;
                     if constexpr (GATEUP)
-                        static_cast<__nv_bfloat16 *>(sg.out)[o] = __float2bfloat16_rn(silu_mul(acc0[c], acc1[c]));
+                        static_cast<__nv_bfloat16 *>(sg.out)[(size_t)(tl.row0 + cbase + c) * sg.N + n] =
+                            __float2bfloat16_rn(silu_mul(acc0[c], acc1[c]));
                     else
-                        static_cast<float *>(sg.out)[o] = acc0[c];
+                        down_out(sg, args, tl.row0 + cbase + c, n, acc0[c]);
                 }
             }
         }
     }
 done:
+    // own asynchronous work first: the producer's last copies of both rings have landed and
+    // the MMAs this CTA issued have completed (both already true unless a role gave up early)
+    if (warp == 0 && lane == 0) {
+        for (uint32_t j = issued_r > (uint32_t)C::NR ? issued_r - C::NR : 0; j < issued_r; ++j)
+            mbar_wait_drain(&rfull[j % C::NR], (j / C::NR) & 1, tmo);
+        for (uint32_t j = issued_b > (uint32_t)C::NB ? issued_b - C::NB : 0; j < issued_b; ++j)
+            mbar_wait_drain(&bfull[j % C::NB], (j / C::NB) & 1, tmo);
+    }
+    if (warp == 1 && lane == 0) mma_drain(drain_bar, tmo);
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {

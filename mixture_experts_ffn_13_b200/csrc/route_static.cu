@@ -14,15 +14,20 @@
 // Properties a caller must know:
 //  * Capacity: T*k + ceil(T/256)*E + 2*(E+1) <= kStaticScratchInts (2^19 int32 = 2 MiB);
 //    larger problems are rejected with MOE_ERR_UNSUPPORTED before any device work.
-//  * The first call on a device looks up the array's device address with
-//    cudaGetSymbolAddress (once per device, under a lock, with that device current).  Make that
-//    first call before any stream capture.
+//  * The first call in a CUDA context (normally: on a device) looks up the array's device
+//    address with cudaGetSymbolAddress (under a lock, with that device current) and keeps it
+//    for the context; a call in a new context of the device (after cudaDeviceReset, say) looks
+//    it up again.  Make the first call on each device before any stream capture.
+//  * `stream` must belong to the current device (its context); a stream of another device is
+//    rejected with MOE_ERR_INVALID_ARG, and the buffers must live on the current device too.
 //  * Every call on a device shares the one array, and it keeps the previous call's contents.
 //    Nothing in it needs to start at zero: each launch writes every entry it later reads.  Two
 //    calls whose kernels overlap on the GPU (different streams, no ordering between them)
 //    race on the array and give undefined results; serialise them.
 //  * No cudaMalloc, cudaFree or allocating library routine is called.
 #include "moe_internal.h"
+
+#include <cudaTypedefs.h>
 
 #include <mutex>
 
@@ -35,25 +40,62 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) int32_t g_route_scratch[kStaticScratchInts];
 
-std::mutex g_scratch_mu;
-int32_t *g_scratch_ptr[kMaxDevices] = {};
+// Driver entry points (through the runtime, so the library links only libcudart).
+PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;
+PFN_cuCtxGetId_v12000 g_ctx_id = nullptr;
+PFN_cuStreamGetCtx_v9020 g_stream_ctx = nullptr;
+std::once_flag g_driver_once;
 
-// Device address of g_route_scratch on the current device (looked up once per device).
-cudaError_t scratch_for_current_device(int32_t **out)
+void load_driver()
 {
+    auto get = [](const char *name, unsigned ver) -> void * {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion(name, &fn, ver, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return fn;
+    };
+    g_ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(get("cuCtxGetCurrent", 4000));
+    g_ctx_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(get("cuCtxGetId", 12000));
+    g_stream_ctx = reinterpret_cast<PFN_cuStreamGetCtx_v9020>(get("cuStreamGetCtx", 9020));
+}
+
+struct ScratchSlot {
+    unsigned long long ctx_id;  // context the address was looked up in (0: none yet)
+    int32_t *ptr;
+};
+std::mutex g_scratch_mu;
+ScratchSlot g_scratch[kMaxDevices] = {};
+
+// Device address of g_route_scratch in the current context, after checking that `stream`
+// belongs to that context.  Looked up once per context.
+int scratch_for_current_context(cudaStream_t stream, int32_t **out)
+{
+    std::call_once(g_driver_once, load_driver);
+    if (!g_ctx_current || !g_ctx_id || !g_stream_ctx) return MOE_ERR_CUDA;
     int dev = -1;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_ptr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_route_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_ptr[dev] = static_cast<int32_t *>(p);
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
+    CUcontext ctx = nullptr, sctx = nullptr;
+    unsigned long long id = 0;
+    if (g_ctx_current(&ctx) != CUDA_SUCCESS) return MOE_ERR_CUDA;
+    if (!ctx) {  // no context yet on this thread: cudaSetDevice makes the primary context current
+        if (cudaSetDevice(dev) != cudaSuccess || g_ctx_current(&ctx) != CUDA_SUCCESS || !ctx) return MOE_ERR_CUDA;
     }
-    *out = g_scratch_ptr[dev];
-    return cudaSuccess;
+    if (g_ctx_id(ctx, &id) != CUDA_SUCCESS) return MOE_ERR_CUDA;
+    if (g_stream_ctx(reinterpret_cast<CUstream>(stream), &sctx) != CUDA_SUCCESS) return MOE_ERR_INVALID_ARG;
+    if (sctx != ctx) return MOE_ERR_INVALID_ARG;  // a stream of another device or context
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    ScratchSlot &slot = g_scratch[dev];
+    if (slot.ctx_id != id || !slot.ptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess) return MOE_ERR_CUDA;
+        slot.ptr = static_cast<int32_t *>(p);
+        slot.ctx_id = id;
+    }
+    *out = slot.ptr;
+    return MOE_OK;
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
@@ -79,9 +121,10 @@ extern "C" int moe_route_static(int32_t T, int32_t E, int32_t k, const float *lo
         !aligned16(offsets) || !aligned16(perm_tok))
         return MOE_ERR_INVALID_ARG;
 
+    cudaStream_t s = (cudaStream_t)stream;
     int32_t *scratch = nullptr;
-    cudaError_t e = scratch_for_current_device(&scratch);
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    const int rc = scratch_for_current_context(s, &scratch);
+    if (rc != MOE_OK) return rc;
 
     RouteBufs b;
     b.topk_idx = topk_idx;
@@ -93,10 +136,10 @@ extern "C" int moe_route_static(int32_t T, int32_t E, int32_t k, const float *lo
     b.chunk_hist = scratch + A;
     b.ttile_a = b.chunk_hist + nch * (size_t)E;
     b.ttile_b = b.ttile_a + (E + 1);
-    cudaStream_t s = (cudaStream_t)stream;
+    b.rowscale = nullptr;
     const long avg = ((long)T * k + E - 1) / E;
     const int bn = avg > 48 ? 64 : 32;
-    e = launch_route(logits, T, E, k, topk_idx, topk_w, s);
+    cudaError_t e = launch_route(logits, T, E, k, topk_idx, topk_w, s);
     if (e == cudaSuccess) e = launch_permute(b, T, E, k, bn, bn, s);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

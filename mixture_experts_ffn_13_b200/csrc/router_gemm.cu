@@ -56,6 +56,7 @@ __global__ void __launch_bounds__(RCfg<BN>::THREADS, 1)
     uint64_t *acce = accf + 2;       // 2
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(acce + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+    uint64_t *drain_bar = reinterpret_cast<uint64_t *>(tmem_holder + 2);  // MMA drain on exit
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::NS; ++s) {
@@ -66,6 +67,7 @@ __global__ void __launch_bounds__(RCfg<BN>::THREADS, 1)
             mbar_init(&accf[s], 1);
             mbar_init(&acce[s], 4);
         }
+        mbar_init(drain_bar, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -89,6 +91,7 @@ __global__ void __launch_bounds__(RCfg<BN>::THREADS, 1)
     const int ntt = (a.T + BN - 1) / BN;
     const int total = net * ntt;
     const int nkc = a.H / kRKE;
+    uint32_t issued = 0;  // producer: stages whose copies have been issued
     if (warp == 0) {
         if (lane == 0) {
             const uint64_t pol_x = l2_policy_evict_last();
@@ -99,6 +102,7 @@ __global__ void __launch_bounds__(RCfg<BN>::THREADS, 1)
                     const int s = it % C::NS;
                     if (!mbar_wait(&empty[s], ((it / C::NS) & 1) ^ 1, abort_flag, a.status, a.timeout_ns)) goto done;
                     uint8_t *st = smem + s * C::STAGE;
+                    issued = it + 1;
                     mbar_arrive_expect_tx(&full[s], C::STAGE);
                     tma_load_2d(st, &map_w, &full[s], kc * kRKE, et * kTileM);
                     tma_load_2d_hint(st + C::A_BYTES, &map_x, &full[s], kc * kRKE, tt * BN, pol_x);
@@ -156,6 +160,11 @@ __global__ void __launch_bounds__(RCfg<BN>::THREADS, 1)
         }
     }
 done:
+    // own asynchronous work first (already finished unless a role gave up early)
+    if (warp == 0 && lane == 0)
+        for (uint32_t j = issued > (uint32_t)C::NS ? issued - C::NS : 0; j < issued; ++j)
+            mbar_wait_drain(&full[j % C::NS], (j / C::NS) & 1, a.timeout_ns);
+    if (warp == 1 && lane == 0) mma_drain(drain_bar, a.timeout_ns);
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -201,6 +210,7 @@ __global__ void __launch_bounds__(SCfg<BN>::THREADS, 1)
     uint64_t *redbar = accf + 1;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(redbar + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+    uint64_t *drain_bar = reinterpret_cast<uint64_t *>(tmem_holder + 2);  // MMA drain on exit
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
     if (threadIdx.x == 0) {
@@ -209,6 +219,7 @@ __global__ void __launch_bounds__(SCfg<BN>::THREADS, 1)
             mbar_init(&empty[s], 1);
         }
         mbar_init(accf, 1);
+        mbar_init(drain_bar, 1);
         mbar_init(redbar, 128 * (S - 1));  // every epilogue thread of CTAs 1..S-1
         *abort_flag = 0;
         fence_mbar_init();
@@ -234,6 +245,7 @@ __global__ void __launch_bounds__(SCfg<BN>::THREADS, 1)
     const int et = tile % net, tt = tile / net;
     const int nkc = a.H / kRKE;
     const int k0 = (int)(((long)nkc * rank) / S), k1 = (int)(((long)nkc * (rank + 1)) / S);
+    uint32_t issued = 0;  // producer: stages whose copies have been issued
     if (warp == 0) {
         if (lane == 0) {
             const uint64_t pol_x = l2_policy_evict_last();
@@ -241,6 +253,7 @@ __global__ void __launch_bounds__(SCfg<BN>::THREADS, 1)
                 const int s = it % C::NS;
                 if (!mbar_wait(&empty[s], ((it / C::NS) & 1) ^ 1, abort_flag, a.status, a.timeout_ns)) break;
                 uint8_t *st = smem + s * C::STAGE;
+                issued = it + 1;
                 mbar_arrive_expect_tx(&full[s], C::STAGE);
                 tma_load_2d(st, &map_w, &full[s], kc * kRKE, et * kTileM);
                 tma_load_2d_hint(st + C::A_BYTES, &map_x, &full[s], kc * kRKE, tt * BN, pol_x);
@@ -304,6 +317,11 @@ __global__ void __launch_bounds__(SCfg<BN>::THREADS, 1)
             }
         }
     }
+    // own asynchronous work first (already finished unless a role gave up early)
+    if (warp == 0 && lane == 0)
+        for (uint32_t j = issued > (uint32_t)C::NS ? issued - C::NS : 0; j < issued; ++j)
+            mbar_wait_drain(&full[j % C::NS], (j / C::NS) & 1, a.timeout_ns);
+    if (warp == 1 && lane == 0) mma_drain(drain_bar, a.timeout_ns);
     tc_fence_before();
     __syncthreads();
     cluster_sync();  // CTA 0 stays resident until every partial has been stored into it

@@ -83,6 +83,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     return true;
 }
 
+// Bounded wait that ignores the abort flag: on the way out of a kernel, a thread waits for its
+// own asynchronous work (TMA copies into shared memory, MMAs into tensor memory) to finish
+// before the CTA releases that memory.  Gives up after `timeout_ns` (what is still in flight
+// then is left to the hardware).
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity, uint64_t timeout_ns)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    uint32_t n = 0;
+    while (!mbar_try_wait(bar, parity))
+        if ((++n & 255u) == 0 && globaltimer_ns() - t0 > timeout_ns) return false;
+    return true;
+}
+
 // ---------------------------------------------------------------------------------------
 // clusters: rank, distributed shared memory, cluster-scope barriers
 // ---------------------------------------------------------------------------------------
@@ -347,6 +361,72 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar)
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                      smem_u32(bar))
                  : "memory");
+}
+
+// ---- CTA pairs (cta_group::2): one MMA of M = 256 over the tensor cores of two SMs ----------
+// Each CTA of a 2-CTA cluster holds half of A (M/2 rows) and half of B (N/2 rows) in its own
+// shared memory at the same offsets, and half of D (its M/2 rows, all N columns) in its own
+// tensor memory.  The even CTA of the pair issues the MMAs and commits; both CTAs allocate
+// tensor memory with the pair form (same warp, same destination address).
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t *dst, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)),
+                 "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair()
+{
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// D[tmem of both CTAs] (+)= A[smem of both] * B[smem of both]^T, FP8, issued by the even CTA.
+__device__ __forceinline__ void mma_f8_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Same for 16-bit operands.
+__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive once on the mbarrier at the same shared-memory offset as `bar` in every CTA of the
+// cluster named by `cta_mask` when all pair MMAs this thread issued so far have completed.
+__device__ __forceinline__ void mma_commit_pair(uint64_t *bar, uint16_t cta_mask)
+{
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"(cta_mask)
+        : "memory");
+}
+
+// Exit path of the MMA-issuing thread: wait (bounded) until every MMA it issued has completed,
+// through a commit to `bar`, an mbarrier initialised with one arrival and used for nothing else.
+__device__ __forceinline__ void mma_drain(uint64_t *bar, uint64_t timeout_ns)
+{
+    mma_commit(bar);
+    mbar_wait_drain(bar, 0, timeout_ns);
 }
 
 // Warp-wide load of 16 consecutive fp32 columns of this warp's 32 TMEM lanes.

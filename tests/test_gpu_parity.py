@@ -28,15 +28,45 @@ def _bf16_to_f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
+# Tokens allowed to have outputs that pass only through the envelope of equally valid outputs
+# (an h code on a rounding boundary, reading R10a), as a fraction of the tokens a check compares.
+# One such code moves every output of its token a little, so the count is per token.
+ENV_ONLY_MAX_TOKEN_FRAC = 0.05
+
+
 def check_out(got_bf16: torch.Tensor, want: np.ndarray, what: str, amb: np.ndarray | None = None):
     """Per-element bound ATOL + RTOL*|oracle|, widened only by the oracle's envelope of equally
-    valid outputs where an h value sits on an FP8/bf16 rounding midpoint (zero elsewhere)."""
+    valid outputs where an h value may round either way (zero elsewhere).  Reports how many
+    elements needed the envelope (outside the plain bound, inside the widened one) and bounds
+    that count."""
     got = _bf16_to_f64(got_bf16)
     err = np.abs(got - want)
-    bound = ATOL + RTOL * np.abs(want) + (amb if amb is not None else 0.0)
+    base = ATOL + RTOL * np.abs(want)
+    bound = base + (amb if amb is not None else 0.0)
     bad = err > bound
+    env = (err > base) & ~bad
+    env_only = int(env.sum())
+    env_tokens = int(env.reshape(env.shape[0], -1).any(axis=1).sum())
+    print(f"{what}: envelope-only elements: {env_only}/{err.size} in {env_tokens}/{env.shape[0]} tokens; "
+          f"max err/bound {(err / base).max():.3f}")
     assert not bad.any(), (f"{what}: {bad.sum()} of {bad.size} outside tolerance; "
                            f"worst excess {(err - bound).max():.3e} at {np.unravel_index(np.argmax(err - bound), err.shape)}")
+    assert env_tokens <= max(1, ENV_ONLY_MAX_TOKEN_FRAC * env.shape[0]), \
+        f"{what}: {env_tokens} tokens have outputs that pass only through the envelope"
+    return env_only
+
+
+def assert_same_up_to_sum_order(a: torch.Tensor, b: torch.Tensor, what: str = "repeat"):
+    """Two results of the same call on the same inputs.  The fused combine adds each token's k+1
+    terms into fp32 in whatever order the additions reach L2 (reading R12: the summation order is
+    free), so a repeat may round differently -- by at most one bf16 step after the final
+    rounding, since order effects in fp32 are ~1e-7 relative and a bf16 step is 2^-8."""
+    if torch.equal(a, b):
+        return
+    fa, fb = a.float(), b.float()
+    ulp = torch.ldexp(torch.ones_like(fa), torch.frexp(torch.maximum(fa.abs(), fb.abs()))[1] - 8)
+    diff = (fa - fb).abs()
+    assert (diff <= ulp).all(), f"{what}: {(diff > ulp).sum().item()} elements differ by more than one bf16 step"
 
 
 def check_route(plan, ws, logits: torch.Tensor, k: int):
@@ -151,10 +181,10 @@ def test_layer_fp8_small(cfg):
     assert moe.moe_get_status(m.plan) == 0
     want, _, amb = oracle.layer(moe_synth.to_numpy(layer), ambiguity=True)
     check_out(out, want, "layer", amb)
-    # a second call on the same workspace gives the same bits
+    # a second call on the same workspace gives the same result (up to the combine's sum order)
     out2 = m(layer["x"], layer["logits"])
     torch.cuda.synchronize()
-    assert torch.equal(out, out2)
+    assert_same_up_to_sum_order(out, out2)
 
 
 def test_layer_fp8_variable_T_within_plan():
@@ -191,7 +221,7 @@ def test_layer_int4_small(cfg):
     check_out(out, want, "int4 layer", amb)
     out2 = m(layer["x"], layer["logits"])
     torch.cuda.synchronize()
-    assert torch.equal(out, out2)
+    assert_same_up_to_sum_order(out, out2)
 
 
 SMALL_FP4 = [
@@ -217,22 +247,48 @@ def test_layer_fp4_small(cfg, fmt):
     check_out(out, want, f"{fmt} layer", amb)
     out2 = m(layer["x"], layer["logits"])
     torch.cuda.synchronize()
-    assert torch.equal(out, out2)
+    assert_same_up_to_sum_order(out, out2)
 
 
-def _sampled_parity(name, n_sample=12):
+def stratified_tokens(logits: np.ndarray, k: int, cap: int = 768, seed: int = 99) -> np.ndarray:
+    """Tokens to check at full size, chosen from the oracle's own routing of the logits: the
+    token owning the last row of every non-empty expert group (the partial last token tile),
+    then the first row of every group, then the rows on either side of every 32-row boundary
+    inside a group (every token-tile width the kernels use is a multiple of 32), then tokens
+    0 and T-1, then random tokens -- in that priority order, up to `cap` distinct tokens."""
+    T, E = logits.shape
+    idx, _ = oracle.route(logits, k)
+    _, offsets, perm, _ = oracle.permute(idx, E)
+    picks = []
+    nonempty = [e for e in range(E) if offsets[e + 1] > offsets[e]]
+    picks += [perm[offsets[e + 1] - 1] for e in nonempty]
+    picks += [perm[offsets[e]] for e in nonempty]
+    for e in nonempty:
+        for r in range(offsets[e] + 32, offsets[e + 1], 32):
+            picks += [perm[r - 1], perm[r]]
+    picks += [0, T - 1]
+    picks += list(np.random.default_rng(seed).permutation(T))
+    seen, sel = set(), []
+    for t in picks:
+        if int(t) not in seen:
+            seen.add(int(t))
+            sel.append(int(t))
+        if len(sel) == cap:
+            break
+    return np.sort(np.array(sel, dtype=np.int32))
+
+
+def _sampled_parity(name):
     cfg = moe_synth.CONFIGS[name]
     layer = moe_synth.make_layer(name, device="cuda")
     m = moe.MoELayer(layer)
     out = m(layer["x"], layer["logits"])
     assert moe.moe_get_status(m.plan) == 0
     torch.cuda.synchronize()
-    T = cfg["T"]
-    rng = np.random.default_rng(99)
-    sel = np.unique(np.concatenate([[0, T - 1], rng.choice(T, n_sample, replace=False)])).astype(np.int32)
     L = moe_synth.to_numpy(layer)
+    sel = stratified_tokens(L["logits"], cfg["k"])
     want, _, amb = oracle.layer(L, sel, ambiguity=True)
-    check_out(out[torch.from_numpy(sel).long().cuda()], want, name, amb)
+    check_out(out[torch.from_numpy(sel).long().cuda()], want, f"{name} ({sel.size} tokens)", amb)
     # the routing of the whole batch is bit-exact as well
     check_route(m.plan, m.workspace, layer["logits"], cfg["k"])
 
@@ -245,7 +301,8 @@ def test_layer_configs_sampled(name):
 def test_forward_replays_in_cuda_graph():
     """moe_forward is stream-ordered and allocates nothing, so it can be captured in a CUDA
     graph (its programmatic-dependent launches become graph edges); replays match the eager
-    call bit for bit, also after new inputs are copied into the captured buffers."""
+    call (up to the combine's fp32 summation order), also after new inputs are copied into the
+    captured buffers."""
     cfg = dict(T=96, H=512, E=16, I=256, k=4, Is=128, seed=30, bias=None, wfmt="fp8")
     layer = moe_synth.make_layer(cfg, device="cuda")
     m = moe.MoELayer(layer)
@@ -260,7 +317,7 @@ def test_forward_replays_in_cuda_graph():
         moe.moe_forward(m.plan, x, logits, m.weights, m.workspace, out=out)
     g.replay()
     torch.cuda.synchronize()
-    assert torch.equal(out, ref)
+    assert_same_up_to_sum_order(out, ref, "graph replay")
     # new inputs through the same captured buffers
     layer2 = moe_synth.make_layer(dict(cfg, seed=31), device="cuda")
     x.copy_(layer2["x"])
