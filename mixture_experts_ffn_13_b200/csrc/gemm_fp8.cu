@@ -428,16 +428,18 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, MODE, EW>::THREADS, 1)
                     const float v = is_up ? silu_mul(other, mine) : silu_mul(mine, other);
                     if (cbase + c + (odd ? 1 : 0) < tl.nrows) orow[(size_t)c * sg.N] = v;
                 }
-            } else {
+            } else if constexpr (C::PAIR) {
 #pragma unroll
-                for (int c = 0; c < C::CPW; ++c) {
-                    if (cbase + c < tl.nrows) {
-                        if constexpr (C::PAIR)
-                            out[(size_t)(tl.row0 + cbase + c) * sg.N + n] = silu_mul(acc0[c], acc1[c]);
-                        else
-                            down_out(sg, args, tl.row0 + cbase + c, n, acc0[c]);
-                    }
-                }
+                for (int c = 0; c < C::CPW; ++c)
+                    if (cbase + c < tl.nrows) out[(size_t)(tl.row0 + cbase + c) * sg.N + n] = silu_mul(acc0[c], acc1[c]);
+            } else {
+                constexpr int NREG = (C::CPW + 31) / 32;
+                int ctok[NREG];
+                float cw[NREG];
+                if (sg.accum) combine_cols(sg, tl.row0 + cbase, tl.nrows - cbase, lane, ctok, cw);
+#pragma unroll
+                for (int c = 0; c < C::CPW; ++c)
+                    if (cbase + c < tl.nrows) down_out(sg, args, tl.row0 + cbase + c, c, n, acc0[c], ctok, cw);
             }
             if constexpr (kSxDouble) {
                 if (wn < total) store_sx(tn, sxbuf + ((ti + 1) & 1) * (BN * kMaxKb));

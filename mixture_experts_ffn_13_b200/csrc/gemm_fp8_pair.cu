@@ -346,9 +346,13 @@ __global__ void __launch_bounds__(PairCfg<GATEUP>::THREADS, 1)
                     if (cbase + c + (odd ? 1 : 0) < tl.nrows) orow[(size_t)c * sg.N] = v;
                 }
             } else {
+                constexpr int NREG = C::CPW / 32;
+                int ctok[NREG];
+                float cw[NREG];
+                if (sg.accum) combine_cols(sg, tl.row0 + cbase, tl.nrows - cbase, lane, ctok, cw);
 #pragma unroll
                 for (int c = 0; c < C::CPW; ++c)
-                    if (cbase + c < tl.nrows) down_out(sg, args, tl.row0 + cbase + c, n, acc[c]);
+                    if (cbase + c < tl.nrows) down_out(sg, args, tl.row0 + cbase + c, c, n, acc[c], ctok, cw);
             }
             if (wn < total) store_sx(tn, sxbuf + ((ti + 1) & 1) * (BN * kMaxKb));
             epi_sync(32 * EW);

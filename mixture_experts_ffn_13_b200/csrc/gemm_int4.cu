@@ -473,6 +473,10 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
                 tc_fence_after();
                 const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + C::A_TMEM + slot * C::SLOT_COLS;
                 const int n = tl.nt * kTileM + r;
+                constexpr int NREG = (BN + 31) / 32;
+                int ctok[NREG];
+                float cw[NREG];
+                if (!GATEUP && sg.accum) combine_cols(sg, tl.row0, tl.nrows, lane, ctok, cw);
                 for (int c0 = 0; c0 < BN && c0 < tl.nrows; c0 += 16) {  // warp-uniform bounds
                     float v[16], u[16];
                     tmem_ld16(tb + c0, v);
@@ -490,7 +494,7 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
                                 static_cast<__nv_bfloat16 *>(sg.out)[o] =
                                     __float2bfloat16_rn(NV ? silu_mul(v[c] * t0, u[c] * t1) : silu_mul(v[c], u[c]));
                             else
-                                down_out(sg, args, tl.row0 + c0 + c, n, NV ? v[c] * t0 : v[c]);
+                                down_out(sg, args, tl.row0 + c0 + c, c0 + c, n, NV ? v[c] * t0 : v[c], ctok, cw);
                         }
                     }
                 }
@@ -545,6 +549,10 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
                 if (lane == 0) mbar_arrive(&acce[slot]);
             }
             const int n = tl.nt * kTileM + r;
+            constexpr int NREG = (C::CPW + 31) / 32;
+            int ctok[NREG];
+            float cw[NREG];
+            if (!GATEUP && sg.accum) combine_cols(sg, tl.row0 + cbase, tl.nrows - cbase, lane, ctok, cw);
 #pragma unroll
             for (int c = 0; c < C::CPW; ++c) {
                 if (cbase + c < tl.nrows) {
@@ -552,7 +560,7 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
                         static_cast<__nv_bfloat16 *>(sg.out)[(size_t)(tl.row0 + cbase + c) * sg.N + n] =
                             __float2bfloat16_rn(silu_mul(acc0[c], acc1[c]));
                     else
-                        down_out(sg, args, tl.row0 + cbase + c, n, acc0[c]);
+                        down_out(sg, args, tl.row0 + cbase + c, c, n, acc0[c], ctok, cw);
                 }
             }
         }

@@ -25,7 +25,7 @@ __global__ void bounded_wait_kernel(int *status, uint64_t timeout_ns)
 // kernels do per stage, and records the cycles spent issuing and until the last MMA completed.
 enum { kRateF16SS = 0, kRateF16TS = 1, kRateF8SS = 2, kRateF16Pair = 3, kRateF8Pair = 4 };
 constexpr int kRateA = 128 * 128, kRateB = 256 * 128;
-constexpr int kRateSmem = 1024 + kRateA + kRateB + 64;  // + done, step[2], holder, abort flag
+constexpr int kRateSmem = 1024 + kRateA + kRateB + 64;  // + done, step[2], fin0, holder, abort flag
 
 template <int FORM>
 __global__ void __launch_bounds__(128, 1)
@@ -39,7 +39,8 @@ __global__ void __launch_bounds__(128, 1)
     uint8_t *A = smem, *B = smem + kRateA;
     uint64_t *done = reinterpret_cast<uint64_t *>(smem + kRateA + kRateB);
     uint64_t *step = done + 1;  // two barriers: step[0], step[1]
-    uint32_t *holder = reinterpret_cast<uint32_t *>(step + 2);
+    uint64_t *fin0 = step + 2;  // completion of the second issuing thread (two-issuer variant)
+    uint32_t *holder = reinterpret_cast<uint32_t *>(fin0 + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(holder + 1);
     const int warp = threadIdx.x >> 5;
     const uint32_t rank = kPair ? cluster_ctarank() : 0;
@@ -49,6 +50,7 @@ __global__ void __launch_bounds__(128, 1)
         mbar_init(done, 1);
         mbar_init(&step[0], 1);
         mbar_init(&step[1], 1);
+        mbar_init(fin0, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -69,7 +71,39 @@ __global__ void __launch_bounds__(128, 1)
         __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *holder;
-    if (threadIdx.x == 0 && rank == 0) {
+    if ((flags & 4) && !kPair) {
+        // two issuing threads in different warps, each with its own accumulator, commit
+        // barrier and half of the MMAs: does one thread's commit hold up the other's issue?
+        __shared__ long long t_end[2];
+        const int who = threadIdx.x == 0 ? 0 : (threadIdx.x == 64 ? 1 : -1);
+        const uint32_t idesc = instr_desc(128, N, kF8 ? 0 : 1, kF8 ? 0 : 1);
+        const uint64_t da = smem_desc_sw128(A), db = smem_desc_sw128(B);
+        __syncthreads();
+        const long long t0 = clock64();
+        if (who >= 0) {
+            const uint32_t d = tmem + (who ? 256 : 0);
+            uint64_t *b = &step[who];
+            const int per = commit_every > 0 ? commit_every : count / 2;
+            for (int i = 0; i < count / 2;) {
+                for (int j = 0; j < per && i < count / 2; ++j, ++i) {
+                    const uint32_t acc = i > 0 ? 1u : 0u;
+                    if constexpr (FORM == kRateF16SS) mma_bf16(d, da, db, idesc, acc);
+                    if constexpr (FORM == kRateF16TS) mma_bf16_ts(d, tmem + 384, db, idesc, acc);
+                    if constexpr (FORM == kRateF8SS) mma_f8(d, da, db, idesc, acc);
+                }
+                if (commit_every > 0) mma_commit(b);
+            }
+            uint64_t *fin = who ? done : fin0;
+            mma_commit(fin);
+            mbar_wait(fin, 0, abort_flag, status, timeout_ns);
+            t_end[who] = clock64();
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            cycles[0] = (t_end[0] > t_end[1] ? t_end[0] : t_end[1]) - t0;
+            cycles[1] = cycles[0];
+        }
+    } else if (threadIdx.x == 0 && rank == 0) {
         const uint32_t idesc = instr_desc(kPair ? 256 : 128, N, kF8 ? 0 : 1, kF8 ? 0 : 1);
         const uint64_t da = smem_desc_sw128(A), db = smem_desc_sw128(B);
         const long long t0 = clock64();
@@ -77,16 +111,19 @@ __global__ void __launch_bounds__(128, 1)
         // the TS form's A then sits at column 384) every commit group; bit 1: alternate the
         // commit between two mbarriers
         const uint32_t ta = tmem + ((flags & 1) ? 384 : 256);
-        for (int i = 0; i < count; ++i) {
-            const int grp = commit_every > 0 ? i / commit_every : 0;
+        const int per = commit_every > 0 ? commit_every : count;  // MMAs per commit group
+        int i = 0;
+        for (int grp = 0; i < count; ++grp) {
             const uint32_t d = tmem + (((flags & 1) && (grp & 1)) ? 256 : 0);
-            const uint32_t acc = (i > 0 && (commit_every == 0 || i % commit_every != 0 || !(flags & 1))) ? 1u : 0u;
-            if constexpr (FORM == kRateF16SS) mma_bf16(d, da, db, idesc, acc);
-            if constexpr (FORM == kRateF16TS) mma_bf16_ts(d, ta, db, idesc, acc);
-            if constexpr (FORM == kRateF8SS) mma_f8(d, da, db, idesc, acc);
-            if constexpr (FORM == kRateF16Pair) mma_bf16_pair(d, da, db, idesc, acc);
-            if constexpr (FORM == kRateF8Pair) mma_f8_pair(d, da, db, idesc, acc);
-            if (commit_every > 0 && (i + 1) % commit_every == 0) {
+            for (int j = 0; j < per && i < count; ++j, ++i) {
+                const uint32_t acc = (j > 0 || (i > 0 && !(flags & 1))) ? 1u : 0u;
+                if constexpr (FORM == kRateF16SS) mma_bf16(d, da, db, idesc, acc);
+                if constexpr (FORM == kRateF16TS) mma_bf16_ts(d, ta, db, idesc, acc);
+                if constexpr (FORM == kRateF8SS) mma_f8(d, da, db, idesc, acc);
+                if constexpr (FORM == kRateF16Pair) mma_bf16_pair(d, da, db, idesc, acc);
+                if constexpr (FORM == kRateF8Pair) mma_f8_pair(d, da, db, idesc, acc);
+            }
+            if (commit_every > 0) {
                 uint64_t *b = &step[(flags & 2) ? (grp & 1) : 0];
                 if constexpr (kPair)
                     mma_commit_pair(b, 1);
@@ -150,12 +187,13 @@ extern "C" int moe_test_mma_rate(int32_t form, int32_t N, int32_t count, int32_t
                                  long long *cycles, int32_t *status, moe_stream_t stream)
 {
     using namespace moe;
-    if (!cycles || !status || count < 1 || count > (1 << 20) || commit_every < 0 || flags < 0 || flags > 3)
+    if (!cycles || !status || count < 2 || count > (1 << 20) || commit_every < 0 || flags < 0 || flags > 7)
         return MOE_ERR_INVALID_ARG;
     const bool pair = form == kRateF16Pair || form == kRateF8Pair;
     // MMA N: a multiple of 16 in [16, 256]; the pair forms split N over the two CTAs
     if (N < 16 || N > 256 || N % 16 || (pair && N < 32)) return MOE_ERR_INVALID_ARG;
-    if (form == kRateF16TS && (flags & 1) && N > 128) return MOE_ERR_INVALID_ARG;  // A sits at column 384
+    if (form == kRateF16TS && (flags & 5) && N > 128) return MOE_ERR_INVALID_ARG;  // A sits at column 384
+    if ((flags & 4) && (pair || (flags & 3))) return MOE_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;
     switch (form) {

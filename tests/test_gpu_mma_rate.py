@@ -69,7 +69,8 @@ def test_mma_rate_argument_errors(L):
 def test_commit_cost_table(L):
     """What a commit costs the issuing thread: 2048 MMAs of the FP8 prefill tile shape (M = 128,
     N = 192, K = 32) and the bf16 4-bit shape (N = 96), committing every 1 .. 64 MMAs, with one
-    accumulator or two alternating ones, and one barrier or two alternating ones."""
+    accumulator or two alternating ones, one barrier or two alternating ones, or (flags 4) two
+    issuing threads in different warps with an accumulator each."""
     cyc = torch.zeros(2, dtype=torch.int64, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     st = torch.cuda.current_stream().cuda_stream
@@ -77,7 +78,7 @@ def test_commit_cost_table(L):
     print("\nform      N  commit/  flags  issue cyc/MMA  done cyc/MMA")
     for form, N in ((2, 192), (0, 96), (1, 96), (4, 192)):
         for every in (1, 2, 4, 8, 16, 64):
-            for flags in (0, 1, 2, 3):
+            for flags in ((0, 1, 2, 3) if form == 4 else (0, 1, 2, 3, 4)):
                 for _ in range(2):
                     assert L.moe_test_mma_rate(form, N, count, every, flags, cyc.data_ptr(), status.data_ptr(), st) == 0
                 torch.cuda.synchronize()

@@ -59,14 +59,16 @@ def check_out(got_bf16: torch.Tensor, want: np.ndarray, what: str, amb: np.ndarr
 def assert_same_up_to_sum_order(a: torch.Tensor, b: torch.Tensor, what: str = "repeat"):
     """Two results of the same call on the same inputs.  The fused combine adds each token's k+1
     terms into fp32 in whatever order the additions reach L2 (reading R12: the summation order is
-    free), so a repeat may round differently -- by at most one bf16 step after the final
-    rounding, since order effects in fp32 are ~1e-7 relative and a bf16 step is 2^-8."""
+    free), so a repeat may round differently: the fp32 sums differ by at most a few roundings of
+    terms of order 1 (k+1 <= 33 additions at 2^-24 each, well below 2^-16 absolute), and the bf16
+    results then by at most one bf16 step of the result plus that."""
     if torch.equal(a, b):
         return
     fa, fb = a.float(), b.float()
     ulp = torch.ldexp(torch.ones_like(fa), torch.frexp(torch.maximum(fa.abs(), fb.abs()))[1] - 8)
     diff = (fa - fb).abs()
-    assert (diff <= ulp).all(), f"{what}: {(diff > ulp).sum().item()} elements differ by more than one bf16 step"
+    tol = ulp + 2.0 ** -16
+    assert (diff <= tol).all(), f"{what}: {(diff > tol).sum().item()} elements differ by more than the order bound"
 
 
 def check_route(plan, ws, logits: torch.Tensor, k: int):

@@ -143,8 +143,8 @@ def _fp8_code(orc, v):
 
 def _fp8_midpoint_layer(orc, cancel: float, rel: float):
     """FP8 layer with two features.  Feature 0: G = 64, U = 7, h = 448 (the block amax, so the
-    h scale is 1).  Feature 1: G = 64 (+ cancel*448 - cancel*448 added in two other MMA chunks of
-    32 K elements, leaving G but not its partial sums unchanged) and U = 2.625 * (1 + rel), so
+    h scale is 1).  Feature 1: G = 64 (+ cancel*448 - cancel*448, leaving G unchanged but not the
+    sum of the magnitudes of its products) and U = 2.625 * (1 + rel), so
     h = 168 (1 + rel): just above the midpoint 168 of the e4m3 values 160 and 176.  The down
     weights of feature 1 are 0.5."""
     H, I = 512, 2
@@ -170,13 +170,12 @@ def _fp8_midpoint_layer(orc, cancel: float, rel: float):
                 s_gate=ones(1, I, 1), s_up=su, s_down=ones(1, H, 1))
 
 
-def test_fp8_window_follows_the_partial_sums(orc):
-    """The window of equally valid h values scales with the partial sums of G's evaluation,
-    not with G itself.  With h = 168 (1 + 2^-12), i.e. 0.04 above the midpoint 168: without
-    cancellation in G the window is far narrower than that and the code 176 is the only valid
-    one (zero envelope); with +-448*448 cancelling across two MMA chunks (G unchanged) the
-    window covers the midpoint and 160 is valid too, so each output moves by up to
-    16 * 0.5 = 8."""
+def test_fp8_window_follows_the_sum_of_magnitudes(orc):
+    """The window of equally valid h values scales with the sum of |products| of G's dot
+    product, not with G itself.  With h = 168 (1 + 2^-12), i.e. 0.04 above the midpoint 168:
+    without cancellation in G the window is far narrower than that and the code 176 is the only
+    valid one (zero envelope); with +-448*448 cancelling inside G (G unchanged) the window covers
+    the midpoint and 160 is valid too, so each output moves by up to 16 * 0.5 = 8."""
     rel = 2.0 ** -12
     out0, _, amb0 = orc.layer(_fp8_midpoint_layer(orc, 0.0, rel), ambiguity=True)
     out1, _, amb1 = orc.layer(_fp8_midpoint_layer(orc, 448.0, rel), ambiguity=True)

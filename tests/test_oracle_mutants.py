@@ -42,7 +42,7 @@ PINS = [
     (NV.test_tensor_scales_apply_to_their_own_matrices, {}),
     (LY.test_shared_expert_adds_with_weight_one, {}),
     (LY.test_h_on_a_rounding_midpoint_reports_the_envelope, {}),
-    (ENV.test_fp8_window_follows_the_partial_sums, {}),
+    (ENV.test_fp8_window_follows_the_sum_of_magnitudes, {}),
     (ENV.test_bf16_h_on_a_rounding_midpoint, {"fmt": "int4"}),
     (ENV.test_bf16_h_on_a_rounding_midpoint, {"fmt": "mxfp4"}),
     (ENV.test_bf16_h_on_a_rounding_midpoint, {"fmt": "nvfp4"}),
@@ -83,8 +83,9 @@ MUTANTS = [
      "double b = hx[i];", 1),
     ("bf16 alternatives ignore the window above h",
      "double hi = orc_bf16_to_double(orc_double_to_bf16(hx[i] + dh[i]));", "double hi = b;", 1),
-    ("FP8 window from the result instead of the partial sums",
-     "mag += sc * pmag + sc * fabs(part) + fabs(acc);", "mag += fabs(acc);", 1),
+    ("FP8 window from the block sums instead of the sum of |products|",
+     "mag += fabs((double)sx[kb] * (double)sw[(size_t)n * nb + kb]) * apart;",
+     "mag += fabs((double)sx[kb] * (double)sw[(size_t)n * nb + kb] * part);", 1),
     ("FP8 envelope one code step too wide", "D *= s;", "D *= 2.0 * s;", 1),
     ("shared expert weighted like a routed one", "            for (int n = 0; n < H; ++n) out[n] += y[n];\n",
      "            for (int n = 0; n < H; ++n) out[n] += p[0] * y[n];\n", 2),
