@@ -497,6 +497,40 @@ def run_ours(args, ws, rank, local, cfg_name):
         "fp8_peak_tflops_measured": fp8_tf,
     }
     del xd, ld, od, xh, lh, oh
+    # small batches of the same layer (the first T tokens): device time per call against each
+    # T's own HBM roofline (the touched experts' weights and scales plus x, logits and out);
+    # T <= 16 runs the single-kernel small-batch path
+    if ws == 1 and not args.no_per_config and cfg["wfmt"] == "fp8":
+        sweep = []
+        for Tq in (1, 2, 4, 8, 16):
+            xs, ls = x[:Tq].contiguous(), logits[:Tq].contiguous()
+            os_ = torch.empty_like(xs)
+            for _ in range(3):
+                m(xs, ls, out=os_)
+            torch.cuda.synchronize()
+            times = []
+            for _ in range(20):
+                flush.zero_()
+                # hold the stream (~100 us) until the call is enqueued: at these sizes the host's
+                # launch latency would otherwise land between the events
+                torch.cuda._sleep(200000)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                m(xs, ls, out=os_)
+                e1.record(stream)
+                torch.cuda.synchronize()
+                times.append(e0.elapsed_time(e1))
+            launches = moe.moe_launch_count(m.plan)
+            cnt = m.route(ls)["counts"].cpu().numpy()
+            alg = algorithmic(dict(cfg, T=Tq), cnt)
+            ms = statistics.median(times)
+            t_roof = alg["layer"] / (pk["hbm_gbs"] * 1e9) * 1e3
+            sweep.append({"T": Tq, "ms": ms, "tokens_per_s": Tq / (ms / 1e3), "hbm_roofline_ms": t_roof,
+                          "frac": t_roof / ms, "kernels": launches})
+        rc = moe.moe_get_status(m.plan)
+        if rc != 0:
+            raise RuntimeError(f"device status after the small-batch sweep: {moe.moe_strerror(rc)}")
+        line["small_batch_sweep"] = sweep
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         del layer, m
         torch.cuda.empty_cache()

@@ -13,7 +13,7 @@ BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libmoe_b200.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 
-SOURCES = ["moe_abi.cu", "route.cu", "route_static.cu", "quant.cu", "combine.cu", "gemm_fp8.cu", "gemm_fp8_pair.cu", "gemm_int4.cu",
+SOURCES = ["moe_abi.cu", "context.cu", "route.cu", "route_static.cu", "quant.cu", "combine.cu", "gemm_fp8.cu", "gemm_int4.cu", "small_batch.cu",
            "testing.cu", "router_gemm.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",

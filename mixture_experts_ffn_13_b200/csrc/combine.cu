@@ -67,36 +67,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
     reinterpret_cast<uint2 *>(out + (size_t)t * H)[c] = o;
 }
 
-// The fused combine's last step: fp32 token-order sums -> bf16 (RNE), 8 values per thread.
-__global__ void __launch_bounds__(256) cast_bf16_kernel(const float4 *__restrict__ acc, long n8,
-                                                        uint4 *__restrict__ out)
-{
-    griddep_wait();
-    griddep_launch_dependents();
-    for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (long)gridDim.x * blockDim.x) {
-        const float4 a = __ldg(acc + 2 * i), b = __ldg(acc + 2 * i + 1);
-        const __nv_bfloat162 p0 = __floats2bfloat162_rn(a.x, a.y), p1 = __floats2bfloat162_rn(a.z, a.w);
-        const __nv_bfloat162 p2 = __floats2bfloat162_rn(b.x, b.y), p3 = __floats2bfloat162_rn(b.z, b.w);
-        uint4 o;
-        o.x = *reinterpret_cast<const uint32_t *>(&p0);
-        o.y = *reinterpret_cast<const uint32_t *>(&p1);
-        o.z = *reinterpret_cast<const uint32_t *>(&p2);
-        o.w = *reinterpret_cast<const uint32_t *>(&p3);
-        out[i] = o;
-    }
-}
-
 }  // namespace
-
-cudaError_t launch_cast_bf16(const float *acc, int T, int H, uint16_t *out, int sms, cudaStream_t s)
-{
-    if (T <= 0) return cudaSuccess;
-    const long n8 = (long)T * H / 8;  // H is a multiple of 128
-    const long want = (n8 + 255) / 256;
-    const unsigned blocks = (unsigned)(want < 8L * sms ? want : 8L * sms);
-    return launch_pdl(cast_bf16_kernel, dim3(blocks), dim3(256), 0, s, reinterpret_cast<const float4 *>(acc), n8,
-                      reinterpret_cast<uint4 *>(out));
-}
 
 cudaError_t launch_combine(const float *y, const float *y_shared, const int32_t *pos, const float *topk_w, int T,
                            int H, int k, uint16_t *out, cudaStream_t s, int *check)

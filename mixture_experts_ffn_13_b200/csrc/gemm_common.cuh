@@ -80,45 +80,6 @@ __device__ __forceinline__ int total_tiles(const GemmArgs &a, int BN, int *tot0,
     return *tot0 + tot1;
 }
 
-// Down GEMM epilogue with the combine fused: the token and p_hat of the `ncols` permuted rows
-// row0 .. row0 + ncols - 1 that this warp's columns cover, one per lane (column j*32 + lane in
-// register j), loaded before the epilogue's adds so that their latency is paid once per tile.
-// Routed rows take them from the permutation; the shared segment's rows are their own tokens
-// with weight 1.  Columns at or beyond `nvalid` get weight 0.
-template <int NREG>
-__device__ __forceinline__ void combine_cols(const GemmSeg &sg, int row0, int nvalid, int lane, int (&tok)[NREG],
-                                             float (&w)[NREG])
-{
-#pragma unroll
-    for (int j = 0; j < NREG; ++j) {
-        const int c = j * 32 + lane;
-        const bool ok = c < nvalid;
-        tok[j] = ok ? (sg.tok ? __ldg(sg.tok + row0 + c) : row0 + c) : 0;
-        w[j] = ok ? (sg.rw ? __ldg(sg.rw + row0 + c) : 1.0f) : 0.0f;
-    }
-}
-
-// One output value v of feature n for column c of the tile: stored as y (plain mode) or, with
-// the combine fused, w * v added into the fp32 accumulator row of the column's token (atomic add
-// in L2; the summation order of a token's k+1 contributions is therefore unspecified).  Lanes of
-// a warp hold consecutive n, so each add instruction of a warp covers 128 contiguous bytes.
-template <int NREG>
-__device__ __forceinline__ void down_out(const GemmSeg &sg, const GemmArgs &a, int row, int c, int n, float v,
-                                         const int (&tok)[NREG], const float (&w)[NREG])
-{
-    if (!sg.accum) {
-        static_cast<float *>(sg.out)[(size_t)row * sg.N + n] = v;
-        return;
-    }
-    const int t = __shfl_sync(0xffffffffu, tok[c >> 5], c & 31);
-    const float wt = __shfl_sync(0xffffffffu, w[c >> 5], c & 31);
-    if (a.check && (unsigned)t >= (unsigned)a.T) {
-        atomicCAS(a.check, 0, MOE_ERR_BOUNDS);
-        return;
-    }
-    atomicAdd(sg.accum + (size_t)t * sg.N + n, wt * v);
-}
-
 // silu(g) * u = g / (1 + e^-g) * u with the hardware exponential and approximate division
 // (a few ulp in fp32, far below the accumulation's own rounding).  For g below about -88 the
 // denominator overflows to infinity and the approximate quotient is the exact limit 0.

@@ -382,7 +382,8 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, MODE, EW>::THREADS, 1)
                     s1 = C::PAIR ? __ldg(sw1 + kb) : 0.0f;
                 }
                 const bool ok = mbar_wait(&accf[slot], aph, abort_flag, status, tmo);
-                if (!__all_sync(0xffffffffu, ok)) goto done;
+                // wide tiles meet at named barriers between tiles: decide for all epilogue warps
+                if (!(kStageSx ? bar_all(2, 32 * EW, ok) : __all_sync(0xffffffffu, ok))) goto done;
                 tc_fence_after();
                 const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + slot * C::SLOT_COLS + cbase;
                 const float *sxk = sxs + kb * BN + cbase;
@@ -428,18 +429,18 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, MODE, EW>::THREADS, 1)
                     const float v = is_up ? silu_mul(other, mine) : silu_mul(mine, other);
                     if (cbase + c + (odd ? 1 : 0) < tl.nrows) orow[(size_t)c * sg.N] = v;
                 }
-            } else if constexpr (C::PAIR) {
-#pragma unroll
-                for (int c = 0; c < C::CPW; ++c)
-                    if (cbase + c < tl.nrows) out[(size_t)(tl.row0 + cbase + c) * sg.N + n] = silu_mul(acc0[c], acc1[c]);
             } else {
-                constexpr int NREG = (C::CPW + 31) / 32;
-                int ctok[NREG];
-                float cw[NREG];
-                if (sg.accum) combine_cols(sg, tl.row0 + cbase, tl.nrows - cbase, lane, ctok, cw);
 #pragma unroll
-                for (int c = 0; c < C::CPW; ++c)
-                    if (cbase + c < tl.nrows) down_out(sg, args, tl.row0 + cbase + c, c, n, acc0[c], ctok, cw);
+                for (int c = 0; c < C::CPW; ++c) {
+                    if (cbase + c < tl.nrows) {
+                        float v;
+                        if constexpr (C::PAIR)
+                            v = silu_mul(acc0[c], acc1[c]);
+                        else
+                            v = acc0[c];
+                        out[(size_t)(tl.row0 + cbase + c) * sg.N + n] = v;
+                    }
+                }
             }
             if constexpr (kSxDouble) {
                 if (wn < total) store_sx(tn, sxbuf + ((ti + 1) & 1) * (BN * kMaxKb));
@@ -470,7 +471,7 @@ cudaError_t launch_t(const GemmMaps &maps, const GemmArgs &args, int num_sms, cu
 {
     using C = Fp8Cfg<BN, MODE, EW>;
     auto kern = gemm_fp8_kernel<BN, MODE, EW>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    cudaError_t e = set_smem_limit(reinterpret_cast<const void *>(kern), C::SMEM);
     if (e != cudaSuccess) return e;
     return launch_pdl(kern, dim3(num_sms), dim3(C::THREADS), C::SMEM, s, maps, args);
 }

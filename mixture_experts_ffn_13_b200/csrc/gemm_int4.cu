@@ -10,16 +10,17 @@
 //    128-byte swizzle; narrower boxes make the TMA issue-bound) by TMA into a ring of raw
 //    stages (evict-first), keeps an L2 prefetch of the raw tiles kPrefetch stages further
 //    ahead, and streams the bf16 activation tiles through their own ring;
-//  * warps 2-5 (one thread per weight row, 64 K-elements at a time) turn the nibbles into the
+//  * warps 3-6 (one thread per weight row, 64 K-elements at a time) turn the nibbles into the
 //    integers q as bf16 (exact: |q| <= 8): flip each nibble's sign bit, place it in the
 //    mantissa of the bf16 value 128 (so it reads 128 + q + 8), subtract 136.  The result goes
 //    to TENSOR memory with tcgen05.st (rows in lanes, two bf16 per 32-bit column): staging
 //    the 4x-expanded weights in shared memory instead costs a write and a tensor-core read of
 //    them per stage, which made the kernel shared-memory-bandwidth bound;
-//  * warp 1 issues tcgen05.mma.kind::f16 (A from tensor memory, B from shared memory) from one
-//    thread: 4 MMAs of K = 16 per stage per matrix; each 128-element K group (2 stages)
-//    accumulates into its own TMEM slot, because the weight scale changes per (row, group);
-//  * warps 6-13 (two per TMEM lane quarter, each owning half of the token columns) promote each
+//  * warps 1 and 2 issue tcgen05.mma.kind::f16 (A from tensor memory, B from shared memory),
+//    one thread each (gate|up: one matrix each; down: half of the token columns each): 4 MMAs of K = 16 per
+//    stage per matrix; each 128-element K group (2 stages) accumulates into its own TMEM slot,
+//    because the weight scale changes per (row, group);
+//  * warps 7-14 (two per TMEM lane quarter, each owning half of the token columns) promote each
 //    finished group, acc += D_g * s[row, g] in fp32 registers, and at the end of the tile write
 //    gate|up h = silu(G) * U rounded to bf16 (the 4-bit layer keeps activations in bf16) or
 //    down y in fp32.
@@ -34,8 +35,8 @@
 // value (at most two significant bits) times its block's power-of-two E8M0 scale is exact in
 // bf16, so the dequantisers write the scaled weights themselves, the whole K accumulates in
 // one TMEM slot, and the epilogue has no promotion to do.  The warp roles shift with that:
-// warps 2-9 dequantise (two per TMEM lane quarter, one 32-element block of each 64-K stage
-// apiece) and warps 10-13 (one per quarter) stream each finished tile out.
+// warps 3-10 dequantise (two per TMEM lane quarter, one 32-element block of each 64-K stage
+// apiece) and warps 11-14 (one per quarter) stream each finished tile out.
 //
 // NVFP4 weights (the NVIDIA co-design commentary, section "讀的時候記得這是廠商文": two levels
 // of scale factors) take the same path: an E2M1 value times its 16-block's E4M3 scale has at
@@ -59,7 +60,7 @@ constexpr int kRawKE = 256;            // K elements per raw weight stage (128 b
 constexpr int kSubs = kRawKE / kKE;    // MMA stages per raw stage
 constexpr int kPrefetch = 8;           // raw stages prefetched into L2 ahead of the loads
 
-// Warp roles: 0 producer, 1 MMA issuer, CONV dequantisers, EW epilogue warps.  int4 keeps two
+// Warp roles: 0 producer, 1 and 2 MMA issuers, CONV dequantisers, EW epilogue warps.  int4 keeps two
 // epilogue warps per TMEM lane quarter (each holds half the token columns' fp32 sums across
 // the scale groups); MXFP4 has no promotion, so one epilogue warp per quarter streams the
 // accumulator out, and the freed warps become a second dequantiser per quarter (each of the
@@ -71,7 +72,7 @@ struct I4Cfg {
     static constexpr int CONV = FP4 ? 8 : 4;                // dequantiser warps
     static constexpr int EW = FP4 ? 4 : 8;                  // epilogue warps
     static constexpr int CPW = BN / (EW / 4);               // token columns per epilogue thread
-    static constexpr int THREADS = 32 * (2 + CONV + EW);
+    static constexpr int THREADS = 32 * (3 + CONV + EW);  // producer, two MMA issuers, roles
     static constexpr int NA = GATEUP ? 2 : 1;
     static constexpr int RAW_BYTES = kTileM * (kRawKE / 2);  // 16 KB per matrix
     static constexpr int B_BYTES = BN * kKE * 2;
@@ -80,14 +81,14 @@ struct I4Cfg {
     static constexpr int NM = GATEUP ? 2 : 3;
     static constexpr int A_COLS = 32;
     static constexpr int A_TMEM = NM * NA * A_COLS;
-    static constexpr int SLOT_COLS = NA * BN;               // one 128-element K group
+    static constexpr int SLOT_COLS = NA * BN;  // one 128-element K group (int4) or a whole tile (E2M1)
     static constexpr int NSLOT = (512 - A_TMEM) / SLOT_COLS;
     static constexpr int STAGES_PER_GROUP = kGroupK / kKE;  // 2
     static constexpr int NR = GATEUP ? 3 : 5;               // raw weight stages (256 K each)
     static constexpr int NB_FIT = (212 * 1024 - NR * NA * RAW_BYTES) / B_BYTES;
     static constexpr int NB = NB_FIT < 12 ? NB_FIT : 12;     // activation stages (64 K each)
     static constexpr int TT_BYTES = (4 * (kMaxE + 1) + 15) & ~15;  // keeps the mbarriers 8-byte aligned
-    static constexpr int BAR_BYTES = 8 * (2 * NR + 2 * NB + 2 * NM + 2 * NSLOT) + 16;
+    static constexpr int BAR_BYTES = 8 * (2 * NR + 2 * NB + 2 * NM + 2 * NSLOT) + 24;
     static constexpr int SMEM = 1024 + NB * B_BYTES + NR * NA * RAW_BYTES + TT_BYTES + BAR_BYTES;
     static_assert(B_BYTES % 1024 == 0, "1024-byte aligned tiles");
     static_assert(NSLOT >= 2, "TMEM slots");
@@ -182,7 +183,7 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
     uint64_t *acce = accf + C::NSLOT;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(acce + C::NSLOT);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
-    uint64_t *drain_bar = reinterpret_cast<uint64_t *>(tmem_holder + 2);  // MMA drain on exit
+    uint64_t *drain_bar = reinterpret_cast<uint64_t *>(tmem_holder + 2);  // MMA drain on exit, one per issuer
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -190,19 +191,21 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
             mbar_init(&rfull[s], 1);
             mbar_init(&rempty[s], C::CONV);
         }
+        // both MMA issuers consume every stage and contribute to every accumulator
         for (int s = 0; s < C::NB; ++s) {
             mbar_init(&bfull[s], 1);
-            mbar_init(&bempty[s], 1);
+            mbar_init(&bempty[s], 2);
         }
         for (int s = 0; s < C::NM; ++s) {
             mbar_init(&mfull[s], C::CONV);
-            mbar_init(&mempty[s], 1);
+            mbar_init(&mempty[s], 2);
         }
         for (int s = 0; s < C::NSLOT; ++s) {
-            mbar_init(&accf[s], 1);
+            mbar_init(&accf[s], 2);
             mbar_init(&acce[s], C::EW);
         }
-        mbar_init(drain_bar, 1);
+        mbar_init(&drain_bar[0], 1);
+        mbar_init(&drain_bar[1], 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -275,13 +278,22 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
                 }
             }
         }
-    } else if (warp == 1) {
-        // ------------------------------ MMA issuer --------------------------------
+    } else if (warp == 1 || warp == 2) {
+        // ------------------------------ MMA issuers -------------------------------
+        // Two threads in different warps share every stage's MMAs: a tcgen05.commit holds up
+        // the issuing thread, and a stage needs two (the tensor-memory and the activation
+        // stage), which one thread alone cannot hide behind the short N <= 96 MMAs.  gate|up:
+        // issuer 0 multiplies the gate weights and issuer 1 the up weights; down: each takes
+        // half of the tile's token columns (the MMA's N), into its half of the accumulator.
+        // Both wait for and release every stage, so each consumes the stage rings in order.
+        const int mt = warp - 1;
         if (lane == 0) {
             uint32_t it = 0, ai = 0;
             for (int w = blockIdx.x; w < total; w += gridDim.x) {
                 const TileInfo tl = decode_tile<BN, true>(args, stt, w, tot0);
-                const int n_mma = min(BN, (tl.nrows + 15) & ~15);  // partial tiles: no work on absent rows
+                // MMA N: the tile's valid rows rounded up to 16 (gate|up) or, split in two halves
+                // of a multiple of 16 each, to 32 (down); partial tiles cost no work on absent rows
+                const int n_mma = GATEUP ? min(BN, (tl.nrows + 15) & ~15) : min(BN, (tl.nrows + 31) & ~31) / 2;
                 const uint32_t kIdesc = instr_desc(kTileM, n_mma, 1, 1);
                 // int4: one TMEM slot per 128-element scale group; E2M1 formats: one for the K
                 const int ngrp = FP4 ? 1 : args.seg[tl.seg].K / kGroupK;
@@ -290,23 +302,22 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
                     const int slot = ai % C::NSLOT;
                     if (!mbar_wait(&acce[slot], ((ai / C::NSLOT) & 1) ^ 1, abort_flag, status, tmo)) goto done;
                     tc_fence_after();
-                    const uint32_t d0 = tmem_base + C::A_TMEM + slot * C::SLOT_COLS;
-                    const uint32_t d1 = d0 + BN;
+                    // gate|up: this issuer's matrix; down: its half of the token columns
+                    const uint32_t d = tmem_base + C::A_TMEM + slot * C::SLOT_COLS + (GATEUP ? mt * BN : mt * n_mma);
                     for (int sk = 0; sk < spg; ++sk, ++it) {
                         const int s = it % C::NM;
                         const int bs = it % C::NB;
                         if (!mbar_wait(&mfull[s], (it / C::NM) & 1, abort_flag, status, tmo)) goto done;
                         if (!mbar_wait(&bfull[bs], (it / C::NB) & 1, abort_flag, status, tmo)) goto done;
                         tc_fence_after();
-                        const uint32_t a0 = tmem_base + s * C::NA * C::A_COLS;
-                        const uint32_t a1 = a0 + C::A_COLS;
-                        const uint64_t db = smem_desc_sw128(bst + bs * C::B_BYTES);
+                        const uint32_t a = tmem_base + s * C::NA * C::A_COLS + (GATEUP ? mt * C::A_COLS : 0);
+                        // down: the second half's token rows start n_mma rows (n_mma * 128 bytes,
+                        // whole 8-row swizzle atoms) into the activation stage
+                        const uint64_t db =
+                            smem_desc_sw128(bst + bs * C::B_BYTES) + (GATEUP ? 0 : (uint64_t)(mt * n_mma * 8));
 #pragma unroll
-                        for (int kk = 0; kk < kKE / 16; ++kk) {
-                            const uint32_t acc = (sk > 0 || kk > 0) ? 1u : 0u;
-                            mma_bf16_ts(d0, a0 + 8 * kk, db + 2 * kk, kIdesc, acc);
-                            if (GATEUP) mma_bf16_ts(d1, a1 + 8 * kk, db + 2 * kk, kIdesc, acc);
-                        }
+                        for (int kk = 0; kk < kKE / 16; ++kk)
+                            mma_bf16_ts(d, a + 8 * kk, db + 2 * kk, kIdesc, (sk > 0 || kk > 0) ? 1u : 0u);
                         mma_commit(&mempty[s]);
                         mma_commit(&bempty[bs]);
                     }
@@ -314,7 +325,7 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
                 }
             }
         }
-    } else if (warp < 2 + C::CONV) {
+    } else if (warp < 3 + C::CONV) {
         // ------------------------------ dequantisers ------------------------------
         const int q = warp & 3;        // TMEM lane quarter reachable from this warp
         const int r = q * 32 + lane;   // weight row of the tile handled by this thread
@@ -384,7 +395,7 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
                     // half hx of the stage: 16-byte chunk ch = 2*sub + hx of the row (the 128-byte
                     // swizzle stores chunk c at position c ^ (r & 7)), K elements 32*ch .. +31 of
                     // the raw stage, written to TMEM columns 16*hx .. 16*hx + 15
-                    const int hx = (warp - 2) >> 2;
+                    const int hx = (warp - 3) >> 2;
                     const int cc = ((2 * sub + hx) ^ (r & 7)) << 4;
 #pragma unroll
                     for (int m = 0; m < C::NA; ++m) {
@@ -452,7 +463,7 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
     } else {
         // ------------------------------ epilogue ----------------------------------
         const int q = warp & 3;                                   // TMEM lane quarter
-        const int cbase = ((warp - 2 - C::CONV) >> 2) * C::CPW;  // first token column
+        const int cbase = ((warp - 3 - C::CONV) >> 2) * C::CPW;  // first token column
         const int r = q * 32 + lane;
         uint32_t ai = 0;
         for (int w = blockIdx.x; w < total; w += gridDim.x) {
@@ -473,10 +484,6 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
                 tc_fence_after();
                 const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + C::A_TMEM + slot * C::SLOT_COLS;
                 const int n = tl.nt * kTileM + r;
-                constexpr int NREG = (BN + 31) / 32;
-                int ctok[NREG];
-                float cw[NREG];
-                if (!GATEUP && sg.accum) combine_cols(sg, tl.row0, tl.nrows, lane, ctok, cw);
                 for (int c0 = 0; c0 < BN && c0 < tl.nrows; c0 += 16) {  // warp-uniform bounds
                     float v[16], u[16];
                     tmem_ld16(tb + c0, v);
@@ -494,7 +501,7 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
                                 static_cast<__nv_bfloat16 *>(sg.out)[o] =
                                     __float2bfloat16_rn(NV ? silu_mul(v[c] * t0, u[c] * t1) : silu_mul(v[c], u[c]));
                             else
-                                down_out(sg, args, tl.row0 + c0 + c, c0 + c, n, NV ? v[c] * t0 : v[c], ctok, cw);
+                                static_cast<float *>(sg.out)[o] = NV ? v[c] * t0 : v[c];
                         }
                     }
                 }
@@ -549,18 +556,14 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
                 if (lane == 0) mbar_arrive(&acce[slot]);
             }
             const int n = tl.nt * kTileM + r;
-            constexpr int NREG = (C::CPW + 31) / 32;
-            int ctok[NREG];
-            float cw[NREG];
-            if (!GATEUP && sg.accum) combine_cols(sg, tl.row0 + cbase, tl.nrows - cbase, lane, ctok, cw);
 #pragma unroll
             for (int c = 0; c < C::CPW; ++c) {
                 if (cbase + c < tl.nrows) {
+                    const size_t o = (size_t)(tl.row0 + cbase + c) * sg.N + n;
                     if constexpr (GATEUP)
-                        static_cast<__nv_bfloat16 *>(sg.out)[(size_t)(tl.row0 + cbase + c) * sg.N + n] =
-                            __float2bfloat16_rn(silu_mul(acc0[c], acc1[c]));
+                        static_cast<__nv_bfloat16 *>(sg.out)[o] = __float2bfloat16_rn(silu_mul(acc0[c], acc1[c]));
                     else
-                        down_out(sg, args, tl.row0 + cbase + c, c, n, acc0[c], ctok, cw);
+                        static_cast<float *>(sg.out)[o] = acc0[c];
                 }
             }
         }
@@ -574,7 +577,7 @@ done:
         for (uint32_t j = issued_b > (uint32_t)C::NB ? issued_b - C::NB : 0; j < issued_b; ++j)
             mbar_wait_drain(&bfull[j % C::NB], (j / C::NB) & 1, tmo);
     }
-    if (warp == 1 && lane == 0) mma_drain(drain_bar, tmo);
+    if ((warp == 1 || warp == 2) && lane == 0) mma_drain(&drain_bar[warp - 1], tmo);
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -589,7 +592,7 @@ cudaError_t launch_t(const GemmMaps &maps, const GemmArgs &args, int num_sms, cu
 {
     using C = I4Cfg<BN, GATEUP, FMT != kFmtInt4>;
     auto kern = gemm_int4_kernel<BN, GATEUP, FMT>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    cudaError_t e = set_smem_limit(reinterpret_cast<const void *>(kern), C::SMEM);
     if (e != cudaSuccess) return e;
     return launch_pdl(kern, dim3(num_sms), dim3(C::THREADS), C::SMEM, s, maps, args);
 }

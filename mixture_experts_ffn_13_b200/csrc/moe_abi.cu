@@ -5,7 +5,6 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
-#include <cstdlib>
 #include <mutex>
 #include <new>
 
@@ -18,7 +17,6 @@ struct moe_plan_s {
     size_t ws_bytes;
     int launches;             // kernels launched by the last route/forward call
     bool checked = false;     // checked mode (moe_set_checked): device-side argument checks
-    bool fused_combine;       // the down GEMM adds into a token-order accumulator (no y rows)
     bool prof;                // stage events enabled
     bool prof_recorded;       // the last forward recorded them
     cudaEvent_t ev[8];        // stage boundaries 0..7
@@ -40,14 +38,13 @@ struct Layout {
     size_t act, act_scale;       // permuted activations (+ scales for FP8)
     size_t h, h_sh;              // gate|up output, routed / shared
     size_t hq, hq_sh, sh, sh_sh; // quantised h (FP8)
-    size_t rowscale;             // p_hat per permuted row (fused combine)
-    size_t y;                    // down output: rows (routed then shared) fp32, or with the
-                                 // combine fused the token-order accumulator [T, H] fp32
+    size_t y;                    // down output rows (routed then shared), fp32
     size_t lg;                   // router logits [T, E] fp32 (moe_forward_x): inside y when they fit
+    size_t small;                // the small-batch kernel's partial sums, y rows and barrier
     size_t total;
 };
 
-Layout make_layout(const moe_dims &d, bool fused)
+Layout make_layout(const moe_dims &d)
 {
     const size_t Tm = (size_t)d.T_max, k = (size_t)d.k, E = (size_t)d.E;
     const size_t H = (size_t)d.H, I = (size_t)d.I, Is = (size_t)d.I_shared;
@@ -71,7 +68,6 @@ Layout make_layout(const moe_dims &d, bool fused)
     L.chunk_hist = take(nch * E * 4);
     L.ttile_a = take((E + 1) * 4);
     L.ttile_b = take((E + 1) * 4);
-    L.rowscale = take(fused ? A * 4 : 0);
     if (fp8) {
         L.act = take(R * H);
         L.act_scale = take(R * nb512(d.H) * 4);
@@ -88,12 +84,12 @@ Layout make_layout(const moe_dims &d, bool fused)
         L.h_sh = take(Tm * Is * 2);
         L.hq = L.hq_sh = L.sh = L.sh_sh = 0;
     }
-    const size_t ybytes = fused ? Tm * H * 4 : R * H * 4;
-    L.y = take(ybytes);
+    L.y = take(R * H * 4);
     // moe_forward_x's logits are read only by the route kernel, the first kernel of the
-    // forward, and y (or the accumulator, cleared by the activation pass after routing) is
-    // written later on the same stream, so they share y's bytes unless they do not fit there
-    L.lg = Tm * E * 4 <= ybytes ? L.y : take(Tm * E * 4);
+    // forward, and y is written by the down GEMM later on the same stream, so they share y's
+    // bytes unless they do not fit there
+    L.lg = Tm * E <= R * H ? L.y : take(Tm * E * 4);
+    L.small = fp8 ? take(small_batch_workspace(d)) : 0;
     L.total = o;
     return L;
 }
@@ -116,21 +112,6 @@ int fail_cuda(moe_plan_t *p, cudaError_t e)
 {
     p->last_cuda_error = (int)e;
     return MOE_ERR_CUDA;
-}
-
-// Environment switches, read once, for comparison and diagnosis: MOE_GEMM_PAIR=0 keeps the
-// 192-row FP8 GEMMs on one SM per tile; MOE_FUSED_COMBINE=0 (read when a plan is made) keeps
-// the down GEMM's y rows and the separate combine kernel.
-bool env_on(const char *name)
-{
-    const char *v = getenv(name);
-    return !(v && v[0] == '0');
-}
-
-bool use_pair_gemm()
-{
-    static const bool on = env_on("MOE_GEMM_PAIR");
-    return on;
 }
 
 // Tile size along the token dimension from the mean rows per expert group: decode-sized
@@ -229,8 +210,7 @@ int moe_plan(const moe_dims *dims, moe_plan_t **out_plan, size_t *workspace_byte
         delete p;
         return MOE_ERR_CUDA;
     }
-    p->fused_combine = env_on("MOE_FUSED_COMBINE");
-    p->ws_bytes = make_layout(d, p->fused_combine).total;
+    p->ws_bytes = make_layout(d).total;
     *workspace_bytes = p->ws_bytes;
     *out_plan = p;
     return MOE_OK;
@@ -309,10 +289,9 @@ static int check_ws(const moe_plan_t *p, void *ws, size_t ws_bytes)
     return MOE_OK;
 }
 
-static RouteBufs route_bufs(const Layout &L, uint8_t *ws, bool fused)
+static RouteBufs route_bufs(const Layout &L, uint8_t *ws)
 {
     RouteBufs b;
-    b.rowscale = fused ? reinterpret_cast<float *>(ws + L.rowscale) : nullptr;
     b.topk_idx = reinterpret_cast<int32_t *>(ws + L.topk_idx);
     b.topk_w = reinterpret_cast<float *>(ws + L.topk_w);
     b.counts = reinterpret_cast<int32_t *>(ws + L.counts);
@@ -370,8 +349,8 @@ int moe_route(moe_plan_t *p, int32_t T, const float *logits, int32_t *topk_idx, 
     int rc = check_ws(p, workspace, ws_bytes);
     if (rc) return rc;
     const moe_dims &d = p->d;
-    const Layout L = make_layout(d, p->fused_combine);
-    RouteBufs b = route_bufs(L, static_cast<uint8_t *>(workspace), false);
+    const Layout L = make_layout(d);
+    RouteBufs b = route_bufs(L, static_cast<uint8_t *>(workspace));
     b.topk_idx = topk_idx;
     b.topk_w = topk_w;
     b.counts = counts;
@@ -395,9 +374,8 @@ static int forward_w4(moe_plan_t *p, int T, const uint16_t *x, const float *logi
     auto mark = [&](int i) {
         if (p->prof) cudaEventRecord(p->ev[i], s);
     };
-    const bool fused = p->fused_combine;
-    const Layout L = make_layout(d, fused);
-    const RouteBufs b = route_bufs(L, ws, fused);
+    const Layout L = make_layout(d);
+    const RouteBufs b = route_bufs(L, ws);
     const int H = d.H, I = d.I, Is = d.I_shared, k = d.k, E = d.E;
     const bool shared = Is > 0;
     const int A = T * k;
@@ -411,14 +389,14 @@ static int forward_w4(moe_plan_t *p, int T, const uint16_t *x, const float *logi
     if (e != cudaSuccess) return fail_cuda(p, e);
     uint16_t *xp = reinterpret_cast<uint16_t *>(ws + L.act);
     uint16_t *xp_sh = shared ? xp + (size_t)A * H : nullptr;
-    float *y = reinterpret_cast<float *>(ws + L.y);  // y rows, or the fused combine's accumulator
-    e = launch_gather_x_bf16(x, T, H, k, b.pos, xp, xp_sh, s, fused ? y : nullptr);
+    e = launch_gather_x_bf16(x, T, H, k, b.pos, xp, xp_sh, s);
     mark(3);
     if (e != cudaSuccess) return fail_cuda(p, e);
 
     uint16_t *h = reinterpret_cast<uint16_t *>(ws + L.h);
     uint16_t *h_sh = reinterpret_cast<uint16_t *>(ws + L.h_sh);
-    float *y_sh = shared && !fused ? y + (size_t)A * H : nullptr;
+    float *y = reinterpret_cast<float *>(ws + L.y);
+    float *y_sh = shared ? y + (size_t)A * H : nullptr;
     const CUtensorMapDataType U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8, BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
 
     GemmMaps mg{};
@@ -453,20 +431,13 @@ static int forward_w4(moe_plan_t *p, int T, const uint16_t *x, const float *logi
     GemmMaps md{};
     GemmArgs ad = ag;
     ad.ttile = b.ttile_b;
-    ad.check = fused ? chk : nullptr;
     ad.seg[0] = GemmSeg{H, I, A, w->s_down, nullptr, nullptr, y};
     ad.seg[0].ts0 = w->t_down;
-    if (fused) {
-        ad.seg[0].accum = y;
-        ad.seg[0].tok = b.perm_tok;
-        ad.seg[0].rw = b.rowscale;
-    }
     rc = encode_map_2d(&md.a0[0], w->w_down, U8, 1, I / 2, (uint64_t)E * H, 128, 128, true);
     rc |= encode_map_2d(&md.b[0], h, BF, 2, I, A, 64, bn, true);
     if (shared) {
         ad.seg[1] = GemmSeg{H, Is, T, w->ss_down, nullptr, nullptr, y_sh};
         ad.seg[1].ts0 = w->ts_down;
-        if (fused) ad.seg[1].accum = y;
         rc |= encode_map_2d(&md.a0[1], w->ws_down, U8, 1, Is / 2, H, 128, 128, true);
         rc |= encode_map_2d(&md.b[1], h_sh, BF, 2, Is, T, 64, bn, true);
     }
@@ -474,7 +445,7 @@ static int forward_w4(moe_plan_t *p, int T, const uint16_t *x, const float *logi
     e = launch_gemm_w4(false, d.wfmt, bn, md, ad, p->num_sms, s);
     mark(6);
     if (e != cudaSuccess) return fail_cuda(p, e);
-    e = fused ? launch_cast_bf16(y, T, H, out, p->num_sms, s) : launch_combine(y, y_sh, b.pos, b.topk_w, T, H, k, out, s, chk);
+    e = launch_combine(y, y_sh, b.pos, b.topk_w, T, H, k, out, s, chk);
     mark(7);
     if (e != cudaSuccess) return fail_cuda(p, e);
     p->launches = route_permute_launches(T, E, k) + 1 + 1 + 1 + 1;
@@ -528,9 +499,24 @@ int moe_forward(moe_plan_t *p, int32_t T, const uint16_t *x, const float *logits
     };
     if (d.wfmt != MOE_W_FP8_SC512) return forward_w4(p, T, x, logits, w, out, static_cast<uint8_t *>(workspace), s);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    const bool fused = p->fused_combine;
-    const Layout L = make_layout(d, fused);
-    const RouteBufs b = route_bufs(L, ws, fused);
+    const Layout L = make_layout(d);
+    // small batches: the whole layer in one kernel (checked mode keeps the regular path, whose
+    // kernels carry the device-side checks); the whole call is reported as stage 3
+    if (!p->checked && small_batch_fits(T, d)) {
+        int launched = 0;
+        for (int i = 0; i <= 3; ++i) mark(i);
+        const cudaError_t es =
+            launch_small_batch(d, T, x, logits, w, out, ws + L.small, p->d_status, p->num_sms, s, &launched);
+        if (es == cudaSuccess) {
+            for (int i = 4; i <= 7; ++i) mark(i);
+            p->launches = 1;
+            p->prof_recorded = p->prof;
+            return MOE_OK;
+        }
+        if (launched || es != cudaErrorNotSupported) return fail_cuda(p, es);
+        // gate and up weights too far apart for the small kernel's tensor map: regular path
+    }
+    const RouteBufs b = route_bufs(L, ws);
     const int H = d.H, I = d.I, Is = d.I_shared, k = d.k, E = d.E;
     const int A = T * k;
     const int bn_b = pick_bn(T, k, E, true);
@@ -555,8 +541,7 @@ int moe_forward(moe_plan_t *p, int32_t T, const uint16_t *x, const float *logits
     const int nbH = nb512(H);
     uint8_t *xq_sh = shared ? xq + (size_t)A * H : nullptr;
     float *sx_sh = shared ? sx + (size_t)A * nbH : nullptr;
-    float *y = reinterpret_cast<float *>(ws + L.y);  // y rows, or the fused combine's accumulator
-    e = launch_quant_x_fp8(x, T, H, k, b.pos, xq, sx, xq_sh, sx_sh, s, fused ? y : nullptr);
+    e = launch_quant_x_fp8(x, T, H, k, b.pos, xq, sx, xq_sh, sx_sh, s);
     mark(3);
     if (e != cudaSuccess) return fail_cuda(p, e);
 
@@ -564,7 +549,8 @@ int moe_forward(moe_plan_t *p, int32_t T, const uint16_t *x, const float *logits
     float *h_sh = reinterpret_cast<float *>(ws + L.h_sh);
     uint8_t *hq = ws + L.hq, *hq_sh = ws + L.hq_sh;
     float *sh = reinterpret_cast<float *>(ws + L.sh), *sh_sh = reinterpret_cast<float *>(ws + L.sh_sh);
-    float *y_sh = shared && !fused ? y + (size_t)A * H : nullptr;
+    float *y = reinterpret_cast<float *>(ws + L.y);
+    float *y_sh = shared ? y + (size_t)A * H : nullptr;
     const CUtensorMapDataType U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
 
     // A4: gate|up
@@ -589,19 +575,15 @@ int moe_forward(moe_plan_t *p, int32_t T, const uint16_t *x, const float *logits
         return encode_map_2d(&m0, wg, U8, 1, H, rows, 128, wbox, true) |
                encode_map_2d(&m1, wu, U8, 1, H, rows, 128, wbox, true);
     };
-    if (shared) ag.seg[1] = GemmSeg{Is, H, T, w->ss_gate, w->ss_up, sx_sh, h_sh};
-    // 192-row token tiles run on CTA pairs (M = 256 over two SMs) where the shapes allow; their
-    // activation boxes are 32 rows (each CTA loads half of a tile's rows)
-    const bool pair_a = ilv && use_pair_gemm() && gemm_fp8_pair_fits(true, ag);
-    const uint32_t xbox_a = pair_a ? 32 : kXBox;
     rc = gateup_maps(ag.seg[0], mg.a0[0], mg.a1[0], w->w_gate, w->w_up, (uint64_t)E * I);
-    rc |= encode_map_2d(&mg.b[0], xq, U8, 1, H, A, 128, xbox_a, true);
+    rc |= encode_map_2d(&mg.b[0], xq, U8, 1, H, A, 128, kXBox, true);
     if (shared) {
+        ag.seg[1] = GemmSeg{Is, H, T, w->ss_gate, w->ss_up, sx_sh, h_sh};
         rc |= gateup_maps(ag.seg[1], mg.a0[1], mg.a1[1], w->ws_gate, w->ws_up, (uint64_t)Is);
-        rc |= encode_map_2d(&mg.b[1], xq_sh, U8, 1, H, T, 128, xbox_a, true);
+        rc |= encode_map_2d(&mg.b[1], xq_sh, U8, 1, H, T, 128, kXBox, true);
     }
     if (rc) return MOE_ERR_CUDA;
-    e = pair_a ? launch_gemm_fp8_pair(true, mg, ag, p->num_sms, s) : launch_gemm_fp8(true, bn_a, mg, ag, p->num_sms, s);
+    e = launch_gemm_fp8(true, bn_a, mg, ag, p->num_sms, s);
     mark(4);
     if (e != cudaSuccess) return fail_cuda(p, e);
 
@@ -614,30 +596,22 @@ int moe_forward(moe_plan_t *p, int32_t T, const uint16_t *x, const float *logits
     GemmMaps md{};
     GemmArgs ad = ag;
     ad.ttile = b.ttile_b;
-    ad.check = fused ? chk : nullptr;
     ad.seg[0] = GemmSeg{H, I, A, w->s_down, nullptr, sh, y};
-    if (shared) ad.seg[1] = GemmSeg{H, Is, T, w->ss_down, nullptr, sh_sh, y_sh};
-    if (fused) {
-        ad.seg[0].accum = y;
-        ad.seg[0].tok = b.perm_tok;
-        ad.seg[0].rw = b.rowscale;
-        if (shared) ad.seg[1].accum = y;
-    }
-    const bool pair_b = bn_b == 192 && use_pair_gemm() && gemm_fp8_pair_fits(false, ad);
-    const uint32_t kHBox = pair_b ? 32 : (bn_b < 64 ? bn_b : 64);
+    const uint32_t kHBox = bn_b < 64 ? bn_b : 64;
     rc = encode_map_2d(&md.a0[0], w->w_down, U8, 1, I, (uint64_t)E * H, 128, 128, true);
     rc |= encode_map_2d(&md.b[0], hq, U8, 1, I, A, 128, kHBox, true);
     if (shared) {
+        ad.seg[1] = GemmSeg{H, Is, T, w->ss_down, nullptr, sh_sh, y_sh};
         rc |= encode_map_2d(&md.a0[1], w->ws_down, U8, 1, Is, H, 128, 128, true);
         rc |= encode_map_2d(&md.b[1], hq_sh, U8, 1, Is, T, 128, kHBox, true);
     }
     if (rc) return MOE_ERR_CUDA;
-    e = pair_b ? launch_gemm_fp8_pair(false, md, ad, p->num_sms, s) : launch_gemm_fp8(false, bn_b, md, ad, p->num_sms, s);
+    e = launch_gemm_fp8(false, bn_b, md, ad, p->num_sms, s);
     mark(6);
     if (e != cudaSuccess) return fail_cuda(p, e);
 
-    // A6: combine (fused: the down GEMM summed into y; round it to bf16)
-    e = fused ? launch_cast_bf16(y, T, H, out, p->num_sms, s) : launch_combine(y, y_sh, b.pos, b.topk_w, T, H, k, out, s, chk);
+    // A6: combine
+    e = launch_combine(y, y_sh, b.pos, b.topk_w, T, H, k, out, s, chk);
     mark(7);
     if (e != cudaSuccess) return fail_cuda(p, e);
     p->launches = route_permute_launches(T, E, k) + 1 + 1 + 1 + 1 + 1;
@@ -658,7 +632,7 @@ int moe_forward_x(moe_plan_t *p, int32_t T, const uint16_t *x, const uint16_t *w
     if (rc) return rc;
     p->launches = 0;
     if (T == 0) return MOE_OK;
-    const Layout L = make_layout(d, p->fused_combine);
+    const Layout L = make_layout(d);
     float *lg = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + L.lg);
     const cudaError_t e =
         launch_router_gemm(x, w_router, lg, T, d.H, d.E, p->d_status, p->num_sms, (cudaStream_t)stream);

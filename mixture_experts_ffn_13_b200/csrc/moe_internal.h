@@ -18,6 +18,17 @@ constexpr int kGroupK = 128;  // int4 scale group along K
 constexpr int kMxBlock = 32;  // MXFP4 scale block along K
 constexpr uint64_t kDefaultTimeoutNs = 1000000000ull;  // device-side waits give up after 1 s
 
+// ---- the current context (context.cu) -----------------------------------------------------
+
+// Current device, context and the context's process-unique id; makes the device's primary
+// context current if the thread has none.  MOE_OK or MOE_ERR_CUDA.
+int current_context(int *dev, CUcontext *ctx, unsigned long long *id);
+// MOE_OK if stream `s` belongs to context `ctx`, else MOE_ERR_INVALID_ARG.
+int stream_in_context(cudaStream_t s, CUcontext ctx);
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (context, kernel): later calls with
+// the same or a smaller size return without a driver call.
+cudaError_t set_smem_limit(const void *func, int smem);
+
 // ---- routing / permutation (route.cu) ---------------------------------------------------
 
 struct RouteBufs {
@@ -30,7 +41,6 @@ struct RouteBufs {
     int32_t *chunk_hist;  // [nchunks, E]
     int32_t *ttile_a;     // [E + 1] token-tile prefix for the gate|up GEMM tile size
     int32_t *ttile_b;     // [E + 1] token-tile prefix for the down GEMM tile size
-    float *rowscale;      // [T * k] p_hat of each permuted row (fused combine), or nullptr
 };
 
 // check != nullptr (checked mode): non-finite logits record MOE_ERR_BOUNDS in *check.
@@ -48,10 +58,8 @@ int route_permute_launches(int T, int E, int k);
 
 // FP8: quantise each bf16 token row of x (per 512-block) and write it to the permuted rows
 // pos[t, 0..k) and, when shared_rows != nullptr, to shared row t.
-// zero (optional, [T, H] fp32): cleared in the same pass (the fused combine's accumulator).
 cudaError_t launch_quant_x_fp8(const uint16_t *x, int T, int H, int k, const int32_t *pos, uint8_t *xq,
-                               float *sx, uint8_t *xq_shared, float *sx_shared, cudaStream_t s,
-                               float *zero = nullptr);
+                               float *sx, uint8_t *xq_shared, float *sx_shared, cudaStream_t s);
 // FP8: quantise fp32 rows (h) per 512-block.
 // h -> e4m3 per (row, 512-block) for two row segments in one launch (segment 1 skipped when
 // h1 is null or R1 == 0).
@@ -59,7 +67,7 @@ cudaError_t launch_quant_rows_fp8(const float *h, int R, int K, uint8_t *q, floa
                                   int K1, uint8_t *q1, float *sq1, cudaStream_t s);
 // int4 layers: copy bf16 token rows into the permuted rows (and the shared rows).
 cudaError_t launch_gather_x_bf16(const uint16_t *x, int T, int H, int k, const int32_t *pos, uint16_t *xp,
-                                 uint16_t *xp_shared, cudaStream_t s, float *zero = nullptr);
+                                 uint16_t *xp_shared, cudaStream_t s);
 
 // ---- combine (combine.cu) ----------------------------------------------------------------
 
@@ -67,8 +75,6 @@ cudaError_t launch_gather_x_bf16(const uint16_t *x, int T, int H, int k, const i
 // MOE_ERR_BOUNDS in *check.
 cudaError_t launch_combine(const float *y, const float *y_shared, const int32_t *pos, const float *topk_w,
                            int T, int H, int k, uint16_t *out, cudaStream_t s, int *check = nullptr);
-// The fused combine's last step: the fp32 token-order sums [T, H] rounded to bf16 (RNE).
-cudaError_t launch_cast_bf16(const float *acc, int T, int H, uint16_t *out, int num_sms, cudaStream_t s);
 
 // ---- grouped GEMMs (gemm_fp8.cu, gemm_int4.cu) -------------------------------------------
 
@@ -86,12 +92,6 @@ struct GemmSeg {
     int up_lo;        // interleaved gate|up: the up rows come first in each 32-row quarter
     const float *ts0; // NVFP4: fp32 tensor scales of the first / second weight matrix, one per
     const float *ts1; //   group (routed: [E], shared: [1]); unused otherwise
-    // down with the combine fused (accum != nullptr): instead of storing y, row r adds
-    // rw[r] * y[r, :] into accum[tok[r], :] (fp32, token order, zeroed beforehand); tok/rw are
-    // the permutation's token and p_hat per row (nullptr for the shared segment: token r, 1)
-    float *accum;
-    const int32_t *tok;
-    const float *rw;
 };
 
 struct GemmArgs {
@@ -103,7 +103,6 @@ struct GemmArgs {
     const int32_t *ttile;    // [E + 1] routed token-tile prefix for this GEMM's tile size
     int *status;             // device status word
     uint64_t timeout_ns;
-    int *check;              // checked mode: out-of-range fused-combine tokens record MOE_ERR_BOUNDS
 };
 
 // Tensor maps of one GEMM launch: A (weights) 0 and 1 per segment, B (activations) per segment.
@@ -114,16 +113,22 @@ struct GemmMaps {
 // FP8 grouped GEMMs.  gateup: h = silu(x Wg^T) * (x Wu^T) in fp32; down: y = h Wd^T in fp32.
 cudaError_t launch_gemm_fp8(bool gateup, int bn, const GemmMaps &maps, const GemmArgs &args, int num_sms,
                             cudaStream_t s);
-// The same FP8 GEMMs with 192-row token tiles on CTA pairs (cta_group::2, M = 256 over two
-// SMs); the activation maps must use 32-row boxes.  gemm_fp8_pair_fits: the shapes it takes
-// (gate|up: N a multiple of 128; down: N a multiple of 256).
-bool gemm_fp8_pair_fits(bool gateup, const GemmArgs &args);
-cudaError_t launch_gemm_fp8_pair(bool gateup, const GemmMaps &maps, const GemmArgs &args, int num_sms,
-                                 cudaStream_t s);
 // 4-bit grouped GEMMs over bf16 activations (wfmt: MOE_W_INT4_G128, MOE_W_MXFP4_G32 or
 // MOE_W_NVFP4_G16): gate|up writes h as bf16, down writes y fp32.
 cudaError_t launch_gemm_w4(bool gateup, int wfmt, int bn, const GemmMaps &maps, const GemmArgs &args,
                            int num_sms, cudaStream_t s);
+
+// Small batches (T <= 16, FP8 weights): the whole layer in one cooperative persistent kernel
+// (small_batch.cu).  small_batch_fits: shapes it takes (H a multiple of 2048 up to 4096, I and
+// I_shared multiples of 512 up to 2048); small_batch_workspace: the bytes it needs in the
+// workspace (partial sums, y rows, a grid-barrier counter).  launch_small_batch returns
+// cudaErrorNotSupported, before any device work, when the gate and up weight arrays are too far
+// apart for one tensor map (the caller then takes the regular path).
+bool small_batch_fits(int T, const moe_dims &d);
+size_t small_batch_workspace(const moe_dims &d);
+cudaError_t launch_small_batch(const moe_dims &d, int T, const uint16_t *x, const float *logits,
+                               const moe_weights *w, uint16_t *out, void *ws, int *status, int num_sms,
+                               cudaStream_t s, int *launched);
 
 // Router logits [T, E] (written) and their softmax top-k (step A1): the router GEMM, then the
 // route kernel.

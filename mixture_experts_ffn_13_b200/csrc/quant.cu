@@ -58,7 +58,7 @@ __device__ __forceinline__ uint4 quant16(const float (&f)[16], bool valid, float
 __global__ void __launch_bounds__(256) quant_x_fp8_kernel(const uint16_t *__restrict__ x, int T, int H, int k,
                                                           const int32_t *__restrict__ pos, uint8_t *__restrict__ xq,
                                                           float *__restrict__ sx, uint8_t *__restrict__ xq_sh,
-                                                          float *__restrict__ sx_sh, float *__restrict__ zero)
+                                                          float *__restrict__ sx_sh)
 {
     griddep_wait();
     griddep_launch_dependents();
@@ -80,14 +80,6 @@ __global__ void __launch_bounds__(256) quant_x_fp8_kernel(const uint16_t *__rest
             f[2 * i] = bf16_bits_to_float(w[i] & 0xffffu);
             f[2 * i + 1] = bf16_bits_to_float(w[i] >> 16);
         }
-    }
-    if (zero && valid) {  // the fused combine's accumulator, same (t, block) footprint in fp32
-        float4 *z = reinterpret_cast<float4 *>(zero + (size_t)t * H + i0);
-        const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
-        z[0] = z4;
-        z[1] = z4;
-        z[2] = z4;
-        z[3] = z4;
     }
     float s;
     const uint4 q = quant16(f, valid, &s);
@@ -152,7 +144,7 @@ __global__ void __launch_bounds__(256) quant_rows_fp8_kernel(RowsSeg s0, RowsSeg
 // grid T: copy bf16 token row t to the permuted rows pos[t, :] and to shared row t.
 __global__ void __launch_bounds__(128) gather_x_bf16_kernel(const uint16_t *__restrict__ x, int H, int k,
                                                             const int32_t *__restrict__ pos, uint16_t *__restrict__ xp,
-                                                            uint16_t *__restrict__ xp_sh, float *__restrict__ zero)
+                                                            uint16_t *__restrict__ xp_sh)
 {
     griddep_wait();
     griddep_launch_dependents();
@@ -166,23 +158,18 @@ __global__ void __launch_bounds__(128) gather_x_bf16_kernel(const uint16_t *__re
             reinterpret_cast<uint4 *>(xp + (size_t)r * H)[c] = v;
         }
         if (xp_sh) reinterpret_cast<uint4 *>(xp_sh + (size_t)t * H)[c] = v;
-        if (zero) {  // the fused combine's accumulator row t, 8 fp32 per chunk
-            float4 *z = reinterpret_cast<float4 *>(zero + (size_t)t * H) + 2 * c;
-            z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-            z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
     }
 }
 
 }  // namespace
 
 cudaError_t launch_quant_x_fp8(const uint16_t *x, int T, int H, int k, const int32_t *pos, uint8_t *xq, float *sx,
-                               uint8_t *xq_shared, float *sx_shared, cudaStream_t s, float *zero)
+                               uint8_t *xq_shared, float *sx_shared, cudaStream_t s)
 {
     if (T <= 0) return cudaSuccess;
     const long warps = (long)T * ((H + kBlockK - 1) / kBlockK);
     return launch_pdl(quant_x_fp8_kernel, dim3((unsigned)((warps + 7) / 8)), dim3(256), 0, s, x, T, H, k, pos, xq, sx,
-                      xq_shared, sx_shared, zero);
+                      xq_shared, sx_shared);
 }
 
 cudaError_t launch_quant_rows_fp8(const float *h, int R, int K, uint8_t *q, float *sq, const float *h1, int R1,
@@ -195,10 +182,10 @@ cudaError_t launch_quant_rows_fp8(const float *h, int R, int K, uint8_t *q, floa
 }
 
 cudaError_t launch_gather_x_bf16(const uint16_t *x, int T, int H, int k, const int32_t *pos, uint16_t *xp,
-                                 uint16_t *xp_shared, cudaStream_t s, float *zero)
+                                 uint16_t *xp_shared, cudaStream_t s)
 {
     if (T <= 0) return cudaSuccess;
-    return launch_pdl(gather_x_bf16_kernel, dim3(T), dim3(128), 0, s, x, H, k, pos, xp, xp_shared, zero);
+    return launch_pdl(gather_x_bf16_kernel, dim3(T), dim3(128), 0, s, x, H, k, pos, xp, xp_shared);
 }
 
 }  // namespace moe

@@ -239,8 +239,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(int nchunks, int E, int32_t 
 // lane loads its 32 expert ids up front so the in-order walks touch shared memory only.
 __global__ void __launch_bounds__(kChunk) scatter_kernel(const int32_t *__restrict__ topk_idx, int T, int E, int k,
                                                          const int32_t *__restrict__ chunk_base,
-                                                         int32_t *__restrict__ perm_tok, int32_t *__restrict__ pos,
-                                                         const float *__restrict__ topk_w, float *__restrict__ rowscale)
+                                                         int32_t *__restrict__ perm_tok, int32_t *__restrict__ pos)
 {
     __shared__ int cnt[kChunk / 32][kMaxE];
     griddep_wait();
@@ -274,7 +273,6 @@ __global__ void __launch_bounds__(kChunk) scatter_kernel(const int32_t *__restri
             const int r = cnt[warp][ids[l]]++;
             perm_tok[r] = t0 + l;
             pos[(size_t)(t0 + l) * k + lane] = r;
-            if (rowscale) rowscale[r] = topk_w[(size_t)(t0 + l) * k + lane];
         }
         __syncwarp();
     }
@@ -290,9 +288,7 @@ __global__ void __launch_bounds__(1024) permute_small_kernel(const int32_t *__re
                                                              int32_t *__restrict__ offsets,
                                                              int32_t *__restrict__ perm_tok, int32_t *__restrict__ pos,
                                                              int bn_a, int32_t *__restrict__ ttile_a, int bn_b,
-                                                             int32_t *__restrict__ ttile_b,
-                                                             const float *__restrict__ topk_w,
-                                                             float *__restrict__ rowscale)
+                                                             int32_t *__restrict__ ttile_b)
 {
     extern __shared__ int sm[];
     const int W = (T + 31) >> 5;
@@ -346,7 +342,6 @@ __global__ void __launch_bounds__(1024) permute_small_kernel(const int32_t *__re
         const int r = pre[w * E + e] + __popc(mask[w * E + e] & ((1u << (t & 31)) - 1u));
         perm_tok[r] = t;
         pos[i] = r;
-        if (rowscale) rowscale[r] = topk_w[i];
     }
 }
 
@@ -371,10 +366,10 @@ cudaError_t launch_permute_any(const RouteBufs &b, int T, int E, int k, int bn_a
     cudaError_t e;
     const size_t smem = small_route_smem(T, E, k);
     if (T < 1 || T > 4096 || smem > 160 * 1024) return launch_permute(b, T, E, k, bn_a, bn_b, s);
-    e = cudaFuncSetAttribute(permute_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = set_smem_limit(reinterpret_cast<const void *>(permute_small_kernel), (int)smem);
     if (e != cudaSuccess) return e;
     return launch_pdl(permute_small_kernel, dim3(1), dim3(1024), smem, s, b.topk_idx, T, E, k, b.counts, b.offsets,
-                      b.perm_tok, b.pos, bn_a, b.ttile_a, bn_b, b.ttile_b, (const float *)b.topk_w, b.rowscale);
+                      b.perm_tok, b.pos, bn_a, b.ttile_a, bn_b, b.ttile_b);
 }
 
 int route_permute_launches(int T, int E, int k)
@@ -409,7 +404,7 @@ cudaError_t launch_permute(const RouteBufs &b, int T, int E, int k, int bn_a, in
                        b.ttile_a, bn_b, b.ttile_b);
     if (e == cudaSuccess && nchunks > 0)
         e = launch_pdl(scatter_kernel, dim3(nchunks), dim3(kChunk), 0, s, b.topk_idx, T, E, k, b.chunk_hist,
-                       b.perm_tok, b.pos, (const float *)b.topk_w, b.rowscale);
+                       b.perm_tok, b.pos);
     return e;
 }
 

@@ -27,8 +27,6 @@
 //  * No cudaMalloc, cudaFree or allocating library routine is called.
 #include "moe_internal.h"
 
-#include <cudaTypedefs.h>
-
 #include <mutex>
 
 namespace moe {
@@ -39,27 +37,6 @@ constexpr size_t kStaticScratchInts = size_t(1) << 19;
 constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) int32_t g_route_scratch[kStaticScratchInts];
-
-// Driver entry points (through the runtime, so the library links only libcudart).
-PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;
-PFN_cuCtxGetId_v12000 g_ctx_id = nullptr;
-PFN_cuStreamGetCtx_v9020 g_stream_ctx = nullptr;
-std::once_flag g_driver_once;
-
-void load_driver()
-{
-    auto get = [](const char *name, unsigned ver) -> void * {
-        void *fn = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPointByVersion(name, &fn, ver, cudaEnableDefault, &q) != cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            return nullptr;
-        return fn;
-    };
-    g_ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(get("cuCtxGetCurrent", 4000));
-    g_ctx_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(get("cuCtxGetId", 12000));
-    g_stream_ctx = reinterpret_cast<PFN_cuStreamGetCtx_v9020>(get("cuStreamGetCtx", 9020));
-}
 
 struct ScratchSlot {
     unsigned long long ctx_id;  // context the address was looked up in (0: none yet)
@@ -72,20 +49,14 @@ ScratchSlot g_scratch[kMaxDevices] = {};
 // belongs to that context.  Looked up once per context.
 int scratch_for_current_context(cudaStream_t stream, int32_t **out)
 {
-    std::call_once(g_driver_once, load_driver);
-    if (!g_ctx_current || !g_ctx_id || !g_stream_ctx) return MOE_ERR_CUDA;
     int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
-    CUcontext ctx = nullptr, sctx = nullptr;
+    CUcontext ctx = nullptr;
     unsigned long long id = 0;
-    if (g_ctx_current(&ctx) != CUDA_SUCCESS) return MOE_ERR_CUDA;
-    if (!ctx) {  // no context yet on this thread: cudaSetDevice makes the primary context current
-        if (cudaSetDevice(dev) != cudaSuccess || g_ctx_current(&ctx) != CUDA_SUCCESS || !ctx) return MOE_ERR_CUDA;
-    }
-    if (g_ctx_id(ctx, &id) != CUDA_SUCCESS) return MOE_ERR_CUDA;
-    if (g_stream_ctx(reinterpret_cast<CUstream>(stream), &sctx) != CUDA_SUCCESS) return MOE_ERR_INVALID_ARG;
-    if (sctx != ctx) return MOE_ERR_INVALID_ARG;  // a stream of another device or context
+    int rc = current_context(&dev, &ctx, &id);
+    if (rc != MOE_OK) return rc;
+    if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
+    rc = stream_in_context(stream, ctx);  // a stream of another device or context is rejected
+    if (rc != MOE_OK) return rc;
     std::lock_guard<std::mutex> lock(g_scratch_mu);
     ScratchSlot &slot = g_scratch[dev];
     if (slot.ctx_id != id || !slot.ptr) {
@@ -136,7 +107,6 @@ extern "C" int moe_route_static(int32_t T, int32_t E, int32_t k, const float *lo
     b.chunk_hist = scratch + A;
     b.ttile_a = b.chunk_hist + nch * (size_t)E;
     b.ttile_b = b.ttile_a + (E + 1);
-    b.rowscale = nullptr;
     const long avg = ((long)T * k + E - 1) / E;
     const int bn = avg > 48 ? 64 : 32;
     cudaError_t e = launch_route(logits, T, E, k, topk_idx, topk_w, s);

@@ -362,7 +362,7 @@ int resident_clusters_query(int S)
 {
     using C = SCfg<BN>;
     auto kern = router_splitk_kernel<BN>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess) return 0;
+    if (set_smem_limit(reinterpret_cast<const void *>(kern), C::SMEM) != cudaSuccess) return 0;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = S;
@@ -401,7 +401,7 @@ cudaError_t launch_rt(const CUtensorMap &mw, const CUtensorMap &mx, const Router
 {
     using C = RCfg<BN>;
     auto kern = router_gemm_kernel<BN>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    cudaError_t e = set_smem_limit(reinterpret_cast<const void *>(kern), C::SMEM);
     if (e != cudaSuccess) return e;
     const int tiles = ((a.E + kTileM - 1) / kTileM) * ((a.T + BN - 1) / BN);
     const int grid = tiles < num_sms ? tiles : num_sms;

@@ -83,6 +83,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     return true;
 }
 
+// True iff `p` holds in every one of the `nthreads` threads that reach named barrier `id`
+// (bar.red.and): a barrier that also gives each participating warp the same answer.  Roles of
+// several warps that also meet at named barriers take a wait's outcome through this, so a
+// timeout seen by one warp sends all of them down the same path and none is left waiting at a
+// barrier the others have left.
+__device__ __forceinline__ bool bar_all(int id, int nthreads, bool p)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\tbar.red.and.pred po, %2, %3, pi;\n\t"
+        "selp.u32 %0, 1, 0, po;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)p), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
+}
+
 // Bounded wait that ignores the abort flag: on the way out of a kernel, a thread waits for its
 // own asynchronous work (TMA copies into shared memory, MMAs into tensor memory) to finish
 // before the CTA releases that memory.  Gives up after `timeout_ns` (what is still in flight

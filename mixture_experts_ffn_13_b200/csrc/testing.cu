@@ -163,7 +163,7 @@ cudaError_t launch_rate(int N, int count, int commit_every, int flags, long long
 {
     constexpr bool kPair = FORM >= kRateF16Pair;
     auto kern = mma_rate_kernel<FORM>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kRateSmem);
+    cudaError_t e = set_smem_limit(reinterpret_cast<const void *>(kern), kRateSmem);
     if (e != cudaSuccess) return e;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
