@@ -75,6 +75,8 @@ struct SmallArgs {
     float *xs;                     // [T, H/512] their scales
     float *partG, *partU;          // [kSbSplit][R][Imax] partial gate / up sums
     float *ybuf;                   // [R][H] down outputs of the selected rows
+    uint8_t *hq;                   // [R][Imax] e4m3 codes of h (phase 1.5 -> 2)
+    float *hs;                     // [R][Imax/512] their scales
     int R, Imax;                   // rows (T*k + T) and features per row of the partial sums
     const uint8_t *ws_warm;        // partials and y rows: pages touched early (address translation)
     size_t ws_warm_bytes;
@@ -605,14 +607,70 @@ __global__ void __launch_bounds__(kSbThreads, 1)
                 if (c < T && ((mask >> c) & 1)) part[(size_t)row_of(g, c) * a.Imax + feat] = acc[c];
         }
         if (!grid_sync_epi(a.bar, 2 * nblk, status, abort_flag, tmo)) goto done;
-        // phase 2: the B operand of segment si (group g) into buffer si & 1: h of the group's
-        // selected rows, e4m3 per 512-block.  Columns of tokens that did not pick the group keep
-        // whatever codes the buffer held: an MMA column depends only on its own B row, and those
-        // columns are never stored.
-        auto build_h = [&](int g, int si) -> bool {
+        // phase 1.5, spread over the epilogue warps of the grid: h = silu(G)*U of every row from
+        // the four partial sums, e4m3 per 512-block (the regular path's quantiser), into hq/hs;
+        // one warp per (row, 512-block), lane = 16 consecutive features
+        {
+            const int nbI = I / kBlockK, nbS = Is / kBlockK;
+            const int units = T * k * nbI + T * nbS;
+            for (int u = blockIdx.x * kSbEW + ew; u < units; u += nblk * kSbEW) {
+                int row, kb;
+                if (u < T * k * nbI) {
+                    row = u / nbI;
+                    kb = u - row * nbI;
+                } else {
+                    row = T * k + (u - T * k * nbI) / nbS;
+                    kb = (u - T * k * nbI) % nbS;
+                }
+                const int f0 = kb * kBlockK + lane * 16;
+                float4 vg[kSbSplit][4], vu[kSbSplit][4];
+#pragma unroll
+                for (int sp = 0; sp < kSbSplit; ++sp) {
+                    const size_t o = ((size_t)sp * a.R + row) * a.Imax + f0;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        vg[sp][i] = __ldcg(reinterpret_cast<const float4 *>(a.partG + o) + i);
+                        vu[sp][i] = __ldcg(reinterpret_cast<const float4 *>(a.partU + o) + i);
+                    }
+                }
+                float h[16], am = 0.0f;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    float g4[4] = {0.f, 0.f, 0.f, 0.f}, u4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int sp = 0; sp < kSbSplit; ++sp) {
+                        g4[0] += vg[sp][i].x;
+                        g4[1] += vg[sp][i].y;
+                        g4[2] += vg[sp][i].z;
+                        g4[3] += vg[sp][i].w;
+                        u4[0] += vu[sp][i].x;
+                        u4[1] += vu[sp][i].y;
+                        u4[2] += vu[sp][i].z;
+                        u4[3] += vu[sp][i].w;
+                    }
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        h[4 * i + j] = silu_mul(g4[j], u4[j]);
+                        am = fmaxf(am, fabsf(h[4 * i + j]));
+                    }
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, off));
+                float sc;
+                const uint4 cw = e4m3_codes16(h, am, &sc);
+                *reinterpret_cast<uint4 *>(a.hq + (size_t)row * a.Imax + f0) = cw;
+                if (lane == 0) a.hs[row * (a.Imax / kBlockK) + kb] = sc;
+            }
+        }
+        if (!grid_sync_epi(a.bar, 3 * nblk, status, abort_flag, tmo)) goto done;
+        // phase 2: the B operand of segment si (group g) into buffer si & 1: the codes and scales
+        // of the group's selected rows, copied from hq/hs.  Columns of tokens that did not pick
+        // the group keep whatever codes the buffer held: an MMA column depends only on its own B
+        // row, and those columns are never stored.
+        auto load_h = [&](int g, int si) -> bool {
             const int b = si & 1;
             const int nbK = (g == Gr ? Is : I) / kBlockK;
-            uint8_t *bops = bt + b * (kSbT * kSbMaxI);
+            const uint32_t bops = smem_u32(bt + b * (kSbT * kSbMaxI));
             float *bsc = bscale + b * kSbT * kSbMaxKb;
             if (si >= 2) {
                 // the MMAs of segment si - 2 have read the buffer, and (the vote is also a
@@ -622,50 +680,23 @@ __global__ void __launch_bounds__(kSbThreads, 1)
             }
             const int mask = s_gmask[g];
             const int nsel = __popc(mask);
-            // one warp per (selected token, 512-block); lane: 16 consecutive features
-            for (int u = ew; u < nsel * nbK; u += kSbEW) {
-                const int j = u / nbK, kb = u - j * nbK;
+            const int per_row = nbK * (kBlockK / 16);  // 16-byte chunks of a row's codes
+            for (int c = et; c < nsel * per_row; c += 32 * kSbEW) {
+                const int j = c / per_row, b16 = (c - j * per_row) * 16;
                 int m = mask;
                 for (int i = 0; i < j; ++i) m &= m - 1;
                 const int t = __ffs(m) - 1;
                 const int row = row_of(g, t);
-                const int f0 = kb * kBlockK + lane * 16;
-                float gs[16], us[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) gs[i] = us[i] = 0.0f;
-#pragma unroll
-                for (int sp = 0; sp < kSbSplit; ++sp) {
-                    const size_t o = ((size_t)sp * a.R + row) * a.Imax + f0;
-                    const float4 *pg = reinterpret_cast<const float4 *>(a.partG + o);
-                    const float4 *pu = reinterpret_cast<const float4 *>(a.partU + o);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float4 vg = __ldcg(pg + i), vu = __ldcg(pu + i);
-                        gs[4 * i] += vg.x;
-                        gs[4 * i + 1] += vg.y;
-                        gs[4 * i + 2] += vg.z;
-                        gs[4 * i + 3] += vg.w;
-                        us[4 * i] += vu.x;
-                        us[4 * i + 1] += vu.y;
-                        us[4 * i + 2] += vu.z;
-                        us[4 * i + 3] += vu.w;
-                    }
-                }
-                float h[16], am = 0.0f;
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    h[i] = silu_mul(gs[i], us[i]);
-                    am = fmaxf(am, fabsf(h[i]));
-                }
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, off));
-                float sc;
-                *reinterpret_cast<uint4 *>(bops + bt_off(t, f0)) = e4m3_codes16(h, am, &sc);
-                if (lane == 0) bsc[t * kSbMaxKb + kb] = sc;
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(bops + bt_off(t, b16)),
+                             "l"(a.hq + (size_t)row * a.Imax + b16)
+                             : "memory");
+                if (b16 % kBlockK == 0) bsc[t * kSbMaxKb + b16 / kBlockK] = __ldcg(a.hs + row * (a.Imax / kBlockK) + b16 / kBlockK);
             }
+            asm volatile("cp.async.wait_all;" ::: "memory");
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // h codes, for the tensor cores
             __syncwarp();
             if (lane == 0) mbar_arrive(&bready[b]);
+            epi_sync();  // the scales are in place for every epilogue warp
             return true;
         };
         // this thread's down-weight scales of item w, loaded one item ahead as in phase 1
@@ -682,11 +713,11 @@ __global__ void __launch_bounds__(kSbThreads, 1)
         float scn2[kB2];
         if (w2lo < w2hi) scales2(w2lo, scn2);
         int si = 0;
-        if (w2lo < w2hi && !build_h(grp2(w2lo), 0)) goto done;
+        if (w2lo < w2hi && !load_h(grp2(w2lo), 0)) goto done;
         for (int w = w2lo; w < w2hi; ++si) {
             const int g = grp2(w);
             const int wend = min(w2hi, (w / ntile + 1) * ntile);  // end of this segment
-            if (wend < w2hi && !build_h(grp2(wend), si + 1)) goto done;
+            if (wend < w2hi && !load_h(grp2(wend), si + 1)) goto done;
             const bool sh = g == Gr;
             const int nbK = (sh ? Is : I) / kBlockK;
             const float *bsc = bscale + (si & 1) * kSbT * kSbMaxKb;
@@ -723,7 +754,7 @@ __global__ void __launch_bounds__(kSbThreads, 1)
                     if (c < T && ((mask >> c) & 1)) a.ybuf[(size_t)row_of(g, c) * H + n] = acc[c];
             }
         }
-        if (!grid_sync_epi(a.bar, 3 * nblk, status, abort_flag, tmo)) goto done;
+        if (!grid_sync_epi(a.bar, 4 * nblk, status, abort_flag, tmo)) goto done;
         // phase 3: combine, 4 hidden features per thread over all CTAs
         for (int i = blockIdx.x * (32 * kSbEW) + et; i < T * H / 4; i += nblk * (32 * kSbEW)) {
             const int t = i / (H / 4), c4 = i - t * (H / 4);
@@ -781,7 +812,7 @@ int env_small_batch()
 // Workspace carve-up for a batch of T tokens (every region 256-byte aligned; sizes grow with T,
 // so the layout for T_max bounds every smaller batch's).
 struct SbLayout {
-    size_t bar, partG, partU, ybuf, tk_idx, tk_w, xq, xs, total;
+    size_t bar, partG, partU, ybuf, hq, hs, tk_idx, tk_w, xq, xs, total;
 };
 
 SbLayout sb_layout(size_t T, const moe_dims &d)
@@ -795,7 +826,9 @@ SbLayout sb_layout(size_t T, const moe_dims &d)
     L.partG = 256;
     L.partU = al(L.partG + part);
     L.ybuf = al(L.partU + part);
-    L.tk_idx = al(L.ybuf + R * (size_t)d.H * 4);
+    L.hq = al(L.ybuf + R * (size_t)d.H * 4);
+    L.hs = al(L.hq + R * Imax);
+    L.tk_idx = al(L.hs + R * (Imax / kBlockK) * 4);
     L.tk_w = al(L.tk_idx + T * (size_t)d.k * 4);
     L.xq = al(L.tk_w + T * (size_t)d.k * 4);
     L.xs = al(L.xq + T * (size_t)d.H);
@@ -866,6 +899,8 @@ cudaError_t launch_small_batch(const moe_dims &d, int T, const uint16_t *x, cons
     a.partG = reinterpret_cast<float *>(p + L.partG);
     a.partU = reinterpret_cast<float *>(p + L.partU);
     a.ybuf = reinterpret_cast<float *>(p + L.ybuf);
+    a.hq = p + L.hq;
+    a.hs = reinterpret_cast<float *>(p + L.hs);
     a.bar = reinterpret_cast<unsigned *>(p + L.bar);
     a.tk_idx = reinterpret_cast<int32_t *>(p + L.tk_idx);
     a.tk_w = reinterpret_cast<float *>(p + L.tk_w);

@@ -62,7 +62,9 @@ def test_mma_rate_argument_errors(L):
     assert L.moe_test_mma_rate(3, 16, 8, 0, 0, cyc.data_ptr(), status.data_ptr(), st) == -1   # pair N < 32
     assert L.moe_test_mma_rate(9, 64, 8, 0, 0, cyc.data_ptr(), status.data_ptr(), st) == -1   # form
     assert L.moe_test_mma_rate(0, 64, 0, 0, 0, cyc.data_ptr(), status.data_ptr(), st) == -1   # count
-    assert L.moe_test_mma_rate(0, 64, 8, 0, 4, cyc.data_ptr(), status.data_ptr(), st) == -1   # flags
+    assert L.moe_test_mma_rate(0, 64, 8, 0, 8, cyc.data_ptr(), status.data_ptr(), st) == -1   # flags > 7
+    assert L.moe_test_mma_rate(0, 64, 8, 0, 5, cyc.data_ptr(), status.data_ptr(), st) == -1   # two issuers + alternation
+    assert L.moe_test_mma_rate(3, 64, 8, 0, 4, cyc.data_ptr(), status.data_ptr(), st) == -1   # two issuers on a pair form
     assert L.moe_test_mma_rate(1, 256, 8, 4, 1, cyc.data_ptr(), status.data_ptr(), st) == -1  # TS A overlap
 
 
