@@ -88,10 +88,11 @@ struct I4Cfg {
     static constexpr int NB_FIT = (212 * 1024 - NR * NA * RAW_BYTES) / B_BYTES;
     static constexpr int NB = NB_FIT < 12 ? NB_FIT : 12;     // activation stages (64 K each)
     static constexpr int TT_BYTES = (4 * (kMaxE + 1) + 15) & ~15;  // keeps the mbarriers 8-byte aligned
-    static constexpr int BAR_BYTES = 8 * (2 * NR + 2 * NB + 2 * NM + 2 * NSLOT) + 24;
+    static constexpr int BAR_BYTES = 8 * (2 * NR + 2 * NB + NM + 2 * NSLOT) + 24;
     static constexpr int SMEM = 1024 + NB * B_BYTES + NR * NA * RAW_BYTES + TT_BYTES + BAR_BYTES;
     static_assert(B_BYTES % 1024 == 0, "1024-byte aligned tiles");
     static_assert(NSLOT >= 2, "TMEM slots");
+    static_assert(NB > NM, "the weight stages' release is read from the deeper activation ring");
     static_assert(CONV % 4 == 0 && EW % 4 == 0, "whole TMEM lane quarters per role");
     static_assert(SMEM <= 227 * 1024, "shared memory");
     static_assert((NR * NA * RAW_BYTES + NB * B_BYTES + TT_BYTES) % 16 == 0, "mbarriers must be 8-byte aligned");
@@ -178,8 +179,7 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
     uint64_t *bfull = rempty + C::NR;
     uint64_t *bempty = bfull + C::NB;
     uint64_t *mfull = bempty + C::NB;
-    uint64_t *mempty = mfull + C::NM;
-    uint64_t *accf = mempty + C::NM;
+    uint64_t *accf = mfull + C::NM;
     uint64_t *acce = accf + C::NSLOT;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(acce + C::NSLOT);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
@@ -196,10 +196,10 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
             mbar_init(&bfull[s], 1);
             mbar_init(&bempty[s], 2);
         }
-        for (int s = 0; s < C::NM; ++s) {
-            mbar_init(&mfull[s], C::CONV);
-            mbar_init(&mempty[s], 2);
-        }
+        // a TMEM weight stage is free again once the MMAs of the stage that used it have
+        // completed, which bempty of that stage records (the ring of activation stages is
+        // deeper than the ring of weight stages, so the phase waited for is never overtaken)
+        for (int s = 0; s < C::NM; ++s) mbar_init(&mfull[s], C::CONV);
         for (int s = 0; s < C::NSLOT; ++s) {
             mbar_init(&accf[s], 2);
             mbar_init(&acce[s], C::EW);
@@ -318,8 +318,7 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
 #pragma unroll
                         for (int kk = 0; kk < kKE / 16; ++kk)
                             mma_bf16_ts(d, a + 8 * kk, db + 2 * kk, kIdesc, (sk > 0 || kk > 0) ? 1u : 0u);
-                        mma_commit(&mempty[s]);
-                        mma_commit(&bempty[bs]);
+                        mma_commit(&bempty[bs]);  // frees the activation stage and the TMEM weight stage
                     }
                     mma_commit(&accf[slot]);
                 }
@@ -386,7 +385,11 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
                 bool ok = true;
                 if (sub == 0) ok = mbar_wait(&rfull[rs_i], (rt / C::NR) & 1, abort_flag, status, tmo);
                 if (!__all_sync(0xffffffffu, ok)) goto done;
-                ok = mbar_wait(&mempty[ms_i], ((it / C::NM) & 1) ^ 1, abort_flag, status, tmo);
+                // TMEM stage ms_i was last read by the MMAs of stage it - NM
+                if (it >= (uint32_t)C::NM) {
+                    const uint32_t j = it - C::NM;
+                    ok = mbar_wait(&bempty[j % C::NB], (j / C::NB) & 1, abort_flag, status, tmo);
+                }
                 if (!__all_sync(0xffffffffu, ok)) goto done;
                 tc_fence_after();
                 const uint8_t *rs = raw + rs_i * C::NA * C::RAW_BYTES + r * 128;

@@ -20,15 +20,18 @@
 //    stores the partial G and U of the selected tokens' rows.  Splitting K four ways gives ~4x
 //    more items than SMs at T = 1;
 //  * grid barrier;
+//  * phase 1.5, spread over the epilogue warps of the grid, one warp per (row, 512-block):
+//    h = silu(G)*U from the four partials, quantised to e4m3 exactly as the regular path does,
+//    into the workspace (each row once, whichever CTAs later stream its expert);
+//  * grid barrier;
 //  * phase 2: down.  Work items are (expert, 128 rows of H), the shared expert's first, and each
 //    CTA takes a contiguous run of them, so consecutive items mostly share an expert.  For each
-//    expert of its run a CTA forms h = silu(G)*U from the four partials of the selected rows,
-//    quantises it per 512-block exactly as the regular path does, and lays it out in shared
-//    memory as the B operand (double-buffered: the next expert's operand is built while the
-//    current one's weights stream); the epilogue promotes and stores y for the selected rows;
+//    expert of its run a CTA copies the selected rows' h codes into shared memory as the B
+//    operand (double-buffered: the next expert's operand is copied while the current one's
+//    weights stream); the epilogue promotes and stores y for the selected rows;
 //  * grid barrier, then phase 3: out[t] = sum_j p_hat[t,j] * y(t, e_j) + y_shared(t) in fp32,
 //    rounded to bf16.
-// The producer warp streams phase 2's weights while the phase-1 barrier is pending.  Every wait
+// The producer warp streams phase 2's weights while the barriers before it are pending.  Every wait
 // is bounded and reports MOE_ERR_DEVICE_TIMEOUT through the status word; the epilogue warps
 // take every wait's outcome together (bar.red), so none is left behind at a named barrier.
 #include "moe_internal.h"

@@ -74,6 +74,9 @@ PROFILE_CONFIGS = {
                           workload="MXFP4 MoE T=128 H=4096 E=16 I=1536 top-8, e2m1 + E8M0/32"),
     "profile-nvfp4": dict(T=128, H=4096, E=16, I=1536, k=8, Is=0, wfmt="nvfp4", seed=11, bias=None,
                           workload="NVFP4 MoE T=128 H=4096 E=16 I=1536 top-8, e2m1 + E4M3/16 + tensor scale"),
+    # 16 tokens: the single-kernel small-batch path
+    "profile-small": dict(T=16, H=4096, E=64, I=1024, k=10, Is=1024, wfmt="fp8", seed=12, bias=None,
+                          workload="decode-shaped MoE T=16 H=4096 E=64 I=1024 top-10 + shared 1024, FP8"),
 }
 
 # tensor ids for the per-tensor generators
