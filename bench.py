@@ -29,11 +29,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM traffic of the gate|up GEMM per algorithmic byte: one ncu capture of
 # dram__bytes_read.sum + dram__bytes_write.sum for the gate|up launch of the decode-shaped
-# profiling workload (moe_synth "profile-decode": 552,512,000 + 3,825,408 bytes against
+# profiling workload (moe_synth "profile-decode": 552,476,416 + 3,635,712 bytes against
 # 549,519,360 algorithmic), scaled to a decode launch by its algorithmic bytes.  Stored with
 # the hash of the kernel source it was taken on; the figure is null once that source changes.
-TRAFFIC = {"decode": {"kernel": "gemm_gateup", "ratio": (552512000 + 3825408) / 549519360,
-                      "src_sha": "7a3b63e6f3243785"}}
+TRAFFIC = {"decode": {"kernel": "gemm_gateup", "ratio": (552476416 + 3635712) / 549519360,
+                      "src_sha": "4beb1fb13146fb9a"}}
 
 
 def parse():
@@ -355,7 +355,13 @@ def measure_layer(cfg_name, steps, warmup, ws, rank, local, pk, pk_src, fp8_tf, 
     ms_step = total_ms / steps
     mean_stage = {k: v / steps for k, v in stage_ms.items()}
     dom = max(("gemm_gateup", "gemm_down"), key=lambda s_: mean_stage[s_])
-    achieved = alg[dom] / (mean_stage[dom] / 1e3) / 1e9
+    dom_ms = mean_stage[dom]
+    if moe.moe_launch_count(m.plan) == 1:
+        # the single-kernel small-batch path: one launch does the whole layer, so the dominant
+        # kernel is that launch and its bytes are the layer's
+        dom, dom_ms = "small_batch", sum(mean_stage.values())
+        alg = dict(alg, small_batch=alg["layer"], flops_small_batch=alg["flops"])
+    achieved = alg[dom] / (dom_ms / 1e3) / 1e9
     layer_gbs = alg["layer"] / (ms_step / 1e3) / 1e9
     if cfg["wfmt"] == "fp8":
         if fp8_tf:
@@ -376,9 +382,9 @@ def measure_layer(cfg_name, steps, warmup, ws, rank, local, pk, pk_src, fp8_tf, 
                      "peak_source": pk_src, "layer_achieved_gbs": layer_gbs, "layer_frac": layer_gbs / pk["hbm_gbs"]},
         # tensor-core view of the same run: FP8 MMAs against the FP8 peak named in peak_source,
         # the 4-bit path's bf16 MMAs against the bf16 peak
-        "tensor": {"kernel": dom, "achieved": alg["flops_" + dom] / (mean_stage[dom] / 1e3) / 1e12,
+        "tensor": {"kernel": dom, "achieved": alg["flops_" + dom] / (dom_ms / 1e3) / 1e12,
                    "peak": tpk, "unit": "TFLOP/s",
-                   "frac": alg["flops_" + dom] / (mean_stage[dom] / 1e3) / 1e12 / tpk,
+                   "frac": alg["flops_" + dom] / (dom_ms / 1e3) / 1e12 / tpk,
                    "layer_achieved": alg["flops"] / (ms_step / 1e3) / 1e12,
                    "layer_frac": alg["flops"] / (ms_step / 1e3) / 1e12 / tpk, "peak_source": tpk_src},
         # the layer's binding roofline: the slower of streaming its algorithmic bytes at the

@@ -527,9 +527,22 @@ int moe_forward(moe_plan_t *p, int32_t T, const uint16_t *x, const float *logits
     const uint32_t wbox = ilv ? 16 : 128;  // weight rows per TMA box (2-D maps)
     const uint32_t kXBox = bn_a < 64 ? bn_a : 64;  // activation rows per TMA box
 
+    // When nearly every expert is picked (T*k >= 2E: each misses with probability < e^-2), the
+    // gate|up GEMM's first wave of work items is the leading experts' weight tiles (items run
+    // expert by expert).  The route kernel asks L2 for the first ~96 MB of them, so that part of
+    // the weight stream overlaps routing, permutation and quantisation instead of following them.
+    WeightPrefetch pf;
+    if ((int64_t)T * k >= 2 * (int64_t)E && aligned16(w->w_gate) && aligned16(w->w_up)) {
+        const size_t per_expert = (size_t)I * H;
+        const size_t budget = 48u << 20;  // per matrix
+        const size_t n_exp = std::min<size_t>((size_t)E, budget / per_expert);
+        pf.a = static_cast<const uint8_t *>(w->w_gate);
+        pf.b = static_cast<const uint8_t *>(w->w_up);
+        pf.chunks = (uint32_t)(n_exp * per_expert / WeightPrefetch::kChunk);
+    }
     mark(0);
     int *chk = p->checked ? p->d_status : nullptr;
-    cudaError_t e = launch_route(logits, T, E, k, b.topk_idx, b.topk_w, s, chk);
+    cudaError_t e = launch_route(logits, T, E, k, b.topk_idx, b.topk_w, s, chk, pf);
     mark(1);
     if (e == cudaSuccess) e = launch_permute_any(b, T, E, k, bn_a, bn_b, s);
     mark(2);

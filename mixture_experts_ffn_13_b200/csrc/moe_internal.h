@@ -43,9 +43,17 @@ struct RouteBufs {
     int32_t *ttile_b;     // [E + 1] token-tile prefix for the down GEMM tile size
 };
 
+// An L2 prefetch the route kernel issues before it waits on the previous kernel: `chunks`
+// blocks of kChunk bytes from each of a and b (16-byte aligned), or nothing (chunks = 0).
+struct WeightPrefetch {
+    static constexpr uint32_t kChunk = 64 * 1024;
+    const uint8_t *a = nullptr, *b = nullptr;
+    uint32_t chunks = 0;
+};
+
 // check != nullptr (checked mode): non-finite logits record MOE_ERR_BOUNDS in *check.
 cudaError_t launch_route(const float *logits, int T, int E, int k, int32_t *topk_idx, float *topk_w,
-                         cudaStream_t s, int *check = nullptr);
+                         cudaStream_t s, int *check = nullptr, WeightPrefetch pf = WeightPrefetch());
 cudaError_t launch_permute(const RouteBufs &b, int T, int E, int k, int bn_a, int bn_b, cudaStream_t s);
 // Permutation: one single-block kernel for small batches, else the three launches above.
 cudaError_t launch_permute_any(const RouteBufs &b, int T, int E, int k, int bn_a, int bn_b, cudaStream_t s);

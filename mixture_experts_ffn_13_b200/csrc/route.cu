@@ -15,6 +15,8 @@
 #include "launch.cuh"
 #include "moe_internal.h"
 
+#include <algorithm>
+
 #include <math.h>
 
 namespace moe {
@@ -82,8 +84,22 @@ __device__ __forceinline__ void route_one(const float *__restrict__ L, int E, in
 template <int EPL>
 __global__ void __launch_bounds__(256) route_kernel(const float *__restrict__ logits, int T, int E, int k,
                                                     int32_t *__restrict__ topk_idx, float *__restrict__ topk_w,
-                                                    int *check)
+                                                    int *check, WeightPrefetch pf)
 {
+    // Blocks past the routing ones only ask L2 for weights that no kernel of this stream writes
+    // (before waiting on the previous kernel), so the weight stream overlaps routing, permutation
+    // and quantisation without delaying the routing blocks, whose issue is latency-bound.
+    const uint32_t nroute = (T + 7) / 8;
+    if (blockIdx.x >= nroute) {
+        const uint32_t npf = gridDim.x - nroute;
+        for (uint32_t c = (blockIdx.x - nroute) + npf * threadIdx.x; c < 2 * pf.chunks; c += npf * blockDim.x) {
+            const uint8_t *src = (c & 1 ? pf.b : pf.a) + (size_t)(c >> 1) * WeightPrefetch::kChunk;
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(WeightPrefetch::kChunk)
+                         : "memory");
+        }
+        griddep_launch_dependents();
+        return;
+    }
     griddep_wait();
     griddep_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -380,12 +396,17 @@ int route_permute_launches(int T, int E, int k)
 }
 
 cudaError_t launch_route(const float *logits, int T, int E, int k, int32_t *topk_idx, float *topk_w,
-                         cudaStream_t s, int *check)
+                         cudaStream_t s, int *check, WeightPrefetch pf)
 {
     if (T <= 0) return cudaSuccess;
-    const dim3 grid((T + 7) / 8), block(256);
+    // prefetching blocks: spread over the SMs (a few 64 KB chunks each), since one SM issues
+    // bulk prefetches at about its share of the L2 bandwidth
+    const int npf = (int)std::min<uint32_t>(128u, 2 * pf.chunks);
+    const dim3 grid((T + 7) / 8 + npf), block(256);
     const int epl = (E + 31) / 32;
-    auto go = [&](auto kern) { return launch_pdl(kern, grid, block, 0, s, logits, T, E, k, topk_idx, topk_w, check); };
+    auto go = [&](auto kern) {
+        return launch_pdl(kern, grid, block, 0, s, logits, T, E, k, topk_idx, topk_w, check, pf);
+    };
     if (epl <= 1) return go(route_kernel<1>);
     if (epl <= 2) return go(route_kernel<2>);
     if (epl <= 4) return go(route_kernel<4>);
