@@ -38,9 +38,10 @@
 //    interleaved weight tile is one 4-D TMA box: (128 K bytes, 16 rows, {gate, up}, 4 row
 //    groups), the {gate, up} dimension's stride being the distance between the two arrays.
 //  * down: one weight tile; y is stored in fp32.
-//  * Wide token tiles load activations in 64-row boxes, only as many as the tile has rows, and
-//    size the MMA's N to the tile's valid rows rounded up to 16.  The producer warp issues a
-//    stage's copies from separate lanes, one copy each.
+//  * Every token tile loads its activations as one BN-row box (a TMA copy has a fixed cost of
+//    the order of 0.1 us in the SM's copy engine, so a stage is as few copies as possible), and
+//    wide tiles size the MMA's N to the tile's valid rows rounded up to 16.  The producer warp
+//    issues a wide stage's copies from separate lanes, one copy each.
 #include "moe_internal.h"
 #include "gemm_common.cuh"
 #include "launch.cuh"
@@ -55,10 +56,14 @@ constexpr int kStagesPerBlock = kBlockK / kKC;
 constexpr int kMaxKb = 16;   // activation-scale staging holds up to 16 blocks (K <= 8192)
 constexpr int kSmemLimit = 227 * 1024;
 
-// Activation boxes: narrow tiles load BN rows in one box; wide tiles load 64-row boxes.
+// Activation boxes: every tile loads its BN rows as one box.  A TMA copy costs the SM's copy
+// engine on the order of a hundred nanoseconds whatever its size (measured: a wide stage of four
+// copies took ~0.48 us to issue whether it held 40 KB or 28 KB), so a stage is as few copies as
+// possible; rows past the tensor's end are zero-filled and rows past the tile's group are never
+// used (the MMA's N covers the valid rows).
 template <int BN>
 struct BoxOf {
-    static constexpr int ROWS = BN >= 64 ? 64 : BN;
+    static constexpr int ROWS = BN;
     static constexpr int BYTES = ROWS * kKC;
 };
 
@@ -72,8 +77,8 @@ struct Fp8Cfg {
     static constexpr int RT = ILV ? kTileM / 2 : kTileM;  // output features per tile
     static constexpr int NA = PAIR ? 2 : 1;
     static constexpr int A_BYTES = kTileM * kKC;
-    // activation rows a stage holds: wide tiles round up to whole 64-row boxes
-    static constexpr int B_ROWS = BN >= 64 ? (BN + 63) / 64 * 64 : BN;
+    // activation rows a stage holds: the tile's box
+    static constexpr int B_ROWS = BN;
     static constexpr int B_BYTES = B_ROWS * kKC;
     static constexpr int STAGE_BYTES = NA * A_BYTES + B_BYTES;
     static constexpr int SLOT_COLS = NA * BN;
@@ -187,9 +192,8 @@ __global__ void __launch_bounds__(Fp8Cfg<BN, MODE, EW>::THREADS, 1)
             const TileInfo tl = decode_tile<BN, kStageSx, RT>(args, ttab, w, tot0);
             const GemmSeg &sg = args.seg[tl.seg];
             const int nkc = sg.K / kKC;
-            // activation boxes: the whole BN-row tile for narrow tiles, else 64-row boxes up to
-            // the tile's valid rows
-            const int nbox = C::WIDE ? (tl.nrows + kBoxRows - 1) / kBoxRows : 1;
+            // activation copies: one box of the whole BN-row tile
+            const int nbox = 1;
             // weight copies: the paired form loads two 128-row tiles; the interleaved form one
             // 4-D box or eight 16-row boxes
             const int nwa = C::ILV ? (sg.ilv4d ? 1 : 8) : C::NA;

@@ -525,7 +525,7 @@ int moe_forward(moe_plan_t *p, int32_t T, const uint16_t *x, const float *logits
     const int bn_a = bn_b;
     const bool ilv = bn_a > 64;
     const uint32_t wbox = ilv ? 16 : 128;  // weight rows per TMA box (2-D maps)
-    const uint32_t kXBox = bn_a < 64 ? bn_a : 64;  // activation rows per TMA box
+    const uint32_t kXBox = bn_a;  // activation rows per TMA box: the whole token tile
 
     // When nearly every expert is picked (T*k >= 2E: each misses with probability < e^-2), the
     // gate|up GEMM's first wave of work items is the leading experts' weight tiles (items run
@@ -610,7 +610,7 @@ int moe_forward(moe_plan_t *p, int32_t T, const uint16_t *x, const float *logits
     GemmArgs ad = ag;
     ad.ttile = b.ttile_b;
     ad.seg[0] = GemmSeg{H, I, A, w->s_down, nullptr, sh, y};
-    const uint32_t kHBox = bn_b < 64 ? bn_b : 64;
+    const uint32_t kHBox = bn_b;  // the whole token tile per TMA box
     rc = encode_map_2d(&md.a0[0], w->w_down, U8, 1, I, (uint64_t)E * H, 128, 128, true);
     rc |= encode_map_2d(&md.b[0], hq, U8, 1, I, A, 128, kHBox, true);
     if (shared) {
