@@ -126,7 +126,7 @@ cudaError_t launch_gemm_fp8(bool gateup, int bn, const GemmMaps &maps, const Gem
 cudaError_t launch_gemm_w4(bool gateup, int wfmt, int bn, const GemmMaps &maps, const GemmArgs &args,
                            int num_sms, cudaStream_t s);
 
-// Small batches (T <= 16, FP8 weights): the whole layer in one cooperative persistent kernel
+// Small batches (2 <= T <= 16, FP8 weights): the whole layer in one cooperative persistent kernel
 // (small_batch.cu).  small_batch_fits: shapes it takes (H a multiple of 2048 up to 4096, I and
 // I_shared multiples of 512 up to 2048); small_batch_workspace: the bytes it needs in the
 // workspace (partial sums, y rows, a grid-barrier counter).  launch_small_batch returns

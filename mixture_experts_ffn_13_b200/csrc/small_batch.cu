@@ -3,7 +3,7 @@
 // Page "TPU推理外部化全面加速：InferenceX首份第三方性能數據發布", sections "优化 MoE 路由与专家内核" and
 // "减少填充和低并发开销": at low concurrency the per-step overheads of routing, permutation and
 // padding dominate, and for small batches the permutation is done as a one-hot selection
-// instead of a sort.  Here, for T <= 16, one cooperative launch (one CTA per SM) does the layer:
+// instead of a sort.  Here, for 2 <= T <= 16, one cooperative launch (one CTA per SM) does the layer:
 //  * phase 0a, spread over the grid, one warp per unit: the softmax top-k of one token, or the
 //    e4m3 quantisation of one (token, 512-block) of x; results go to the workspace.  Meanwhile
 //    every CTA asks L2 to prefetch its slice of the shared expert's weights, which no routing
@@ -51,7 +51,7 @@ constexpr int kSbT = 16;                        // token columns of every MMA (t
 constexpr int kSbKC = 128;                      // K bytes per weight stage
 constexpr int kSbSplit = 4;                     // gate|up: K split into quarters
 constexpr int kSbStage = 128 * kSbKC;           // 16 KB weight tile per stage
-constexpr int kSbNS = 8;                        // weight stages
+constexpr int kSbNS = 5;                        // weight stages: a smaller shared-memory carve-out leaves more L1 (measured: 5 beats 4, 6, 8 and 9)
 constexpr int kSbEW = 4;                        // epilogue warps (one per TMEM lane quarter)
 constexpr int kSbWarps = 2 + kSbEW;
 constexpr int kSbThreads = 32 * kSbWarps;       // producer, MMA issuer, epilogue
@@ -843,7 +843,9 @@ SbLayout sb_layout(size_t T, const moe_dims &d)
 
 bool small_batch_fits(int T, const moe_dims &d)
 {
-    return env_small_batch() && d.wfmt == MOE_W_FP8_SC512 && T >= 1 && T <= kSbT && d.H <= kSbMaxH &&
+    // T = 1 stays on the multi-kernel path, which measured faster there (66.6 against ~70 us on
+    // the decode-shaped layer); from 2 to 16 tokens the single kernel is as fast or faster
+    return env_small_batch() && d.wfmt == MOE_W_FP8_SC512 && T >= 2 && T <= kSbT && d.H <= kSbMaxH &&
            d.H % (kSbSplit * kBlockK) == 0 && d.I <= kSbMaxI && d.I % kBlockK == 0 &&
            (d.I_shared == 0 || (d.I_shared <= kSbMaxI && d.I_shared % kBlockK == 0)) && d.E <= kMaxE &&
            d.k <= kMaxK;

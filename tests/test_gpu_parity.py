@@ -337,7 +337,8 @@ def test_layer_small_batch_single_kernel(cfg):
     m = moe.MoELayer(layer)
     out = m(layer["x"], layer["logits"])
     assert moe.moe_get_status(m.plan) == 0
-    assert moe.moe_launch_count(m.plan) == 1  # the single-kernel path ran
+    # the single-kernel path runs from 2 to 16 tokens; one token takes the multi-kernel path
+    assert (moe.moe_launch_count(m.plan) == 1) == (cfg["T"] >= 2)
     want, _, amb = oracle.layer(moe_synth.to_numpy(layer), ambiguity=True)
     check_out(out, want, "small batch", amb)
     # no atomics decide any value: repeated calls are bit-identical (a race between the kernel's
