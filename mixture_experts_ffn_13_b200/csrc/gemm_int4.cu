@@ -85,8 +85,13 @@ struct I4Cfg {
     static constexpr int NSLOT = (512 - A_TMEM) / SLOT_COLS;
     static constexpr int STAGES_PER_GROUP = kGroupK / kKE;  // 2
     static constexpr int NR = GATEUP ? 3 : 5;               // raw weight stages (256 K each)
-    static constexpr int NB_FIT = (212 * 1024 - NR * NA * RAW_BYTES) / B_BYTES;
-    static constexpr int NB = NB_FIT < 12 ? NB_FIT : 12;     // activation stages (64 K each)
+    // activation stages (64 K each).  int4 keeps the block within 196 KB of shared memory, so
+    // that the carve-out leaves ~60 KB of L1 for its epilogue's scale loads (int4 layer 1.061
+    // against 1.064 ms); the E2M1 formats have no such loads and keep the deeper ring (MXFP4
+    // 1.185 against 1.206 ms with the int4 budget, NVFP4 even).
+    static constexpr int SMEM_BUDGET = FP4 ? 212 * 1024 : 190 * 1024;
+    static constexpr int NB_FIT = (SMEM_BUDGET - NR * NA * RAW_BYTES) / B_BYTES;
+    static constexpr int NB = NB_FIT < 12 ? NB_FIT : 12;
     static constexpr int TT_BYTES = (4 * (kMaxE + 1) + 15) & ~15;  // keeps the mbarriers 8-byte aligned
     static constexpr int BAR_BYTES = 8 * (2 * NR + 2 * NB + NM + 2 * NSLOT) + 24;
     static constexpr int SMEM = 1024 + NB * B_BYTES + NR * NA * RAW_BYTES + TT_BYTES + BAR_BYTES;
@@ -94,7 +99,7 @@ struct I4Cfg {
     static_assert(NSLOT >= 2, "TMEM slots");
     static_assert(NB > NM, "the weight stages' release is read from the deeper activation ring");
     static_assert(CONV % 4 == 0 && EW % 4 == 0, "whole TMEM lane quarters per role");
-    static_assert(SMEM <= 227 * 1024, "shared memory");
+    static_assert(SMEM <= (FP4 ? 227 : 196) * 1024, "shared memory (int4: within the carve-out that leaves ~60 KB of L1)");
     static_assert((NR * NA * RAW_BYTES + NB * B_BYTES + TT_BYTES) % 16 == 0, "mbarriers must be 8-byte aligned");
 };
 
