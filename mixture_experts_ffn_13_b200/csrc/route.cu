@@ -221,10 +221,26 @@ __global__ void __launch_bounds__(1024) scan_kernel(int nchunks, int E, int32_t 
     __shared__ int scratch[33];
     griddep_wait();
     griddep_launch_dependents();
+    // Each thread walks its expert's column of chunk counts.  A store and the next load go
+    // through the same pointer, so the compiler keeps them in order; the column is therefore
+    // walked kBatch entries at a time, all loads of a batch issued before its stores, so that
+    // a long column (4096 chunks at 2^20 tokens) costs nchunks / kBatch memory round trips.
+    constexpr int kBatch = 16;
     const int e = threadIdx.x;
     int c = 0;
     if (e < E) {
-        for (int ch = 0; ch < nchunks; ++ch) {
+        int ch = 0;
+        for (; ch + kBatch <= nchunks; ch += kBatch) {
+            int v[kBatch];
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j) v[j] = chunk_hist[(size_t)(ch + j) * E + e];
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j) {
+                chunk_hist[(size_t)(ch + j) * E + e] = c;
+                c += v[j];
+            }
+        }
+        for (; ch < nchunks; ++ch) {
             const int v = chunk_hist[(size_t)ch * E + e];
             chunk_hist[(size_t)ch * E + e] = c;
             c += v;
@@ -235,7 +251,15 @@ __global__ void __launch_bounds__(1024) scan_kernel(int nchunks, int E, int32_t 
     const int off = block_exclusive_scan(e < E ? c : 0, scratch, &total);
     if (e < E) {
         offsets[e] = off;
-        for (int ch = 0; ch < nchunks; ++ch) chunk_hist[(size_t)ch * E + e] += off;
+        int ch = 0;
+        for (; ch + kBatch <= nchunks; ch += kBatch) {
+            int v[kBatch];
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j) v[j] = chunk_hist[(size_t)(ch + j) * E + e];
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j) chunk_hist[(size_t)(ch + j) * E + e] = v[j] + off;
+        }
+        for (; ch < nchunks; ++ch) chunk_hist[(size_t)ch * E + e] += off;
     }
     if (e == 0) offsets[E] = total;
     const int ta = (e < E) ? (c + bn_a - 1) / bn_a : 0;

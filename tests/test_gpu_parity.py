@@ -86,6 +86,17 @@ def test_route_random(T, E, k):
     check_route(plan, ws, logits, k)
 
 
+def test_route_long_chunk_column():
+    """70000 tokens: 274 chunks of 256 in the multi-kernel permutation, so the per-expert
+    chunk scan runs many full batches of chunks and a remainder; bit-exact against the oracle."""
+    T, E, k = 70000, 256, 8
+    plan = moe.Plan(T, 128, E, 128, k)
+    ws = plan.new_workspace()
+    g = torch.Generator(device="cuda").manual_seed(11)
+    logits = torch.randn((T, E), generator=g, device="cuda")
+    check_route(plan, ws, logits, k)
+
+
 def test_route_ties_and_plateaus():
     T, E, k = 600, 96, 7
     plan = moe.Plan(T, 128, E, 128, k)
