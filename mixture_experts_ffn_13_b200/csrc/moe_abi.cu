@@ -389,7 +389,7 @@ static int forward_w4(moe_plan_t *p, int T, const uint16_t *x, const float *logi
     if (e != cudaSuccess) return fail_cuda(p, e);
     uint16_t *xp = reinterpret_cast<uint16_t *>(ws + L.act);
     uint16_t *xp_sh = shared ? xp + (size_t)A * H : nullptr;
-    e = launch_gather_x_bf16(x, T, H, k, b.pos, xp, xp_sh, s);
+    e = launch_gather_x_bf16(x, T, H, k, b.pos, xp, xp_sh, d.wfmt == MOE_W_INT4_G128, s);
     mark(3);
     if (e != cudaSuccess) return fail_cuda(p, e);
 

@@ -73,9 +73,10 @@ cudaError_t launch_quant_x_fp8(const uint16_t *x, int T, int H, int k, const int
 // h1 is null or R1 == 0).
 cudaError_t launch_quant_rows_fp8(const float *h, int R, int K, uint8_t *q, float *sq, const float *h1, int R1,
                                   int K1, uint8_t *q1, float *sq1, cudaStream_t s);
-// int4 layers: copy bf16 token rows into the permuted rows (and the shared rows).
+// 4-bit layers: copy bf16 token rows into the permuted rows (and the shared rows); with
+// `interleave` (int4), each aligned block of 8 elements in the order 0, 4, 1, 5, 2, 6, 3, 7.
 cudaError_t launch_gather_x_bf16(const uint16_t *x, int T, int H, int k, const int32_t *pos, uint16_t *xp,
-                                 uint16_t *xp_shared, cudaStream_t s);
+                                 uint16_t *xp_shared, bool interleave, cudaStream_t s);
 
 // ---- combine (combine.cu) ----------------------------------------------------------------
 

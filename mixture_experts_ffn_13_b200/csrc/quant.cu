@@ -141,10 +141,12 @@ __global__ void __launch_bounds__(256) quant_rows_fp8_kernel(RowsSeg s0, RowsSeg
     if (lane == 0) sq[(size_t)r * nb + kb] = s;
 }
 
-// grid T: copy bf16 token row t to the permuted rows pos[t, :] and to shared row t.
+// grid T: copy bf16 token row t to the permuted rows pos[t, :] and to shared row t.  With
+// `interleave`, every aligned block of 8 elements is stored in the order 0, 4, 1, 5, 2, 6, 3, 7
+// (the K order in which the int4 GEMM unpacks its weights), else as it is.
 __global__ void __launch_bounds__(128) gather_x_bf16_kernel(const uint16_t *__restrict__ x, int H, int k,
                                                             const int32_t *__restrict__ pos, uint16_t *__restrict__ xp,
-                                                            uint16_t *__restrict__ xp_sh)
+                                                            uint16_t *__restrict__ xp_sh, bool interleave)
 {
     griddep_wait();
     griddep_launch_dependents();
@@ -152,7 +154,16 @@ __global__ void __launch_bounds__(128) gather_x_bf16_kernel(const uint16_t *__re
     const int n16 = H / 8;  // uint4 chunks of 8 bf16
     const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * H);
     for (int c = threadIdx.x; c < n16; c += blockDim.x) {
-        const uint4 v = __ldg(src + c);
+        uint4 v = __ldg(src + c);
+        if (interleave) {
+            // words hold elements (0, 1), (2, 3), (4, 5), (6, 7); make them (0, 4), (1, 5), ...
+            uint4 u;
+            asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(u.x) : "r"(v.x), "r"(v.z));
+            asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(u.y) : "r"(v.x), "r"(v.z));
+            asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(u.z) : "r"(v.y), "r"(v.w));
+            asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(u.w) : "r"(v.y), "r"(v.w));
+            v = u;
+        }
         for (int j = 0; j < k; ++j) {
             const int r = pos[(size_t)t * k + j];
             reinterpret_cast<uint4 *>(xp + (size_t)r * H)[c] = v;
@@ -182,10 +193,10 @@ cudaError_t launch_quant_rows_fp8(const float *h, int R, int K, uint8_t *q, floa
 }
 
 cudaError_t launch_gather_x_bf16(const uint16_t *x, int T, int H, int k, const int32_t *pos, uint16_t *xp,
-                                 uint16_t *xp_shared, cudaStream_t s)
+                                 uint16_t *xp_shared, bool interleave, cudaStream_t s)
 {
     if (T <= 0) return cudaSuccess;
-    return launch_pdl(gather_x_bf16_kernel, dim3(T), dim3(128), 0, s, x, H, k, pos, xp, xp_shared);
+    return launch_pdl(gather_x_bf16_kernel, dim3(T), dim3(128), 0, s, x, H, k, pos, xp, xp_shared, interleave);
 }
 
 }  // namespace moe
