@@ -10,8 +10,8 @@
 //    128-byte swizzle; narrower boxes make the TMA issue-bound) by TMA into a ring of raw
 //    stages (evict-first), keeps an L2 prefetch of the raw tiles kPrefetch stages further
 //    ahead, and streams the bf16 activation tiles through their own ring;
-//  * warps 3-6 (one thread per weight row, 64 K-elements at a time) turn the nibbles into the
-//    integers q as bf16 (exact: |q| <= 8): flip each nibble's sign bit, place it in the
+//  * warps 4-11 (two per TMEM lane quarter; a thread handles one weight row and one 32-element
+//    half of every 64-K stage) turn the nibbles into the integers q as bf16 (exact: |q| <= 8): flip each nibble's sign bit, place it in the
 //    mantissa of the bf16 value 128 (so it reads 128 + q + 8), subtract 136.  A 32-bit word of
 //    8 nibbles holds elements i and i + 4 sixteen bits apart, so each bf16 pair is one shift,
 //    one mask and one subtract when it pairs element i with element i + 4: int4 tiles keep
@@ -27,7 +27,7 @@
 //    one thread each (gate|up: one matrix each; down: half of the token columns each): 4 MMAs of K = 16 per
 //    stage per matrix; each 128-element K group (2 stages) accumulates into its own TMEM slot,
 //    because the weight scale changes per (row, group);
-//  * warps 7-14 (two per TMEM lane quarter, each owning half of the token columns) promote each
+//  * warps 12-19 (two per TMEM lane quarter, each owning half of the token columns) promote each
 //    finished group, acc += D_g * s[row, g] in fp32 registers, and at the end of the tile write
 //    gate|up h = silu(G) * U rounded to bf16 (the 4-bit layer keeps activations in bf16) or
 //    down y in fp32.
@@ -43,7 +43,8 @@
 // bf16, so the dequantisers write the scaled weights themselves, the whole K accumulates in
 // one TMEM slot, and the epilogue has no promotion to do.  The warp roles shift with that:
 // warps 3-10 dequantise (two per TMEM lane quarter, one 32-element block of each 64-K stage
-// apiece) and warps 11-14 (one per quarter) stream each finished tile out.
+// apiece, as for int4) and warps 11-14 (one per quarter) stream each finished tile out; with
+// 15 warps at one register count nothing spills, so these formats keep that layout.
 //
 // NVFP4 weights (the NVIDIA co-design commentary, section "讀的時候記得這是廠商文": two levels
 // of scale factors) take the same path: an E2M1 value times its 16-block's E4M3 scale has at
@@ -67,19 +68,31 @@ constexpr int kRawKE = 256;            // K elements per raw weight stage (128 b
 constexpr int kSubs = kRawKE / kKE;    // MMA stages per raw stage
 constexpr int kPrefetch = 8;           // raw stages prefetched into L2 ahead of the loads
 
-// Warp roles: 0 producer, 1 and 2 MMA issuers, CONV dequantisers, EW epilogue warps.  int4 keeps two
-// epilogue warps per TMEM lane quarter (each holds half the token columns' fp32 sums across
-// the scale groups); MXFP4 has no promotion, so one epilogue warp per quarter streams the
-// accumulator out, and the freed warps become a second dequantiser per quarter (each of the
-// pair converts one 32-element block of a 64-K stage).
+// Warp roles: 0 producer, 1 and 2 MMA issuers, then CONV dequantisers from warp D0 (two per TMEM
+// lane quarter, each converting one 32-element half of every 64-K stage), then EW epilogue
+// warps from warp E0.  int4 keeps two epilogue warps per quarter (each holds half the token
+// columns' fp32 sums across the scale groups) and lays the roles out by warpgroup (warp 3
+// idle, warpgroups 1-2 dequantise, 3-4 promote) so that each can set its own register count:
+// the promotion needs ~128 per thread, the rest far fewer, and 20 warps at one count would
+// leave the promotion 96.  MXFP4/NVFP4 have no promotion: one epilogue warp per quarter
+// streams the accumulator out, and 15 warps fit without a split.
 enum { kFmtInt4 = 0, kFmtMx = 1, kFmtNv = 2 };
 
 template <int BN, bool GATEUP, bool FP4>
 struct I4Cfg {
-    static constexpr int CONV = FP4 ? 8 : 4;                // dequantiser warps
+    static constexpr int CONV = 8;                          // dequantiser warps
     static constexpr int EW = FP4 ? 4 : 8;                  // epilogue warps
+    static constexpr int D0 = FP4 ? 3 : 4;                  // first dequantiser warp
+    static constexpr int E0 = D0 + CONV;                    // first epilogue warp
     static constexpr int CPW = BN / (EW / 4);               // token columns per epilogue thread
-    static constexpr int THREADS = 32 * (3 + CONV + EW);  // producer, two MMA issuers, roles
+    static constexpr int THREADS = 32 * (E0 + EW);
+    // int4 register split (per thread, multiples of 8): warpgroup 0 (producer, issuers),
+    // warpgroups 1-2 (dequantisers), warpgroups 3-4 (promotion).  Their sum over the five
+    // warpgroups must not exceed what the block is launched with (checked on the host before
+    // every launch), or an increase would wait for registers that never come.
+    static constexpr int REG_PI = 56, REG_D = 80, REG_E = 128;
+    static constexpr int REG_SUM = REG_PI + 2 * REG_D + 2 * REG_E;  // x 128 threads
+    static_assert(FP4 || THREADS == 640, "int4: five whole warpgroups");
     static constexpr int NA = GATEUP ? 2 : 1;
     static constexpr int RAW_BYTES = kTileM * (kRawKE / 2);  // 16 KB per matrix
     static constexpr int B_BYTES = BN * kKE * 2;
@@ -242,102 +255,109 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
     const uint64_t tmo = args.timeout_ns;
     uint32_t issued_r = 0, issued_b = 0;  // producer: raw and activation stages issued
 
-    if (warp == 0) {
-        // --------------------- raw weight + activation producer ---------------------
-        if (lane == 0) {
-            const uint64_t pol_w = l2_policy_evict_first();
-            const uint64_t pol_x = l2_policy_evict_last();
-            uint32_t it = 0, rt = 0;  // MMA-stage and raw-stage counters
-            // L2 prefetch cursor: raw stage (pw tile, pk index) runs kPrefetch raw stages ahead
-            // of the shared-memory loads, across tile boundaries
-            int pw = blockIdx.x, pk = 0;
-            TileInfo pt;
-            if (pw < total) pt = decode_tile<BN, true>(args, stt, pw, tot0);
-            auto prefetch_next = [&]() {
-                if (pw >= total) return;
-                const int x = pk * (kRawKE / 2);
-                tma_prefetch_l2_2d(&maps.a0[pt.seg], x, pt.wrow);
-                if (GATEUP) tma_prefetch_l2_2d(&maps.a1[pt.seg], x, pt.wrow);
-                if (++pk * kRawKE >= args.seg[pt.seg].K) {
-                    pk = 0;
-                    pw += gridDim.x;
-                    if (pw < total) pt = decode_tile<BN, true>(args, stt, pw, tot0);
-                }
-            };
-            for (int i = 0; i < kPrefetch; ++i) prefetch_next();
-            for (int w = blockIdx.x; w < total; w += gridDim.x) {
-                const TileInfo tl = decode_tile<BN, true>(args, stt, w, tot0);
-                const int nkc = args.seg[tl.seg].K / kKE;
-                for (int kc = 0; kc < nkc; ++kc, ++it) {
-                    if (kc % kSubs == 0) {
-                        prefetch_next();
-                        // raw weights for the next 256 K-elements (the last stage of a K that is
-                        // not a multiple of 256 reads zeros past the end)
-                        const int s = rt % C::NR;
-                        if (!mbar_wait(&rempty[s], ((rt / C::NR) & 1) ^ 1, abort_flag, status, tmo)) goto done;
-                        uint8_t *rs = raw + s * C::NA * C::RAW_BYTES;
-                        issued_r = rt + 1;
-                        mbar_arrive_expect_tx(&rfull[s], C::NA * C::RAW_BYTES);
-                        const int x = (kc / kSubs) * (kRawKE / 2);
-                        tma_load_2d_hint(rs, &maps.a0[tl.seg], &rfull[s], x, tl.wrow, pol_w);
-                        if (GATEUP) tma_load_2d_hint(rs + C::RAW_BYTES, &maps.a1[tl.seg], &rfull[s], x, tl.wrow, pol_w);
-                        ++rt;
+    if (warp < C::D0) {
+        // int4: warpgroup 0 (producer, issuers and an idle warp) gives registers back; the
+        // register counts are set at the top of each role's branch, where the compiler can
+        // budget the role's code with them
+        if constexpr (!FP4) regs_dec<C::REG_PI>();
+        if (warp == 0) {
+            // --------------------- raw weight + activation producer ---------------------
+            if (lane == 0) {
+                const uint64_t pol_w = l2_policy_evict_first();
+                const uint64_t pol_x = l2_policy_evict_last();
+                uint32_t it = 0, rt = 0;  // MMA-stage and raw-stage counters
+                // L2 prefetch cursor: raw stage (pw tile, pk index) runs kPrefetch raw stages ahead
+                // of the shared-memory loads, across tile boundaries
+                int pw = blockIdx.x, pk = 0;
+                TileInfo pt;
+                if (pw < total) pt = decode_tile<BN, true>(args, stt, pw, tot0);
+                auto prefetch_next = [&]() {
+                    if (pw >= total) return;
+                    const int x = pk * (kRawKE / 2);
+                    tma_prefetch_l2_2d(&maps.a0[pt.seg], x, pt.wrow);
+                    if (GATEUP) tma_prefetch_l2_2d(&maps.a1[pt.seg], x, pt.wrow);
+                    if (++pk * kRawKE >= args.seg[pt.seg].K) {
+                        pk = 0;
+                        pw += gridDim.x;
+                        if (pw < total) pt = decode_tile<BN, true>(args, stt, pw, tot0);
                     }
-                    const int b = it % C::NB;
-                    if (!mbar_wait(&bempty[b], ((it / C::NB) & 1) ^ 1, abort_flag, status, tmo)) goto done;
-                    issued_b = it + 1;
-                    mbar_arrive_expect_tx(&bfull[b], C::B_BYTES);
-                    tma_load_2d_hint(bst + b * C::B_BYTES, &maps.b[tl.seg], &bfull[b], kc * kKE, tl.row0, pol_x);
+                };
+                for (int i = 0; i < kPrefetch; ++i) prefetch_next();
+                for (int w = blockIdx.x; w < total; w += gridDim.x) {
+                    const TileInfo tl = decode_tile<BN, true>(args, stt, w, tot0);
+                    const int nkc = args.seg[tl.seg].K / kKE;
+                    for (int kc = 0; kc < nkc; ++kc, ++it) {
+                        if (kc % kSubs == 0) {
+                            prefetch_next();
+                            // raw weights for the next 256 K-elements (the last stage of a K that is
+                            // not a multiple of 256 reads zeros past the end)
+                            const int s = rt % C::NR;
+                            if (!mbar_wait(&rempty[s], ((rt / C::NR) & 1) ^ 1, abort_flag, status, tmo)) goto done;
+                            uint8_t *rs = raw + s * C::NA * C::RAW_BYTES;
+                            issued_r = rt + 1;
+                            mbar_arrive_expect_tx(&rfull[s], C::NA * C::RAW_BYTES);
+                            const int x = (kc / kSubs) * (kRawKE / 2);
+                            tma_load_2d_hint(rs, &maps.a0[tl.seg], &rfull[s], x, tl.wrow, pol_w);
+                            if (GATEUP) tma_load_2d_hint(rs + C::RAW_BYTES, &maps.a1[tl.seg], &rfull[s], x, tl.wrow, pol_w);
+                            ++rt;
+                        }
+                        const int b = it % C::NB;
+                        if (!mbar_wait(&bempty[b], ((it / C::NB) & 1) ^ 1, abort_flag, status, tmo)) goto done;
+                        issued_b = it + 1;
+                        mbar_arrive_expect_tx(&bfull[b], C::B_BYTES);
+                        tma_load_2d_hint(bst + b * C::B_BYTES, &maps.b[tl.seg], &bfull[b], kc * kKE, tl.row0, pol_x);
+                    }
                 }
             }
-        }
-    } else if (warp == 1 || warp == 2) {
-        // ------------------------------ MMA issuers -------------------------------
-        // Two threads in different warps share every stage's MMAs: a tcgen05.commit holds up
-        // the issuing thread, and a stage needs two (the tensor-memory and the activation
-        // stage), which one thread alone cannot hide behind the short N <= 96 MMAs.  gate|up:
-        // issuer 0 multiplies the gate weights and issuer 1 the up weights; down: each takes
-        // half of the tile's token columns (the MMA's N), into its half of the accumulator.
-        // Both wait for and release every stage, so each consumes the stage rings in order.
-        const int mt = warp - 1;
-        if (lane == 0) {
-            uint32_t it = 0, ai = 0;
-            for (int w = blockIdx.x; w < total; w += gridDim.x) {
-                const TileInfo tl = decode_tile<BN, true>(args, stt, w, tot0);
-                // MMA N: the tile's valid rows rounded up to 16 (gate|up) or, split in two halves
-                // of a multiple of 16 each, to 32 (down); partial tiles cost no work on absent rows
-                const int n_mma = GATEUP ? min(BN, (tl.nrows + 15) & ~15) : min(BN, (tl.nrows + 31) & ~31) / 2;
-                const uint32_t kIdesc = instr_desc(kTileM, n_mma, 1, 1);
-                // int4: one TMEM slot per 128-element scale group; E2M1 formats: one for the K
-                const int ngrp = FP4 ? 1 : args.seg[tl.seg].K / kGroupK;
-                const int spg = FP4 ? args.seg[tl.seg].K / kKE : C::STAGES_PER_GROUP;
-                for (int g = 0; g < ngrp; ++g, ++ai) {
-                    const int slot = ai % C::NSLOT;
-                    if (!mbar_wait(&acce[slot], ((ai / C::NSLOT) & 1) ^ 1, abort_flag, status, tmo)) goto done;
-                    tc_fence_after();
-                    // gate|up: this issuer's matrix; down: its half of the token columns
-                    const uint32_t d = tmem_base + C::A_TMEM + slot * C::SLOT_COLS + (GATEUP ? mt * BN : mt * n_mma);
-                    for (int sk = 0; sk < spg; ++sk, ++it) {
-                        const int s = it % C::NM;
-                        const int bs = it % C::NB;
-                        if (!mbar_wait(&mfull[s], (it / C::NM) & 1, abort_flag, status, tmo)) goto done;
-                        if (!mbar_wait(&bfull[bs], (it / C::NB) & 1, abort_flag, status, tmo)) goto done;
+        } else if (warp == 1 || warp == 2) {
+            // ------------------------------ MMA issuers -------------------------------
+            // Two threads in different warps share every stage's MMAs: a tcgen05.commit holds up
+            // the issuing thread, and a stage needs two (the tensor-memory and the activation
+            // stage), which one thread alone cannot hide behind the short N <= 96 MMAs.  gate|up:
+            // issuer 0 multiplies the gate weights and issuer 1 the up weights; down: each takes
+            // half of the tile's token columns (the MMA's N), into its half of the accumulator.
+            // Both wait for and release every stage, so each consumes the stage rings in order.
+            const int mt = warp - 1;
+            if (lane == 0) {
+                uint32_t it = 0, ai = 0;
+                for (int w = blockIdx.x; w < total; w += gridDim.x) {
+                    const TileInfo tl = decode_tile<BN, true>(args, stt, w, tot0);
+                    // MMA N: the tile's valid rows rounded up to 16 (gate|up) or, split in two halves
+                    // of a multiple of 16 each, to 32 (down); partial tiles cost no work on absent rows
+                    const int n_mma = GATEUP ? min(BN, (tl.nrows + 15) & ~15) : min(BN, (tl.nrows + 31) & ~31) / 2;
+                    const uint32_t kIdesc = instr_desc(kTileM, n_mma, 1, 1);
+                    // int4: one TMEM slot per 128-element scale group; E2M1 formats: one for the K
+                    const int ngrp = FP4 ? 1 : args.seg[tl.seg].K / kGroupK;
+                    const int spg = FP4 ? args.seg[tl.seg].K / kKE : C::STAGES_PER_GROUP;
+                    for (int g = 0; g < ngrp; ++g, ++ai) {
+                        const int slot = ai % C::NSLOT;
+                        if (!mbar_wait(&acce[slot], ((ai / C::NSLOT) & 1) ^ 1, abort_flag, status, tmo)) goto done;
                         tc_fence_after();
-                        const uint32_t a = tmem_base + s * C::NA * C::A_COLS + (GATEUP ? mt * C::A_COLS : 0);
-                        // down: the second half's token rows start n_mma rows (n_mma * 128 bytes,
-                        // whole 8-row swizzle atoms) into the activation stage
-                        const uint64_t db =
-                            smem_desc_sw128(bst + bs * C::B_BYTES) + (GATEUP ? 0 : (uint64_t)(mt * n_mma * 8));
-#pragma unroll
-                        for (int kk = 0; kk < kKE / 16; ++kk)
-                            mma_bf16_ts(d, a + 8 * kk, db + 2 * kk, kIdesc, (sk > 0 || kk > 0) ? 1u : 0u);
-                        mma_commit(&bempty[bs]);  // frees the activation stage and the TMEM weight stage
+                        // gate|up: this issuer's matrix; down: its half of the token columns
+                        const uint32_t d = tmem_base + C::A_TMEM + slot * C::SLOT_COLS + (GATEUP ? mt * BN : mt * n_mma);
+                        for (int sk = 0; sk < spg; ++sk, ++it) {
+                            const int s = it % C::NM;
+                            const int bs = it % C::NB;
+                            if (!mbar_wait(&mfull[s], (it / C::NM) & 1, abort_flag, status, tmo)) goto done;
+                            if (!mbar_wait(&bfull[bs], (it / C::NB) & 1, abort_flag, status, tmo)) goto done;
+                            tc_fence_after();
+                            const uint32_t a = tmem_base + s * C::NA * C::A_COLS + (GATEUP ? mt * C::A_COLS : 0);
+                            // down: the second half's token rows start n_mma rows (n_mma * 128 bytes,
+                            // whole 8-row swizzle atoms) into the activation stage
+                            const uint64_t db =
+                                smem_desc_sw128(bst + bs * C::B_BYTES) + (GATEUP ? 0 : (uint64_t)(mt * n_mma * 8));
+    #pragma unroll
+                            for (int kk = 0; kk < kKE / 16; ++kk)
+                                mma_bf16_ts(d, a + 8 * kk, db + 2 * kk, kIdesc, (sk > 0 || kk > 0) ? 1u : 0u);
+                            mma_commit(&bempty[bs]);  // frees the activation stage and the TMEM weight stage
+                        }
+                        mma_commit(&accf[slot]);
                     }
-                    mma_commit(&accf[slot]);
                 }
             }
-        }
-    } else if (warp < 3 + C::CONV) {
+    }
+    } else if (warp < C::E0) {
+        if constexpr (!FP4) regs_dec<C::REG_D>();
         // ------------------------------ dequantisers ------------------------------
         const int q = warp & 3;        // TMEM lane quarter reachable from this warp
         const int r = q * 32 + lane;   // weight row of the tile handled by this thread
@@ -411,7 +431,7 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
                     // half hx of the stage: 16-byte chunk ch = 2*sub + hx of the row (the 128-byte
                     // swizzle stores chunk c at position c ^ (r & 7)), K elements 32*ch .. +31 of
                     // the raw stage, written to TMEM columns 16*hx .. 16*hx + 15
-                    const int hx = (warp - 3) >> 2;
+                    const int hx = (warp - C::D0) >> 2;
                     const int cc = ((2 * sub + hx) ^ (r & 7)) << 4;
 #pragma unroll
                     for (int m = 0; m < C::NA; ++m) {
@@ -445,24 +465,25 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
                         tmem_st16(ta + m * C::A_COLS + 16 * hx, v);  // 32 bf16 = 16 packed columns
                     }
                 } else {
-                    // this sub-stage's 32 raw bytes are 16-byte chunks 2*sub and 2*sub+1 of the
-                    // row, stored by the 128-byte swizzle at chunk positions (c ^ (r & 7))
-                    const int c0 = ((2 * sub) ^ (r & 7)) << 4, c1 = ((2 * sub + 1) ^ (r & 7)) << 4;
+                    // half hx of the sub-stage: 16-byte chunk 2*sub + hx of the row (the 128-byte
+                    // swizzle stores chunk c at position c ^ (r & 7)), K elements 32*hx .. +31 of
+                    // the 64, written to TMEM columns 16*hx .. 16*hx + 15
+                    const int hx = (warp - C::D0) >> 2;
+                    const int cc = ((2 * sub + hx) ^ (r & 7)) << 4;
 #pragma unroll
                     for (int m = 0; m < C::NA; ++m) {
-                        const uint4 q0 = *reinterpret_cast<const uint4 *>(rs + m * C::RAW_BYTES + c0);
-                        const uint4 q1 = *reinterpret_cast<const uint4 *>(rs + m * C::RAW_BYTES + c1);
-                        const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-                        uint32_t v[32];
+                        const uint4 qq = *reinterpret_cast<const uint4 *>(rs + m * C::RAW_BYTES + cc);
+                        const uint32_t words[4] = {qq.x, qq.y, qq.z, qq.w};
+                        uint32_t v[16];
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) {
+                        for (int j = 0; j < 4; ++j) {
                             const uint4 u = unpack8(words[j]);
                             v[4 * j] = u.x;
                             v[4 * j + 1] = u.y;
                             v[4 * j + 2] = u.z;
                             v[4 * j + 3] = u.w;
                         }
-                        tmem_st32(ta + m * C::A_COLS, v);  // row r: 64 bf16 = 32 packed columns
+                        tmem_st16(ta + m * C::A_COLS + 16 * hx, v);  // 32 bf16 = 16 packed columns
                     }
                 }
                 tmem_wait_st();
@@ -477,9 +498,10 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
             }
         }
     } else {
+        if constexpr (!FP4) regs_inc<C::REG_E>();
         // ------------------------------ epilogue ----------------------------------
-        const int q = warp & 3;                                   // TMEM lane quarter
-        const int cbase = ((warp - 3 - C::CONV) >> 2) * C::CPW;  // first token column
+        const int q = warp & 3;                            // TMEM lane quarter
+        const int cbase = ((warp - C::E0) >> 2) * C::CPW;  // first token column
         const int r = q * 32 + lane;
         uint32_t ai = 0;
         for (int w = blockIdx.x; w < total; w += gridDim.x) {
@@ -611,6 +633,14 @@ cudaError_t launch_t(const GemmMaps &maps, const GemmArgs &args, int num_sms, cu
     auto kern = gemm_int4_kernel<BN, GATEUP, FMT>;
     cudaError_t e = set_smem_limit(reinterpret_cast<const void *>(kern), C::SMEM);
     if (e != cudaSuccess) return e;
+    if constexpr (FMT == kFmtInt4) {
+        // the register split must fit in what the block is launched with
+        static const int launch_regs = [&] {
+            cudaFuncAttributes fa{};
+            return cudaFuncGetAttributes(&fa, reinterpret_cast<const void *>(kern)) == cudaSuccess ? fa.numRegs : 0;
+        }();
+        if (launch_regs * C::THREADS < 128 * C::REG_SUM || launch_regs < C::REG_D) return cudaErrorInvalidConfiguration;
+    }
     return launch_pdl(kern, dim3(num_sms), dim3(C::THREADS), C::SMEM, s, maps, args);
 }
 

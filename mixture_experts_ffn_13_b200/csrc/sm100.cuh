@@ -282,6 +282,23 @@ __device__ __forceinline__ void tc_fence_after()
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
+// Per-warpgroup register counts (setmaxnreg): every thread of a warpgroup executes the same
+// one.  A decrease returns registers to the block's pool; an increase waits until the pool
+// holds enough, so the counts of all warpgroups must add up to at most what the block was
+// launched with.
+template <int N>
+__device__ __forceinline__ void regs_dec()
+{
+    static_assert(N % 8 == 0 && N >= 24 && N <= 256, "setmaxnreg count");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc()
+{
+    static_assert(N % 8 == 0 && N >= 24 && N <= 256, "setmaxnreg count");
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // Shared-memory matrix descriptor of a K-major operand tile stored with the 128-byte
 // swizzle: rows of 128 bytes, 8-row groups 1024 bytes apart (stride byte offset), tile base
 // 1024-byte aligned.  Fields: start address >> 4 in bits 0-13, leading byte offset (unused
