@@ -43,8 +43,9 @@
 // bf16, so the dequantisers write the scaled weights themselves, the whole K accumulates in
 // one TMEM slot, and the epilogue has no promotion to do.  The warp roles shift with that:
 // warps 3-10 dequantise (two per TMEM lane quarter, one 32-element block of each 64-K stage
-// apiece, as for int4) and warps 11-14 (one per quarter) stream each finished tile out; with
-// 15 warps at one register count nothing spills, so these formats keep that layout.
+// apiece, as for int4; the gate|up tiles take four per quarter, one half of one matrix apiece,
+// warps 3-18) and one warp per quarter streams each finished tile out; at one register count
+// for all warps nothing spills, so these formats need no register split.
 //
 // NVFP4 weights (the NVIDIA co-design commentary, section "讀的時候記得這是廠商文": two levels
 // of scale factors) take the same path: an E2M1 value times its 16-block's E4M3 scale has at
@@ -80,7 +81,11 @@ enum { kFmtInt4 = 0, kFmtMx = 1, kFmtNv = 2 };
 
 template <int BN, bool GATEUP, bool FP4>
 struct I4Cfg {
-    static constexpr int CONV = 8;                          // dequantiser warps
+    // dequantiser warps: two per TMEM lane quarter (one 32-element half of each 64-K stage
+    // apiece); the E2M1 gate|up tiles, whose conversion is the longest, take four (one half
+    // of one matrix apiece)
+    static constexpr int CONV = FP4 && GATEUP ? 16 : 8;
+    static constexpr int MSPLIT = CONV / 8;                 // dequantiser sets sharing the matrices
     static constexpr int EW = FP4 ? 4 : 8;                  // epilogue warps
     static constexpr int D0 = FP4 ? 3 : 4;                  // first dequantiser warp
     static constexpr int E0 = D0 + CONV;                    // first epilogue warp
@@ -369,6 +374,9 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
         constexpr int SBLK = NV ? 16 : 32;         // K elements per block scale
         constexpr int SW = kRawKE / SBLK / 4;      // scale words per raw stage: 2 (MX), 4 (NV)
         uint32_t scur[C::NA][SW] = {}, snxt[C::NA][SW] = {};
+        const int unit = (warp - C::D0) >> 2;               // which share of each stage
+        const int hx = C::MSPLIT == 2 ? (unit & 1) : unit;   // 32-element half of the 64-K stage
+        const int mown = unit >> 1;                         // MSPLIT 2: the one matrix converted
         auto load_scales = [&](int wi, int kr, uint32_t (&dst)[C::NA][SW]) {
             const TileInfo t = decode_tile<BN, true>(args, stt, wi, tot0);
             const GemmSeg &s = args.seg[t.seg];
@@ -377,8 +385,9 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
             const int b0 = kr * (4 * SW);          // first byte of raw stage kr
             const int half = 2 * SW;               // bytes of the first 128 K of the raw stage
 #pragma unroll
-            for (int m = 0; m < C::NA; ++m) {
-                const uint8_t *base = static_cast<const uint8_t *>(m == 0 ? s.sw0 : s.sw1);
+            for (int m = 0; m < C::NA / C::MSPLIT; ++m) {
+                const int ms = C::MSPLIT == 2 ? mown : m;
+                const uint8_t *base = static_cast<const uint8_t *>(ms == 0 ? s.sw0 : s.sw1);
                 const uint8_t *p = base + (size_t)(t.wrow + r) * nbk + b0;
                 // a last raw stage of 128 K has only its first half: b0 + half <= nbk always
                 if constexpr (NV) {
@@ -430,26 +439,27 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
                 if constexpr (FP4) {
                     // half hx of the stage: 16-byte chunk ch = 2*sub + hx of the row (the 128-byte
                     // swizzle stores chunk c at position c ^ (r & 7)), K elements 32*ch .. +31 of
-                    // the raw stage, written to TMEM columns 16*hx .. 16*hx + 15
-                    const int hx = (warp - C::D0) >> 2;
+                    // the raw stage, written to TMEM columns 16*hx .. 16*hx + 15; with MSPLIT 2
+                    // only matrix mown, whose scale bytes sit in slot 0
                     const int cc = ((2 * sub + hx) ^ (r & 7)) << 4;
 #pragma unroll
-                    for (int m = 0; m < C::NA; ++m) {
+                    for (int mi = 0; mi < C::NA / C::MSPLIT; ++mi) {
+                        const int m = C::MSPLIT == 2 ? mown : mi;
                         const uint4 qq = *reinterpret_cast<const uint4 *>(rs + m * C::RAW_BYTES + cc);
                         // scales of the chunk's elements 0-15 (sa) and 16-31 (sb)
                         __nv_bfloat162 sa, sb;
                         if constexpr (NV) {
                             // 16-blocks 2*ch and 2*ch + 1: bytes 2*ch, 2*ch + 1 = word sub, bytes
                             // 2*hx and 2*hx + 1 of it
-                            const uint32_t sw = sub == 0   ? scur[m][0]
-                                                : sub == 1 ? scur[m][1]
-                                                : sub == 2 ? scur[m][SW - 2]
-                                                           : scur[m][SW - 1];
+                            const uint32_t sw = sub == 0   ? scur[mi][0]
+                                                : sub == 1 ? scur[mi][1]
+                                                : sub == 2 ? scur[mi][SW - 2]
+                                                           : scur[mi][SW - 1];
                             sa = e4m3_pair((sw >> (hx * 16)) & 0xFFu);
                             sb = e4m3_pair((sw >> (hx * 16 + 8)) & 0xFFu);
                         } else {
                             // 32-block ch: byte ch = word sub >> 1, byte (sub & 1) * 2 + hx of it
-                            const uint32_t sw = (sub >> 1) ? scur[m][SW - 1] : scur[m][0];
+                            const uint32_t sw = (sub >> 1) ? scur[mi][SW - 1] : scur[mi][0];
                             sa = sb = e8m0_pair((sw >> ((sub & 1) * 16 + hx * 8)) & 0xFFu);
                         }
                         const uint32_t words[4] = {qq.x, qq.y, qq.z, qq.w};
@@ -468,7 +478,6 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
                     // half hx of the sub-stage: 16-byte chunk 2*sub + hx of the row (the 128-byte
                     // swizzle stores chunk c at position c ^ (r & 7)), K elements 32*hx .. +31 of
                     // the 64, written to TMEM columns 16*hx .. 16*hx + 15
-                    const int hx = (warp - C::D0) >> 2;
                     const int cc = ((2 * sub + hx) ^ (r & 7)) << 4;
 #pragma unroll
                     for (int m = 0; m < C::NA; ++m) {
