@@ -199,6 +199,7 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
 {
     constexpr bool FP4 = FMT != kFmtInt4;  // E2M1 elements with exact bf16 scaling (MXFP4, NVFP4)
     constexpr bool NV = FMT == kFmtNv;
+    constexpr bool DALT = !GATEUP && !FP4;  // int4 down: the two issuers alternate scale groups
     using C = I4Cfg<BN, GATEUP, FP4>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -222,17 +223,18 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
             mbar_init(&rfull[s], 1);
             mbar_init(&rempty[s], C::CONV);
         }
-        // both MMA issuers consume every stage and contribute to every accumulator
+        // gate|up and the E2M1 down: both MMA issuers consume every stage and contribute to
+        // every accumulator; int4 down: the issuers take alternate scale groups
         for (int s = 0; s < C::NB; ++s) {
             mbar_init(&bfull[s], 1);
-            mbar_init(&bempty[s], 2);
+            mbar_init(&bempty[s], DALT ? 1 : 2);
         }
         // a TMEM weight stage is free again once the MMAs of the stage that used it have
         // completed, which bempty of that stage records (the ring of activation stages is
         // deeper than the ring of weight stages, so the phase waited for is never overtaken)
         for (int s = 0; s < C::NM; ++s) mbar_init(&mfull[s], C::CONV);
         for (int s = 0; s < C::NSLOT; ++s) {
-            mbar_init(&accf[s], 2);
+            mbar_init(&accf[s], DALT ? 1 : 2);
             mbar_init(&acce[s], C::EW);
         }
         mbar_init(&drain_bar[0], 1);
@@ -316,30 +318,38 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
             }
         } else if (warp == 1 || warp == 2) {
             // ------------------------------ MMA issuers -------------------------------
-            // Two threads in different warps share every stage's MMAs: a tcgen05.commit holds up
-            // the issuing thread, and a stage needs two (the tensor-memory and the activation
-            // stage), which one thread alone cannot hide behind the short N <= 96 MMAs.  gate|up:
-            // issuer 0 multiplies the gate weights and issuer 1 the up weights; down: each takes
-            // half of the tile's token columns (the MMA's N), into its half of the accumulator.
-            // Both wait for and release every stage, so each consumes the stage rings in order.
+            // Two threads in different warps share the MMAs: a tcgen05.commit holds up the
+            // issuing thread, which one thread alone cannot hide behind the short N <= 96 MMAs.
+            // gate|up: issuer 0 multiplies the gate weights and issuer 1 the up weights; E2M1
+            // down: each takes half of the tile's token columns (the MMA's N), into its half of
+            // the accumulator; both wait for and release every stage.  int4 down: the issuers
+            // take alternate 128-element scale groups (each its own TMEM slot) with the whole N,
+            // so a stage costs four MMAs instead of eight; each waits for and releases the
+            // stages of its groups only.
             const int mt = warp - 1;
             if (lane == 0) {
                 uint32_t it = 0, ai = 0;
                 for (int w = blockIdx.x; w < total; w += gridDim.x) {
                     const TileInfo tl = decode_tile<BN, true>(args, stt, w, tot0);
-                    // MMA N: the tile's valid rows rounded up to 16 (gate|up) or, split in two halves
-                    // of a multiple of 16 each, to 32 (down); partial tiles cost no work on absent rows
-                    const int n_mma = GATEUP ? min(BN, (tl.nrows + 15) & ~15) : min(BN, (tl.nrows + 31) & ~31) / 2;
+                    // MMA N: the tile's valid rows rounded up to 16 (gate|up, int4 down) or, split in
+                    // two halves of a multiple of 16 each, to 32 (E2M1 down); partial tiles cost no
+                    // work on absent rows
+                    const int n_mma = GATEUP || DALT ? min(BN, (tl.nrows + 15) & ~15) : min(BN, (tl.nrows + 31) & ~31) / 2;
                     const uint32_t kIdesc = instr_desc(kTileM, n_mma, 1, 1);
                     // int4: one TMEM slot per 128-element scale group; E2M1 formats: one for the K
                     const int ngrp = FP4 ? 1 : args.seg[tl.seg].K / kGroupK;
                     const int spg = FP4 ? args.seg[tl.seg].K / kKE : C::STAGES_PER_GROUP;
                     for (int g = 0; g < ngrp; ++g, ++ai) {
+                        if (DALT && (int)(ai & 1) != mt) {  // the other issuer's group
+                            it += spg;
+                            continue;
+                        }
                         const int slot = ai % C::NSLOT;
                         if (!mbar_wait(&acce[slot], ((ai / C::NSLOT) & 1) ^ 1, abort_flag, status, tmo)) goto done;
                         tc_fence_after();
-                        // gate|up: this issuer's matrix; down: its half of the token columns
-                        const uint32_t d = tmem_base + C::A_TMEM + slot * C::SLOT_COLS + (GATEUP ? mt * BN : mt * n_mma);
+                        // gate|up: this issuer's matrix; E2M1 down: its half of the token columns
+                        const uint32_t d =
+                            tmem_base + C::A_TMEM + slot * C::SLOT_COLS + (GATEUP ? mt * BN : DALT ? 0 : mt * n_mma);
                         for (int sk = 0; sk < spg; ++sk, ++it) {
                             const int s = it % C::NM;
                             const int bs = it % C::NB;
@@ -350,8 +360,8 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
                             // down: the second half's token rows start n_mma rows (n_mma * 128 bytes,
                             // whole 8-row swizzle atoms) into the activation stage
                             const uint64_t db =
-                                smem_desc_sw128(bst + bs * C::B_BYTES) + (GATEUP ? 0 : (uint64_t)(mt * n_mma * 8));
-    #pragma unroll
+                                smem_desc_sw128(bst + bs * C::B_BYTES) + (GATEUP || DALT ? 0 : (uint64_t)(mt * n_mma * 8));
+#pragma unroll
                             for (int kk = 0; kk < kKE / 16; ++kk)
                                 mma_bf16_ts(d, a + 8 * kk, db + 2 * kk, kIdesc, (sk > 0 || kk > 0) ? 1u : 0u);
                             mma_commit(&bempty[bs]);  // frees the activation stage and the TMEM weight stage
