@@ -325,7 +325,11 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
             // the accumulator; both wait for and release every stage.  int4 down: the issuers
             // take alternate 128-element scale groups (each its own TMEM slot) with the whole N,
             // so a stage costs four MMAs instead of eight; each waits for and releases the
-            // stages of its groups only.
+            // stages of its groups only.  That is safe with parity waits because an issuer skips
+            // only two stages at a time: the dequantisers cannot complete a stage more than NM
+            // stages past an MMA stage that has not been issued, so no barrier an issuer waits
+            // on is ever two phases ahead of it.  (Alternating whole E2M1 tiles, 24 stages
+            // apiece, let the full-size MXFP4 layer time out, so those keep the N split.)
             const int mt = warp - 1;
             if (lane == 0) {
                 uint32_t it = 0, ai = 0;
