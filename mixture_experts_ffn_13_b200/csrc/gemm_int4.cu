@@ -11,26 +11,30 @@
 //    stages (evict-first), keeps an L2 prefetch of the raw tiles kPrefetch stages further
 //    ahead, and streams the bf16 activation tiles through their own ring;
 //  * warps 4-11 (two per TMEM lane quarter; a thread handles one weight row and one 32-element
-//    half of every 64-K stage) turn the nibbles into the integers q as bf16 (exact: |q| <= 8): flip each nibble's sign bit, place it in the
-//    mantissa of the bf16 value 128 (so it reads 128 + q + 8), subtract 136.  A 32-bit word of
-//    8 nibbles holds elements i and i + 4 sixteen bits apart, so each bf16 pair is one shift,
-//    one mask and one subtract when it pairs element i with element i + 4: int4 tiles keep
-//    their K elements in that interleaved order inside every aligned block of 8, and so do the
-//    activations and h they multiply (the gather kernel and the int4 gate|up epilogue store
-//    them so); the products and their sums are the same, only the order the MMA adds them in
-//    changes (11 instructions per 8 nibbles instead of 16; the int4 layer went from 1.054 to
-//    0.946 ms, since the conversion is what the dequantisers spend their time on).  The
-//    result goes to TENSOR memory with tcgen05.st (rows in lanes, two bf16 per 32-bit column): staging
-//    the 4x-expanded weights in shared memory instead costs a write and a tensor-core read of
-//    them per stage, which made the kernel shared-memory-bandwidth bound;
+//    half of every 64-K stage) turn the nibbles into the integers q as bf16 (exact: |q| <= 8):
+//    flip each nibble's sign bit, place it in the mantissa of the bf16 value 128 (so it reads
+//    128 + q + 8), subtract 136.  A 32-bit word of 8 nibbles holds elements i and i + 4 sixteen
+//    bits apart, so each bf16 pair is one shift, one mask and one subtract when it pairs
+//    element i with element i + 4: int4 tiles keep their K elements in that interleaved order
+//    inside every aligned block of 8, and so do the activations and h they multiply (the
+//    gather kernel and the int4 gate|up epilogue store them so); the products and their sums
+//    are the same, only the order the MMA adds them in changes (11 instructions per 8 nibbles
+//    instead of 16; the int4 layer went from 1.054 to 0.946 ms, since the conversion is what
+//    the dequantisers spend their time on).  The result goes to TENSOR memory with tcgen05.st
+//    (rows in lanes, two bf16 per 32-bit column): staging the 4x-expanded weights in shared
+//    memory instead costs a write and a tensor-core read of them per stage, which made the
+//    kernel shared-memory-bandwidth bound;
 //  * warps 1 and 2 issue tcgen05.mma.kind::f16 (A from tensor memory, B from shared memory),
-//    one thread each (gate|up: one matrix each; down: half of the token columns each): 4 MMAs of K = 16 per
-//    stage per matrix; each 128-element K group (2 stages) accumulates into its own TMEM slot,
+//    one thread each, 4 MMAs of K = 16 per 64-K stage and matrix: gate|up, one matrix each;
+//    int4 down, alternate 128-element scale groups with the whole N; E2M1 down, half of the
+//    token columns each.  Each int4 K group (2 stages) accumulates into its own TMEM slot,
 //    because the weight scale changes per (row, group);
 //  * warps 12-19 (two per TMEM lane quarter, each owning half of the token columns) promote each
 //    finished group, acc += D_g * s[row, g] in fp32 registers, and at the end of the tile write
 //    gate|up h = silu(G) * U rounded to bf16 (the 4-bit layer keeps activations in bf16) or
-//    down y in fp32.
+//    down y in fp32;
+//  * the five warpgroups (warp 3 idles) set their own register counts with setmaxnreg: 56 for
+//    the producer and issuers, 80 for the dequantisers, 128 for the promotion's 96 sums.
 // Multiplying the exact integers on the tensor cores and applying the bf16 scale to fp32
 // partial sums reproduces sum_i x_i * q_i * s_i up to fp32 rounding; rounding q * s to bf16
 // before the MMA would not (that costs ~2^-9 relative per weight and fails the layer's
