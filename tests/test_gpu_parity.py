@@ -203,6 +203,7 @@ SMALL_INT4 = [
     dict(T=37, H=512, E=8, I=384, k=3, Is=256, seed=42, bias="normal"),   # shared expert, ragged groups
     dict(T=200, H=1024, E=4, I=256, k=2, Is=0, seed=43, bias="zipf"),     # 64-row token tiles, several per group
     dict(T=3, H=128, E=16, I=128, k=4, Is=128, seed=44, bias=None),       # mostly empty experts
+    dict(T=64, H=512, E=8, I=256, k=4, Is=128, seed=46, bias="normal"),   # ~32 rows per expert: 64-row tiles
     # more than 4096 tokens (multi-kernel permutation), groups of many 96-row token tiles
     dict(T=4500, H=256, E=8, I=128, k=2, Is=0, seed=45, bias="zipf"),
 ]
@@ -228,6 +229,7 @@ SMALL_FP4 = [
     dict(T=37, H=384, E=8, I=384, k=3, Is=256, seed=82, bias="normal"),
     dict(T=200, H=1024, E=4, I=256, k=2, Is=0, seed=83, bias="zipf"),     # several token tiles per group
     dict(T=3, H=128, E=16, I=128, k=4, Is=128, seed=84, bias=None),       # K = 128: half a raw stage
+    dict(T=64, H=512, E=8, I=256, k=4, Is=128, seed=86, bias="normal"),   # ~32 rows per expert: 64-row tiles
     # many tiles per CTA: the scale prefetch crosses tile boundaries all the time
     dict(T=4500, H=256, E=8, I=128, k=2, Is=0, seed=85, bias="zipf"),
 ]
