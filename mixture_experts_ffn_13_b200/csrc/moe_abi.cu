@@ -123,6 +123,8 @@ int pick_bn(int T, int k, int E, bool fp8)
     if (avg <= 48) return fp8 || avg <= 24 ? 32 : 64;
     if (!fp8) return 96;  // 4-bit: one tile per group up to ~1.5x the mean (dequant is per tile)
     return avg <= 96 ? 64 : 192;  // 192: one pass over each weight tile for groups up to 192 rows
+    // (the FP8 GEMM also builds 128- and 160-row tiles; both measured slower at prefill, 3.88 and
+    // 3.69 against 3.37 ms, and are not picked)
 }
 
 }  // namespace
