@@ -26,8 +26,8 @@
 //    kernel shared-memory-bandwidth bound;
 //  * warps 1 and 2 issue tcgen05.mma.kind::f16 (A from tensor memory, B from shared memory),
 //    one thread each, 4 MMAs of K = 16 per 64-K stage and matrix: gate|up, one matrix each;
-//    int4 down, alternate 128-element scale groups with the whole N; E2M1 down, half of the
-//    token columns each.  Each int4 K group (2 stages) accumulates into its own TMEM slot,
+//    int4 down, alternate 128-element scale groups with the whole N; E2M1 down, issuer 0
+//    alone with the whole N.  Each int4 K group (2 stages) accumulates into its own TMEM slot,
 //    because the weight scale changes per (row, group);
 //  * warps 12-19 (two per TMEM lane quarter, each owning half of the token columns) promote each
 //    finished group, acc += D_g * s[row, g] in fp32 registers, and at the end of the tile write
@@ -203,7 +203,8 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
 {
     constexpr bool FP4 = FMT != kFmtInt4;  // E2M1 elements with exact bf16 scaling (MXFP4, NVFP4)
     constexpr bool NV = FMT == kFmtNv;
-    constexpr bool DALT = !GATEUP && !FP4;  // int4 down: the two issuers alternate scale groups
+    constexpr bool DALT = !GATEUP;         // down: one issuer per group, with the whole N
+    constexpr bool ONE = !GATEUP && FP4;   // E2M1 down: one tile = one group, so issuer 0 takes all
     using C = I4Cfg<BN, GATEUP, FP4>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -324,40 +325,39 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
             // ------------------------------ MMA issuers -------------------------------
             // Two threads in different warps share the MMAs: a tcgen05.commit holds up the
             // issuing thread, which one thread alone cannot hide behind the short N <= 96 MMAs.
-            // gate|up: issuer 0 multiplies the gate weights and issuer 1 the up weights; E2M1
-            // down: each takes half of the tile's token columns (the MMA's N), into its half of
-            // the accumulator; both wait for and release every stage.  int4 down: the issuers
+            // gate|up: issuer 0 multiplies the gate weights and issuer 1 the up weights; both
+            // wait for and release every stage.  int4 down: the issuers
             // take alternate 128-element scale groups (each its own TMEM slot) with the whole N,
             // so a stage costs four MMAs instead of eight; each waits for and releases the
             // stages of its groups only.  That is safe with parity waits because an issuer skips
             // only two stages at a time: the dequantisers cannot complete a stage more than NM
             // stages past an MMA stage that has not been issued, so no barrier an issuer waits
-            // on is ever two phases ahead of it.  (Alternating whole E2M1 tiles, 24 stages
-            // apiece, let the full-size MXFP4 layer time out, so those keep the N split.)
+            // on is ever two phases ahead of it.  E2M1 down: a tile's whole K is one group, and
+            // alternating whole tiles (24 stages and more apiece) lets the barriers run phases
+            // ahead of the skipping issuer (the full-size MXFP4 layer timed out), so issuer 0
+            // issues every stage with the whole N and issuer 1 idles.
             const int mt = warp - 1;
-            if (lane == 0) {
+            if (lane == 0 && !(ONE && mt == 1)) {
                 uint32_t it = 0, ai = 0;
                 for (int w = blockIdx.x; w < total; w += gridDim.x) {
                     const TileInfo tl = decode_tile<BN, true>(args, stt, w, tot0);
-                    // MMA N: the tile's valid rows rounded up to 16 (gate|up, int4 down) or, split in
-                    // two halves of a multiple of 16 each, to 32 (E2M1 down); partial tiles cost no
-                    // work on absent rows
-                    const int n_mma = GATEUP || DALT ? min(BN, (tl.nrows + 15) & ~15) : min(BN, (tl.nrows + 31) & ~31) / 2;
+                    // MMA N: the tile's valid rows rounded up to 16; partial tiles cost no work on
+                    // absent rows
+                    const int n_mma = min(BN, (tl.nrows + 15) & ~15);
                     const uint32_t kIdesc = instr_desc(kTileM, n_mma, 1, 1);
                     // int4: one TMEM slot per 128-element scale group; E2M1 formats: one for the K
                     const int ngrp = FP4 ? 1 : args.seg[tl.seg].K / kGroupK;
                     const int spg = FP4 ? args.seg[tl.seg].K / kKE : C::STAGES_PER_GROUP;
                     for (int g = 0; g < ngrp; ++g, ++ai) {
-                        if (DALT && (int)(ai & 1) != mt) {  // the other issuer's group
+                        if (DALT && !ONE && (int)(ai & 1) != mt) {  // the other issuer's group
                             it += spg;
                             continue;
                         }
                         const int slot = ai % C::NSLOT;
                         if (!mbar_wait(&acce[slot], ((ai / C::NSLOT) & 1) ^ 1, abort_flag, status, tmo)) goto done;
                         tc_fence_after();
-                        // gate|up: this issuer's matrix; E2M1 down: its half of the token columns
-                        const uint32_t d =
-                            tmem_base + C::A_TMEM + slot * C::SLOT_COLS + (GATEUP ? mt * BN : DALT ? 0 : mt * n_mma);
+                        // gate|up: this issuer's matrix; down: the whole slot
+                        const uint32_t d = tmem_base + C::A_TMEM + slot * C::SLOT_COLS + (GATEUP ? mt * BN : 0);
                         for (int sk = 0; sk < spg; ++sk, ++it) {
                             const int s = it % C::NM;
                             const int bs = it % C::NB;
@@ -367,8 +367,7 @@ __global__ void __launch_bounds__(I4Cfg<BN, GATEUP, FMT != kFmtInt4>::THREADS, 1
                             const uint32_t a = tmem_base + s * C::NA * C::A_COLS + (GATEUP ? mt * C::A_COLS : 0);
                             // down: the second half's token rows start n_mma rows (n_mma * 128 bytes,
                             // whole 8-row swizzle atoms) into the activation stage
-                            const uint64_t db =
-                                smem_desc_sw128(bst + bs * C::B_BYTES) + (GATEUP || DALT ? 0 : (uint64_t)(mt * n_mma * 8));
+                            const uint64_t db = smem_desc_sw128(bst + bs * C::B_BYTES);
 #pragma unroll
                             for (int kk = 0; kk < kKE / 16; ++kk)
                                 mma_bf16_ts(d, a + 8 * kk, db + 2 * kk, kIdesc, (sk > 0 || kk > 0) ? 1u : 0u);
